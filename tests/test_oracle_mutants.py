@@ -1,0 +1,84 @@
+"""Mutation check of the oracle's pins.
+
+Each case below plants one plausible mistake in a copy of the oracle's C source
+(on the CPU, in a temporary directory), builds it, and runs the pin tests of
+``test_oracle_pins`` against that build.  The pins must reject every mutant;
+a mutant that survives means a mistake of that kind would go unnoticed.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import tests.test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")
+
+# (name, original text, replacement) -- every replacement keeps memory accesses in bounds.
+MUTANTS = [
+    ("no_decay", "for (int i = 0; i < DK * DV; ++i) S[i] *= a;", "(void)a;"),
+    ("error_sign", "e[j] = v[j] - p;", "e[j] = v[j] + p;"),
+    ("no_beta", "S[i * DV + j] += b * kh[i] * e[j];", "S[i * DV + j] += kh[i] * e[j];"),
+    ("error_from_undecayed_state",
+     "    for (int i = 0; i < DK * DV; ++i) S[i] *= a;\n    /* (2) e = v - St^T kh */\n"
+     "    for (int j = 0; j < DV; ++j) {\n        double p = 0.0;\n"
+     "        for (int i = 0; i < DK; ++i) p += S[i * DV + j] * kh[i];\n"
+     "        e[j] = v[j] - p;\n    }\n",
+     "    for (int j = 0; j < DV; ++j) {\n        double p = 0.0;\n"
+     "        for (int i = 0; i < DK; ++i) p += S[i * DV + j] * kh[i];\n"
+     "        e[j] = v[j] - p;\n    }\n    for (int i = 0; i < DK * DV; ++i) S[i] *= a;\n"),
+    ("output_reads_query_unnormalised", "l2norm_vec(J->q + th * DK, DK, J->eps, J->l2norm, qh);\n"
+     "        gdn_step(S, kh, qh, J->v + th * DV, J->alpha[th], J->beta[th], J->scale,\n"
+     "                 J->y ? J->y + th * DV : NULL, e, DK, DV);",
+     "l2norm_vec(J->q + th * DK, DK, J->eps, 0, qh);\n"
+     "        gdn_step(S, kh, qh, J->v + th * DV, J->alpha[th], J->beta[th], J->scale,\n"
+     "                 J->y ? J->y + th * DV : NULL, e, DK, DV);"),
+    ("norm_without_sqrt", "double r = 1.0 / sqrt(ss + eps);", "double r = 1.0 / (ss + eps);"),
+    ("y_scale_dropped", "y[j] = scale * acc;", "y[j] = acc;"),
+    ("bwd_dalpha_uses_dS", "for (size_t i = 0; i < ssz; ++i) da += dSt[i] * Sprev[i];",
+     "for (size_t i = 0; i < ssz; ++i) da += dS[i] * Sprev[i];"),
+    ("bwd_dk_sign", "dkh[i] -= acc;", "dkh[i] += acc;"),
+    ("bwd_state_grad_not_decayed", "for (size_t i = 0; i < ssz; ++i) dS[i] = a * dSt[i];",
+     "for (size_t i = 0; i < ssz; ++i) dS[i] = dSt[i];"),
+    ("bwd_norm_projection_dropped", "for (int i = 0; i < n; ++i) dx[i] = (dxh[i] - xh[i] * dot) * r;",
+     "for (int i = 0; i < n; ++i) dx[i] = dxh[i] * r;"),
+    ("bwd_dbeta_missing_error", "db += kh[i] * acc;", "db += kh[i];"),
+    ("bwd_output_grad_unscaled", "dS[i * DV + j] += J->scale * qh[i] * dyv[j];",
+     "dS[i * DV + j] += qh[i] * dyv[j];"),
+]
+
+# Pin tests that only use the C oracle (the chunked form is a separate implementation).
+PIN_TESTS = [
+    lambda: pins.test_hand_worked_examples("scalar_three_tokens.txt"),
+    lambda: pins.test_hand_worked_examples("two_by_three.txt"),
+    lambda: pins.test_hand_worked_examples("l2norm_one_token.txt"),
+    pins.test_alpha1_beta0_is_identity,
+    pins.test_one_token_outer_product,
+    pins.test_beta1_unit_key_writes_exactly,
+    pins.test_beta0_closed_form,
+    pins.test_scale_multiplies_y_only,
+    lambda: pins.test_chunked_form_matches_token_loop(16, True),
+    lambda: pins.test_chunked_form_matches_token_loop(16, False),
+    lambda: pins.test_backward_matches_central_differences(True),
+    lambda: pins.test_backward_matches_central_differences(False),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_reject_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mut = tmp_path / f"{name}.c"
+    mut.write_text(src.replace(old, new))
+    lib = tmp_path / f"{name}.so"
+    subprocess.check_call(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-pthread", "-o",
+                           str(lib), str(mut), "-lm"])
+    caught = []
+    with oracle.use_library(str(lib)):
+        for t in PIN_TESTS:
+            try:
+                t()
+            except AssertionError:
+                caught.append(t)
+    assert caught, f"no pin rejects the planted mistake {name!r}"
