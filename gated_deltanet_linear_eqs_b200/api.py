@@ -1,0 +1,192 @@
+"""Python binding of libgdn.so with the C ABI's names.
+
+Argument marshalling only: every function checks that the torch tensors are CUDA,
+contiguous and of the expected dtype, allocates the outputs (and workspace) it is not
+given, and calls the C entry point on the current CUDA stream.  Every arithmetic step
+runs in the library's kernels; a non-OK status raises ``GdnError``.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import GdnError
+
+_DT = {torch.bfloat16: _abi.GDN_BF16, torch.float32: _abi.GDN_FP32}
+
+
+def _lib():
+    return _abi.load()
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _p(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t, name, dtype=None, shape=None, optional=False):
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _check(rc, what):
+    if rc != _abi.GDN_OK:
+        raise GdnError(rc, what)
+
+
+def gdn_workspace_bytes(op, B, T, H, dk, dv, num_seqs=0):
+    n = ctypes.c_size_t(0)
+    _check(_lib().gdn_workspace_bytes(int(op), B, T, H, dk, dv, num_seqs, ctypes.byref(n)),
+           "gdn_workspace_bytes")
+    return int(n.value)
+
+
+def _workspace(op, device, B, T, H, dk, dv, num_seqs=0, ws=None):
+    n = gdn_workspace_bytes(op, B, T, H, dk, dv, num_seqs)
+    if n == 0:
+        return None, 0
+    if ws is None:
+        ws = torch.empty(n, dtype=torch.uint8, device=device)
+    return ws, ws.numel() * ws.element_size()
+
+
+def gdn_prefill(q, k, v, alpha, beta, s0=None, scale=1.0, l2norm_qk=True, y=None,
+                s_final=None, want_final=True, ws=None, stream=None):
+    """q,k [B,T,H,dk], v [B,T,H,dv] (bf16 or fp32), alpha,beta [B,T,H] fp32,
+    s0 [B,H,dk,dv] fp32 or None.  Returns (y, s_final)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _need(q, "q", dt)
+    _need(k, "k", dt, q.shape)
+    _need(v, "v", dt, (B, T, H, dv))
+    _need(alpha, "alpha", torch.float32, (B, T, H))
+    _need(beta, "beta", torch.float32, (B, T, H))
+    _need(s0, "s0", torch.float32, (B, H, dk, dv), optional=True)
+    if y is None:
+        y = torch.empty((B, T, H, dv), dtype=dt, device=q.device)
+    _need(y, "y", dt, (B, T, H, dv))
+    if s_final is None and want_final:
+        s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(s_final, "s_final", torch.float32, (B, H, dk, dv), optional=True)
+    ws, wsb = _workspace(_abi.GDN_OP_PREFILL, q.device, B, T, H, dk, dv, ws=ws)
+    rc = _lib().gdn_prefill(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(s0), _p(y),
+                            _p(s_final), B, T, H, dk, dv, _DT[dt], float(scale),
+                            int(bool(l2norm_qk)), _p(ws), wsb, _stream(stream))
+    _check(rc, "gdn_prefill")
+    return y, s_final
+
+
+def gdn_prefill_varlen(q, k, v, alpha, beta, cu_seqlens, s0=None, scale=1.0, l2norm_qk=True,
+                       y=None, s_final=None, ws=None, stream=None):
+    """Packed documents: q,k [1,T,H,dk] (or [T,H,dk]), v likewise, alpha,beta [1,T,H],
+    cu_seqlens int32 [N+1] on the device, s0 [N,H,dk,dv] or None.  Returns (y, s_final)."""
+    if q.dim() == 3:
+        q, k, v, alpha, beta = (x.unsqueeze(0) for x in (q, k, v, alpha, beta))
+    _, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError("q/k/v must be bf16 or fp32")
+    N = cu_seqlens.numel() - 1
+    _need(q, "q", dt)
+    _need(k, "k", dt, q.shape)
+    _need(v, "v", dt, (1, T, H, dv))
+    _need(alpha, "alpha", torch.float32, (1, T, H))
+    _need(beta, "beta", torch.float32, (1, T, H))
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,))
+    _need(s0, "s0", torch.float32, (N, H, dk, dv), optional=True)
+    if y is None:
+        y = torch.empty((1, T, H, dv), dtype=dt, device=q.device)
+    _need(y, "y", dt, (1, T, H, dv))
+    if s_final is None:
+        s_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(s_final, "s_final", torch.float32, (N, H, dk, dv))
+    ws, wsb = _workspace(_abi.GDN_OP_PREFILL_VARLEN, q.device, 1, T, H, dk, dv, N, ws=ws)
+    rc = _lib().gdn_prefill_varlen(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(cu_seqlens), N,
+                                   _p(s0), _p(y), _p(s_final), T, H, dk, dv, _DT[dt],
+                                   float(scale), int(bool(l2norm_qk)), _p(ws), wsb,
+                                   _stream(stream))
+    _check(rc, "gdn_prefill_varlen")
+    return y, s_final
+
+
+def gdn_decode_step(q, k, v, alpha, beta, state, scale=1.0, l2norm_qk=True, y=None,
+                    stream=None):
+    """q,k [N,H,dk], v [N,H,dv], alpha,beta [N,H], state [N,H,dk,dv] fp32 (updated in
+    place).  Returns y [N,H,dv]."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _need(q, "q", dt)
+    _need(k, "k", dt, q.shape)
+    _need(v, "v", dt, (N, H, dv))
+    _need(alpha, "alpha", torch.float32, (N, H))
+    _need(beta, "beta", torch.float32, (N, H))
+    _need(state, "state", torch.float32, (N, H, dk, dv))
+    if y is None:
+        y = torch.empty((N, H, dv), dtype=dt, device=q.device)
+    _need(y, "y", dt, (N, H, dv))
+    rc = _lib().gdn_decode_step(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(state), _p(y), N, H,
+                                dk, dv, _DT[dt], float(scale), int(bool(l2norm_qk)),
+                                _stream(stream))
+    _check(rc, "gdn_decode_step")
+    return y
+
+
+def gdn_backward(q, k, v, alpha, beta, dy, s0=None, ds_final=None, scale=1.0, l2norm_qk=True,
+                 want_ds0=True, ws=None, stream=None):
+    """Gradients of (y, s_final) w.r.t. (q, k, v, alpha, beta, s0) given dy and ds_final.
+    Returns dict dq, dk, dv, dalpha, dbeta, ds0."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _need(q, "q", dt)
+    _need(k, "k", dt, q.shape)
+    _need(v, "v", dt, (B, T, H, dv))
+    _need(alpha, "alpha", torch.float32, (B, T, H))
+    _need(beta, "beta", torch.float32, (B, T, H))
+    _need(dy, "dy", dt, (B, T, H, dv))
+    _need(s0, "s0", torch.float32, (B, H, dk, dv), optional=True)
+    _need(ds_final, "ds_final", torch.float32, (B, H, dk, dv), optional=True)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               dalpha=torch.empty_like(alpha), dbeta=torch.empty_like(beta),
+               ds0=torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+               if want_ds0 else None)
+    ws, wsb = _workspace(_abi.GDN_OP_BACKWARD, q.device, B, T, H, dk, dv, ws=ws)
+    rc = _lib().gdn_backward(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(s0), _p(dy),
+                             _p(ds_final), _p(out["dq"]), _p(out["dk"]), _p(out["dv"]),
+                             _p(out["dalpha"]), _p(out["dbeta"]), _p(out["ds0"]), B, T, H, dk,
+                             dv, _DT[dt], float(scale), int(bool(l2norm_qk)), _p(ws), wsb,
+                             _stream(stream))
+    _check(rc, "gdn_backward")
+    return out
+
+
+def gdn_read_device_status(reset=True):
+    st = ctypes.c_int(0)
+    _check(_lib().gdn_read_device_status(int(bool(reset)), ctypes.byref(st)),
+           "gdn_read_device_status")
+    return int(st.value)

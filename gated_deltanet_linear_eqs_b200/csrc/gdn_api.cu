@@ -1,0 +1,196 @@
+// gdn_api.cu -- the C ABI of libgdn.so: argument validation, device checks, dispatch.
+//
+// Every entry point validates its arguments on the host first and launches nothing when
+// they are rejected; see include/gdn.h for the contract of each call.
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+// Device status word: kernels record the first device-side error here (bounded waits
+// that ran out).  One per device; its address is looked up once per device.
+__device__ int g_device_status;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    bool sm100 = false;
+    int* status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+int current_device_info(DeviceInfo* out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return GDN_ERR_CUDA;
+        }
+        d.sm100 = (major == 10);
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
+            cudaGetLastError();
+            return GDN_ERR_CUDA;
+        }
+        d.status = static_cast<int*>(p);
+        d.ready = true;
+    }
+    *out = d;
+    return d.sm100 ? GDN_OK : GDN_ERR_UNSUPPORTED_DEVICE;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+bool ok_opt_ptr(const void* p) { return p == nullptr || aligned16(p); }
+
+int check_dims(int dk, int dv, int dtype) {
+    if (dtype != GDN_BF16 && dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (dk != dv || (dk != 64 && dk != 128)) return GDN_ERR_UNSUPPORTED_SHAPE;
+    return GDN_OK;
+}
+
+int map_cuda(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* gdn_status_string(int status) {
+    switch (status) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: null/misaligned pointer or bad size";
+        case GDN_ERR_UNSUPPORTED_SHAPE: return "GDN_ERR_UNSUPPORTED_SHAPE: need dk == dv in {64, 128}";
+        case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing or too small";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA call or kernel launch failed";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: a device-side bounded wait ran out";
+        case GDN_ERR_UNSUPPORTED_DEVICE: return "GDN_ERR_UNSUPPORTED_DEVICE: needs an sm_100 GPU";
+        default: return "GDN_ERR_UNKNOWN";
+    }
+}
+
+const char* gdn_version(void) { return "gdn-b200 0.1"; }
+
+int gdn_workspace_bytes(int op, int B, int T, int H, int dk, int dv, int num_seqs,
+                        size_t* bytes) {
+    if (!bytes) return GDN_ERR_INVALID_ARG;
+    *bytes = 0;
+    if (T < 1 || H < 1 || dk < 1 || dv < 1) return GDN_ERR_INVALID_ARG;
+    switch (op) {
+        case GDN_OP_PREFILL:
+        case GDN_OP_DECODE:
+            if (B < 1) return GDN_ERR_INVALID_ARG;
+            return GDN_OK;
+        case GDN_OP_PREFILL_VARLEN:
+            if (num_seqs < 1) return GDN_ERR_INVALID_ARG;
+            return GDN_OK;
+        case GDN_OP_BACKWARD:
+            if (B < 1) return GDN_ERR_INVALID_ARG;
+            *bytes = gdn::backward_workspace_bytes(B, T, H, dk, dv);
+            return GDN_OK;
+        default:
+            return GDN_ERR_INVALID_ARG;
+    }
+}
+
+int gdn_prefill(const void* q, const void* k, const void* v, const float* alpha,
+                const float* beta, const float* s0, void* y, float* s_final, int B, int T, int H,
+                int dk, int dv, int dtype, float scale, int l2norm_qk, void* ws, size_t ws_bytes,
+                void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
+        !ok_ptr(y) || !ok_opt_ptr(s0) || !ok_opt_ptr(s_final))
+        return GDN_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (int rc = check_dims(dk, dv, dtype)) return rc;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::PrefillArgs a{q, k, v, alpha, beta, s0, y, s_final, nullptr, B, T, H, dk, dv,
+                       dtype, scale, l2norm_qk ? 1 : 0, dev.status};
+    return map_cuda(gdn::launch_prefill(a, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float* alpha,
+                       const float* beta, const int32_t* cu_seqlens, int num_seqs,
+                       const float* s0, void* y, float* s_final, int T, int H, int dk, int dv,
+                       int dtype, float scale, int l2norm_qk, void* ws, size_t ws_bytes,
+                       void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
+        !ok_ptr(y) || cu_seqlens == nullptr || !ok_opt_ptr(s0) || !ok_opt_ptr(s_final))
+        return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 1 || T < 1 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (int rc = check_dims(dk, dv, dtype)) return rc;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::PrefillArgs a{q, k, v, alpha, beta, s0, y, s_final, cu_seqlens, num_seqs, T, H, dk, dv,
+                       dtype, scale, l2norm_qk ? 1 : 0, dev.status};
+    return map_cuda(gdn::launch_prefill(a, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_decode_step(const void* q, const void* k, const void* v, const float* alpha,
+                    const float* beta, float* state, void* y, int N, int H, int dk, int dv,
+                    int dtype, float scale, int l2norm_qk, void* stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
+        !ok_ptr(state) || !ok_ptr(y))
+        return GDN_ERR_INVALID_ARG;
+    if (N < 1 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (int rc = check_dims(dk, dv, dtype)) return rc;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::DecodeArgs a{q, k, v, alpha, beta, state, y, N, H, dk, dv, dtype, scale,
+                      l2norm_qk ? 1 : 0};
+    return map_cuda(gdn::launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_backward(const void* q, const void* k, const void* v, const float* alpha,
+                 const float* beta, const float* s0, const void* dy, const float* ds_final,
+                 void* dq, void* dk_out, void* dv_out, float* dalpha, float* dbeta, float* ds0,
+                 int B, int T, int H, int dk, int dv, int dtype, float scale, int l2norm_qk,
+                 void* ws, size_t ws_bytes, void* stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
+        !ok_ptr(dy) || !ok_ptr(dq) || !ok_ptr(dk_out) || !ok_ptr(dv_out) || !ok_ptr(dalpha) ||
+        !ok_ptr(dbeta) || !ok_opt_ptr(s0) || !ok_opt_ptr(ds_final) || !ok_opt_ptr(ds0))
+        return GDN_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (int rc = check_dims(dk, dv, dtype)) return rc;
+    const size_t need = gdn::backward_workspace_bytes(B, T, H, dk, dv);
+    if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return GDN_ERR_WORKSPACE;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::BackwardArgs a{q, k, v, alpha, beta, s0, dy, ds_final, dq, dk_out, dv_out, dalpha,
+                        dbeta, ds0, B, T, H, dk, dv, dtype, scale, l2norm_qk ? 1 : 0, ws,
+                        ws_bytes, dev.status};
+    return map_cuda(gdn::launch_backward(a, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_read_device_status(int reset, int* device_status) {
+    if (!device_status) return GDN_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    int h = 0;
+    if (cudaMemcpy(&h, dev.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (reset && h != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(dev.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    *device_status = h;
+    return GDN_OK;
+}
+
+}  // extern "C"

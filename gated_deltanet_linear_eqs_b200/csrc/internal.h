@@ -1,0 +1,58 @@
+// internal.h -- host-side launch interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdn {
+
+struct DecodeArgs {
+    const void *q, *k, *v;
+    const float *alpha, *beta;
+    float* state;
+    void* y;
+    int N, H, dk, dv, dtype;
+    float scale;
+    int l2norm;
+};
+
+// Dense prefill is the varlen case with B documents of T tokens each (cu_seqlens == nullptr).
+struct PrefillArgs {
+    const void *q, *k, *v;
+    const float *alpha, *beta;
+    const float* s0;
+    void* y;
+    float* s_final;
+    const int32_t* cu_seqlens;  // device, [num_seqs+1]; nullptr for the dense layout
+    int num_seqs;               // documents (dense: B)
+    int T;                      // tokens per sequence (dense) or packed total (varlen)
+    int H, dk, dv, dtype;
+    float scale;
+    int l2norm;
+    int* status;                // device status word
+};
+
+struct BackwardArgs {
+    const void *q, *k, *v;
+    const float *alpha, *beta, *s0;
+    const void* dy;
+    const float* ds_final;
+    void *dq, *dk, *dv;
+    float *dalpha, *dbeta, *ds0;
+    int B, T, H, dkdim, dvdim, dtype;
+    float scale;
+    int l2norm;
+    void* ws;
+    size_t ws_bytes;
+    int* status;
+};
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st);
+cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st);
+
+// Workspace the backward pass needs (chunk-start states), bytes.
+size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv);
+
+}  // namespace gdn

@@ -1,0 +1,148 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: the Gated DeltaNet token-mixer recurrence on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (Qwen3.8-Flash-Next summary, picx.dev, "Theoretical
+ * foundations", eqs. (1)-(4)), per sequence and head, with a state
+ * S in R^{dk x dv}:
+ *
+ *     St  = alpha_t S_{t-1}            e_t = v_t - St^T k_t
+ *     S_t = St + beta_t k_t e_t^T      y_t = scale * S_t^T q_t
+ *
+ * alpha_t, beta_t are one scalar per (token, head); the pages give their range
+ * as (0, 1) (same passage).  When l2norm_qk != 0, q and k are first replaced by
+ * x / sqrt(sum(x^2) + 1e-6) (same page, "Methodology", "1. GDN Hybrid Token
+ * Mixing": L2 normalisation of queries and keys; the exact formula and epsilon
+ * are this library's reading).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers to dense, row-major (C-order)
+ *    arrays, last index fastest, each 16-byte aligned.  The caller owns every
+ *    buffer; the library allocates nothing and keeps no state between calls.
+ *  - Token tensors: q, k [B, T, H, dk]; v, y, dy [B, T, H, dv] in `dtype`
+ *    (bf16 or fp32).  alpha, beta, dalpha, dbeta [B, T, H] fp32.  States
+ *    s0, s_final, ds_final, ds0 [B, H, dk, dv] fp32 (varlen: [num_seqs, ...]).
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *    asynchronous and stream ordered; arguments are validated on the host before
+ *    anything is launched, and a rejected call launches nothing.
+ *  - Supported sizes: dk == dv, both 64 or 128.  H >= 1, T >= 1, B >= 1.
+ *  - Domain: alpha in (0, 1], beta in [0, 1]; not checked on the device.
+ *  - Return value: a gdn_status.  Launch failures map to GDN_ERR_CUDA.  Errors
+ *    found inside a kernel (a bounded wait that ran out) are recorded in a
+ *    device status word read with gdn_read_device_status().  Nothing throws.
+ *  - The calls are thread safe: no global mutable host state is touched after
+ *    the first call on a device (which caches its properties).
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,       /* null pointer, bad size, misaligned pointer, bad cu_seqlens */
+    GDN_ERR_UNSUPPORTED_SHAPE = 2, /* dk/dv outside the supported set */
+    GDN_ERR_WORKSPACE = 3,         /* workspace missing or smaller than gdn_workspace_bytes() */
+    GDN_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
+    GDN_ERR_TIMEOUT = 5,           /* a device-side bounded wait ran out (device status word) */
+    GDN_ERR_UNSUPPORTED_DEVICE = 6 /* the current device is not sm_100 */
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
+
+typedef enum {
+    GDN_OP_PREFILL = 0,
+    GDN_OP_PREFILL_VARLEN = 1,
+    GDN_OP_DECODE = 2,
+    GDN_OP_BACKWARD = 3
+} gdn_op;
+
+/* Static description of a status code.  Never NULL. */
+const char* gdn_status_string(int status);
+
+/* Library version string, e.g. "gdn-b200 0.1". */
+const char* gdn_version(void);
+
+/*
+ * Workspace (device scratch memory, caller-allocated) needed by `op` at the given
+ * sizes, in bytes, written to *bytes.  num_seqs is only read for
+ * GDN_OP_PREFILL_VARLEN (T is then the packed token count).  A size of 0 means
+ * the op needs no workspace and ws may be NULL.
+ * Errors: GDN_ERR_INVALID_ARG (bytes NULL, bad sizes, unknown op).
+ */
+int gdn_workspace_bytes(int op, int B, int T, int H, int dk, int dv, int num_seqs,
+                        size_t* bytes);
+
+/*
+ * gdn_prefill -- chunked (64-token chunks) forward over B independent sequences
+ * of T tokens: writes y and, if s_final is non-NULL, the state after the last
+ * token.  s0 == NULL means S_0 = 0.  The computation is exactly eqs. (1)-(4)
+ * above, rearranged chunk-wise (WY/UT form), on the tensor cores.
+ *   q, k  [B,T,H,dk]  dtype        v [B,T,H,dv] dtype
+ *   alpha, beta [B,T,H] fp32       s0 [B,H,dk,dv] fp32 or NULL
+ *   y [B,T,H,dv] dtype (output)    s_final [B,H,dk,dv] fp32 or NULL (output)
+ *   ws/ws_bytes: see gdn_workspace_bytes(GDN_OP_PREFILL, ...).
+ */
+int gdn_prefill(const void* q, const void* k, const void* v, const float* alpha,
+                const float* beta, const float* s0, void* y, float* s_final, int B, int T, int H,
+                int dk, int dv, int dtype, float scale, int l2norm_qk, void* ws, size_t ws_bytes,
+                void* stream);
+
+/*
+ * gdn_prefill_varlen -- as gdn_prefill over ONE packed stream of T tokens
+ * (tensors laid out with B = 1) holding num_seqs documents: document n covers
+ * tokens cu_seqlens[n] .. cu_seqlens[n+1]-1 and starts from s0[n] (zero if s0
+ * is NULL); its final state goes to s_final[n].
+ *   cu_seqlens: DEVICE int32 [num_seqs+1], cu_seqlens[0] = 0, non-decreasing,
+ *   cu_seqlens[num_seqs] = T.  Empty documents are allowed (their s_final is
+ *   s0 or 0).  The kernel reads cu_seqlens on the device (no host sync); the
+ *   values themselves are not validated on the host.
+ */
+int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float* alpha,
+                       const float* beta, const int32_t* cu_seqlens, int num_seqs,
+                       const float* s0, void* y, float* s_final, int T, int H, int dk, int dv,
+                       int dtype, float scale, int l2norm_qk, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/*
+ * gdn_decode_step -- one new token for each of N independent sequences
+ * (eqs. (1)-(4) with T = 1).  The state is read once and written once, in place.
+ *   q, k [N,H,dk] dtype   v [N,H,dv] dtype   alpha, beta [N,H] fp32
+ *   state [N,H,dk,dv] fp32 (input and output)   y [N,H,dv] dtype (output)
+ */
+int gdn_decode_step(const void* q, const void* k, const void* v, const float* alpha,
+                    const float* beta, float* state, void* y, int N, int H, int dk, int dv,
+                    int dtype, float scale, int l2norm_qk, void* stream);
+
+/*
+ * gdn_backward -- gradients of L(y, s_final) given dy and ds_final (NULL = 0),
+ * with respect to the raw q, k (through the normalisation when l2norm_qk), v,
+ * alpha (d/d alpha itself), beta and s0 (ds0 may be NULL if not wanted).
+ * Dense layout as gdn_prefill.  dq, dk_out, dv_out have q/k/v's dtype; dalpha,
+ * dbeta [B,T,H] fp32; ds0 [B,H,dk,dv] fp32.
+ *   ws/ws_bytes: see gdn_workspace_bytes(GDN_OP_BACKWARD, ...).
+ */
+int gdn_backward(const void* q, const void* k, const void* v, const float* alpha,
+                 const float* beta, const float* s0, const void* dy, const float* ds_final,
+                 void* dq, void* dk_out, void* dv_out, float* dalpha, float* dbeta, float* ds0,
+                 int B, int T, int H, int dk, int dv, int dtype, float scale, int l2norm_qk,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Device status word of the current device: 0 when no kernel has recorded an
+ * error, otherwise the first gdn_status a kernel recorded (GDN_ERR_TIMEOUT).
+ * Synchronises the current device.  If reset != 0 the word is cleared.
+ */
+int gdn_read_device_status(int reset, int* device_status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

@@ -1,0 +1,142 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every entry
+point that include/gdn.h declares, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_deltanet_linear_eqs_b200 import _abi
+from gated_deltanet_linear_eqs_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return _abi.load()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = _declared_functions()
+    for n in ("gdn_prefill", "gdn_prefill_varlen", "gdn_decode_step", "gdn_backward"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _abi.SIGNATURES, f"{name} has no ctypes signature"
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = lib.gdn_status_string(code).decode()
+        assert s.startswith("GDN_")
+    assert lib.gdn_status_string(99).decode() == "GDN_ERR_UNKNOWN"
+    assert lib.gdn_version().decode().startswith("gdn-b200")
+
+
+def test_workspace_bytes(lib):
+    n = ctypes.c_size_t(7)
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL, 1, 4096, 16, 128, 128, 0,
+                                   ctypes.byref(n)) == 0
+    assert n.value == 0
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_BACKWARD, 8, 4096, 32, 128, 128, 0,
+                                   ctypes.byref(n)) == 0
+    assert n.value == 64 * 8 * 32 * 128 * 128 * 4  # one fp32 state per 64-token chunk
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_BACKWARD, 1, 65, 1, 64, 64, 0,
+                                   ctypes.byref(n)) == 0
+    assert n.value == 2 * 64 * 64 * 4
+    assert lib.gdn_workspace_bytes(42, 1, 1, 1, 64, 64, 0, ctypes.byref(n)) == \
+        _abi.GDN_ERR_INVALID_ARG
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL_VARLEN, 1, 10, 1, 64, 64, 0,
+                                   ctypes.byref(n)) == _abi.GDN_ERR_INVALID_ARG
+    assert lib.gdn_workspace_bytes(0, 1, 1, 1, 64, 64, 0, None) == _abi.GDN_ERR_INVALID_ARG
+
+
+A = 0x10000  # a 16-byte-aligned fake address: validation must reject before any access
+
+
+def _prefill(lib, **kw):
+    args = dict(q=A, k=A, v=A, alpha=A, beta=A, s0=0, y=A, sf=0, B=1, T=64, H=1, dk=128, dv=128,
+                dt=0, scale=1.0, l2=1, ws=0, wsb=0)
+    args.update(kw)
+    return lib.gdn_prefill(args["q"], args["k"], args["v"], args["alpha"], args["beta"],
+                           args["s0"], args["y"], args["sf"], args["B"], args["T"], args["H"],
+                           args["dk"], args["dv"], args["dt"], args["scale"], args["l2"],
+                           args["ws"], args["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), _abi.GDN_ERR_INVALID_ARG),
+    (dict(v=0), _abi.GDN_ERR_INVALID_ARG),
+    (dict(y=0), _abi.GDN_ERR_INVALID_ARG),
+    (dict(k=A + 2), _abi.GDN_ERR_INVALID_ARG),        # misaligned
+    (dict(s0=A + 4), _abi.GDN_ERR_INVALID_ARG),       # misaligned optional pointer
+    (dict(B=0), _abi.GDN_ERR_INVALID_ARG),
+    (dict(T=0), _abi.GDN_ERR_INVALID_ARG),
+    (dict(H=-1), _abi.GDN_ERR_INVALID_ARG),
+    (dict(dt=7), _abi.GDN_ERR_INVALID_ARG),
+    (dict(dk=96, dv=96), _abi.GDN_ERR_UNSUPPORTED_SHAPE),
+    (dict(dk=64, dv=128), _abi.GDN_ERR_UNSUPPORTED_SHAPE),
+])
+def test_prefill_rejects_bad_arguments(lib, kw, code):
+    assert _prefill(lib, **kw) == code
+
+
+def test_varlen_rejects_bad_arguments(lib):
+    f = lib.gdn_prefill_varlen
+    ok = dict(q=A, k=A, v=A, al=A, be=A, cu=A, n=2, s0=0, y=A, sf=A, T=100, H=2, dk=64, dv=64,
+              dt=0)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["q"], a["k"], a["v"], a["al"], a["be"], a["cu"], a["n"], a["s0"], a["y"],
+                 a["sf"], a["T"], a["H"], a["dk"], a["dv"], a["dt"], 1.0, 1, None, 0, None)
+
+    assert call(cu=0) == _abi.GDN_ERR_INVALID_ARG
+    assert call(n=0) == _abi.GDN_ERR_INVALID_ARG
+    assert call(T=0) == _abi.GDN_ERR_INVALID_ARG
+    assert call(dk=32, dv=32) == _abi.GDN_ERR_UNSUPPORTED_SHAPE
+
+
+def test_decode_rejects_bad_arguments(lib):
+    f = lib.gdn_decode_step
+    assert f(A, A, A, A, A, 0, A, 4, 2, 128, 128, 0, 1.0, 1, None) == _abi.GDN_ERR_INVALID_ARG
+    assert f(A, A, A, A, A, A, A, 0, 2, 128, 128, 0, 1.0, 1, None) == _abi.GDN_ERR_INVALID_ARG
+    assert f(A, A, A, A, A, A, A, 4, 2, 256, 256, 0, 1.0, 1, None) == \
+        _abi.GDN_ERR_UNSUPPORTED_SHAPE
+
+
+def test_backward_needs_its_workspace(lib):
+    f = lib.gdn_backward
+    args = [A] * 6 + [A, 0] + [A] * 5 + [A] + [1, 64, 1, 64, 64, 0, 1.0, 1]
+    assert f(*args, None, 0, None) == _abi.GDN_ERR_WORKSPACE
+    assert f(*args, A, 16, None) == _abi.GDN_ERR_WORKSPACE
+    bad = list(args)
+    bad[6] = 0  # dy missing
+    assert f(*bad, A, 1 << 30, None) == _abi.GDN_ERR_INVALID_ARG
+
+
+def test_device_status_rejects_null(lib):
+    assert lib.gdn_read_device_status(0, None) == _abi.GDN_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    saved = _abi._lib
+    try:
+        _abi._lib = None
+        with pytest.raises(ImportError):
+            _abi.load(str(tmp_path / "missing" / "libgdn.so"))
+    finally:
+        _abi._lib = saved
