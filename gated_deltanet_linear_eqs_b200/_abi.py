@@ -9,7 +9,11 @@ import os
 import threading
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libgdn.so")
+# GDN_LIBRARY selects another build of the library (e.g. libgdn_debug.so, the self-checking
+# build); the default is the in-tree libgdn.so.
+LIB_PATH = os.environ.get("GDN_LIBRARY") or os.path.join(PKG, "libgdn.so")
+if not os.path.isabs(LIB_PATH):
+    LIB_PATH = os.path.join(PKG, LIB_PATH)
 
 GDN_OK = 0
 GDN_ERR_INVALID_ARG = 1

@@ -20,6 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgdn.so")
+LIB_DEBUG = os.path.join(PKG, "libgdn_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2",
@@ -45,8 +46,8 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src, obj, verbose_ptxas):
-    cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose_ptxas else []) + \
+def _compile(src, obj, verbose_ptxas, extra=()):
+    cmd = [nvcc()] + NVCC_FLAGS + list(extra) + (["-Xptxas", "-v"] if verbose_ptxas else []) + \
         ["-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
@@ -54,37 +55,45 @@ def _compile(src, obj, verbose_ptxas):
     return r.stderr
 
 
-def build(force: bool = False, verbose_ptxas: bool = False, jobs: int = 0) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, jobs: int = 0,
+          debug: bool = False) -> str:
+    """Compile and link libgdn.so; with debug=True, libgdn_debug.so instead (self-checking
+    kernels: bounds guards that record the failing index rather than fault)."""
+    bdir = os.path.join(BUILD, "debug") if debug else BUILD
+    lib = LIB_DEBUG if debug else LIB
+    extra = ["-DGDN_DEBUG"] if debug else []
+    os.makedirs(bdir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdrs = _headers()
-    objs = [os.path.join(BUILD, os.path.basename(s)[:-3] + ".o") for s in srcs]
+    objs = [os.path.join(bdir, os.path.basename(s)[:-3] + ".o") for s in srcs]
     todo = [(s, o) for s, o in zip(srcs, objs) if force or verbose_ptxas or _stale(o, [s] + hdrs)]
     logs = []
     if todo:
         with cf.ThreadPoolExecutor(max_workers=jobs or min(8, len(todo))) as ex:
-            for s, log in zip(todo, ex.map(lambda so: _compile(so[0], so[1], verbose_ptxas), todo)):
+            for s, log in zip(todo, ex.map(lambda so: _compile(so[0], so[1], verbose_ptxas, extra),
+                                           todo)):
                 if log.strip():
                     logs.append(f"== {os.path.basename(s[0])}\n{log}")
-    if todo or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if todo or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcudart_static", "-ldl",
                                                                  "-lrt", "-lpthread"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
+        os.replace(tmp, lib)
     if verbose_ptxas:
         print("\n".join(logs))
-    return LIB
+    return lib
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="build libgdn_debug.so")
     args = ap.parse_args(argv)
-    print(build(force=args.force, verbose_ptxas=args.verbose_ptxas))
+    print(build(force=args.force, verbose_ptxas=args.verbose_ptxas, debug=args.debug))
 
 
 if __name__ == "__main__":

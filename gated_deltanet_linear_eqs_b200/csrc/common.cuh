@@ -55,3 +55,30 @@ __device__ __forceinline__ void record_status(int* status, int code) {
 }
 
 }  // namespace gdn
+
+// ---- debug-build self checks ---------------------------------------------------------------
+// Compiled in only with -DGDN_DEBUG (libgdn_debug.so).  A failed check records
+// (code, detail, block) in the device status words and the guarded access is skipped, so a
+// bad index is reported instead of faulting.  In the normal build every guard is `true`.
+namespace gdn {
+enum DebugCode {
+    DBG_GLOBAL_OOB = 100,   // global index out of the tensor's extent
+    DBG_SMEM_OOB = 101,     // shared-memory offset outside the kernel's layout
+    DBG_TMEM_OOB = 102,     // TMEM column outside the allocation
+    DBG_WAIT = 103          // bounded wait gave up (detail = barrier id * 65536 + chunk)
+};
+#ifdef GDN_DEBUG
+__device__ __forceinline__ bool debug_fail(int* status, int code, long long detail) {
+    if (status && atomicCAS(status, 0, code) == 0) {
+        status[1] = (int)detail;
+        status[2] = (int)(detail >> 32);
+        status[3] = (int)blockIdx.x;
+    }
+    return false;
+}
+#define GDN_GUARD(cond, status, code, detail) \
+    ((cond) || ::gdn::debug_fail((status), (code), (long long)(detail)))
+#else
+#define GDN_GUARD(cond, status, code, detail) true
+#endif
+}  // namespace gdn

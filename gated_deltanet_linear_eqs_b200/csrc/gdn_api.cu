@@ -9,9 +9,10 @@
 
 namespace {
 
-// Device status word: kernels record the first device-side error here (bounded waits
-// that ran out).  One per device; its address is looked up once per device.
-__device__ int g_device_status;
+// Device status words: kernels record the first device-side error in word 0 (bounded waits
+// that ran out); debug builds add the failing check's detail and block in words 1-3.  One set
+// per device; its address is looked up once per device.
+__device__ int g_device_status[4];
 
 constexpr int kMaxDevices = 64;
 
@@ -185,12 +186,24 @@ int gdn_read_device_status(int reset, int* device_status) {
     if (cudaMemcpy(&h, dev.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return GDN_ERR_CUDA;
     if (reset && h != 0) {
-        const int zero = 0;
-        if (cudaMemcpy(dev.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+        const int zero[4] = {0, 0, 0, 0};
+        if (cudaMemcpy(dev.status, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
             return GDN_ERR_CUDA;
     }
     *device_status = h;
     return GDN_OK;
 }
+
+#ifdef GDN_DEBUG
+// Debug builds only: the four status words (code, detail low, detail high, block).
+int gdn_debug_words(int* out4) {
+    if (!out4) return GDN_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    if (cudaMemcpy(out4, dev.status, 4 * sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    return GDN_OK;
+}
+#endif
 
 }  // extern "C"

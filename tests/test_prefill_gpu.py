@@ -1,0 +1,147 @@
+"""GPU parity of gdn_prefill / gdn_prefill_varlen (through the C ABI) against the fp64 oracle.
+
+Bars: y max|dy|/max|y_ref| <= 1e-2, final states relative Frobenius <= 1e-3."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_linear_eqs_b200 import api
+from gated_deltanet_linear_eqs_b200.inputs import (make_inputs, make_varlen_inputs,
+                                                   varlen_lengths)
+from tests._metrics import S_TOL, Y_TOL, frob_rel, max_rel
+
+pytestmark = pytest.mark.gpu
+
+
+def _cuda(d):
+    return {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in d.items()}
+
+
+def _run_dense(inp, scale=1.0, l2norm=True):
+    g = _cuda(inp)
+    y, sf = api.gdn_prefill(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["s0"], scale=scale,
+                            l2norm_qk=l2norm)
+    torch.cuda.synchronize()
+    return y, sf
+
+
+@pytest.mark.parametrize("B,T,H,d,with_s0", [
+    (1, 64, 1, 128, False),     # one full chunk
+    (1, 256, 2, 64, False),     # several chunks, d = 64
+    (2, 200, 3, 128, True),     # ragged tail (200 = 3*64 + 8), initial state
+    (3, 1, 2, 128, True),       # single token
+    (1, 130, 2, 64, True),      # ragged, d = 64
+])
+def test_prefill_dense_small(B, T, H, d, with_s0):
+    inp = make_inputs(B, T, H, d, d, seed=B * 1000 + T, with_s0=with_s0)
+    y, sf = _run_dense(inp)
+    yr, sr = oracle.forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["s0"])
+    assert max_rel(y, yr) <= Y_TOL
+    assert frob_rel(sf, sr) <= S_TOL
+
+
+def test_prefill_scale_and_no_norm():
+    B, T, H, d = 1, 150, 2, 128
+    inp = make_inputs(B, T, H, d, d, seed=7, with_s0=True)
+    for n in ("q", "k"):  # unit rows, so the un-normalised path sees the method's domain
+        x = inp[n].double()
+        inp[n] = (x / x.norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+    y, sf = _run_dense(inp, scale=0.125, l2norm=False)
+    yr, sr = oracle.forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["s0"],
+                            scale=0.125, l2norm=False)
+    assert max_rel(y, yr) <= Y_TOL
+    assert frob_rel(sf, sr) <= S_TOL
+
+
+def test_prefill_chunked_config_full():
+    """Chunked prefill workload: B=1, H=16, T=4096, dk=dv=128, bf16, S0 = 0 (whole tensors)."""
+    inp = make_inputs(1, 4096, 16, 128, 128, seed=0)
+    y, sf = _run_dense(inp)
+    yr, sr = oracle.forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"])
+    assert max_rel(y, yr) <= Y_TOL
+    assert frob_rel(sf, sr) <= S_TOL
+    for h in range(16):  # per-head state error stays under the bar too
+        assert frob_rel(sf[0, h], sr[0, h]) <= S_TOL
+
+
+def test_prefill_extreme_decay():
+    """alpha ~ 1e-6 (cumulative log-decay far below -88 inside a chunk) and alpha = 1."""
+    B, T, H, d = 1, 192, 2, 128
+    inp = make_inputs(B, T, H, d, d, seed=3, with_s0=True)
+    a = inp["alpha"].clone()
+    a[:, :64] = 1e-6
+    a[:, 64:128] = 1.0
+    inp["alpha"] = a
+    y, sf = _run_dense(inp)
+    yr, sr = oracle.forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["s0"])
+    assert max_rel(y, yr) <= Y_TOL
+    assert frob_rel(sf, sr) <= S_TOL
+
+
+@pytest.mark.parametrize("lengths", [[1, 63, 64, 65, 130], [0, 100, 0, 5], [4096]])
+def test_prefill_varlen_small(lengths):
+    H, d = 2, 128
+    inp = make_varlen_inputs(lengths, H, d, d, seed=sum(lengths))
+    g = _cuda(inp)
+    y, sf = api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                   g["cu_seqlens"], g["s0"])
+    torch.cuda.synchronize()
+    yr, sr = oracle.forward_varlen(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                                   inp["cu_seqlens"].numpy(), inp["s0"])
+    assert max_rel(y, yr) <= Y_TOL
+    assert frob_rel(sf, sr) <= S_TOL
+
+
+def test_prefill_varlen_long_config_sampled_heads():
+    """Long varlen workload: T=32768 packed, 4 seeded documents, H=16, d=128, S0 ~ N(0,0.02).
+    The oracle runs 3 of the 16 heads over every document (all tokens)."""
+    lengths = varlen_lengths(32768, 4, seed=0)
+    H, d = 16, 128
+    inp = make_varlen_inputs(lengths, H, d, d, seed=0)
+    g = _cuda(inp)
+    y, sf = api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                   g["cu_seqlens"], g["s0"])
+    torch.cuda.synchronize()
+    heads = [0, 7, 15]
+    sub = {n: inp[n][:, :, heads].contiguous() for n in ("q", "k", "v", "alpha", "beta")}
+    yr, sr = oracle.forward_varlen(sub["q"], sub["k"], sub["v"], sub["alpha"], sub["beta"],
+                                   inp["cu_seqlens"].numpy(), inp["s0"][:, heads].contiguous())
+    assert max_rel(y[:, :, heads], yr) <= Y_TOL
+    assert frob_rel(sf[:, heads], sr) <= S_TOL
+    assert torch.isfinite(y).all() and torch.isfinite(sf).all()
+
+
+def test_prefill_resume_invariant_on_gpu():
+    """prefill(T1) then prefill(T2, S0 = S_T1) equals prefill(T1 + T2) (GPU against GPU)."""
+    B, T, H, d = 2, 320, 4, 128
+    inp = _cuda(make_inputs(B, T, H, d, d, seed=21, with_s0=True))
+    y, sf = api.gdn_prefill(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["s0"])
+    T1 = 128
+    sl = lambda x, a, b: x[:, a:b].contiguous()
+    y1, s1 = api.gdn_prefill(sl(inp["q"], 0, T1), sl(inp["k"], 0, T1), sl(inp["v"], 0, T1),
+                             sl(inp["alpha"], 0, T1), sl(inp["beta"], 0, T1), inp["s0"])
+    y2, s2 = api.gdn_prefill(sl(inp["q"], T1, T), sl(inp["k"], T1, T), sl(inp["v"], T1, T),
+                             sl(inp["alpha"], T1, T), sl(inp["beta"], T1, T), s1)
+    assert max_rel(torch.cat([y1, y2], 1), y) <= Y_TOL
+    assert frob_rel(s2, sf) <= S_TOL
+
+
+def test_prefill_matches_decode_steps():
+    """T decode steps (fp32 state kernel) equal one chunked prefill of the same T tokens."""
+    B, T, H, d = 2, 70, 2, 128
+    inp = _cuda(make_inputs(B, T, H, d, d, seed=5, with_s0=True))
+    y, sf = api.gdn_prefill(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["s0"])
+    S = inp["s0"].clone()
+    ys = []
+    for t in range(T):
+        ys.append(api.gdn_decode_step(*(inp[n][:, t].contiguous() for n in
+                                        ("q", "k", "v", "alpha", "beta")), S))
+    assert max_rel(y, torch.stack(ys, 1)) <= Y_TOL
+    assert frob_rel(sf, S) <= S_TOL
+
+
+def test_prefill_device_status_clean():
+    inp = make_inputs(1, 128, 2, 128, 128, seed=1)
+    _run_dense(inp)
+    assert api.gdn_read_device_status(reset=True) == 0
