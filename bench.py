@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the Gated DeltaNet hot path on B200.
+
+Headline workload: one packed T = 32768 token stream of 4 seeded documents
+(lengths 16749/4122/7000/4897), H = 16 heads, dk = dv = 128, bf16 q/k/v, fp32 alpha/beta,
+per-document initial state S0 ~ N(0, 0.02^2): one step = one gdn_prefill_varlen over the
+stream (norms, decay, intra-chunk WY, state passes, outputs, final states).  Also measured:
+the decode step (256 sequences x 16 heads, fp32 128x128 states, 1000 consecutive steps with
+fresh tokens) as a secondary object.
+
+Prints ONE JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own stream (weak
+scaling, no data-path collective); time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the reference implementation of the method)
+on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill tokens/s & % bf16 tensor peak; decode-step state GB/s vs HBM peak"
+H, D = 16, 128
+T_TOTAL, NDOCS = 32768, 4
+DEC_N = 256
+FLOP_PER_TOKEN_HEAD = 180224        # dense chunk-64 tile FLOPs at dk = dv = 128
+BYTES_PER_TOKEN_HEAD = 1032         # q,k,v,y bf16 (4 x 256) + alpha, beta fp32
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profile_traffic(name, source):
+    """Per-launch DRAM bytes recorded by an ncu capture in profiles/<name>; None when the summary
+    is missing or was taken on a different version of the kernel source."""
+    path = os.path.join(ROOT, "profiles", name)
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", txt)
+    if not m or not h:
+        return None
+    cur = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()
+    return float(m.group(1)) if h.group(1) == cur else None
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [x.strip() for x in l.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- inputs
+def varlen_workload(seed):
+    from gated_deltanet_linear_eqs_b200.inputs import make_varlen_inputs, varlen_lengths
+    lengths = varlen_lengths(T_TOTAL, NDOCS, seed=0)
+    return lengths, make_varlen_inputs(lengths, H, D, D, seed=seed)
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from gated_deltanet_linear_eqs_b200 import api
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks, peak_src = load_peaks()
+    props = torch.cuda.get_device_properties(dev)
+    uuid = "GPU-" + str(props.uuid)
+
+    lengths, inp = varlen_workload(seed=rank)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    y = torch.empty((1, T_TOTAL, H, D), dtype=torch.bfloat16, device=dev)
+    sf = torch.empty((NDOCS, H, D, D), dtype=torch.float32, device=dev)
+
+    def step():
+        api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["cu_seqlens"],
+                               g["s0"], y=y, s_final=sf)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    out = {}
+    if args.only in ("all", "prefill"):
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        with ClockSampler(uuid) as clk:
+            for i in range(args.steps):
+                starts[i].record()
+                step()
+                ends[i].record()
+            torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        total_ms = max_over_ranks(starts[0].elapsed_time(ends[-1]))
+        kern_ms = max_over_ranks(statistics.mean(per))
+        assert api.gdn_read_device_status() == 0, "device status word set during the bench"
+
+        tokens = T_TOTAL
+        flops = FLOP_PER_TOKEN_HEAD * tokens * H
+        state_bytes = 2 * NDOCS * H * D * D * 4
+        hbm_bytes = BYTES_PER_TOKEN_HEAD * tokens * H + state_bytes
+        ms_per_step = total_ms / args.steps
+        value = world * tokens / (ms_per_step / 1e3)
+        tflops = flops / (kern_ms / 1e3) / 1e12
+        gbs = hbm_bytes / (kern_ms / 1e3) / 1e9
+        traffic = profile_traffic("prefill_varlen_T32768.md",
+                                  "gated_deltanet_linear_eqs_b200/csrc/prefill.cu")
+        out["prefill"] = dict(
+            value=value, ms_per_step=ms_per_step, kern_ms=kern_ms, clocks=clk.summary(),
+            roofline={"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
+                      "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
+                      "traffic": traffic, "peak_source": peak_src + " bf16 burst",
+                      "flops_per_launch": flops},
+            roofline_hbm={"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                          "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                          "bytes_per_launch": hbm_bytes, "peak_source": peak_src},
+            frac_bf16_sustained=tflops / peaks["bf16_tflops_sustained"])
+
+        # end to end through the public API with host buffers: H2D of the step's inputs from
+        # pinned memory, the call, D2H of the outputs, all inside the timed region
+        host = {k: v.pin_memory() for k, v in inp.items() if isinstance(v, torch.Tensor)}
+        y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        sf_h = torch.empty(sf.shape, dtype=sf.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = y_h.numel() * y_h.element_size() + sf_h.numel() * sf_h.element_size()
+
+        def e2e_step():
+            d = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+            yy, ss = api.gdn_prefill_varlen(d["q"], d["k"], d["v"], d["alpha"], d["beta"],
+                                            d["cu_seqlens"], d["s0"])
+            y_h.copy_(yy, non_blocking=True)
+            sf_h.copy_(ss, non_blocking=True)
+
+        for _ in range(max(1, min(args.warmup, 3))):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, min(args.steps, 10))
+        e0.record()
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e)
+        out["e2e"] = {"value": world * tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "ms_per_step": e2e_ms}
+
+    if args.only in ("all", "decode") and args.decode_steps > 0:
+        out["decode"] = run_decode(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier)
+    return out
+
+
+def run_decode(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier):
+    import torch
+    from gated_deltanet_linear_eqs_b200 import api
+    from gated_deltanet_linear_eqs_b200.inputs import make_decode_state, make_decode_step_inputs
+
+    nsteps = args.decode_steps
+    S = make_decode_state(DEC_N, H, D, D, seed=0).to(dev)
+    q = torch.empty((nsteps, DEC_N, H, D), dtype=torch.bfloat16, device=dev)
+    k = torch.empty_like(q)
+    v = torch.empty_like(q)
+    a = torch.empty((nsteps, DEC_N, H), dtype=torch.float32, device=dev)
+    b = torch.empty_like(a)
+    for t in range(nsteps):  # fresh seeded tokens per step, staged in HBM before timing
+        d = make_decode_step_inputs(DEC_N, H, D, D, step=t)
+        q[t].copy_(d["q"]); k[t].copy_(d["k"]); v[t].copy_(d["v"])
+        a[t].copy_(d["alpha"]); b[t].copy_(d["beta"])
+    y = torch.empty((DEC_N, H, D), dtype=torch.bfloat16, device=dev)
+    for t in range(min(3, nsteps)):  # warm-up on a copy of the state
+        Sw = S.clone()
+        api.gdn_decode_step(q[t], k[t], v[t], a[t], b[t], Sw, y=y)
+    del Sw
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(uuid) as clk:
+        e0.record()
+        for t in range(nsteps):
+            api.gdn_decode_step(q[t], k[t], v[t], a[t], b[t], S, y=y)
+        e1.record()
+        torch.cuda.synchronize()
+    step_ms = max_over_ranks(e0.elapsed_time(e1) / nsteps)
+    bytes_step = DEC_N * H * (2 * D * D * 4 + BYTES_PER_TOKEN_HEAD)
+    gbs = bytes_step / (step_ms / 1e3) / 1e9
+    return {"metric": "decode-step state GB/s", "value": gbs, "unit": "GB/s",
+            "ms_per_step": step_ms, "steps": nsteps, "gpu_launches": nsteps,
+            "config": {"workload": f"decode: {DEC_N} sequences x {H} heads, dk=dv={D}, fp32 "
+                                   f"state updated in place, bf16 tokens, {nsteps} steps",
+                       "l2": "state (537 MB) exceeds the 126 MB L2; no flush"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "bytes_per_launch": bytes_step,
+                         "traffic": profile_traffic("decode_N256_H16.md",
+                                                    "gated_deltanet_linear_eqs_b200/csrc/decode.cu"),
+                         "peak_source": peak_src},
+            "clocks": clk.summary()}
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def oracle_sample(n_tok, nthreads):
+    """Time the fp64 oracle on the first n_tok tokens of document 0 (all 16 heads)."""
+    import oracle
+    from gated_deltanet_linear_eqs_b200.inputs import make_varlen_inputs, varlen_lengths
+    lengths = varlen_lengths(T_TOTAL, NDOCS, seed=0)
+    inp = make_varlen_inputs([n_tok], H, D, D, seed=0)
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.forward_varlen(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                          inp["cu_seqlens"].numpy(), inp["s0"], nthreads=nthreads)
+    return time.perf_counter() - t0, lengths
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(target_s=12.0):
+    cores = cpu_cores()
+    threads = min(cores, H)
+    dt, _ = oracle_sample(128, threads)
+    n = int(min(16749, max(128, 128 * target_s / max(dt, 1e-6))))
+    dt, _ = oracle_sample(n, threads)
+    return {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 token-loop oracle on the first {n} tokens of the 16749-token "
+                      f"document, all {H} heads (threads over heads), {dt:.1f} s"}
+
+
+def run_reference(args):
+    cores = cpu_cores()
+    threads = min(cores, H)
+    n_tok = args.ref_tokens
+    for _ in range(args.warmup):
+        oracle_sample(n_tok, threads)
+    times = []
+    for _ in range(args.steps):
+        dt, _ = oracle_sample(n_tok, threads)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = n_tok / (ms / 1e3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAME, "sample_tokens_per_step": n_tok},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: fp64 oracle on {n_tok} tokens x {H} heads of "
+                                   "the longest document"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+WORKLOAD_NAME = ("varlen prefill: packed T=32768 stream of 4 seeded documents "
+                 "(16749/4122/7000/4897 tokens), H=16, dk=dv=128, bf16 q/k/v, fp32 alpha/beta, "
+                 "S0 ~ N(0,0.02^2) per document")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=512)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic"}
+    if "prefill" in res:
+        p = res["prefill"]
+        line.update(value=p["value"], unit="tokens/s", ms_per_step=p["ms_per_step"],
+                    config={"workload": WORKLOAD_NAME, "tokens_per_step_per_gpu": T_TOTAL,
+                            "parallelism": f"dp{world} (independent streams, no collective)",
+                            "l2": "inputs (403 MB) exceed the 126 MB L2; no flush"},
+                    roofline=p["roofline"], roofline_hbm=p["roofline_hbm"],
+                    frac_bf16_sustained=p["frac_bf16_sustained"], kernel_ms=p["kern_ms"],
+                    clocks=p["clocks"], e2e=res["e2e"], gpu_launches=args.steps)
+    if "decode" in res:
+        line["decode"] = res["decode"]
+        if "prefill" not in res:
+            d = res["decode"]
+            line.update(metric=METRIC, value=d["value"], unit="GB/s", ms_per_step=d["ms_per_step"],
+                        config=d["config"], roofline=d["roofline"], clocks=d["clocks"],
+                        gpu_launches=d["gpu_launches"])
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
