@@ -235,7 +235,93 @@ def run_ours(args, rank, world, local_rank):
 
     if args.only in ("all", "decode") and args.decode_steps > 0:
         out["decode"] = run_decode(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier)
+    if args.only in ("all", "train") and args.train_steps > 0:
+        out["train"] = run_train(args, dev, uuid, max_over_ranks, barrier, rank)
     return out
+
+
+TRAIN_B, TRAIN_T, TRAIN_H = 8, 4096, 32
+
+
+def train_inputs(dev, seed=0):
+    import torch
+    from gated_deltanet_linear_eqs_b200.inputs import make_inputs
+    inp = make_inputs(TRAIN_B, TRAIN_T, TRAIN_H, D, D, seed=seed, with_dy=True)
+    return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+
+
+def run_train(args, dev, uuid, max_over_ranks, barrier, rank):
+    """Training shape: forward (gdn_prefill) + backward (gdn_backward) per step."""
+    import torch
+    from gated_deltanet_linear_eqs_b200 import api
+    from gated_deltanet_linear_eqs_b200._abi import GDN_OP_BACKWARD
+    g = train_inputs(dev, seed=rank)
+    ws = torch.empty(api.gdn_workspace_bytes(GDN_OP_BACKWARD, TRAIN_B, TRAIN_T, TRAIN_H, D, D),
+                     dtype=torch.uint8, device=dev)
+
+    def fwd():
+        return api.gdn_prefill(g["q"], g["k"], g["v"], g["alpha"], g["beta"])
+
+    def bwd():
+        return api.gdn_backward(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["dy"], ws=ws)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    barrier()
+    steps = max(1, min(args.steps, args.train_steps))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    with ClockSampler(uuid) as clk:
+        for i in range(steps):
+            ev[i][0].record()
+            fwd()
+            ev[i][1].record()
+            bwd()
+            ev[i][2].record()
+        torch.cuda.synchronize()
+    f_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
+    b_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
+    tokens = TRAIN_B * TRAIN_T
+    return {"metric": "GDN fwd+bwd tokens/s (training shape)", "unit": "tokens/s",
+            "value": tokens / ((f_ms + b_ms) / 1e3), "ms_per_step": f_ms + b_ms,
+            "fwd_ms": f_ms, "bwd_ms": b_ms, "steps": steps, "gpu_launches": 3 * steps,
+            "config": {"workload": f"train: B={TRAIN_B}, T={TRAIN_T}, H={TRAIN_H}, dk=dv={D}, "
+                                   "bf16, dy ~ N(0,1), S0 = 0"},
+            "clocks": clk.summary()}
+
+
+def run_profile(args):
+    """Launch-only driver for ncu: one warm-up plus --launches launches of one op on the bench
+    workload, no timing and no host-side extras."""
+    import torch
+    from gated_deltanet_linear_eqs_b200 import api
+    dev = torch.device("cuda", 0)
+    n = args.launches
+    if args.profile == "prefill":
+        _, inp = varlen_workload(seed=0)
+        g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        for _ in range(n + 1):
+            api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                   g["cu_seqlens"], g["s0"])
+    elif args.profile == "decode":
+        from gated_deltanet_linear_eqs_b200.inputs import make_decode_state, make_decode_step_inputs
+        S = make_decode_state(DEC_N, H, D, D, seed=0).to(dev)
+        d = {k: v.to(dev) for k, v in make_decode_step_inputs(DEC_N, H, D, D, step=0).items()
+             if isinstance(v, torch.Tensor)}
+        for _ in range(n + 1):
+            api.gdn_decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S)
+    else:
+        from gated_deltanet_linear_eqs_b200._abi import GDN_OP_BACKWARD
+        g = train_inputs(dev)
+        ws = torch.empty(api.gdn_workspace_bytes(GDN_OP_BACKWARD, TRAIN_B, TRAIN_T, TRAIN_H, D, D),
+                         dtype=torch.uint8, device=dev)
+        for _ in range(n + 1):
+            api.gdn_backward(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["dy"], ws=ws)
+    torch.cuda.synchronize()
+    assert api.gdn_read_device_status() == 0
+    print("ok", flush=True)
+    return 0
 
 
 def run_decode(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier):
@@ -356,8 +442,12 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "train"], default="all")
     ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--train-steps", type=int, default=3)
+    ap.add_argument("--profile", choices=["prefill", "decode", "backward"], default=None,
+                    help="launch-only mode for ncu (no timing, no JSON)")
+    ap.add_argument("--launches", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=512)
     args = ap.parse_args()
@@ -368,6 +458,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.profile:
+        return run_profile(args)
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
@@ -400,6 +492,8 @@ def main():
                     roofline=p["roofline"], roofline_hbm=p["roofline_hbm"],
                     frac_bf16_sustained=p["frac_bf16_sustained"], kernel_ms=p["kern_ms"],
                     clocks=p["clocks"], e2e=res["e2e"], gpu_launches=args.steps)
+    if "train" in res:
+        line["train"] = res["train"]
     if "decode" in res:
         line["decode"] = res["decode"]
         if "prefill" not in res:
