@@ -52,10 +52,11 @@ def test_workspace_bytes(lib):
     assert n.value == 0
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_BACKWARD, 8, 4096, 32, 128, 128, 0,
                                    ctypes.byref(n)) == 0
-    assert n.value == 64 * 8 * 32 * 128 * 128 * 4  # one fp32 state per 64-token chunk
+    # one fp32 state per 64-token chunk (checkpoints) + 64 per chain (replayed chunk)
+    assert n.value == (64 + 64) * 8 * 32 * 128 * 128 * 4
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_BACKWARD, 1, 65, 1, 64, 64, 0,
                                    ctypes.byref(n)) == 0
-    assert n.value == 2 * 64 * 64 * 4
+    assert n.value == (2 + 64) * 64 * 64 * 4
     assert lib.gdn_workspace_bytes(42, 1, 1, 1, 64, 64, 0, ctypes.byref(n)) == \
         _abi.GDN_ERR_INVALID_ARG
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL_VARLEN, 1, 10, 1, 64, 64, 0,
