@@ -7,7 +7,8 @@ library; the first call does, and fails loudly if it has not been built.
 from ._abi import GdnError  # noqa: F401
 
 __all__ = ["gdn_prefill", "gdn_prefill_varlen", "gdn_decode_step", "gdn_backward",
-           "gdn_workspace_bytes", "gdn_read_device_status", "GdnError"]
+           "gdn_backward_noalloc", "gdn_backward_noalloc_max_workspace", "gdn_workspace_bytes",
+           "gdn_read_device_status", "GdnError"]
 
 
 def __getattr__(name):

@@ -47,6 +47,8 @@ SIGNATURES = {
                                 _I, _P, _S, _P]),
     "gdn_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gdn_backward": (_I, [_P] * 14 + [_I] * 6 + [_F, _I, _P, _S, _P]),
+    "gdn_backward_noalloc": (_I, [_P] * 14 + [_I] * 6 + [_F, _I, _P]),
+    "gdn_backward_noalloc_max_workspace": (_S, []),
     "gdn_read_device_status": (_I, [_I, ctypes.POINTER(_I)]),
 }
 

@@ -185,6 +185,43 @@ def gdn_backward(q, k, v, alpha, beta, dy, s0=None, ds_final=None, scale=1.0, l2
     return out
 
 
+def gdn_backward_noalloc(q, k, v, alpha, beta, dy, s0=None, ds_final=None, scale=1.0,
+                         l2norm_qk=True, want_ds0=True, out=None, stream=None):
+    """gdn_backward on the library's fixed device scratch: no workspace is passed and the
+    library allocates nothing.  ``out`` may supply preallocated gradient tensors (a dict with
+    the keys of gdn_backward's result), so that a caller without an allocator can pass its
+    own buffers.  Returns the gradient dict."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _need(q, "q", dt)
+    _need(k, "k", dt, q.shape)
+    _need(v, "v", dt, (B, T, H, dv))
+    _need(alpha, "alpha", torch.float32, (B, T, H))
+    _need(beta, "beta", torch.float32, (B, T, H))
+    _need(dy, "dy", dt, (B, T, H, dv))
+    _need(s0, "s0", torch.float32, (B, H, dk, dv), optional=True)
+    _need(ds_final, "ds_final", torch.float32, (B, H, dk, dv), optional=True)
+    if out is None:
+        out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                   dalpha=torch.empty_like(alpha), dbeta=torch.empty_like(beta),
+                   ds0=torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+                   if want_ds0 else None)
+    rc = _lib().gdn_backward_noalloc(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(s0), _p(dy),
+                                     _p(ds_final), _p(out["dq"]), _p(out["dk"]), _p(out["dv"]),
+                                     _p(out["dalpha"]), _p(out["dbeta"]), _p(out.get("ds0")), B,
+                                     T, H, dk, dv, _DT[dt], float(scale), int(bool(l2norm_qk)),
+                                     _stream(stream))
+    _check(rc, "gdn_backward_noalloc")
+    return out
+
+
+def gdn_backward_noalloc_max_workspace():
+    return int(_lib().gdn_backward_noalloc_max_workspace())
+
+
 def gdn_read_device_status(reset=True):
     st = ctypes.c_int(0)
     _check(_lib().gdn_read_device_status(int(bool(reset)), ctypes.byref(st)),

@@ -20,6 +20,8 @@
 // Thread layout: warp w owns rows 8w..8w+7 of the dk x dv state, lane l owns columns
 // [l*CPL, l*CPL + CPL).  Column (dk) reductions go through shared memory, row (dv) reductions
 // through warp shuffles.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -444,6 +446,37 @@ cudaError_t launch_t(const BackwardArgs& a, cudaStream_t st) {
 }
 
 }  // namespace
+
+// ----------------------------------------------------------------------------- fixed scratch
+// Scratch for gdn_backward_noalloc: a file-scope device array that every GPU loading the
+// library holds until the process exits.  Host code must never hand g_bwd_fixed_scratch itself
+// to a kernel (on the host the name is only a stand-in for the symbol, not a device address);
+// the device address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_bwd_fixed_scratch[kBackwardFixedScratchBytes];
+
+namespace {
+std::mutex g_fixed_mu;
+void* g_fixed_ptr[64] = {};
+}  // namespace
+
+int backward_fixed_scratch(void** ptr) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lk(g_fixed_mu);
+    if (!g_fixed_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_bwd_fixed_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return GDN_ERR_CUDA;
+        }
+        g_fixed_ptr[dev] = p;
+    }
+    *ptr = g_fixed_ptr[dev];
+    return GDN_OK;
+}
 
 size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv) {
     const size_t chunks = (size_t)(T + kC - 1) / kC;

@@ -178,6 +178,31 @@ int gdn_backward(const void* q, const void* k, const void* v, const float* alpha
     return map_cuda(gdn::launch_backward(a, static_cast<cudaStream_t>(stream)));
 }
 
+int gdn_backward_noalloc(const void* q, const void* k, const void* v, const float* alpha,
+                         const float* beta, const float* s0, const void* dy,
+                         const float* ds_final, void* dq, void* dk_out, void* dv_out,
+                         float* dalpha, float* dbeta, float* ds0, int B, int T, int H, int dk,
+                         int dv, int dtype, float scale, int l2norm_qk, void* stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
+        !ok_ptr(dy) || !ok_ptr(dq) || !ok_ptr(dk_out) || !ok_ptr(dv_out) || !ok_ptr(dalpha) ||
+        !ok_ptr(dbeta) || !ok_opt_ptr(s0) || !ok_opt_ptr(ds_final) || !ok_opt_ptr(ds0))
+        return GDN_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (int rc = check_dims(dk, dv, dtype)) return rc;
+    const size_t need = gdn::backward_workspace_bytes(B, T, H, dk, dv);
+    if (need > gdn::kBackwardFixedScratchBytes) return GDN_ERR_WORKSPACE;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    void* scratch = nullptr;
+    if (int rc = gdn::backward_fixed_scratch(&scratch)) return rc;
+    gdn::BackwardArgs a{q, k, v, alpha, beta, s0, dy, ds_final, dq, dk_out, dv_out, dalpha,
+                        dbeta, ds0, B, T, H, dk, dv, dtype, scale, l2norm_qk ? 1 : 0, scratch,
+                        gdn::kBackwardFixedScratchBytes, dev.status};
+    return map_cuda(gdn::launch_backward(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t gdn_backward_noalloc_max_workspace(void) { return gdn::kBackwardFixedScratchBytes; }
+
 int gdn_read_device_status(int reset, int* device_status) {
     if (!device_status) return GDN_ERR_INVALID_ARG;
     DeviceInfo dev;

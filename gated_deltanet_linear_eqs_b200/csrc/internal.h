@@ -55,4 +55,9 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st);
 // Workspace the backward pass needs (chunk-start states), bytes.
 size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv);
 
+// Size of the fixed device scratch array behind gdn_backward_noalloc.
+constexpr size_t kBackwardFixedScratchBytes = size_t(32) << 20;
+// Device address of that array on the current device (looked up on first use per device).
+int backward_fixed_scratch(void** ptr);
+
 }  // namespace gdn

@@ -135,6 +135,38 @@ int gdn_backward(const void* q, const void* k, const void* v, const float* alpha
                  void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * gdn_backward_noalloc -- gdn_backward for callers that cannot allocate device memory.
+ * (The pages describe no such call; it exists for the library's users.)
+ *
+ * Some callers may not call cudaMalloc, or any allocator, on the path where they run the
+ * backward pass: a plugin inside a host framework whose device memory is owned by that
+ * framework's pool, or a server that reserves all of its memory at start-up and forbids later
+ * allocations.  This entry point takes no workspace argument: it uses a fixed 32 MiB scratch
+ * array compiled into the library, which every GPU that loads the library keeps until the
+ * process exits.  It allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
+ *   - Arguments, layouts, results and error codes are those of gdn_backward; inputs and
+ *     outputs are still the caller's buffers.
+ *   - Sizes whose workspace (gdn_workspace_bytes(GDN_OP_BACKWARD, ...)) exceeds
+ *     gdn_backward_noalloc_max_workspace() are rejected with GDN_ERR_WORKSPACE before any
+ *     launch.  At dk = dv = 128 that is B*H*(ceil(T/64) + 64) <= 512.
+ *   - The first call on each device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls share the one array and it keeps the last call's contents; every byte a call
+ *     reads from it is written earlier by the same call, so nothing needs clearing.  Calls
+ *     whose kernels overlap on the GPU (other streams, other host threads) race on the array:
+ *     order them on one stream.
+ */
+int gdn_backward_noalloc(const void* q, const void* k, const void* v, const float* alpha,
+                         const float* beta, const float* s0, const void* dy,
+                         const float* ds_final, void* dq, void* dk_out, void* dv_out,
+                         float* dalpha, float* dbeta, float* ds0, int B, int T, int H, int dk,
+                         int dv, int dtype, float scale, int l2norm_qk, void* stream);
+
+/* Capacity in bytes of the fixed scratch behind gdn_backward_noalloc (32 MiB). */
+size_t gdn_backward_noalloc_max_workspace(void);
+
+/*
  * Device status word of the current device: 0 when no kernel has recorded an
  * error, otherwise the first gdn_status a kernel recorded (GDN_ERR_TIMEOUT).
  * Synchronises the current device.  If reset != 0 the word is cleared.
