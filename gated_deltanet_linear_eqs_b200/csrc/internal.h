@@ -50,6 +50,8 @@ struct BackwardArgs {
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st);
+// Token-by-token prefill on CUDA cores (used for fp32 inputs).
+cudaError_t launch_prefill_seq(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st);
 
 // Workspace the backward pass needs (chunk-start states), bytes.

@@ -712,7 +712,8 @@ cudaError_t launch_dk(const PrefillArgs& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st) {
-    if (a.dtype != GDN_BF16) return cudaErrorNotSupported;
+    // bf16 inputs run the tensor-core kernel; fp32 inputs the exact-fp32 token loop.
+    if (a.dtype != GDN_BF16) return launch_prefill_seq(a, st);
     return a.dk == 128 ? launch_dk<128>(a, st) : launch_dk<64>(a, st);
 }
 

@@ -41,6 +41,31 @@ def test_prefill_dense_small(B, T, H, d, with_s0):
     assert frob_rel(sf, sr) <= S_TOL
 
 
+def test_prefill_pr1_config_fp32():
+    """PR1 reference config: B=1, H=2, T=256, dk=dv=64, fp32, S0 = 0, seed 0 (whole tensors)."""
+    inp = make_inputs(1, 256, 2, 64, 64, dtype="fp32", seed=0)
+    y, sf = _run_dense(inp)
+    assert y.dtype == torch.float32
+    yr, sr = oracle.forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"])
+    assert max_rel(y, yr) <= Y_TOL
+    assert frob_rel(sf, sr) <= S_TOL
+    assert max_rel(y, yr) <= 1e-5 and frob_rel(sf, sr) <= 1e-5  # exact fp32 arithmetic
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_fp32_varlen(d):
+    lengths = [1, 64, 100, 0, 7]
+    inp = make_varlen_inputs(lengths, 3, d, d, dtype="fp32", seed=d)
+    g = _cuda(inp)
+    y, sf = api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                   g["cu_seqlens"], g["s0"], scale=0.5)
+    torch.cuda.synchronize()
+    yr, sr = oracle.forward_varlen(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                                   inp["cu_seqlens"].numpy(), inp["s0"], scale=0.5)
+    assert max_rel(y, yr) <= 1e-5
+    assert frob_rel(sf, sr) <= 1e-5
+
+
 def test_prefill_scale_and_no_norm():
     B, T, H, d = 1, 150, 2, 128
     inp = make_inputs(B, T, H, d, d, seed=7, with_s0=True)
