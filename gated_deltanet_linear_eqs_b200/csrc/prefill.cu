@@ -75,8 +75,8 @@ struct Layout {
     static constexpr int TF = AF + 64 * kLd * 2;         // T, bf16 64 x kLd
     static constexpr int XB = TF + 64 * kLd * 2;         // 4 warps x 16 x 24 bf16
     static constexpr int AB = XB + 4 * 16 * 24 * 2;      // per stage alpha[64], beta[64]
-    static constexpr int SC = AB + kStages * 512;        // scalars: 2 buffers x 8 x 64 floats
-    static constexpr int BAR = SC + 2 * 8 * 256;         // mbarriers
+    static constexpr int SC = AB + kStages * 512;        // scalars: 2 buffers x 9 x 64 floats
+    static constexpr int BAR = SC + 2 * 9 * 256;         // mbarriers
     static constexpr int MISC = BAR + 32 * 8;            // tmem base, abort, exit flags
     static constexpr int BYTES = MISC + 64;
     static constexpr int TX = 2 * KB * 8192 + VT;        // TMA bytes per stage
@@ -90,7 +90,7 @@ struct Layout {
 };
 
 // scalar arrays (64 floats each) inside one scalar buffer
-enum { SC_G = 0, SC_GAM, SC_BETA, SC_RK, SC_RQ, SC_USC, SC_YSC, SC_CARRY };
+enum { SC_G = 0, SC_GAM, SC_BETA, SC_RK, SC_RQ, SC_USC, SC_YSC, SC_FTW, SC_CARRY, SC_SLOTS };
 // barriers
 enum {
     B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1,  // input ring
@@ -142,15 +142,15 @@ __device__ __forceinline__ void load_half_row(const uint8_t* tile, int row, int 
 }
 // Sum of squares of one swizzled bf16 row of 64 elements.
 __device__ __forceinline__ float row_sumsq(const uint8_t* tile, int row) {
-    float s = 0.f;
+    float s[8] = {};
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         float x[8];
         unpack8(*reinterpret_cast<const uint4*>(tile + swz(row, c)), x);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s = fmaf(x[e], x[e], s);
+        for (int e = 0; e < 8; ++e) s[e] = fmaf(x[e], x[e], s[e]);
     }
-    return s;
+    return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
 }
 
 template <int DK>
@@ -229,7 +229,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         return ok;
     };
     auto stage_of = [&](int c) { return sm + (c & 1) * L::STAGE; };
-    auto scal = [&](int c, int which) { return reinterpret_cast<float*>(sm + L::SC + (c & 1) * 2048 + which * 256); };
+    auto scal = [&](int c, int which) { return reinterpret_cast<float*>(sm + L::SC + (c & 1) * (SC_SLOTS * 256) + which * 256); };
 
     if (warp == 0) {
         // ================================================================ TMA producer
@@ -291,82 +291,101 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             constexpr uint32_t ID_KN = idesc_bf16(128, kNV, false, true);
             constexpr uint32_t ID_M5 = idesc_bf16(128, kNV, true, true);
             const uint32_t lbo_k = (DK == 128) ? L::KQW_BLOCK : 0;  // DK=64: rows 64-127 repeat 0-63
-            const uint32_t s_tw = smem_u32(sm + L::TW), s_av = smem_u32(sm + L::AV);
-            const uint32_t s_sb = smem_u32(sm + L::SB), s_uhi = smem_u32(sm + L::UHI);
-            const uint32_t s_ulo = smem_u32(sm + L::ULO), s_ub = smem_u32(sm + L::UB);
-            const uint32_t s_p0 = smem_u32(sm + L::P0);
+            // Descriptors of every operand, built once; a K step only adds its byte offset / 16
+            // to the start-address field (all addresses stay far below 2^18).
+            // stage 0 descriptors; stage 1 is the same plus STAGE / 16 in the address field
+            const uint32_t st0 = smem_u32(sm);
+            const uint64_t dK0 = sdesc(st0, 16, 1024);                // K-major K / [K;Q] rows
+            const uint64_t dM3b0 = sdesc(st0, L::KQW_BLOCK, 1024);    // K as MN-major B (N = dk)
+            const uint64_t dV0 = sdesc(st0 + L::KQW, 8192, 1024);     // V as MN-major B
+            const uint64_t dQW0 = sdesc(st0 + 8192, 16, 1024);        // [Q;-W] rows, K-major A
+            const uint64_t dM5a0 = sdesc(st0, lbo_k, 1024);           // K^T as MN-major A
+            constexpr uint64_t SST = L::STAGE >> 4;
+            const uint64_t dTW = sdesc(smem_u32(sm + L::TW), 16, 1024);
+            const uint64_t dAV = sdesc(smem_u32(sm + L::AV), 16, 1024);
+            const uint64_t dSB = sdesc(smem_u32(sm + L::SB), DK * 128, 1024);
+            const uint64_t dUHI = sdesc(smem_u32(sm + L::UHI), 8192, 1024);
+            const uint64_t dULO = sdesc(smem_u32(sm + L::ULO), 8192, 1024);
+            const uint64_t dUB = sdesc(smem_u32(sm + L::UB), 8192, 1024);
+            const uint64_t dP0 = sdesc(smem_u32(sm + L::P0), 16, 1024);
+            constexpr uint64_t PST = 8192 >> 4;
+            constexpr uint64_t KS = 32 >> 4;     // K-major: +32 bytes per 16-element K step
+            constexpr uint64_t MS = 2048 >> 4;   // MN-major: +2048 bytes per 16-row K step
+            constexpr uint64_t BLK = L::KQW_BLOCK >> 4;
             int c1 = 0, c3 = 0, c4 = 0, c5 = 0;
-            uint64_t t_last = globaltimer_ns();
+            long long t_last = clock64();
+            int idle = 0;
             while (c5 < nchunks) {
                 bool did = true;
                 if (c5 < c4 && mbar_test(&bars[B_RB5], c5 & 1)) {
                     tc_fence_after();
-                    const uint32_t st = smem_u32(stage_of(c5));
+                    const int s2 = c5 & 1;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + L::T_S, sdesc(st + kk * 2048, lbo_k, 1024),
-                                 sdesc(s_uhi + kk * 2048, 8192, 1024), ID_M5, 1);
+                        mma_bf16(tmem + L::T_S, dM5a0 + s2 * SST + kk * MS, dUHI + kk * MS, ID_M5, 1);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + L::T_S, sdesc(st + kk * 2048, lbo_k, 1024),
-                                 sdesc(s_ulo + kk * 2048, 8192, 1024), ID_M5, 1);
-                    const uint32_t s_p = s_p0 + (c5 & 1) * 8192;
+                        mma_bf16(tmem + L::T_S, dM5a0 + s2 * SST + kk * MS, dULO + kk * MS, ID_M5, 1);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + L::T_D6 + (c5 & 1) * 64, sdesc(s_p + kk * 32, 16, 1024),
-                                 sdesc(s_ub + kk * 2048, 8192, 1024), ID_KN, kk != 0);
+                        mma_bf16(tmem + L::T_D6 + s2 * 64, dP0 + s2 * PST + kk * KS, dUB + kk * MS, ID_KN, kk != 0);
                     mma_commit(&bars[B_M56]);
-                    mma_commit(&bars[B_EMPTY0 + (c5 & 1)]);
+                    mma_commit(&bars[B_EMPTY0 + s2]);
                     ++c5;
                 } else if (c4 < c3 && mbar_test(&bars[B_RAD], c4 & 1) &&
                            mbar_test(&bars[B_RB4], c4 & 1)) {
                     tc_fence_after();
-                    const uint32_t st = smem_u32(stage_of(c4));
-                    const uint32_t d4 = tmem + L::T_D4 + (c4 & 1) * 64;
+                    const int s2 = c4 & 1;
+                    const uint32_t d4 = tmem + L::T_D4 + s2 * 64;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(d4, sdesc(s_av + kk * 32, 16, 1024),
-                                 sdesc(st + L::KQW + kk * 2048, 8192, 1024), ID_KN, kk != 0);
+                        mma_bf16(d4, dAV + kk * KS, dV0 + s2 * SST + kk * MS, ID_KN, kk != 0);
+#pragma unroll
                     for (int b = 0; b < L::KB; ++b)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16(d4, sdesc(st + b * L::KQW_BLOCK + 8192 + kk * 32, 16, 1024),
-                                     sdesc(s_sb + (b * 4 + kk) * 2048, DK * 128, 1024), ID_KN, 1);
+                            mma_bf16(d4, dQW0 + s2 * SST + b * BLK + kk * KS, dSB + (b * 4 + kk) * MS, ID_KN, 1);
                     mma_commit(&bars[B_M4]);
                     ++c4;
                 } else if (c3 < c1 && mbar_test(&bars[B_RA1], c3 & 1)) {
                     tc_fence_after();
-                    const uint32_t st = smem_u32(stage_of(c3));
+                    const int s2 = c3 & 1;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + L::T_D3, sdesc(s_tw + kk * 32, 16, 1024),
-                                 sdesc(st + kk * 2048, L::KQW_BLOCK, 1024), ID_M3, kk != 0);
+                        mma_bf16(tmem + L::T_D3, dTW + kk * KS, dM3b0 + s2 * SST + kk * MS, ID_M3, kk != 0);
                     mma_commit(&bars[B_M3]);
                     ++c3;
                 } else if (c1 < nchunks && c1 <= c3 &&
                            mbar_test(&bars[B_FULL0 + (c1 & 1)], (c1 >> 1) & 1)) {
                     tc_fence_after();
-                    const uint32_t st = smem_u32(stage_of(c1));
+                    const int s2 = c1 & 1;
+#pragma unroll
                     for (int b = 0; b < L::KB; ++b)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t a = st + b * L::KQW_BLOCK + kk * 32;
-                            mma_bf16(tmem + L::T_D1, sdesc(a, 16, 1024), sdesc(a, 16, 1024),
-                                     ID_M1, (b | kk) != 0);
+                            const uint64_t a = dK0 + s2 * SST + b * BLK + kk * KS;
+                            mma_bf16(tmem + L::T_D1, a, a, ID_M1, (b | kk) != 0);
                         }
                     mma_commit(&bars[B_M1]);
                     ++c1;
                 } else {
                     did = false;
                 }
+                if (!did) __nanosleep(32);  // leave the issue slots to the warpgroups
                 if (did) {
-                    t_last = globaltimer_ns();
-                } else if (*abort_flag) {
-                    break;
-                } else if (globaltimer_ns() - t_last > 2000000000ull) {
-                    fail(B_COUNT, c5);
-                    break;
+                    idle = 0;
+                } else if (++idle >= 64) {  // about 2 s of cycles without progress: give up
+                    idle = 0;
+                    const long long now = clock64();
+                    if (*abort_flag) break;
+                    if (t_last == 0) t_last = now;
+                    if (now - t_last > 4000000000ll) {
+                        fail(B_COUNT, c5);
+                        break;
+                    }
+                    continue;
                 }
+                if (did) t_last = 0;
             }
             // no MMA may still be writing TMEM when the warpgroups leave
             mma_commit(&bars[B_FIN]);
@@ -400,7 +419,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ok = wwait(B_FULL0 + (c & 1), (c >> 1) & 1, c) && ok;
             if (ok) {
                 if (t < 64) {
-                    float g = log2f(ab[t]);
+                    float g = lg2(ab[t]);
 #pragma unroll
                     for (int o = 1; o < 32; o <<= 1) {
                         const float x = __shfl_up_sync(0xffffffffu, g, o);
@@ -427,9 +446,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float Glast = sG[nvalid - 1];
             if (ok) {
                 if (t < 64) {
-                    const float G = sG[t];
-                    sGam[t] = ex2(G);
+                    const float G = sG[t], gam = ex2(G);
+                    sGam[t] = gam;
                     sUsc[t] = (t < nvalid) ? ex2(Glast - G) * sRk[t] : 0.f;
+                    scal(c, SC_FTW)[t] = sBeta[t] * gam * sRk[t];
                 } else {
                     const int r = t - 64;
                     sYsc[r] = p.scale * ex2(sG[r]) * sRq[r];
@@ -499,10 +519,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const __nv_bfloat16* src = AF + (16 * b + r) * kLd + 16 * b;
                     unpack8(*reinterpret_cast<const uint4*>(src), arow);
                     unpack8(*reinterpret_cast<const uint4*>(src + 8), arow + 8);
-                    float acc = 0.f;
+                    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-                    for (int m = 0; m < r; ++m) acc = fmaf(arow[m], x[m], acc);
-                    x[r] = (r < l) ? 0.f : (r == l ? 1.f : -acc);
+                    for (int m = 0; m < r; m += 2) {
+                        acc0 = fmaf(arow[m], x[m], acc0);
+                        if (m + 1 < r) acc1 = fmaf(arow[m + 1], x[m + 1], acc1);
+                    }
+                    x[r] = (r < l) ? 0.f : (r == l ? 1.f : -(acc0 + acc1));
                 }
 #pragma unroll
                 for (int r = 0; r < 16; ++r) TF[(16 * b + r) * kLd + 16 * b + l] = __float2bfloat16_rn(x[r]);
@@ -564,12 +587,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         const int j = half * 32 + j4;
                         const float4 b4 = *reinterpret_cast<const float4*>(sBeta + j);
                         if (t < 64) {
-                            const float4 g4 = *reinterpret_cast<const float4*>(sGam + j);
-                            const float4 k4 = *reinterpret_cast<const float4*>(sRk + j);
-                            x[j4 + 0] = (j + 0 <= i) ? x[j4 + 0] * b4.x * g4.x * k4.x : 0.f;
-                            x[j4 + 1] = (j + 1 <= i) ? x[j4 + 1] * b4.y * g4.y * k4.y : 0.f;
-                            x[j4 + 2] = (j + 2 <= i) ? x[j4 + 2] * b4.z * g4.z * k4.z : 0.f;
-                            x[j4 + 3] = (j + 3 <= i) ? x[j4 + 3] * b4.w * g4.w * k4.w : 0.f;
+                            const float4 f4 = *reinterpret_cast<const float4*>(scal(c, SC_FTW) + j);
+                            x[j4 + 0] = (j + 0 <= i) ? x[j4 + 0] * f4.x : 0.f;
+                            x[j4 + 1] = (j + 1 <= i) ? x[j4 + 1] * f4.y : 0.f;
+                            x[j4 + 2] = (j + 2 <= i) ? x[j4 + 2] * f4.z : 0.f;
+                            x[j4 + 3] = (j + 3 <= i) ? x[j4 + 3] * f4.w : 0.f;
                         } else {
                             x[j4 + 0] = (j + 0 < i) ? x[j4 + 0] * b4.x : 0.f;
                             x[j4 + 1] = (j + 1 < i) ? x[j4 + 1] * b4.y : 0.f;
@@ -699,18 +721,27 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     float dv[32], vv[32];
                     tmem_ld32(tmem + L::T_D4 + (c & 1) * 64 + lane_base + 32 * half, dv);
                     if (smem_ok(stage + L::KQW + i * 128, 128, 28)) load_half_row(stage + L::KQW, i, half * 4, vv);
-                    float hi[32];
+                    uint32_t phi[16], plo[16], pub[16];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float u = valid ? fmaf(bi, vv[j], dv[j]) : 0.f;
-                        const float up = u * us;
-                        hi[j] = __bfloat162float(__float2bfloat16_rn(up));
-                        dv[j] = up - hi[j];
-                        vv[j] = u;
+                    for (int j = 0; j < 32; j += 2) {
+                        const float u0 = valid ? fmaf(bi, vv[j], dv[j]) : 0.f;
+                        const float u1 = valid ? fmaf(bi, vv[j + 1], dv[j + 1]) : 0.f;
+                        const float p0 = u0 * us, p1 = u1 * us;
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                        const float2 hf = __bfloat1622float2(h2);
+                        const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(u0, u1);
+                        phi[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                        plo[j / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+                        pub[j / 2] = *reinterpret_cast<const uint32_t*>(&b2);
                     }
-                    if (smem_ok(sm + L::UHI + i * 128, 128, 29)) store_half_row(sm + L::UHI, i, half * 4, hi);
-                    if (smem_ok(sm + L::ULO + i * 128, 128, 30)) store_half_row(sm + L::ULO, i, half * 4, dv);
-                    if (smem_ok(sm + L::UB + i * 128, 128, 31)) store_half_row(sm + L::UB, i, half * 4, vv);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int ch = half * 4 + q;
+                        *reinterpret_cast<uint4*>(sm + L::UHI + swz(i, ch)) = make_uint4(phi[4 * q], phi[4 * q + 1], phi[4 * q + 2], phi[4 * q + 3]);
+                        *reinterpret_cast<uint4*>(sm + L::ULO + swz(i, ch)) = make_uint4(plo[4 * q], plo[4 * q + 1], plo[4 * q + 2], plo[4 * q + 3]);
+                        *reinterpret_cast<uint4*>(sm + L::UB + swz(i, ch)) = make_uint4(pub[4 * q], pub[4 * q + 1], pub[4 * q + 2], pub[4 * q + 3]);
+                    }
                 }
             }
             fence_proxy_async_smem();

@@ -71,18 +71,23 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
-// Wait for the phase with the given parity to complete.  Gives up after `limit_ns` or as soon
-// as *abort becomes non-zero; returns false in both cases (the caller then unwinds).  Lanes of
-// one warp may leave the polling loop at different times: callers that go on to aligned
-// (warp-collective) instructions use mbar_wait_warp, which reconverges the warp.
+// Wait for the phase with the given parity to complete.  Gives up after about `limit_ns`
+// (measured in SM clock cycles at a nominal 2 GHz, read only every 64 polls: the SM-local cycle
+// counter is cheap, unlike the global timer) or as soon as *abort becomes non-zero; returns
+// false in both cases (the caller then unwinds).  Lanes of one warp may leave the polling loop
+// at different times: callers that go on to aligned (warp-collective) instructions use
+// mbar_wait_warp, which reconverges the warp.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                           uint64_t limit_ns = 2000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const long long c0 = clock64();
+    const long long limit = static_cast<long long>(limit_ns) * 2;
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > limit_ns) return false;
+        if (clock64() - c0 > limit) return false;
     }
 }
 
@@ -269,6 +274,11 @@ __device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
