@@ -90,11 +90,15 @@ int gdn_workspace_bytes(int op, int B, int T, int H, int dk, int dv, int num_seq
     if (T < 1 || H < 1 || dk < 1 || dv < 1) return GDN_ERR_INVALID_ARG;
     switch (op) {
         case GDN_OP_PREFILL:
+            if (B < 1) return GDN_ERR_INVALID_ARG;
+            *bytes = gdn::prefill_workspace(B, T, H, dk, false).total;
+            return GDN_OK;
         case GDN_OP_DECODE:
             if (B < 1) return GDN_ERR_INVALID_ARG;
             return GDN_OK;
         case GDN_OP_PREFILL_VARLEN:
             if (num_seqs < 1) return GDN_ERR_INVALID_ARG;
+            *bytes = gdn::prefill_workspace(num_seqs, T, H, dk, true).total;
             return GDN_OK;
         case GDN_OP_BACKWARD:
             if (B < 1) return GDN_ERR_INVALID_ARG;
@@ -109,17 +113,19 @@ int gdn_prefill(const void* q, const void* k, const void* v, const float* alpha,
                 const float* beta, const float* s0, void* y, float* s_final, int B, int T, int H,
                 int dk, int dv, int dtype, float scale, int l2norm_qk, void* ws, size_t ws_bytes,
                 void* stream) {
-    (void)ws;
-    (void)ws_bytes;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
         !ok_ptr(y) || !ok_opt_ptr(s0) || !ok_opt_ptr(s_final))
         return GDN_ERR_INVALID_ARG;
     if (B < 1 || T < 1 || H < 1) return GDN_ERR_INVALID_ARG;
     if (int rc = check_dims(dk, dv, dtype)) return rc;
+    if (dtype == GDN_BF16) {
+        const size_t need = gdn::prefill_workspace(B, T, H, dk, false).total;
+        if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return GDN_ERR_WORKSPACE;
+    }
     DeviceInfo dev;
     if (int rc = current_device_info(&dev)) return rc;
     gdn::PrefillArgs a{q, k, v, alpha, beta, s0, y, s_final, nullptr, B, T, H, dk, dv,
-                       dtype, scale, l2norm_qk ? 1 : 0, dev.status};
+                       dtype, scale, l2norm_qk ? 1 : 0, dev.status, ws, ws_bytes};
     return map_cuda(gdn::launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -128,17 +134,19 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
                        const float* s0, void* y, float* s_final, int T, int H, int dk, int dv,
                        int dtype, float scale, int l2norm_qk, void* ws, size_t ws_bytes,
                        void* stream) {
-    (void)ws;
-    (void)ws_bytes;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
         !ok_ptr(y) || cu_seqlens == nullptr || !ok_opt_ptr(s0) || !ok_opt_ptr(s_final))
         return GDN_ERR_INVALID_ARG;
     if (num_seqs < 1 || T < 1 || H < 1) return GDN_ERR_INVALID_ARG;
     if (int rc = check_dims(dk, dv, dtype)) return rc;
+    if (dtype == GDN_BF16) {
+        const size_t need = gdn::prefill_workspace(num_seqs, T, H, dk, true).total;
+        if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return GDN_ERR_WORKSPACE;
+    }
     DeviceInfo dev;
     if (int rc = current_device_info(&dev)) return rc;
     gdn::PrefillArgs a{q, k, v, alpha, beta, s0, y, s_final, cu_seqlens, num_seqs, T, H, dk, dv,
-                       dtype, scale, l2norm_qk ? 1 : 0, dev.status};
+                       dtype, scale, l2norm_qk ? 1 : 0, dev.status, ws, ws_bytes};
     return map_cuda(gdn::launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -31,7 +31,17 @@ struct PrefillArgs {
     float scale;
     int l2norm;
     int* status;                // device status word
+    void* ws;                   // workspace (bf16 path), see prefill_workspace
+    size_t ws_bytes;
 };
+
+// Workspace of the bf16 prefill: per (chunk record, head) the operand tiles that the prep kernel
+// writes and the chain kernel reads, plus the chunk-record base of every packed document.
+struct PrefillWorkspace {
+    int nrec_chunks;  // chunk records (an upper bound for packed documents)
+    size_t off_cb, off_w, off_p, off_u, off_s, total;
+};
+PrefillWorkspace prefill_workspace(int num_seqs, int T, int H, int d, bool varlen);
 
 struct BackwardArgs {
     const void *q, *k, *v;

@@ -47,7 +47,20 @@ def test_status_strings(lib):
 
 def test_workspace_bytes(lib):
     n = ctypes.c_size_t(7)
+    # prefill: per (chunk record, head) -W (d*64 bf16), P (64*64 bf16), Ut (64*d fp32) and
+    # 256 fp32 scalars; packed documents add the chunk-record base array
+    rec = lambda d: d * 128 + 8192 + d * 256 + 1024
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL, 1, 4096, 16, 128, 128, 0,
+                                   ctypes.byref(n)) == 0
+    assert n.value == 64 * 16 * rec(128)
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL, 3, 65, 2, 64, 64, 0,
+                                   ctypes.byref(n)) == 0
+    assert n.value == 3 * 2 * 2 * rec(64)
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL_VARLEN, 1, 32768, 16, 128, 128, 4,
+                                   ctypes.byref(n)) == 0
+    nrec = (32768 + 63 * 4) // 64  # bound on sum(ceil(len / 64)) over the documents
+    assert n.value == 256 + nrec * 16 * rec(128)
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_DECODE, 4, 1, 2, 128, 128, 0,
                                    ctypes.byref(n)) == 0
     assert n.value == 0
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_BACKWARD, 8, 4096, 32, 128, 128, 0,
@@ -92,6 +105,12 @@ def _prefill(lib, **kw):
 ])
 def test_prefill_rejects_bad_arguments(lib, kw, code):
     assert _prefill(lib, **kw) == code
+
+
+def test_bf16_prefill_needs_its_workspace(lib):
+    assert _prefill(lib, ws=0, wsb=0) == _abi.GDN_ERR_WORKSPACE
+    assert _prefill(lib, ws=A, wsb=4096) == _abi.GDN_ERR_WORKSPACE
+    assert _prefill(lib, ws=A + 8, wsb=1 << 30) == _abi.GDN_ERR_WORKSPACE  # misaligned
 
 
 def test_varlen_rejects_bad_arguments(lib):
