@@ -142,10 +142,13 @@ def run_ours(args, rank, world, local_rank):
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     y = torch.empty((1, T_TOTAL, H, D), dtype=torch.bfloat16, device=dev)
     sf = torch.empty((NDOCS, H, D, D), dtype=torch.float32, device=dev)
+    from gated_deltanet_linear_eqs_b200._abi import GDN_OP_PREFILL_VARLEN
+    ws = torch.empty(api.gdn_workspace_bytes(GDN_OP_PREFILL_VARLEN, 1, T_TOTAL, H, D, D, NDOCS),
+                     dtype=torch.uint8, device=dev)
 
     def step():
         api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["cu_seqlens"],
-                               g["s0"], y=y, s_final=sf)
+                               g["s0"], y=y, s_final=sf, ws=ws)
 
     def barrier():
         if world > 1:
@@ -249,13 +252,15 @@ def run_train(args, dev, uuid, max_over_ranks, barrier, rank):
     """Training shape: forward (gdn_prefill) + backward (gdn_backward) per step."""
     import torch
     from gated_deltanet_linear_eqs_b200 import api
-    from gated_deltanet_linear_eqs_b200._abi import GDN_OP_BACKWARD
+    from gated_deltanet_linear_eqs_b200._abi import GDN_OP_BACKWARD, GDN_OP_PREFILL
     g = train_inputs(dev, seed=rank)
     ws = torch.empty(api.gdn_workspace_bytes(GDN_OP_BACKWARD, TRAIN_B, TRAIN_T, TRAIN_H, D, D),
                      dtype=torch.uint8, device=dev)
+    wsf = torch.empty(api.gdn_workspace_bytes(GDN_OP_PREFILL, TRAIN_B, TRAIN_T, TRAIN_H, D, D),
+                      dtype=torch.uint8, device=dev)
 
     def fwd():
-        return api.gdn_prefill(g["q"], g["k"], g["v"], g["alpha"], g["beta"])
+        return api.gdn_prefill(g["q"], g["k"], g["v"], g["alpha"], g["beta"], ws=wsf)
 
     def bwd():
         return api.gdn_backward(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["dy"], ws=ws)
@@ -280,7 +285,7 @@ def run_train(args, dev, uuid, max_over_ranks, barrier, rank):
     tokens = TRAIN_B * TRAIN_T
     return {"metric": "GDN fwd+bwd tokens/s (training shape)", "unit": "tokens/s",
             "value": tokens / ((f_ms + b_ms) / 1e3), "ms_per_step": f_ms + b_ms,
-            "fwd_ms": f_ms, "bwd_ms": b_ms, "steps": steps, "gpu_launches": 3 * steps,
+            "fwd_ms": f_ms, "bwd_ms": b_ms, "steps": steps, "gpu_launches": 4 * steps,
             "config": {"workload": f"train: B={TRAIN_B}, T={TRAIN_T}, H={TRAIN_H}, dk=dv={D}, "
                                    "bf16, dy ~ N(0,1), S0 = 0"},
             "clocks": clk.summary()}
@@ -294,11 +299,14 @@ def run_profile(args):
     dev = torch.device("cuda", 0)
     n = args.launches
     if args.profile == "prefill":
+        from gated_deltanet_linear_eqs_b200._abi import GDN_OP_PREFILL_VARLEN
         _, inp = varlen_workload(seed=0)
         g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        ws = torch.empty(api.gdn_workspace_bytes(GDN_OP_PREFILL_VARLEN, 1, T_TOTAL, H, D, D, NDOCS),
+                         dtype=torch.uint8, device=dev)
         for _ in range(n + 1):
             api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
-                                   g["cu_seqlens"], g["s0"])
+                                   g["cu_seqlens"], g["s0"], ws=ws)
     elif args.profile == "decode":
         from gated_deltanet_linear_eqs_b200.inputs import make_decode_state, make_decode_step_inputs
         S = make_decode_state(DEC_N, H, D, D, seed=0).to(dev)
@@ -486,7 +494,7 @@ def main():
                             "l2": "inputs (403 MB) exceed the 126 MB L2; no flush"},
                     roofline=p["roofline"], roofline_hbm=p["roofline_hbm"],
                     frac_bf16_sustained=p["frac_bf16_sustained"], kernel_ms=p["kern_ms"],
-                    clocks=p["clocks"], e2e=res["e2e"], gpu_launches=args.steps)
+                    clocks=p["clocks"], e2e=res["e2e"], gpu_launches=3 * args.steps)
     if "train" in res:
         line["train"] = res["train"]
     if "decode" in res:

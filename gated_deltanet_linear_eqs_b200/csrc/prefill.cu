@@ -70,6 +70,26 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
     return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
                       pack_bf16(x[6], x[7]));
 }
+// Round-to-nearest bf16 pair on the FP32 pipe instead of the conversion unit (which runs at a
+// fraction of the FP32 rate): Veltkamp's splitting with the factor 2^16 + 1 leaves the 8
+// leading significand bits of x in hi (the low 16 bits of hi are zero), and the two upper halves
+// are packed with one byte permute.  Valid for |x| < 2^111.
+__device__ __forceinline__ uint32_t pack_bf16_fma(float a, float b) {
+    const float ca = __fmul_rn(a, 65537.f), cb = __fmul_rn(b, 65537.f);
+    const float ha = __fsub_rn(ca, __fsub_rn(ca, a)), hb = __fsub_rn(cb, __fsub_rn(cb, b));
+    return __byte_perm(__float_as_uint(ha), __float_as_uint(hb), 0x7632);
+}
+__device__ __forceinline__ uint4 pack8_fma(const float* x) {
+    return make_uint4(pack_bf16_fma(x[0], x[1]), pack_bf16_fma(x[2], x[3]),
+                      pack_bf16_fma(x[4], x[5]), pack_bf16_fma(x[6], x[7]));
+}
+// 32 floats -> 4 swizzled 16-byte chunks, half of them rounded on each pipe
+__device__ __forceinline__ void store_half_row_mixed(uint8_t* tile, int row, int c0, const float* x) {
+    *reinterpret_cast<uint4*>(tile + swz(row, c0 + 0)) = pack8(x);
+    *reinterpret_cast<uint4*>(tile + swz(row, c0 + 1)) = pack8_fma(x + 8);
+    *reinterpret_cast<uint4*>(tile + swz(row, c0 + 2)) = pack8(x + 16);
+    *reinterpret_cast<uint4*>(tile + swz(row, c0 + 3)) = pack8_fma(x + 24);
+}
 // 32 floats -> 4 swizzled 16-byte chunks (chunk index c0..c0+3) of a 128-byte bf16 row
 // (shared or global memory: the same tile image)
 __device__ __forceinline__ void store_half_row(uint8_t* tile, int row, int c0, const float* x) {
@@ -146,13 +166,14 @@ struct PrepLayout {
     static constexpr int KB = D / 64;
     static constexpr int KQ = 0;                      // per dk block: K rows 0-63, Q rows 64-127
     static constexpr int V = KB * 16384;              // V: dv/64 blocks of 64 tokens x 64 columns
-    static constexpr int TWN = V + KB * 8192;         // 128 rows: T_w (0-63), N_b (64-127)
-    static constexpr int AF = TWN + 16384;            // A, bf16 64 x kLd
+    static constexpr int AF = V + KB * 8192;          // A, bf16 64 x kLd
     static constexpr int TF = AF + 64 * kLd * 2;      // T, bf16 64 x kLd
+    static constexpr int TWN = AF;                    // 128 rows: T_w (0-63), N_b (64-127), written
+                                                      // over A and T once T is in registers
     static constexpr int XB = TF + 64 * kLd * 2;      // 4 warps x 16 x 24 bf16
     static constexpr int AB = XB + 4 * 16 * 24 * 2;   // alpha[64], beta[64]
     static constexpr int SC = AB + 512;               // scalar arrays, 64 floats each
-    static constexpr int BAR = SC + 7 * 256;
+    static constexpr int BAR = SC + 8 * 256;
     static constexpr int MISC = BAR + 8 * 8;          // tmem base, abort flag, zero word
     static constexpr int BYTES = MISC + 16;
     static constexpr int TX = KB * 16384 + KB * 8192;
@@ -160,10 +181,11 @@ struct PrepLayout {
     static constexpr uint32_t T_D3 = 0;               // W (D columns, lanes 0-63)
     static constexpr uint32_t T_DU = D;               // N_b V (D columns, lanes 64-127)
     static constexpr uint32_t T_COLS = 2 * D;
-    static_assert(2 * (BYTES + 1024) <= 232448 - 2048, "two prep CTAs per SM");
+    static_assert(TWN % 1024 == 0 && TF + 64 * kLd * 2 >= TWN + 16384, "T_w / N_b tile");
+    static_assert(3 * (BYTES + 1024 + 1024) <= 233472, "three prep CTAs per SM");
 };
-enum { PS_G = 0, PS_GAM, PS_BETA, PS_RK, PS_RQ, PS_FTW, PS_CARRY };
-enum { PB_FULL = 0, PB_M1, PB_RA1, PB_M3, PB_FIN, PB_COUNT };
+enum { PS_G = 0, PS_GAM, PS_BETA, PS_RK, PS_RQ, PS_FTW, PS_CARRY, PS_COLF };
+enum { PB_FULL = 0, PB_TMEM, PB_M1, PB_RA1, PB_M3, PB_FIN, PB_COUNT };
 
 struct PrepParams {
     const float* alpha;
@@ -184,8 +206,11 @@ struct PrepParams {
 
 constexpr int kPrepThreads = 192;
 
+// Up to three CTAs share an SM (shared memory and registers allow it), but TMEM holds two
+// allocations: the third CTA's allocation waits until one of the others frees its columns.
+// Everything that needs no TMEM (the input copies, decay and norms) runs before that point.
 template <int D>
-__global__ void __launch_bounds__(kPrepThreads, 2)
+__global__ void __launch_bounds__(kPrepThreads, 3)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const PrepParams p) {
     using L = PrepLayout<D>;
@@ -224,16 +249,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     volatile int* never = reinterpret_cast<volatile int*>(sm + L::MISC + 8);
     if (tid == 0) {
         mbar_init(&bars[PB_FULL], 32);
-        for (int b = PB_M1; b < PB_COUNT; ++b) mbar_init(&bars[b], 1);
+        for (int b = PB_TMEM; b < PB_COUNT; ++b) mbar_init(&bars[b], 1);
         *abort_flag = 0;
         *never = 0;
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(tmem_slot, L::T_COLS);
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
 
 #define GUARD(cond, code, detail) GDN_GUARD(cond, p.status, code, detail)
     auto fail = [&](int bar) {
@@ -250,10 +271,17 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     if (warp == 0) {
         // ---------------------------------------------------------------- loads
+        // the tile copies first (lane 0's arrival carries the byte count), then alpha and beta;
+        // the other 31 arrivals follow the alpha / beta stores of all lanes
         if (lane == 0) {
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
+            mbar_arrive_expect_tx(&bars[PB_FULL], L::TX);
+            const int z = (int)base;
+#pragma unroll
+            for (int b = 0; b < KB; ++b) {
+                tma_load_3d(sm + L::KQ + b * 16384, &tm_k, 64 * b, h, z, &bars[PB_FULL]);
+                tma_load_3d(sm + L::KQ + b * 16384 + 8192, &tm_q, 64 * b, h, z, &bars[PB_FULL]);
+                tma_load_3d(sm + L::V + b * 8192, &tm_v, 64 * b, h, z, &bars[PB_FULL]);
+            }
         }
         float* ab = reinterpret_cast<float*>(sm + L::AB);
 #pragma unroll
@@ -265,22 +293,17 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             ab[64 + i] = ok ? p.beta[t * p.H + h] : 0.f;
         }
         __syncwarp();
-        if (lane == 0) {
-            mbar_arrive_expect_tx(&bars[PB_FULL], L::TX);
-            const int z = (int)base;
-#pragma unroll
-            for (int b = 0; b < KB; ++b) {
-                tma_load_3d(sm + L::KQ + b * 16384, &tm_k, 64 * b, h, z, &bars[PB_FULL]);
-                tma_load_3d(sm + L::KQ + b * 16384 + 8192, &tm_q, 64 * b, h, z, &bars[PB_FULL]);
-                tma_load_3d(sm + L::V + b * 8192, &tm_v, 64 * b, h, z, &bars[PB_FULL]);
-            }
-        } else {
-            mbar_arrive(&bars[PB_FULL]);
-        }
+        if (lane != 0) mbar_arrive(&bars[PB_FULL]);
         // do not leave while the copies are still writing shared memory
         mbar_wait_warp(&bars[PB_FULL], 0, never, 100000000ull);
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- tensor-core issue
+        // ---------------------------------------------------------------- TMEM and tensor cores
+        tmem_alloc(tmem_slot, L::T_COLS);  // may wait for another CTA on this SM to free TMEM
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[PB_TMEM]);
+        tc_fence_after();
+        const uint32_t tmem = *tmem_slot;
         if (lane == 0) {
             constexpr uint32_t ID_M1 = idesc_bf16(128, 64, false, false);
             constexpr uint32_t ID_N = idesc_bf16(128, D, false, true);
@@ -335,6 +358,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         float* sRq = scal(PS_RQ);
         float* sFtw = scal(PS_FTW);
         float* sCarry = scal(PS_CARRY);
+        float* sColf = scal(PS_COLF);
         float* rs = p.ws_s + rec * (kRecS / 4);
 
         // (1) decay and norms
@@ -370,6 +394,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (t < 64) {
                 const float G = sG[t], gam = ex2(G);
                 sGam[t] = gam;
+                sColf[t] = ex2(sG[t | 15] - G);  // decay from token t to the end of its 16-block
                 sFtw[t] = sBeta[t] * gam * sRk[t];
                 rs[t] = (t < nvalid) ? ex2(Glast - G) * sRk[t] : 0.f;
                 if (t == 0) rs[128] = ex2(Glast);
@@ -381,49 +406,51 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         named_sync(1, 128);
 
         // (2) A (rows 0-63 of M1, to shared memory) and P (rows 64-127, to the workspace)
+        ok = wwait(PB_TMEM, 0) && ok;
+        tc_fence_after();
+        const uint32_t tmem = *tmem_slot;
         ok = wwait(PB_M1, 0) && ok;
         tc_fence_after();
+        // Gam_ij = 2^(G_i - G_j) for j <= i.  Within the row's own 16-token block it is computed
+        // directly; for an earlier block b it is the product 2^(G_i - G_e) 2^(G_e - G_j) through
+        // the block's last token e = 16 b + 15.  Both exponents are <= 0 (G does not increase),
+        // so neither factor can overflow, and the row needs 19 exponentials instead of 64.
         if (ok) {
-            if (t < 64) {
-                const int i = t;
-                const float Gi = sG[i], bi = sBeta[i] * sRk[i];
+            const int i = t & 63, blk = i >> 4;
+            const bool arow = t < 64;  // rows of A (strictly lower) or of P (lower, diagonal incl.)
+            const float Gi = sG[i];
+            const float sc = arow ? sBeta[i] * sRk[i] : p.scale * sRq[i];
+            float rowf[3], dg[16];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float d[32];
-                    tmem_ld32(tmem + L::T_D1 + lane_base + half * 32, d);
+            for (int b = 0; b < 3; ++b) rowf[b] = ex2(Gi - sG[16 * b + 15]);
 #pragma unroll
-                    for (int j4 = 0; j4 < 32; j4 += 4) {
-                        const int j = half * 32 + j4;
-                        const float4 rk4 = *reinterpret_cast<const float4*>(sRk + j);
-                        const float4 g4 = *reinterpret_cast<const float4*>(sG + j);
-                        d[j4 + 0] = (j + 0 < i) ? bi * rk4.x * d[j4 + 0] * ex2(Gi - g4.x) : 0.f;
-                        d[j4 + 1] = (j + 1 < i) ? bi * rk4.y * d[j4 + 1] * ex2(Gi - g4.y) : 0.f;
-                        d[j4 + 2] = (j + 2 < i) ? bi * rk4.z * d[j4 + 2] * ex2(Gi - g4.z) : 0.f;
-                        d[j4 + 3] = (j + 3 < i) ? bi * rk4.w * d[j4 + 3] * ex2(Gi - g4.w) : 0.f;
+            for (int u = 0; u < 16; ++u) dg[u] = ex2(Gi - sG[16 * blk + u]);
+            const int lim = arow ? i : i + 1;  // columns j < lim are kept
+            uint8_t* P = p.ws_p + rec * kRecP;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float d[32];
+                tmem_ld32(tmem + L::T_D1 + lane_base + half * 32, d);
+#pragma unroll
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const int j = half * 32 + j4, cb = j >> 4;
+                    const float4 rk4 = *reinterpret_cast<const float4*>(sRk + j);
+                    const float4 cf4 = *reinterpret_cast<const float4*>(sColf + j);
+                    const float rk[4] = {rk4.x, rk4.y, rk4.z, rk4.w};
+                    const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float f = (cb < blk) ? rowf[cb < 3 ? cb : 2] * cf[u] : dg[(j & 15) + u];
+                        d[j4 + u] = (j + u < lim) ? sc * rk[u] * d[j4 + u] * f : 0.f;
                     }
+                }
+                if (arow) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<uint4*>(AF + i * kLd + half * 32 + 8 * q) = pack8(d + 8 * q);
-                }
-            } else {
-                const int r = t - 64;
-                const float Gr = sG[r], pr = p.scale * sRq[r];
-                uint8_t* P = p.ws_p + rec * kRecP;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float d[32];
-                    tmem_ld32(tmem + L::T_D1 + lane_base + half * 32, d);
-#pragma unroll
-                    for (int j4 = 0; j4 < 32; j4 += 4) {
-                        const int j = half * 32 + j4;
-                        const float4 rk4 = *reinterpret_cast<const float4*>(sRk + j);
-                        const float4 g4 = *reinterpret_cast<const float4*>(sG + j);
-                        d[j4 + 0] = (j + 0 <= r) ? pr * rk4.x * d[j4 + 0] * ex2(Gr - g4.x) : 0.f;
-                        d[j4 + 1] = (j + 1 <= r) ? pr * rk4.y * d[j4 + 1] * ex2(Gr - g4.y) : 0.f;
-                        d[j4 + 2] = (j + 2 <= r) ? pr * rk4.z * d[j4 + 2] * ex2(Gr - g4.z) : 0.f;
-                        d[j4 + 3] = (j + 3 <= r) ? pr * rk4.w * d[j4 + 3] * ex2(Gr - g4.w) : 0.f;
-                    }
-                    store_half_row(P, r, half * 4, d);
+                        *reinterpret_cast<uint4*>(AF + i * kLd + half * 32 + 8 * q) =
+                            (q & 1) ? pack8_fma(d + 8 * q) : pack8(d + 8 * q);
+                } else {
+                    store_half_row_mixed(P, i, half * 4, d);
                 }
             }
         }
@@ -492,33 +519,39 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         }
 
-        // (4) T_w = T diag(beta gamma rk) -> rows 0-63;  N_b = strict(T) diag(beta) -> rows 64-127
-        if (ok) {
+        // (4) T_w = T diag(beta gamma rk) -> rows 0-63;  N_b = strict(T) diag(beta) -> rows 64-127.
+        // The tile overlays A and T, so every thread first takes its T row into registers.
+        {
             const int i = t & 63;
-            const __nv_bfloat16* trow = TF + i * kLd;
+            uint4 tr[8];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float x[32];
+            for (int q = 0; q < 8; ++q) tr[q] = *reinterpret_cast<const uint4*>(TF + i * kLd + 8 * q);
+            named_sync(1, 128);
+            if (ok) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) unpack8(*reinterpret_cast<const uint4*>(trow + half * 32 + 8 * q), x + 8 * q);
+                for (int half = 0; half < 2; ++half) {
+                    float x[32];
 #pragma unroll
-                for (int j4 = 0; j4 < 32; j4 += 4) {
-                    const int j = half * 32 + j4;
-                    if (t < 64) {
-                        const float4 f4 = *reinterpret_cast<const float4*>(sFtw + j);
-                        x[j4 + 0] = (j + 0 <= i) ? x[j4 + 0] * f4.x : 0.f;
-                        x[j4 + 1] = (j + 1 <= i) ? x[j4 + 1] * f4.y : 0.f;
-                        x[j4 + 2] = (j + 2 <= i) ? x[j4 + 2] * f4.z : 0.f;
-                        x[j4 + 3] = (j + 3 <= i) ? x[j4 + 3] * f4.w : 0.f;
-                    } else {
-                        const float4 b4 = *reinterpret_cast<const float4*>(sBeta + j);
-                        x[j4 + 0] = (j + 0 < i) ? x[j4 + 0] * b4.x : 0.f;
-                        x[j4 + 1] = (j + 1 < i) ? x[j4 + 1] * b4.y : 0.f;
-                        x[j4 + 2] = (j + 2 < i) ? x[j4 + 2] * b4.z : 0.f;
-                        x[j4 + 3] = (j + 3 < i) ? x[j4 + 3] * b4.w : 0.f;
+                    for (int q = 0; q < 4; ++q) unpack8(tr[half * 4 + q], x + 8 * q);
+#pragma unroll
+                    for (int j4 = 0; j4 < 32; j4 += 4) {
+                        const int j = half * 32 + j4;
+                        if (t < 64) {
+                            const float4 f4 = *reinterpret_cast<const float4*>(sFtw + j);
+                            x[j4 + 0] = (j + 0 <= i) ? x[j4 + 0] * f4.x : 0.f;
+                            x[j4 + 1] = (j + 1 <= i) ? x[j4 + 1] * f4.y : 0.f;
+                            x[j4 + 2] = (j + 2 <= i) ? x[j4 + 2] * f4.z : 0.f;
+                            x[j4 + 3] = (j + 3 <= i) ? x[j4 + 3] * f4.w : 0.f;
+                        } else {
+                            const float4 b4 = *reinterpret_cast<const float4*>(sBeta + j);
+                            x[j4 + 0] = (j + 0 < i) ? x[j4 + 0] * b4.x : 0.f;
+                            x[j4 + 1] = (j + 1 < i) ? x[j4 + 1] * b4.y : 0.f;
+                            x[j4 + 2] = (j + 2 < i) ? x[j4 + 2] * b4.z : 0.f;
+                            x[j4 + 3] = (j + 3 < i) ? x[j4 + 3] * b4.w : 0.f;
+                        }
                     }
+                    store_half_row_mixed(sm + L::TWN, t, half * 4, x);
                 }
-                store_half_row(sm + L::TWN, t, half * 4, x);
             }
         }
         fence_proxy_async_smem();
@@ -539,7 +572,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         tmem_ld32(tmem + L::T_D3 + lane_base + 64 * b + 32 * half, w);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) w[j] = -w[j];
-                        store_half_row(wrec + b * 8192, t, half * 4, w);
+                        store_half_row_mixed(wrec + b * 8192, t, half * 4, w);
                     }
             } else {
                 const int i = t - 64;
@@ -573,7 +606,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, L::T_COLS);
+        tmem_dealloc(*tmem_slot, L::T_COLS);
     }
 }
 
@@ -592,20 +625,19 @@ struct ChainLayout {
     static constexpr int ULO = UHI + 8192;
     static constexpr int UB = ULO + 8192;
     static constexpr int BAR = UB + 8192;
-    static constexpr int MISC = BAR + 16 * 8;     // tmem base, abort flag, zero word
-    static constexpr int BYTES = MISC + 16;
+    static constexpr int MISC = BAR + 16 * 8;     // tmem base, abort flag, zero word, 2 counters
+    static constexpr int BYTES = MISC + 32;
     static constexpr int TX = KB * 16384 + KB * 8192 + 8192 + 16384 + 1024;
-    static constexpr uint32_t T_S = 0;            // K^T U' of the current chunk, 64 columns
-    static constexpr uint32_t T_D4 = 64;          // [Q S ; -W S], 2 x 64 columns
-    static constexpr uint32_t T_D6 = 192;         // P U, 2 x 64 columns
+    static constexpr uint32_t T_S = 0;            // [K^T U'_hi | K^T U'_lo] of the chunk, 128 columns
+    static constexpr uint32_t T_D4 = 128;         // [Q S ; -W S], 2 x 64 columns
+    static constexpr uint32_t T_D6 = 256;         // P U, 2 x 64 columns
     static constexpr uint32_t T_COLS = 512;
     static_assert(STAGE % 1024 == 0, "stage tiles stay 1024-byte aligned");
     static_assert(BYTES + 1024 <= 232448 - 1024, "shared memory budget");
 };
 enum {
     CB_FULL0 = 0, CB_FULL1, CB_EMPTY0, CB_EMPTY1,  // input ring
-    CB_M4, CB_M5, CB_M6_0, CB_M6_1, CB_FIN,        // tensor-core completions
-    CB_RB4, CB_RB5, CB_YD0, CB_YD1,                // epilogue warps -> MMA issuer
+    CB_M4, CB_M5, CB_M6_0, CB_M6_1,                // tensor-core completions
     CB_COUNT
 };
 
@@ -627,10 +659,12 @@ struct ChainParams {
 
 constexpr int kChainThreads = 384;
 
-// Warp roles: 0 loads (TMA for K and Q, bulk copies for the workspace record), 1 issues the
-// tensor-core work, 4..11 are the epilogue warps.  Epilogue warp w reads TMEM lanes
-// 32 (w % 4) .. +31 and columns 32 ((w - 4) / 4) .. +31; lanes 0-63 carry the output rows (Y)
-// and lanes 64-127 the pseudo-value rows (U); all eight hold a 32-column strip of S.
+// Warp roles: 0 loads (TMA for K and Q, bulk copies for the workspace record), 1 owns the TMEM
+// allocation, 4..11 are the epilogue warps.  Epilogue warp w reads TMEM lanes 32 (w % 4) .. +31
+// and columns 32 ((w - 4) / 4) .. +31; lanes 0-63 carry the output rows (Y) and lanes 64-127 the
+// pseudo-value rows (U); all eight hold a 32-column strip of S.  There is no separate MMA warp:
+// the last epilogue warp to finish a step (found with a shared-memory arrival counter) issues the
+// tensor-core products that depend on it, which saves a wake-up on the sequential path.
 template <int D>
 __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -680,18 +714,17 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
     volatile int* never = reinterpret_cast<volatile int*>(sm + L::MISC + 8);
+    int* arrivals = reinterpret_cast<int*>(sm + L::MISC + 16);  // (A) and (B) completions
     if (tid == 0) {
         mbar_init(&bars[CB_FULL0], 1);
         mbar_init(&bars[CB_FULL1], 1);
         mbar_init(&bars[CB_EMPTY0], 5);  // MMA commit + 4 output warps
         mbar_init(&bars[CB_EMPTY1], 5);
-        for (int b = CB_M4; b <= CB_FIN; ++b) mbar_init(&bars[b], 1);
-        mbar_init(&bars[CB_RB4], 8);
-        mbar_init(&bars[CB_RB5], 4);
-        mbar_init(&bars[CB_YD0], 4);
-        mbar_init(&bars[CB_YD1], 4);
+        for (int b = CB_M4; b < CB_COUNT; ++b) mbar_init(&bars[b], 1);
         *abort_flag = 0;
         *never = 0;
+        arrivals[0] = 0;
+        arrivals[1] = 0;
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, L::T_COLS);
@@ -706,7 +739,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         record_status(p.status, GDN_ERR_TIMEOUT);
     };
     auto wwait = [&](int bar, uint32_t parity, int c) {
-        const bool ok = mbar_wait_warp(&bars[bar], parity, abort_flag);
+        const bool ok = mbar_spin_warp(&bars[bar], parity, abort_flag);
         if (!ok && lane == 0) fail(bar, c);
         return ok;
     };
@@ -761,55 +794,26 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- tensor-core issue
+        // ---------------------------------------------------------------- output product M6
         if (lane == 0) {
             constexpr uint32_t ID_KN = idesc_bf16(128, kNV, false, true);
-            constexpr uint32_t ID_M5 = idesc_bf16(128, kNV, true, true);
-            const uint32_t st0 = smem_u32(sm);
-            const uint64_t dQW0 = sdesc(st0 + 8192, 16, 1024);                    // [Q; -W] rows
-            const uint64_t dKt0 = sdesc(st0, D == 128 ? L::KQW_BLOCK : 0, 1024);  // K^T, MN-major
-            const uint64_t dP0 = sdesc(st0 + L::P, 16, 1024);
-            const uint64_t dSB = sdesc(smem_u32(sm + L::SB), D * 128, 1024);
-            const uint64_t dUHI = sdesc(smem_u32(sm + L::UHI), 8192, 1024);
-            const uint64_t dULO = sdesc(smem_u32(sm + L::ULO), 8192, 1024);
+            constexpr uint64_t KS = 32 >> 4, MS = 2048 >> 4;
             const uint64_t dUB = sdesc(smem_u32(sm + L::UB), 8192, 1024);
-            constexpr uint64_t SST = L::STAGE >> 4;
-            constexpr uint64_t KS = 32 >> 4, MS = 2048 >> 4, BLK = L::KQW_BLOCK >> 4;
-            int bad = -1;
             for (int c = 0; c < nch; ++c) {
                 const int s = c & 1;
-                if (!mbar_wait(&bars[CB_FULL0 + s], (c >> 1) & 1, abort_flag)) { bad = CB_FULL0 + s; break; }
-                if (!mbar_wait(&bars[CB_RB4], c & 1, abort_flag)) { bad = CB_RB4; break; }
-                if (c >= 2 && !mbar_wait(&bars[CB_YD0 + s], ((c - 2) >> 1) & 1, abort_flag)) { bad = CB_YD0 + s; break; }
+                // U_bf16 of chunk c is complete once M5(c) is (M5 is issued after it is written)
+                if (!mbar_wait(&bars[CB_M5], c & 1, abort_flag)) {
+                    if (!*abort_flag) fail(CB_M5, c);
+                    break;
+                }
                 tc_fence_after();
-                // M4: [Q; -W] S  ->  Q S (lanes 0-63), -W S (lanes 64-127)
-                const uint32_t d4 = tmem + L::T_D4 + s * 64;
-#pragma unroll
-                for (int b = 0; b < KB; ++b)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(d4, dQW0 + s * SST + b * BLK + kk * KS, dSB + (b * 4 + kk) * MS, ID_KN, (b | kk) != 0);
-                mma_commit(&bars[CB_M4]);
-                if (!mbar_wait(&bars[CB_RB5], c & 1, abort_flag)) { bad = CB_RB5; break; }
-                tc_fence_after();
-                // M5: K^T U'_hi + K^T U'_lo (U' = diag(Gam_C,. rk) U in two bf16 terms)
+                const uint64_t dP = sdesc(smem_u32(sm + s * L::STAGE + L::P), 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + L::T_S, dKt0 + s * SST + kk * MS, dUHI + kk * MS, ID_M5, kk != 0);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + L::T_S, dKt0 + s * SST + kk * MS, dULO + kk * MS, ID_M5, 1);
-                mma_commit(&bars[CB_M5]);
-                // M6: P U_bf16
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + L::T_D6 + s * 64, dP0 + s * SST + kk * KS, dUB + kk * MS, ID_KN, kk != 0);
+                    mma_bf16(tmem + L::T_D6 + s * 64, dP + kk * KS, dUB + kk * MS, ID_KN, kk != 0);
                 mma_commit(&bars[CB_M6_0 + s]);
                 mma_commit(&bars[CB_EMPTY0 + s]);
             }
-            if (bad >= 0 && !*abort_flag) fail(bad, 0);
-            mma_commit(&bars[CB_FIN]);
-            mbar_wait(&bars[CB_FIN], 0, never, 100000000ull);
         }
         __syncwarp();
     } else if (warp >= 4) {
@@ -833,6 +837,55 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         float gprev = 1.f;
         bool ok = true;
 
+        constexpr uint32_t ID_KN = idesc_bf16(128, kNV, false, true);
+        constexpr uint32_t ID_M5 = idesc_bf16(128, 2 * kNV, true, true);  // B = [U'_hi | U'_lo]
+        constexpr uint64_t KS = 32 >> 4, MS = 2048 >> 4, BLK = L::KQW_BLOCK >> 4;
+        static_assert(L::ULO == L::UHI + 8192, "U'_lo is the second 64-column atom of U'");
+        // M4: [Q; -W] S_bf16  ->  Q S (lanes 0-63), -W S (lanes 64-127)
+        auto issue_m4 = [&](int c) {
+            const int s = c & 1;
+            const uint64_t dQW = sdesc(smem_u32(sm + s * L::STAGE + 8192), 16, 1024);
+            const uint64_t dSB = sdesc(smem_u32(sm + L::SB), D * 128, 1024);
+            const uint32_t d4 = tmem + L::T_D4 + s * 64;
+#pragma unroll
+            for (int b = 0; b < KB; ++b)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(d4, dQW + b * BLK + kk * KS, dSB + (b * 4 + kk) * MS, ID_KN, (b | kk) != 0);
+            mma_commit(&bars[CB_M4]);
+        };
+        // M5: K^T [U'_hi | U'_lo] (U' = diag(Gam_C,. rk) U in two bf16 terms, side by side in N:
+        // an N = 128 product costs the tensor core what an N = 64 one does).  The output product
+        // M6 is issued by warp 1 once M5 is done, so that it does not delay M5's completion.
+        auto issue_m56 = [&](int c) {
+            const int s = c & 1;
+            const uint64_t dKt = sdesc(smem_u32(sm + s * L::STAGE), D == 128 ? L::KQW_BLOCK : 0, 1024);
+            const uint64_t dUHI = sdesc(smem_u32(sm + L::UHI), 8192, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem + L::T_S, dKt + kk * MS, dUHI + kk * MS, ID_M5, kk != 0);
+            mma_commit(&bars[CB_M5]);
+        };
+        // Arrival of this warp at the end of a step; the last of `n` arrivals for chunk c issues
+        // the dependent products.  The warp's shared-memory and TMEM accesses are ordered before
+        // the counter update (proxy and tcgen05 fences, then a CTA-scope fence), and the issuing
+        // thread orders the counter read before its tcgen05 operations the same way.
+        auto arrive = [&](int which, int n, int c) {
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence_block();
+                const int old = atomicAdd(arrivals + which, 1);
+                if (old == n * c + n - 1) {
+                    __threadfence_block();
+                    tc_fence_after();
+                    if (which == 0) issue_m4(c); else issue_m56(c);
+                }
+            }
+            __syncwarp();
+        };
+
         auto y_epilogue = [&](int cy) {
             const int s = cy & 1;
             ok = wwait(CB_M6_0 + s, (cy >> 1) & 1, cy) && ok;
@@ -841,8 +894,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 const uint8_t* st = sm + s * L::STAGE;
                 const int nv = min(kChunk, len - cy * kChunk);
                 float a[32], b[32];
-                tmem_ld32(tmem + L::T_D4 + s * 64 + lane_base + col, a);
-                tmem_ld32(tmem + L::T_D6 + s * 64 + lane_base + col, b);
+                tmem_ld32x2(tmem + L::T_D4 + s * 64 + lane_base + col, tmem + L::T_D6 + s * 64 + lane_base + col, a, b);
                 const float ys = reinterpret_cast<const float*>(st + L::SC)[64 + srow];
                 const size_t yoff = ((size_t)(t0 + (long)cy * kChunk + srow) * p.H + h) * p.DV + jsl * kNV + col;
                 if (srow < nv && GUARD((long long)(yoff + 32) <= p.y_elems, DBG_GLOBAL_OOB, 3)) {
@@ -855,10 +907,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars[CB_YD0 + s]);
-                mbar_arrive(&bars[CB_EMPTY0 + s]);
-            }
+            if (lane == 0) mbar_arrive(&bars[CB_EMPTY0 + s]);
         };
 
         for (int c = 0; c < nch; ++c) {
@@ -870,22 +919,24 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 ok = wwait(CB_M5, (c - 1) & 1, c) && ok;
                 tc_fence_after();
                 if (ok) {
-                    float d[32];
-                    tmem_ld32(tmem + L::T_S + lane_base + col, d);
+                    float d[32], e[32];
+                    tmem_ld32x2(tmem + L::T_S + lane_base + col, tmem + L::T_S + lane_base + kNV + col, d, e);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) S[j] = fmaf(gprev, S[j], d[j]);
+                    for (int j = 0; j < 32; ++j) S[j] = fmaf(gprev, S[j], d[j] + e[j]);
                 }
             }
-            if (ok && srow < D) store_half_row(sm + L::SB, srow, 4 * hf, S);
+            if (ok && srow < D) store_half_row_mixed(sm + L::SB, srow, 4 * hf, S);
             gprev = reinterpret_cast<const float*>(st + L::SC)[128];
-            tc_fence_before();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[CB_RB4]);
+            // M4 of this chunk may overwrite the output accumulators of chunk c - 2: the output
+            // warps read them in iteration c - 1, before this arrival
+            arrive(0, 8, c);
 
             if (uwarp) {
-                // (B) U = Ut + (-W S) -> U'_hi, U'_lo (scaled for the state update), U_bf16
+                // (B) U = Ut + (-W S) -> U'_hi, U'_lo (scaled for the state update), U_bf16.
+                // M6 of the previous chunk (issued by another thread, so not covered by this
+                // chunk's M4 commit) must have finished reading U_bf16.
                 ok = wwait(CB_M4, c & 1, c) && ok;
+                if (c >= 1) ok = wwait(CB_M6_0 + ((c - 1) & 1), ((c - 1) >> 1) & 1, c) && ok;
                 tc_fence_after();
                 if (ok) {
                     const int i = srow - 64;
@@ -900,14 +951,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                         const float u[4] = {ut.x + d[4 * q], ut.y + d[4 * q + 1], ut.z + d[4 * q + 2], ut.w + d[4 * q + 3]};
 #pragma unroll
                         for (int e = 0; e < 4; e += 2) {
-                            const float p0 = u[e] * us, p1 = u[e + 1] * us;
-                            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                            const float2 hfl = __bfloat1622float2(h2);
-                            const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - hfl.x, p1 - hfl.y);
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(u[e], u[e + 1]);
-                            phi[2 * q + e / 2] = *reinterpret_cast<const uint32_t*>(&h2);
-                            plo[2 * q + e / 2] = *reinterpret_cast<const uint32_t*>(&l2);
-                            pub[2 * q + e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+                            // U' = hi + lo with hi = U' truncated to bf16 and lo = the exact fp32
+                            // rest, itself truncated: |U' - hi - lo| < 2^-14 |U'|.  Bit operations
+                            // only, no conversion instructions.
+                            const uint32_t b0 = __float_as_uint(u[e] * us), b1 = __float_as_uint(u[e + 1] * us);
+                            const float l0 = __uint_as_float(b0) - __uint_as_float(b0 & 0xffff0000u);
+                            const float l1 = __uint_as_float(b1) - __uint_as_float(b1 & 0xffff0000u);
+                            phi[2 * q + e / 2] = __byte_perm(b0, b1, 0x7632);
+                            plo[2 * q + e / 2] = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
+                            pub[2 * q + e / 2] = pack_bf16(u[e], u[e + 1]);
                         }
                     }
 #pragma unroll
@@ -918,10 +970,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                         *reinterpret_cast<uint4*>(sm + L::UB + off) = make_uint4(pub[4 * q], pub[4 * q + 1], pub[4 * q + 2], pub[4 * q + 3]);
                     }
                 }
-                tc_fence_before();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[CB_RB5]);
+                arrive(1, 4, c);
             } else if (c >= 1) {
                 // (C) outputs of the previous chunk, while this chunk's M4 runs
                 y_epilogue(c - 1);
@@ -931,10 +980,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         ok = wwait(CB_M5, (nch - 1) & 1, nch) && ok;
         tc_fence_after();
         if (ok) {
-            float d[32];
-            tmem_ld32(tmem + L::T_S + lane_base + col, d);
+            float d[32], e[32];
+            tmem_ld32x2(tmem + L::T_S + lane_base + col, tmem + L::T_S + lane_base + kNV + col, d, e);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) S[j] = fmaf(gprev, S[j], d[j]);
+            for (int j = 0; j < 32; ++j) S[j] = fmaf(gprev, S[j], d[j] + e[j]);
             const size_t o = soff + (size_t)srow * p.DV + col;
             if (p.s_final && srow < D && GUARD((long long)(o + 32) <= p.state_elems, DBG_GLOBAL_OOB, 4)) {
                 float4* dst = reinterpret_cast<float4*>(p.s_final + o);
@@ -949,6 +998,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     __syncwarp();
     __syncthreads();
     if (warp == 1) {
+        if (*abort_flag) {  // a wait gave up: let products already issued drain first
+            const long long t = clock64();
+            while (clock64() - t < 400000) {}
+        }
         tc_fence_after();
         tmem_dealloc(tmem, L::T_COLS);
     }

@@ -100,6 +100,29 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
     return __all_sync(0xffffffffu, ok);
 }
 
+// Busy-polling form of mbar_wait for latency-critical waits: test_wait never suspends the
+// thread, so the wait ends within a few cycles of the phase completing.  Same limits and result
+// as mbar_wait.
+__device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                          uint64_t limit_ns = 2000000000ull) {
+    if (mbar_test(bar, parity)) return true;
+    const long long c0 = clock64();
+    const long long limit = static_cast<long long>(limit_ns) * 2;
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 256; ++i)
+            if (mbar_test(bar, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - c0 > limit) return false;
+    }
+}
+__device__ __forceinline__ bool mbar_spin_warp(uint64_t* bar, uint32_t parity,
+                                               const volatile int* abort,
+                                               uint64_t limit_ns = 2000000000ull) {
+    const bool ok = mbar_spin(bar, parity, abort, limit_ns);
+    return __all_sync(0xffffffffu, ok);
+}
+
 // ------------------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -244,6 +267,32 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
         : "memory");
 #pragma unroll
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Two 32-column loads (a, b) with one wait: the second load does not wait for the first.
+__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, float* a, float* b) {
+    uint32_t r[32], w[32];
+    __syncwarp();
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : GDN_R8(0), GDN_R8(8), GDN_R8(16), GDN_R8(24),
+          "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7]),
+          "=r"(w[8]), "=r"(w[9]), "=r"(w[10]), "=r"(w[11]), "=r"(w[12]), "=r"(w[13]), "=r"(w[14]), "=r"(w[15]),
+          "=r"(w[16]), "=r"(w[17]), "=r"(w[18]), "=r"(w[19]), "=r"(w[20]), "=r"(w[21]), "=r"(w[22]), "=r"(w[23]),
+          "=r"(w[24]), "=r"(w[25]), "=r"(w[26]), "=r"(w[27]), "=r"(w[28]), "=r"(w[29]), "=r"(w[30]), "=r"(w[31])
+        : "r"(ta), "r"(tb)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        a[i] = __uint_as_float(r[i]);
+        b[i] = __uint_as_float(w[i]);
+    }
 }
 
 // v[0..31] -> 32 consecutive columns, completed before returning.
