@@ -43,7 +43,6 @@
 #include "sm100.cuh"
 
 namespace gdn {
-
 namespace {
 
 using namespace sm100;
@@ -119,10 +118,15 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 // ============================================================================ chunk-base scan
 // cb[n] = sum over documents m < n of ceil(len_m / 64); cb[num_seqs] = total chunk records.
+// Then, for every record g < nrec, map[g] = (first token, valid tokens) of the chunk it holds
+// ((0, 0) past the last record), so that a prep CTA finds its chunk with one load.
+constexpr int kMapSmem = 8192;  // documents whose bases are searched in shared memory
 __global__ void __launch_bounds__(1024) chunk_base_kernel(const int32_t* __restrict__ cu, int n,
-                                                           int32_t* __restrict__ cb) {
+                                                           int nrec, int32_t* __restrict__ cb,
+                                                           int2* __restrict__ map) {
     __shared__ int wsum[32];
     __shared__ int carry;
+    __shared__ int scb[kMapSmem + 1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) carry = 0;
     __syncthreads();
@@ -158,6 +162,25 @@ __global__ void __launch_bounds__(1024) chunk_base_kernel(const int32_t* __restr
         __syncthreads();
     }
     if (tid == 0) cb[n] = carry;
+    __syncthreads();
+    const bool in_smem = n <= kMapSmem;
+    if (in_smem)
+        for (int i = tid; i <= n; i += 1024) scb[i] = cb[i];
+    __syncthreads();
+    const int total = carry;
+    for (int g = tid; g < nrec; g += 1024) {
+        int2 m = make_int2(0, 0);
+        if (g < total) {
+            int lo = 0, hi = n;  // the last document whose first record is <= g
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if ((in_smem ? scb[mid] : cb[mid]) <= g) lo = mid; else hi = mid - 1;
+            }
+            const int t0 = cu[lo] + (g - (in_smem ? scb[lo] : cb[lo])) * kChunk;
+            m = make_int2(t0, min(kChunk, cu[lo + 1] - t0));
+        }
+        map[g] = m;
+    }
 }
 
 // ============================================================================ prep kernel
@@ -190,8 +213,7 @@ enum { PB_FULL = 0, PB_TMEM, PB_M1, PB_RA1, PB_M3, PB_FIN, PB_COUNT };
 struct PrepParams {
     const float* alpha;
     const float* beta;
-    const int32_t* cu_seqlens;  // varlen: document offsets; nullptr for the dense layout
-    const int32_t* cb;          // varlen: chunk-record base per document
+    const int2* map;            // varlen: (first token, valid tokens) per record; nullptr if dense
     int num_seqs, T, H;
     int nchunk_dense;           // dense: chunks per sequence
     float scale;
@@ -204,13 +226,13 @@ struct PrepParams {
     long long ab_elems;
 };
 
-constexpr int kPrepThreads = 192;
+constexpr int kPrepThreads = 320;  // warp 0 loads, warp 1 TMEM + tensor cores, 2..9 compute
 
-// Up to three CTAs share an SM (shared memory and registers allow it), but TMEM holds two
-// allocations: the third CTA's allocation waits until one of the others frees its columns.
-// Everything that needs no TMEM (the input copies, decay and norms) runs before that point.
+// Two CTAs share an SM (registers and TMEM allow two).  The TMEM allocation is made by warp 1
+// alone; everything that needs no TMEM (the input copies, decay and norms) runs before it is
+// awaited, so a CTA that must wait for columns still gets its inputs in.
 template <int D>
-__global__ void __launch_bounds__(kPrepThreads, 3)
+__global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const PrepParams p) {
     using L = PrepLayout<D>;
@@ -218,26 +240,18 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int bid = blockIdx.x;
     const int h = bid % p.H;
     const int g = bid / p.H;
-    long t0, t1;
-    int c;
-    if (p.cu_seqlens) {
-        if (g >= p.cb[p.num_seqs]) return;  // grid sized for the worst case
-        int lo = 0, hi = p.num_seqs;        // the last document whose first record is <= g
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (p.cb[mid] <= g) lo = mid; else hi = mid - 1;
-        }
-        c = g - p.cb[lo];
-        t0 = p.cu_seqlens[lo];
-        t1 = p.cu_seqlens[lo + 1];
+    long base;
+    int nvalid;
+    if (p.map) {
+        const int2 m = p.map[g];
+        if (m.y <= 0) return;  // grid sized for the worst case
+        base = m.x;
+        nvalid = m.y;
     } else {
-        const int n = g / p.nchunk_dense;
-        c = g % p.nchunk_dense;
-        t0 = (long)n * p.T;
-        t1 = t0 + p.T;
+        const int n = g / p.nchunk_dense, c = g % p.nchunk_dense;
+        base = (long)n * p.T + (long)c * kChunk;
+        nvalid = min(kChunk, p.T - c * kChunk);
     }
-    const long base = t0 + (long)c * kChunk;
-    const int nvalid = (int)min((long)kChunk, t1 - base);
     const size_t rec = (size_t)g * p.H + h;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -258,7 +272,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
 #define GUARD(cond, code, detail) GDN_GUARD(cond, p.status, code, detail)
     auto fail = [&](int bar) {
-        (void)GUARD(false, DBG_WAIT, (long)bar * 65536 + c);
+        (void)GUARD(false, DBG_WAIT, (long)bar * 65536 + g);
         *abort_flag = 1;
         record_status(p.status, GDN_ERR_TIMEOUT);
     };
@@ -343,9 +357,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------------------- prep warpgroup
-        const int t = ((warp & 3) << 5) | lane;  // 0..127 == TMEM lane
+        // ---------------------------------------------------------------- prep warps
+        // Warps 2..9: two per TMEM lane quadrant.  t is the TMEM lane (the row of the 128-row
+        // accumulators); hf selects the half of the columns this warp handles.
+        const int t = ((warp & 3) << 5) | lane;
         const int wa = t >> 5;
+        const int hf = (warp - 2) >> 2;
         const uint32_t lane_base = static_cast<uint32_t>(wa * 32) << 16;
         __nv_bfloat16* AF = reinterpret_cast<__nv_bfloat16*>(sm + L::AF);
         __nv_bfloat16* TF = reinterpret_cast<__nv_bfloat16*>(sm + L::TF);
@@ -363,7 +380,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
         // (1) decay and norms
         bool ok = wwait(PB_FULL, 0);
-        if (ok) {
+        if (ok && hf == 0) {
             if (t < 64) {
                 float gl = lg2(ab[t]);
 #pragma unroll
@@ -386,11 +403,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 sRq[r] = p.l2norm ? 1.0f / sqrtf(ss + kNormEps) : 1.0f;
             }
         }
-        named_sync(1, 128);
-        if (ok && t >= 32 && t < 64) sG[t] += sCarry[0];
-        named_sync(1, 128);
+        named_sync(1, 256);
+        if (ok && hf == 0 && t >= 32 && t < 64) sG[t] += sCarry[0];
+        named_sync(1, 256);
         const float Glast = sG[nvalid - 1];
-        if (ok) {
+        if (ok && hf == 0) {
             if (t < 64) {
                 const float G = sG[t], gam = ex2(G);
                 sGam[t] = gam;
@@ -403,7 +420,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 rs[64 + r] = p.scale * ex2(sG[r]) * sRq[r];
             }
         }
-        named_sync(1, 128);
+        named_sync(1, 256);
 
         // (2) A (rows 0-63 of M1, to shared memory) and P (rows 64-127, to the workspace)
         ok = wwait(PB_TMEM, 0) && ok;
@@ -414,51 +431,55 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // Gam_ij = 2^(G_i - G_j) for j <= i.  Within the row's own 16-token block it is computed
         // directly; for an earlier block b it is the product 2^(G_i - G_e) 2^(G_e - G_j) through
         // the block's last token e = 16 b + 15.  Both exponents are <= 0 (G does not increase),
-        // so neither factor can overflow, and the row needs 19 exponentials instead of 64.
+        // so neither factor can overflow, and a row needs 20 exponentials instead of 64.
         if (ok) {
             const int i = t & 63, blk = i >> 4;
             const bool arow = t < 64;  // rows of A (strictly lower) or of P (lower, diagonal incl.)
             const float Gi = sG[i];
             const float sc = arow ? sBeta[i] * sRk[i] : p.scale * sRq[i];
-            float rowf[3], dg[16];
+            // this warp's columns: blocks 2 hf and 2 hf + 1; the row's own block is among them
+            // when blk / 2 == hf (the same for the whole warp)
+            float rf[2], dg[16];
 #pragma unroll
-            for (int b = 0; b < 3; ++b) rowf[b] = ex2(Gi - sG[16 * b + 15]);
+            for (int k = 0; k < 2; ++k) rf[k] = ex2(Gi - sG[16 * (2 * hf + k) + 15]);
+            if ((blk >> 1) == hf) {
 #pragma unroll
-            for (int u = 0; u < 16; ++u) dg[u] = ex2(Gi - sG[16 * blk + u]);
+                for (int u = 0; u < 16; ++u) dg[u] = ex2(Gi - sG[16 * blk + u]);
+            } else {
+#pragma unroll
+                for (int u = 0; u < 16; ++u) dg[u] = 0.f;
+            }
             const int lim = arow ? i : i + 1;  // columns j < lim are kept
             uint8_t* P = p.ws_p + rec * kRecP;
+            float d[32];
+            tmem_ld32(tmem + L::T_D1 + lane_base + hf * 32, d);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float d[32];
-                tmem_ld32(tmem + L::T_D1 + lane_base + half * 32, d);
+            for (int j4 = 0; j4 < 32; j4 += 4) {
+                const int j = hf * 32 + j4, cb = j >> 4;
+                const float4 rk4 = *reinterpret_cast<const float4*>(sRk + j);
+                const float4 cf4 = *reinterpret_cast<const float4*>(sColf + j);
+                const float rk[4] = {rk4.x, rk4.y, rk4.z, rk4.w};
+                const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
 #pragma unroll
-                for (int j4 = 0; j4 < 32; j4 += 4) {
-                    const int j = half * 32 + j4, cb = j >> 4;
-                    const float4 rk4 = *reinterpret_cast<const float4*>(sRk + j);
-                    const float4 cf4 = *reinterpret_cast<const float4*>(sColf + j);
-                    const float rk[4] = {rk4.x, rk4.y, rk4.z, rk4.w};
-                    const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float f = (cb < blk) ? rowf[cb < 3 ? cb : 2] * cf[u] : dg[(j & 15) + u];
-                        d[j4 + u] = (j + u < lim) ? sc * rk[u] * d[j4 + u] * f : 0.f;
-                    }
-                }
-                if (arow) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<uint4*>(AF + i * kLd + half * 32 + 8 * q) =
-                            (q & 1) ? pack8_fma(d + 8 * q) : pack8(d + 8 * q);
-                } else {
-                    store_half_row_mixed(P, i, half * 4, d);
+                for (int u = 0; u < 4; ++u) {
+                    const float f = (cb < blk) ? rf[j4 >> 4] * cf[u] : dg[(j4 & 15) + u];
+                    d[j4 + u] = (j + u < lim) ? sc * rk[u] * d[j4 + u] * f : 0.f;
                 }
             }
+            if (arow) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4*>(AF + i * kLd + hf * 32 + 8 * q) =
+                        (q & 1) ? pack8_fma(d + 8 * q) : pack8(d + 8 * q);
+            } else {
+                store_half_row_mixed(P, i, hf * 4, d);
+            }
         }
-        named_sync(1, 128);
+        named_sync(1, 256);
 
         // (3) T = (I + A)^-1.  16x16 diagonal blocks by forward substitution (fp32), then the
         // off-diagonal blocks T_ij = -D_i sum_m A_im T_mj by diagonals on mma.sync.
-        if (ok && t < 64) {
+        if (ok && hf == 0 && t < 64) {
             const int b = t >> 4, l = t & 15;
             float x[16];
 #pragma unroll
@@ -478,13 +499,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
             for (int r = 0; r < 16; ++r) TF[(16 * b + r) * kLd + 16 * b + l] = __float2bfloat16_rn(x[r]);
         }
-        named_sync(1, 128);
+        named_sync(1, 256);
         {
             const int mrow = (lane & 7) + ((lane >> 3) & 1) * 8;  // ldmatrix row of this lane
             const int mcol = (lane >> 4) * 8;                      // ldmatrix column offset
             const int gid = lane >> 2, tig = lane & 3;
             for (int dd = 1; dd < 4; ++dd) {
-                if (ok && wa < 4 - dd) {
+                if (ok && hf == 0 && wa < 4 - dd) {
                     const int bi = wa + dd, bj = wa;
                     float cx[2][4] = {};
                     for (int m = bj; m < bi; ++m) {
@@ -515,7 +536,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     }
                     __syncwarp();
                 }
-                named_sync(1, 128);
+                named_sync(1, 256);
             }
         }
 
@@ -523,83 +544,86 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // The tile overlays A and T, so every thread first takes its T row into registers.
         {
             const int i = t & 63;
-            uint4 tr[8];
+            uint4 tr[4];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) tr[q] = *reinterpret_cast<const uint4*>(TF + i * kLd + 8 * q);
-            named_sync(1, 128);
+            for (int q = 0; q < 4; ++q) tr[q] = *reinterpret_cast<const uint4*>(TF + i * kLd + hf * 32 + 8 * q);
+            named_sync(1, 256);
             if (ok) {
+                float x[32];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float x[32];
+                for (int q = 0; q < 4; ++q) unpack8(tr[q], x + 8 * q);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) unpack8(tr[half * 4 + q], x + 8 * q);
-#pragma unroll
-                    for (int j4 = 0; j4 < 32; j4 += 4) {
-                        const int j = half * 32 + j4;
-                        if (t < 64) {
-                            const float4 f4 = *reinterpret_cast<const float4*>(sFtw + j);
-                            x[j4 + 0] = (j + 0 <= i) ? x[j4 + 0] * f4.x : 0.f;
-                            x[j4 + 1] = (j + 1 <= i) ? x[j4 + 1] * f4.y : 0.f;
-                            x[j4 + 2] = (j + 2 <= i) ? x[j4 + 2] * f4.z : 0.f;
-                            x[j4 + 3] = (j + 3 <= i) ? x[j4 + 3] * f4.w : 0.f;
-                        } else {
-                            const float4 b4 = *reinterpret_cast<const float4*>(sBeta + j);
-                            x[j4 + 0] = (j + 0 < i) ? x[j4 + 0] * b4.x : 0.f;
-                            x[j4 + 1] = (j + 1 < i) ? x[j4 + 1] * b4.y : 0.f;
-                            x[j4 + 2] = (j + 2 < i) ? x[j4 + 2] * b4.z : 0.f;
-                            x[j4 + 3] = (j + 3 < i) ? x[j4 + 3] * b4.w : 0.f;
-                        }
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const int j = hf * 32 + j4;
+                    if (t < 64) {
+                        const float4 f4 = *reinterpret_cast<const float4*>(sFtw + j);
+                        x[j4 + 0] = (j + 0 <= i) ? x[j4 + 0] * f4.x : 0.f;
+                        x[j4 + 1] = (j + 1 <= i) ? x[j4 + 1] * f4.y : 0.f;
+                        x[j4 + 2] = (j + 2 <= i) ? x[j4 + 2] * f4.z : 0.f;
+                        x[j4 + 3] = (j + 3 <= i) ? x[j4 + 3] * f4.w : 0.f;
+                    } else {
+                        const float4 b4 = *reinterpret_cast<const float4*>(sBeta + j);
+                        x[j4 + 0] = (j + 0 < i) ? x[j4 + 0] * b4.x : 0.f;
+                        x[j4 + 1] = (j + 1 < i) ? x[j4 + 1] * b4.y : 0.f;
+                        x[j4 + 2] = (j + 2 < i) ? x[j4 + 2] * b4.z : 0.f;
+                        x[j4 + 3] = (j + 3 < i) ? x[j4 + 3] * b4.w : 0.f;
                     }
-                    store_half_row_mixed(sm + L::TWN, t, half * 4, x);
                 }
+                store_half_row_mixed(sm + L::TWN, t, hf * 4, x);
             }
         }
         fence_proxy_async_smem();
-        named_sync(1, 128);
-        if (t == 0) mbar_arrive(&bars[PB_RA1]);
+        named_sync(1, 256);
+        if (t == 0 && hf == 0) mbar_arrive(&bars[PB_RA1]);
 
-        // (5) -W (lanes 0-63 of the W accumulator) and Ut = beta V + N_b V (lanes 64-127)
+        // (5) -W (lanes 0-63 of the W accumulator) and Ut = beta V + N_b V (lanes 64-127), built
+        // as the record's byte images in shared memory that the products no longer read (-W over
+        // the T_w / N_b tile, Ut over K and Q), then written out by two bulk copies
         ok = wwait(PB_M3, 0) && ok;
         tc_fence_after();
+        static_assert(L::KB * 16384 >= D * 256 && 16384 >= D * 128, "staging space");
         if (ok) {
             if (t < 64) {
-                uint8_t* wrec = p.ws_w + rec * (size_t)(D * 128);
 #pragma unroll
-                for (int b = 0; b < KB; ++b)
+                for (int b = 0; b < KB; ++b) {
+                    float w[32];
+                    tmem_ld32(tmem + L::T_D3 + lane_base + 64 * b + 32 * hf, w);
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        float w[32];
-                        tmem_ld32(tmem + L::T_D3 + lane_base + 64 * b + 32 * half, w);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) w[j] = -w[j];
-                        store_half_row_mixed(wrec + b * 8192, t, half * 4, w);
-                    }
+                    for (int j = 0; j < 32; ++j) w[j] = -w[j];
+                    store_half_row_mixed(sm + L::TWN + b * 8192, t, hf * 4, w);
+                }
             } else {
                 const int i = t - 64;
                 const bool valid = i < nvalid;
                 const float bi = sBeta[i];
-                uint8_t* urec = p.ws_u + rec * (size_t)(D * 256) + (size_t)i * 256;
+                uint8_t* urec = sm + L::KQ + (size_t)i * 256;
 #pragma unroll
-                for (int s = 0; s < KB; ++s)
+                for (int s = 0; s < KB; ++s) {
+                    float d[32], vv[32];
+                    tmem_ld32(tmem + L::T_DU + lane_base + 64 * s + 32 * hf, d);
+                    load_half_row(sm + L::V + s * 8192, i, hf * 4, vv);
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        float d[32], vv[32];
-                        tmem_ld32(tmem + L::T_DU + lane_base + 64 * s + 32 * half, d);
-                        load_half_row(sm + L::V + s * 8192, i, half * 4, vv);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float4 u;
-                            u.x = valid ? fmaf(bi, vv[4 * q + 0], d[4 * q + 0]) : 0.f;
-                            u.y = valid ? fmaf(bi, vv[4 * q + 1], d[4 * q + 1]) : 0.f;
-                            u.z = valid ? fmaf(bi, vv[4 * q + 2], d[4 * q + 2]) : 0.f;
-                            u.w = valid ? fmaf(bi, vv[4 * q + 3], d[4 * q + 3]) : 0.f;
-                            const int ch = half * 8 + q;
-                            *reinterpret_cast<float4*>(urec + s * 16384 + ((ch ^ (i & 7)) << 4)) = u;
-                        }
+                    for (int q = 0; q < 8; ++q) {
+                        float4 u;
+                        u.x = valid ? fmaf(bi, vv[4 * q + 0], d[4 * q + 0]) : 0.f;
+                        u.y = valid ? fmaf(bi, vv[4 * q + 1], d[4 * q + 1]) : 0.f;
+                        u.z = valid ? fmaf(bi, vv[4 * q + 2], d[4 * q + 2]) : 0.f;
+                        u.w = valid ? fmaf(bi, vv[4 * q + 3], d[4 * q + 3]) : 0.f;
+                        const int ch = hf * 8 + q;
+                        *reinterpret_cast<float4*>(urec + s * 16384 + ((ch ^ (i & 7)) << 4)) = u;
                     }
+                }
             }
         }
         tc_fence_before();
+        fence_proxy_async_smem();
+        named_sync(1, 256);
+        if (ok && t == 0 && hf == 0) {
+            bulk_store(p.ws_w + rec * (size_t)(D * 128), sm + L::TWN, D * 128);
+            bulk_store(p.ws_u + rec * (size_t)(D * 256), sm + L::KQ, D * 256);
+            bulk_commit();
+            bulk_wait_read();  // the CTA's shared memory must outlive the copies' reads
+        }
     }
 #undef GUARD
     __syncwarp();
@@ -1049,6 +1073,7 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st) {
     if (a.ws == nullptr || a.ws_bytes < w.total) return cudaErrorInvalidValue;
     uint8_t* ws = static_cast<uint8_t*>(a.ws);
     int32_t* cb = reinterpret_cast<int32_t*>(ws + w.off_cb);
+    int2* map = reinterpret_cast<int2*>(ws + w.off_map);
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, a.q, tokens, a.H, D) || !make_map(&mk, a.k, tokens, a.H, D) ||
         !make_map(&mv, a.v, tokens, a.H, D))
@@ -1056,10 +1081,10 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st) {
     const int nchunk_dense = (a.T + kChunk - 1) / kChunk;
     cudaError_t e;
     if (varlen) {
-        chunk_base_kernel<<<1, 1024, 0, st>>>(a.cu_seqlens, a.num_seqs, cb);
+        chunk_base_kernel<<<1, 1024, 0, st>>>(a.cu_seqlens, a.num_seqs, w.nrec_chunks, cb, map);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    PrepParams pp{a.alpha, a.beta, a.cu_seqlens, varlen ? cb : nullptr, a.num_seqs, a.T, a.H,
+    PrepParams pp{a.alpha, a.beta, varlen ? map : nullptr, a.num_seqs, a.T, a.H,
                   nchunk_dense, a.scale, a.l2norm, ws + w.off_w, ws + w.off_p, ws + w.off_u,
                   reinterpret_cast<float*>(ws + w.off_s), a.status, (long long)tokens * a.H};
     const int smem1 = PrepLayout<D>::BYTES + 1024;
@@ -1095,6 +1120,8 @@ PrefillWorkspace prefill_workspace(int num_seqs, int T, int H, int d, bool varle
     size_t off = 0;
     w.off_cb = off;
     off += up(varlen ? ((size_t)num_seqs + 1) * 4 : 0);
+    w.off_map = off;
+    off += up(varlen ? (size_t)nrec * 8 : 0);
     w.off_w = off;
     off += up(R * (size_t)d * 128);
     w.off_p = off;

@@ -59,7 +59,9 @@ def test_workspace_bytes(lib):
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL_VARLEN, 1, 32768, 16, 128, 128, 4,
                                    ctypes.byref(n)) == 0
     nrec = (32768 + 63 * 4) // 64  # bound on sum(ceil(len / 64)) over the documents
-    assert n.value == 256 + nrec * 16 * rec(128)
+    up = lambda x: (x + 255) // 256 * 256
+    # + the document chunk bases and one (first token, length) pair per record
+    assert n.value == 256 + up(nrec * 8) + nrec * 16 * rec(128)
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_DECODE, 4, 1, 2, 128, 128, 0,
                                    ctypes.byref(n)) == 0
     assert n.value == 0
