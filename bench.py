@@ -33,7 +33,9 @@ METRIC = "GDN prefill tokens/s & % bf16 tensor peak; decode-step state GB/s vs H
 H, D = 16, 128
 T_TOTAL, NDOCS = 32768, 4
 DEC_N = 256
-FLOP_PER_TOKEN_HEAD = 180224        # dense chunk-64 tile FLOPs at dk = dv = 128
+FLOP_PER_TOKEN_HEAD = 180224        # dense chunk-64 tile FLOPs at dk = dv = 128, of which
+PREP_FLOP_PER_TOKEN_HEAD = 65536     # chunk-parallel: K K^T, Q K^T, W, Ut (8 C d)
+CHAIN_FLOP_PER_TOKEN_HEAD = 114688   # sequential: W S, Q S, K^T U (6 d^2), masked (Q K^T) U (2 C d)
 BYTES_PER_TOKEN_HEAD = 1032         # q,k,v,y bf16 (4 x 256) + alpha, beta fp32
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -48,15 +50,15 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def profile_traffic(name, source):
-    """Per-launch DRAM bytes recorded by an ncu capture in profiles/<name>; None when the summary
-    is missing or was taken on a different version of the kernel source."""
+def profile_traffic(name, source, key="dram_bytes_per_launch"):
+    """Per-launch DRAM bytes recorded by an ncu capture in profiles/<name> (the line `<key>: N`);
+    None when the summary is missing or was taken on a different version of the kernel source."""
     path = os.path.join(ROOT, "profiles", name)
     try:
         txt = open(path).read()
     except OSError:
         return None
-    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    m = re.search(r"(?m)^" + re.escape(key) + r":\s*([0-9.eE+]+)", txt)
     h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", txt)
     if not m or not h:
         return None
@@ -146,9 +148,19 @@ def run_ours(args, rank, world, local_rank):
     ws = torch.empty(api.gdn_workspace_bytes(GDN_OP_PREFILL_VARLEN, 1, T_TOTAL, H, D, D, NDOCS),
                      dtype=torch.uint8, device=dev)
 
+    # one step = one gdn_prefill_varlen, issued as its two phases (the same kernels) so that
+    # each phase's device time is measured on its own
+    def prepare():
+        api.gdn_prefill_varlen_prepare(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                       g["cu_seqlens"], ws)
+
+    def finish():
+        api.gdn_prefill_varlen_finish(g["q"], g["k"], g["cu_seqlens"], ws, s0=g["s0"], y=y,
+                                      s_final=sf)
+
     def step():
-        api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["cu_seqlens"],
-                               g["s0"], y=y, s_final=sf, ws=ws)
+        prepare()
+        finish()
 
     def barrier():
         if world > 1:
@@ -164,16 +176,21 @@ def run_ours(args, rank, world, local_rank):
         barrier()
         torch.cuda.synchronize()
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         with ClockSampler(uuid) as clk:
             for i in range(args.steps):
                 starts[i].record()
-                step()
+                prepare()
+                mids[i].record()
+                finish()
                 ends[i].record()
             torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
         per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        prep_ms = max_over_ranks(statistics.mean(s.elapsed_time(m) for s, m in zip(starts, mids)))
+        chain_ms = max_over_ranks(statistics.mean(m.elapsed_time(e) for m, e in zip(mids, ends)))
         total_ms = max_over_ranks(starts[0].elapsed_time(ends[-1]))
         kern_ms = max_over_ranks(statistics.mean(per))
         assert api.gdn_read_device_status() == 0, "device status word set during the bench"
@@ -184,20 +201,30 @@ def run_ours(args, rank, world, local_rank):
         hbm_bytes = BYTES_PER_TOKEN_HEAD * tokens * H + state_bytes
         ms_per_step = total_ms / args.steps
         value = world * tokens / (ms_per_step / 1e3)
-        tflops = flops / (kern_ms / 1e3) / 1e12
         gbs = hbm_bytes / (kern_ms / 1e3) / 1e9
-        traffic = profile_traffic("prefill_varlen_T32768.md",
-                                  "gated_deltanet_linear_eqs_b200/csrc/prefill.cu")
+        src = "gated_deltanet_linear_eqs_b200/csrc/prefill.cu"
+        phases = {}
+        for name, ms, fl in (("prep", prep_ms, PREP_FLOP_PER_TOKEN_HEAD),
+                             ("chain", chain_ms, CHAIN_FLOP_PER_TOKEN_HEAD)):
+            f = fl * tokens * H
+            tf = f / (ms / 1e3) / 1e12
+            phases[name] = {"ms": ms, "flops_per_launch": f, "tflops": tf,
+                            "frac": tf / peaks["bf16_tflops"],
+                            "traffic": profile_traffic("prefill_varlen_T32768.md", src,
+                                                       key=f"{name}_dram_bytes_per_launch")}
+        dom = max(phases, key=lambda n: phases[n]["ms"])  # the dominant kernel
+        d = phases[dom]
         out["prefill"] = dict(
             value=value, ms_per_step=ms_per_step, kern_ms=kern_ms, clocks=clk.summary(),
-            roofline={"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
-                      "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
-                      "traffic": traffic, "peak_source": peak_src + " bf16 burst",
-                      "flops_per_launch": flops},
+            roofline={"bound": "tensor", "kernel": f"{dom}_kernel", "achieved": d["tflops"],
+                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": d["frac"],
+                      "traffic": d["traffic"], "peak_source": peak_src + " bf16 burst",
+                      "flops_per_launch": d["flops_per_launch"], "launch_ms": d["ms"]},
+            kernels=phases,
+            step_tflops=flops / (kern_ms / 1e3) / 1e12,
             roofline_hbm={"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                           "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-                          "bytes_per_launch": hbm_bytes, "peak_source": peak_src},
-            frac_bf16_sustained=tflops / peaks["bf16_tflops_sustained"])
+                          "bytes_per_launch": hbm_bytes, "peak_source": peak_src})
 
         # end to end through the public API with host buffers: H2D of the step's inputs from
         # pinned memory, the call, D2H of the outputs, all inside the timed region
@@ -493,7 +520,7 @@ def main():
                             "parallelism": f"dp{world} (independent streams, no collective)",
                             "l2": "inputs (403 MB) exceed the 126 MB L2; no flush"},
                     roofline=p["roofline"], roofline_hbm=p["roofline_hbm"],
-                    frac_bf16_sustained=p["frac_bf16_sustained"], kernel_ms=p["kern_ms"],
+                    kernels=p["kernels"], step_tflops=p["step_tflops"], kernel_ms=p["kern_ms"],
                     clocks=p["clocks"], e2e=res["e2e"], gpu_launches=3 * args.steps)
     if "train" in res:
         line["train"] = res["train"]

@@ -45,6 +45,10 @@ SIGNATURES = {
                          _S, _P]),
     "gdn_prefill_varlen": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _F,
                                 _I, _P, _S, _P]),
+    "gdn_prefill_varlen_prepare": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I,
+                                        _P, _S, _P]),
+    "gdn_prefill_varlen_finish": (_I, [_P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _S,
+                                       _P]),
     "gdn_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gdn_backward": (_I, [_P] * 14 + [_I] * 6 + [_F, _I, _P, _S, _P]),
     "gdn_backward_noalloc": (_I, [_P] * 14 + [_I] * 6 + [_F, _I, _P]),

@@ -129,6 +129,54 @@ def gdn_prefill_varlen(q, k, v, alpha, beta, cu_seqlens, s0=None, scale=1.0, l2n
     return y, s_final
 
 
+def gdn_prefill_varlen_prepare(q, k, v, alpha, beta, cu_seqlens, ws, scale=1.0,
+                               l2norm_qk=True, stream=None):
+    """First phase of gdn_prefill_varlen (bf16): the state-independent chunk work, into ``ws``
+    (a uint8 device tensor of gdn_workspace_bytes(GDN_OP_PREFILL_VARLEN, ...) bytes)."""
+    if q.dim() == 3:
+        q, k, v, alpha, beta = (x.unsqueeze(0) for x in (q, k, v, alpha, beta))
+    _, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    _need(q, "q", torch.bfloat16)
+    _need(k, "k", torch.bfloat16, q.shape)
+    _need(v, "v", torch.bfloat16, (1, T, H, dv))
+    _need(alpha, "alpha", torch.float32, (1, T, H))
+    _need(beta, "beta", torch.float32, (1, T, H))
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,))
+    rc = _lib().gdn_prefill_varlen_prepare(_p(q), _p(k), _p(v), _p(alpha), _p(beta),
+                                           _p(cu_seqlens), N, T, H, dk, dv, _DT[torch.bfloat16],
+                                           float(scale), int(bool(l2norm_qk)), _p(ws),
+                                           ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "gdn_prefill_varlen_prepare")
+
+
+def gdn_prefill_varlen_finish(q, k, cu_seqlens, ws, s0=None, y=None, s_final=None, dv=None,
+                              stream=None):
+    """Second phase of gdn_prefill_varlen (bf16): the sequential chunk pass from s0 over the
+    records gdn_prefill_varlen_prepare wrote into ``ws``.  Returns (y, s_final)."""
+    if q.dim() == 3:
+        q, k = q.unsqueeze(0), k.unsqueeze(0)
+    _, T, H, dk = q.shape
+    dv = dk if dv is None else dv
+    N = cu_seqlens.numel() - 1
+    _need(q, "q", torch.bfloat16)
+    _need(k, "k", torch.bfloat16, q.shape)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,))
+    _need(s0, "s0", torch.float32, (N, H, dk, dv), optional=True)
+    if y is None:
+        y = torch.empty((1, T, H, dv), dtype=torch.bfloat16, device=q.device)
+    _need(y, "y", torch.bfloat16, (1, T, H, dv))
+    if s_final is None:
+        s_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(s_final, "s_final", torch.float32, (N, H, dk, dv))
+    rc = _lib().gdn_prefill_varlen_finish(_p(q), _p(k), _p(cu_seqlens), N, _p(s0), _p(y),
+                                          _p(s_final), T, H, dk, dv, _DT[torch.bfloat16], _p(ws),
+                                          ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "gdn_prefill_varlen_finish")
+    return y, s_final
+
+
 def gdn_decode_step(q, k, v, alpha, beta, state, scale=1.0, l2norm_qk=True, y=None,
                     stream=None):
     """q,k [N,H,dk], v [N,H,dv], alpha,beta [N,H], state [N,H,dk,dv] fp32 (updated in

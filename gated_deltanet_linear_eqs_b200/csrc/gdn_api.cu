@@ -150,6 +150,44 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
     return map_cuda(gdn::launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 
+int gdn_prefill_varlen_prepare(const void* q, const void* k, const void* v, const float* alpha,
+                               const float* beta, const int32_t* cu_seqlens, int num_seqs, int T,
+                               int H, int dk, int dv, int dtype, float scale, int l2norm_qk,
+                               void* ws, size_t ws_bytes, void* stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
+        cu_seqlens == nullptr)
+        return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 1 || T < 1 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (int rc = check_dims(dk, dv, dtype)) return rc;
+    if (dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn::prefill_workspace(num_seqs, T, H, dk, true).total;
+    if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return GDN_ERR_WORKSPACE;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::PrefillArgs a{q, k, v, alpha, beta, nullptr, nullptr, nullptr, cu_seqlens, num_seqs,
+                       T, H, dk, dv, dtype, scale, l2norm_qk ? 1 : 0, dev.status, ws, ws_bytes};
+    return map_cuda(gdn::launch_prefill_phase(a, 0, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_prefill_varlen_finish(const void* q, const void* k, const int32_t* cu_seqlens,
+                              int num_seqs, const float* s0, void* y, float* s_final, int T,
+                              int H, int dk, int dv, int dtype, void* ws, size_t ws_bytes,
+                              void* stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(y) || cu_seqlens == nullptr || !ok_opt_ptr(s0) ||
+        !ok_opt_ptr(s_final))
+        return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 1 || T < 1 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (int rc = check_dims(dk, dv, dtype)) return rc;
+    if (dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn::prefill_workspace(num_seqs, T, H, dk, true).total;
+    if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return GDN_ERR_WORKSPACE;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::PrefillArgs a{q, k, nullptr, nullptr, nullptr, s0, y, s_final, cu_seqlens, num_seqs,
+                       T, H, dk, dv, dtype, 1.0f, 1, dev.status, ws, ws_bytes};
+    return map_cuda(gdn::launch_prefill_phase(a, 1, static_cast<cudaStream_t>(stream)));
+}
+
 int gdn_decode_step(const void* q, const void* k, const void* v, const float* alpha,
                     const float* beta, float* state, void* y, int N, int H, int dk, int dv,
                     int dtype, float scale, int l2norm_qk, void* stream) {

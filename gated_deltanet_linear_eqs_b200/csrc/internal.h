@@ -60,6 +60,9 @@ struct BackwardArgs {
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st);
+// One phase of the bf16 prefill: 0 = state-independent part (chunk map + prep kernel),
+// 1 = sequential part (chain kernel).  launch_prefill runs both.
+cudaError_t launch_prefill_phase(const PrefillArgs& a, int phase, cudaStream_t st);
 // Token-by-token prefill on CUDA cores (used for fp32 inputs).
 cudaError_t launch_prefill_seq(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st);

@@ -1065,8 +1065,16 @@ bool make_map(CUtensorMap* m, const void* base, long tokens, int H, int d) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor maps of the [tokens, H, d] bf16 token tensors; nullptr arguments are skipped.
+bool make_maps(const PrefillArgs& a, int D, CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv) {
+    const long tokens = a.cu_seqlens ? (long)a.T : (long)a.num_seqs * a.T;
+    return (!mq || make_map(mq, a.q, tokens, a.H, D)) && (!mk || make_map(mk, a.k, tokens, a.H, D)) &&
+           (!mv || make_map(mv, a.v, tokens, a.H, D));
+}
+
+// The state-independent phase: chunk map (packed documents) and the prep kernel.
 template <int D>
-cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st) {
+cudaError_t launch_prep(const PrefillArgs& a, cudaStream_t st) {
     const bool varlen = a.cu_seqlens != nullptr;
     const long tokens = varlen ? (long)a.T : (long)a.num_seqs * a.T;
     const PrefillWorkspace w = prefill_workspace(a.num_seqs, a.T, a.H, D, varlen);
@@ -1075,9 +1083,7 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st) {
     int32_t* cb = reinterpret_cast<int32_t*>(ws + w.off_cb);
     int2* map = reinterpret_cast<int2*>(ws + w.off_map);
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, a.q, tokens, a.H, D) || !make_map(&mk, a.k, tokens, a.H, D) ||
-        !make_map(&mv, a.v, tokens, a.H, D))
-        return cudaErrorInvalidValue;
+    if (!make_maps(a, D, &mq, &mk, &mv)) return cudaErrorInvalidValue;
     const int nchunk_dense = (a.T + kChunk - 1) / kChunk;
     cudaError_t e;
     if (varlen) {
@@ -1092,14 +1098,28 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st) {
                                   smem1)) != cudaSuccess)
         return e;
     prep_kernel<D><<<(unsigned)((size_t)w.nrec_chunks * a.H), kPrepThreads, smem1, st>>>(mq, mk, mv, pp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return cudaGetLastError();
+}
 
+// The sequential phase: the chain kernel over the workspace records.
+template <int D>
+cudaError_t launch_chain(const PrefillArgs& a, cudaStream_t st) {
+    const bool varlen = a.cu_seqlens != nullptr;
+    const long tokens = varlen ? (long)a.T : (long)a.num_seqs * a.T;
+    const PrefillWorkspace w = prefill_workspace(a.num_seqs, a.T, a.H, D, varlen);
+    if (a.ws == nullptr || a.ws_bytes < w.total) return cudaErrorInvalidValue;
+    uint8_t* ws = static_cast<uint8_t*>(a.ws);
+    int32_t* cb = reinterpret_cast<int32_t*>(ws + w.off_cb);
+    CUtensorMap mq, mk;
+    if (!make_maps(a, D, &mq, &mk, nullptr)) return cudaErrorInvalidValue;
+    const int nchunk_dense = (a.T + kChunk - 1) / kChunk;
     ChainParams cp{a.s0, static_cast<__nv_bfloat16*>(a.y), a.s_final, a.cu_seqlens,
                    varlen ? cb : nullptr, a.num_seqs, a.T, a.H, a.dv, nchunk_dense,
                    w.nrec_chunks, ws + w.off_w, ws + w.off_p, ws + w.off_u,
                    reinterpret_cast<const float*>(ws + w.off_s), a.status,
                    (long long)tokens * a.H * a.dv, (long long)a.num_seqs * a.H * a.dk * a.dv};
     const int smem2 = ChainLayout<D>::BYTES + 1024;
+    cudaError_t e;
     if ((e = cudaFuncSetAttribute(chain_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   smem2)) != cudaSuccess)
         return e;
@@ -1137,7 +1157,14 @@ PrefillWorkspace prefill_workspace(int num_seqs, int T, int H, int d, bool varle
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st) {
     // bf16 inputs run the tensor-core kernels; fp32 inputs the exact-fp32 token loop.
     if (a.dtype != GDN_BF16) return launch_prefill_seq(a, st);
-    return a.dk == 128 ? launch_d<128>(a, st) : launch_d<64>(a, st);
+    cudaError_t e = launch_prefill_phase(a, 0, st);
+    return e != cudaSuccess ? e : launch_prefill_phase(a, 1, st);
+}
+
+cudaError_t launch_prefill_phase(const PrefillArgs& a, int phase, cudaStream_t st) {
+    if (a.dtype != GDN_BF16) return cudaErrorInvalidValue;
+    if (phase == 0) return a.dk == 128 ? launch_prep<128>(a, st) : launch_prep<64>(a, st);
+    return a.dk == 128 ? launch_chain<128>(a, st) : launch_chain<64>(a, st);
 }
 
 }  // namespace gdn

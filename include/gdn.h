@@ -83,7 +83,9 @@ int gdn_workspace_bytes(int op, int B, int T, int H, int dk, int dv, int num_seq
  * gdn_prefill -- chunked (64-token chunks) forward over B independent sequences
  * of T tokens: writes y and, if s_final is non-NULL, the state after the last
  * token.  s0 == NULL means S_0 = 0.  The computation is exactly eqs. (1)-(4)
- * above, rearranged chunk-wise (WY/UT form), on the tensor cores.
+ * above, rearranged chunk-wise (WY/UT form), on the tensor cores.  bf16 inputs
+ * need the workspace (gdn_workspace_bytes); the fp32 path (a token loop) uses
+ * none and accepts ws == NULL.
  *   q, k  [B,T,H,dk]  dtype        v [B,T,H,dv] dtype
  *   alpha, beta [B,T,H] fp32       s0 [B,H,dk,dv] fp32 or NULL
  *   y [B,T,H,dv] dtype (output)    s_final [B,H,dk,dv] fp32 or NULL (output)
@@ -110,6 +112,30 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
                        int dtype, float scale, int l2norm_qk, void* ws, size_t ws_bytes,
                        void* stream);
 
+/*
+ * gdn_prefill_varlen_prepare / gdn_prefill_varlen_finish -- gdn_prefill_varlen (bf16) in two
+ * calls.  The chunked form splits into a part that depends on the chunk alone (decay, norms,
+ * the 64x64 triangular inverse and the W / U~ / P operands of every chunk of every document,
+ * all computed at once) and a sequential part that walks the chunks from s0 (same page,
+ * eqs. (1)-(4), chunk-wise).  prepare runs the first part into the workspace; finish runs the
+ * second and writes y and s_final.  The pair computes exactly what one gdn_prefill_varlen call
+ * does (which is these two phases back to back); prepare needs no initial state, so it may run
+ * before s0 is known.
+ *   - finish must get the same q, k, cu_seqlens, num_seqs, T, H, dk, dv and workspace as the
+ *     prepare call whose records it reads, be ordered after it (same stream, or an event), and
+ *     nothing may write the workspace in between.  scale and l2norm_qk are applied by prepare.
+ *   - dtype must be GDN_BF16 (the fp32 path has no split; use gdn_prefill_varlen).
+ *   - ws/ws_bytes: gdn_workspace_bytes(GDN_OP_PREFILL_VARLEN, ...).  Errors and validation as
+ *     for gdn_prefill_varlen; a non-bf16 dtype is GDN_ERR_INVALID_ARG.
+ */
+int gdn_prefill_varlen_prepare(const void* q, const void* k, const void* v, const float* alpha,
+                               const float* beta, const int32_t* cu_seqlens, int num_seqs, int T,
+                               int H, int dk, int dv, int dtype, float scale, int l2norm_qk,
+                               void* ws, size_t ws_bytes, void* stream);
+int gdn_prefill_varlen_finish(const void* q, const void* k, const int32_t* cu_seqlens,
+                              int num_seqs, const float* s0, void* y, float* s_final, int T,
+                              int H, int dk, int dv, int dtype, void* ws, size_t ws_bytes,
+                              void* stream);
 /*
  * gdn_decode_step -- one new token for each of N independent sequences
  * (eqs. (1)-(4) with T = 1).  The state is read once and written once, in place.

@@ -115,6 +115,27 @@ def test_bf16_prefill_needs_its_workspace(lib):
     assert _prefill(lib, ws=A + 8, wsb=1 << 30) == _abi.GDN_ERR_WORKSPACE  # misaligned
 
 
+def test_split_phase_validation(lib):
+    prep = lambda **kw: lib.gdn_prefill_varlen_prepare(
+        *[kw.get(n, A) for n in ("q", "k", "v", "al", "be", "cu")], kw.get("n", 2),
+        kw.get("T", 100), 2, kw.get("dk", 64), kw.get("dv", 64), kw.get("dt", 0), 1.0, 1,
+        kw.get("ws", A), kw.get("wsb", 1 << 30), None)
+    fin = lambda **kw: lib.gdn_prefill_varlen_finish(
+        kw.get("q", A), kw.get("k", A), kw.get("cu", A), kw.get("n", 2), kw.get("s0", 0),
+        kw.get("y", A), kw.get("sf", 0), kw.get("T", 100), 2, kw.get("dk", 64), kw.get("dv", 64),
+        kw.get("dt", 0), kw.get("ws", A), kw.get("wsb", 1 << 30), None)
+    for f in (prep, fin):
+        assert f(q=0) == _abi.GDN_ERR_INVALID_ARG
+        assert f(cu=0) == _abi.GDN_ERR_INVALID_ARG
+        assert f(n=0) == _abi.GDN_ERR_INVALID_ARG
+        assert f(dt=1) == _abi.GDN_ERR_INVALID_ARG          # fp32 has no split
+        assert f(dk=96, dv=96) == _abi.GDN_ERR_UNSUPPORTED_SHAPE
+        assert f(ws=0) == _abi.GDN_ERR_WORKSPACE
+        assert f(wsb=16) == _abi.GDN_ERR_WORKSPACE
+    assert fin(y=0) == _abi.GDN_ERR_INVALID_ARG
+    assert fin(s0=A + 4) == _abi.GDN_ERR_INVALID_ARG
+
+
 def test_varlen_rejects_bad_arguments(lib):
     f = lib.gdn_prefill_varlen
     ok = dict(q=A, k=A, v=A, al=A, be=A, cu=A, n=2, s0=0, y=A, sf=A, T=100, H=2, dk=64, dv=64,

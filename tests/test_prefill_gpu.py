@@ -7,6 +7,7 @@ import torch
 
 import oracle
 from gated_deltanet_linear_eqs_b200 import api
+from gated_deltanet_linear_eqs_b200._abi import GDN_OP_PREFILL_VARLEN
 from gated_deltanet_linear_eqs_b200.inputs import (make_inputs, make_varlen_inputs,
                                                    varlen_lengths)
 from tests._metrics import S_TOL, Y_TOL, frob_rel, max_rel
@@ -169,4 +170,32 @@ def test_prefill_matches_decode_steps():
 def test_prefill_device_status_clean():
     inp = make_inputs(1, 128, 2, 128, 128, seed=1)
     _run_dense(inp)
+    assert api.gdn_read_device_status(reset=True) == 0
+
+
+def test_prefill_split_phases():
+    """prepare + finish equals one gdn_prefill_varlen call bit for bit, and the prepared records
+    serve any initial state: a second finish from S0 = 0 matches the oracle from S0 = 0."""
+    lengths = [100, 0, 300, 64]
+    H, d = 2, 128
+    inp = make_varlen_inputs(lengths, H, d, d, seed=77)
+    g = _cuda(inp)
+    T, N = int(inp["cu_seqlens"][-1]), len(lengths)
+    y1, s1 = api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                    g["cu_seqlens"], g["s0"], scale=0.7)
+    ws = torch.empty(api.gdn_workspace_bytes(GDN_OP_PREFILL_VARLEN, 1, T, H, d, d, N),
+                     dtype=torch.uint8, device="cuda")
+    api.gdn_prefill_varlen_prepare(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                   g["cu_seqlens"], ws, scale=0.7)
+    y2, s2 = api.gdn_prefill_varlen_finish(g["q"], g["k"], g["cu_seqlens"], ws, s0=g["s0"])
+    y3, s3 = api.gdn_prefill_varlen_finish(g["q"], g["k"], g["cu_seqlens"], ws, s0=None)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(s1, s2)
+    cu = inp["cu_seqlens"].numpy()
+    yr, sr = oracle.forward_varlen(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], cu,
+                                   inp["s0"], scale=0.7)
+    assert max_rel(y2, yr) <= Y_TOL and frob_rel(s2, sr) <= S_TOL
+    yr0, sr0 = oracle.forward_varlen(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], cu,
+                                     None, scale=0.7)
+    assert max_rel(y3, yr0) <= Y_TOL and frob_rel(s3, sr0) <= S_TOL
     assert api.gdn_read_device_status(reset=True) == 0
