@@ -216,6 +216,8 @@ struct PrepParams {
     const int2* map;            // varlen: (first token, valid tokens) per record; nullptr if dense
     int num_seqs, T, H;
     int nchunk_dense;           // dense: chunks per sequence
+    int ntask;                  // CTAs of the grid: chunk records x heads
+    int ahead;                  // CTA index distance of the L2 prefetch (two CTAs per SM)
     float scale;
     int l2norm;
     uint8_t* ws_w;
@@ -308,6 +310,27 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         __syncwarp();
         if (lane != 0) mbar_arrive(&bars[PB_FULL]);
+        // Warm L2 with the tiles of the CTA that will most likely run next on this SM (CTAs are
+        // dispatched in index order as slots free up), so that its loads do not wait on DRAM.
+        const int nt = bid + p.ahead;
+        if (lane == 0 && nt < p.ntask) {
+            const int g2 = nt / p.H, h2 = nt % p.H;
+            int z2 = -1;
+            if (p.map) {
+                const int2 m = p.map[g2];
+                if (m.y > 0) z2 = m.x;
+            } else {
+                z2 = (g2 / p.nchunk_dense) * p.T + (g2 % p.nchunk_dense) * kChunk;
+            }
+            if (z2 >= 0) {
+#pragma unroll
+                for (int b = 0; b < KB; ++b) {
+                    tma_prefetch_3d(&tm_k, 64 * b, h2, z2);
+                    tma_prefetch_3d(&tm_q, 64 * b, h2, z2);
+                    tma_prefetch_3d(&tm_v, 64 * b, h2, z2);
+                }
+            }
+        }
         // do not leave while the copies are still writing shared memory
         mbar_wait_warp(&bars[PB_FULL], 0, never, 100000000ull);
     } else if (warp == 1) {
@@ -1090,14 +1113,20 @@ cudaError_t launch_prep(const PrefillArgs& a, cudaStream_t st) {
         chunk_base_kernel<<<1, 1024, 0, st>>>(a.cu_seqlens, a.num_seqs, w.nrec_chunks, cb, map);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    int dev = 0, nsm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    const int ntask = w.nrec_chunks * a.H;
     PrepParams pp{a.alpha, a.beta, varlen ? map : nullptr, a.num_seqs, a.T, a.H,
-                  nchunk_dense, a.scale, a.l2norm, ws + w.off_w, ws + w.off_p, ws + w.off_u,
-                  reinterpret_cast<float*>(ws + w.off_s), a.status, (long long)tokens * a.H};
+                  nchunk_dense, ntask, 2 * nsm, a.scale, a.l2norm, ws + w.off_w, ws + w.off_p,
+                  ws + w.off_u, reinterpret_cast<float*>(ws + w.off_s), a.status,
+                  (long long)tokens * a.H};
     const int smem1 = PrepLayout<D>::BYTES + 1024;
     if ((e = cudaFuncSetAttribute(prep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   smem1)) != cudaSuccess)
         return e;
-    prep_kernel<D><<<(unsigned)((size_t)w.nrec_chunks * a.H), kPrepThreads, smem1, st>>>(mq, mk, mv, pp);
+    prep_kernel<D><<<(unsigned)ntask, kPrepThreads, smem1, st>>>(mq, mk, mv, pp);
     return cudaGetLastError();
 }
 
