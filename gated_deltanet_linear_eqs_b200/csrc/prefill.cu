@@ -49,7 +49,7 @@ using namespace sm100;
 
 constexpr int kChunk = 64;
 constexpr int kLd = 72;  // bf16 row stride (elements) of the A / T scratch: 144-byte rows
-constexpr int kNV = 64;  // dv columns per chain CTA
+constexpr int kNV = 32;  // dv columns per chain CTA (operand tiles stay 64 columns wide)
 constexpr uint32_t kRecP = 8192;
 constexpr uint32_t kRecS = 1024;
 
@@ -664,20 +664,21 @@ struct ChainLayout {
     static constexpr int KQW_BLOCK = 192 * 128;   // per dk block: K rows 0-63, Q 64-127, -W 128-191
     static constexpr int KQW = KB * KQW_BLOCK;
     static constexpr int P = KQW;                 // P, 64 rows (read as 128 rows: then U)
-    static constexpr int U = P + 8192;            // Ut slice: fp32, 64 rows x 256 B
+    static constexpr int U = P + 8192;            // Ut image of the 64-column slice: fp32, 64 x 256 B
     static constexpr int SC = U + 16384;          // record scalars
     static constexpr int STAGE = SC + 1024;
-    static constexpr int SB = 2 * STAGE;          // S in bf16: D rows x 64 columns
-    static constexpr int UHI = SB + D * 128;
-    static constexpr int ULO = UHI + 8192;
-    static constexpr int UB = ULO + 8192;
+    // The CTA's 32 state columns use the first half of 64-column operand tiles; an N = 64 MMA
+    // costs the tensor core what an N = 32 one does.
+    static constexpr int SB = 2 * STAGE;          // S in bf16: D rows x 64 columns (0-31 used)
+    static constexpr int UHL = SB + D * 128;      // [U'_hi (columns 0-31) | U'_lo (32-63)], 64 rows
+    static constexpr int UB = UHL + 8192;         // U in bf16, 64 rows (columns 0-31 used)
     static constexpr int BAR = UB + 8192;
     static constexpr int MISC = BAR + 16 * 8;     // tmem base, abort flag, zero word, 2 counters
     static constexpr int BYTES = MISC + 32;
     static constexpr int TX = KB * 16384 + KB * 8192 + 8192 + 16384 + 1024;
-    static constexpr uint32_t T_S = 0;            // [K^T U'_hi | K^T U'_lo] of the chunk, 128 columns
-    static constexpr uint32_t T_D4 = 128;         // [Q S ; -W S], 2 x 64 columns
-    static constexpr uint32_t T_D6 = 256;         // P U, 2 x 64 columns
+    static constexpr uint32_t T_S = 0;            // [K^T U'_hi | K^T U'_lo] of the chunk, 64 columns
+    static constexpr uint32_t T_D4 = 64;          // [Q S ; -W S], 2 x 64 columns (0-31 used)
+    static constexpr uint32_t T_D6 = 192;         // P U, 2 x 64 columns (0-31 used)
     static constexpr uint32_t T_COLS = 512;
     static_assert(STAGE % 1024 == 0, "stage tiles stay 1024-byte aligned");
     static_assert(BYTES + 1024 <= 232448 - 1024, "shared memory budget");
@@ -707,9 +708,10 @@ struct ChainParams {
 constexpr int kChainThreads = 384;
 
 // Warp roles: 0 loads (TMA for K and Q, bulk copies for the workspace record), 1 owns the TMEM
-// allocation, 4..11 are the epilogue warps.  Epilogue warp w reads TMEM lanes 32 (w % 4) .. +31
-// and columns 32 ((w - 4) / 4) .. +31; lanes 0-63 carry the output rows (Y) and lanes 64-127 the
-// pseudo-value rows (U); all eight hold a 32-column strip of S.  There is no separate MMA warp:
+// allocation and issues the output product, 4..11 are the epilogue warps.  Epilogue warp w reads
+// TMEM lanes 32 (w % 4) .. +31 and columns 16 ((w - 4) / 4) .. +15 of the CTA's 32; lanes 0-63
+// carry the output rows (Y) and lanes 64-127 the pseudo-value rows (U); all eight hold a
+// 16-column strip of S.  There is no separate MMA warp:
 // the last epilogue warp to finish a step (found with a shared-memory arrival counter) issues the
 // tensor-core products that depend on it, which saves a wake-up on the sequential path.
 template <int D>
@@ -816,7 +818,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     bulk_load(st + b * L::KQW_BLOCK + 16384, p.ws_w + rec * kRecW + b * 8192, 8192, full);
                 }
                 bulk_load(st + L::P, p.ws_p + rec * kRecP, kRecP, full);
-                bulk_load(st + L::U, p.ws_u + rec * kRecU + (size_t)jsl * 16384, 16384, full);
+                bulk_load(st + L::U, p.ws_u + rec * kRecU + (size_t)(jsl >> 1) * 16384, 16384, full);
                 bulk_load(st + L::SC, p.ws_s + rec * (kRecS / 4), kRecS, full);
                 if (c + 2 < nch) {  // warm L2 for the chunk that will reuse this stage
                     const size_t rec2 = rec + 2 * (size_t)p.H;
@@ -827,7 +829,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     }
                     bulk_prefetch_l2(p.ws_w + rec2 * kRecW, kRecW);
                     bulk_prefetch_l2(p.ws_p + rec2 * kRecP, kRecP);
-                    bulk_prefetch_l2(p.ws_u + rec2 * kRecU + (size_t)jsl * 16384, 16384);
+                    bulk_prefetch_l2(p.ws_u + rec2 * kRecU + (size_t)(jsl >> 1) * 16384, 16384);
                     bulk_prefetch_l2(p.ws_s + rec2 * (kRecS / 4), kRecS);
                 }
                 ++issued;
@@ -843,7 +845,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     } else if (warp == 1) {
         // ---------------------------------------------------------------- output product M6
         if (lane == 0) {
-            constexpr uint32_t ID_KN = idesc_bf16(128, kNV, false, true);
+            constexpr uint32_t ID_KN = idesc_bf16(128, 64, false, true);  // U_bf16 tile is 64 wide
             constexpr uint64_t KS = 32 >> 4, MS = 2048 >> 4;
             const uint64_t dUB = sdesc(smem_u32(sm + L::UB), 8192, 1024);
             for (int c = 0; c < nch; ++c) {
@@ -868,26 +870,33 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const int qd = warp & 3, hf = (warp - 4) >> 2;
         const int srow = qd * 32 + lane;               // TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
-        const uint32_t col = 32 * hf;
+        const uint32_t col = 16 * hf;
         const bool uwarp = qd >= 2;                    // U rows; the others write Y
-        float S[32];
+        float S[16];
         {
             // D = 64: lanes 64-127 of the state product mirror rows 0-63
             const size_t o = soff + (size_t)(srow % D) * p.DV + col;
-            const bool in = p.s0 && GUARD((long long)(o + 32) <= p.state_elems, DBG_GLOBAL_OOB, 2);
+            const bool in = p.s0 && GUARD((long long)(o + 16) <= p.state_elems, DBG_GLOBAL_OOB, 2);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < 4; ++q) {
                 const float4 v = in ? *reinterpret_cast<const float4*>(p.s0 + o + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
                 S[4 * q] = v.x; S[4 * q + 1] = v.y; S[4 * q + 2] = v.z; S[4 * q + 3] = v.w;
             }
+            // the unused halves of the operand tiles feed only unused accumulator columns;
+            // zero them once so that they hold finite values
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            for (int e = tid - 128; e < (D * 128 + 16384) / 16; e += 256)
+                reinterpret_cast<uint4*>(sm + L::SB)[e] = z;
+            fence_proxy_async_smem();
+            named_sync(1, 256);
         }
         float gprev = 1.f;
         bool ok = true;
 
-        constexpr uint32_t ID_KN = idesc_bf16(128, kNV, false, true);
-        constexpr uint32_t ID_M5 = idesc_bf16(128, 2 * kNV, true, true);  // B = [U'_hi | U'_lo]
+        constexpr uint32_t ID_KN = idesc_bf16(128, 64, false, true);
+        constexpr uint32_t ID_M5 = idesc_bf16(128, 64, true, true);  // B = [U'_hi | U'_lo]
         constexpr uint64_t KS = 32 >> 4, MS = 2048 >> 4, BLK = L::KQW_BLOCK >> 4;
-        static_assert(L::ULO == L::UHI + 8192, "U'_lo is the second 64-column atom of U'");
+        static_assert(L::SB + D * 128 + 16384 == L::UB + 8192, "tiles zeroed at start");
         // M4: [Q; -W] S_bf16  ->  Q S (lanes 0-63), -W S (lanes 64-127)
         auto issue_m4 = [&](int c) {
             const int s = c & 1;
@@ -901,16 +910,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     mma_bf16(d4, dQW + b * BLK + kk * KS, dSB + (b * 4 + kk) * MS, ID_KN, (b | kk) != 0);
             mma_commit(&bars[CB_M4]);
         };
-        // M5: K^T [U'_hi | U'_lo] (U' = diag(Gam_C,. rk) U in two bf16 terms, side by side in N:
-        // an N = 128 product costs the tensor core what an N = 64 one does).  The output product
-        // M6 is issued by warp 1 once M5 is done, so that it does not delay M5's completion.
+        // M5: K^T [U'_hi | U'_lo] (U' = diag(Gam_C,. rk) U in two bf16 terms, side by side in one
+        // 64-column tile).  The output product M6 is issued by warp 1 once M5 is done, so that it
+        // does not delay M5's completion.
         auto issue_m56 = [&](int c) {
             const int s = c & 1;
             const uint64_t dKt = sdesc(smem_u32(sm + s * L::STAGE), D == 128 ? L::KQW_BLOCK : 0, 1024);
-            const uint64_t dUHI = sdesc(smem_u32(sm + L::UHI), 8192, 1024);
+            const uint64_t dUHL = sdesc(smem_u32(sm + L::UHL), 8192, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + L::T_S, dKt + kk * MS, dUHI + kk * MS, ID_M5, kk != 0);
+                mma_bf16(tmem + L::T_S, dKt + kk * MS, dUHL + kk * MS, ID_M5, kk != 0);
             mma_commit(&bars[CB_M5]);
         };
         // Arrival of this warp at the end of a step; the last of `n` arrivals for chunk c issues
@@ -940,16 +949,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (ok) {
                 const uint8_t* st = sm + s * L::STAGE;
                 const int nv = min(kChunk, len - cy * kChunk);
-                float a[32], b[32];
-                tmem_ld32x2(tmem + L::T_D4 + s * 64 + lane_base + col, tmem + L::T_D6 + s * 64 + lane_base + col, a, b);
+                float a[16], b[16];
+                tmem_ld16x2(tmem + L::T_D4 + s * 64 + lane_base + col, tmem + L::T_D6 + s * 64 + lane_base + col, a, b);
                 const float ys = reinterpret_cast<const float*>(st + L::SC)[64 + srow];
                 const size_t yoff = ((size_t)(t0 + (long)cy * kChunk + srow) * p.H + h) * p.DV + jsl * kNV + col;
-                if (srow < nv && GUARD((long long)(yoff + 32) <= p.y_elems, DBG_GLOBAL_OOB, 3)) {
+                if (srow < nv && GUARD((long long)(yoff + 16) <= p.y_elems, DBG_GLOBAL_OOB, 3)) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) a[j] = fmaf(ys, a[j], b[j]);
+                    for (int j = 0; j < 16; ++j) a[j] = fmaf(ys, a[j], b[j]);
                     uint4* dst = reinterpret_cast<uint4*>(p.y + yoff);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) dst[q] = pack8(a + 8 * q);
+                    for (int q = 0; q < 2; ++q) dst[q] = pack8(a + 8 * q);
                 }
             }
             tc_fence_before();
@@ -966,13 +975,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 ok = wwait(CB_M5, (c - 1) & 1, c) && ok;
                 tc_fence_after();
                 if (ok) {
-                    float d[32], e[32];
-                    tmem_ld32x2(tmem + L::T_S + lane_base + col, tmem + L::T_S + lane_base + kNV + col, d, e);
+                    float d[16], e[16];
+                    tmem_ld16x2(tmem + L::T_S + lane_base + col, tmem + L::T_S + lane_base + 32 + col, d, e);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) S[j] = fmaf(gprev, S[j], d[j] + e[j]);
+                    for (int j = 0; j < 16; ++j) S[j] = fmaf(gprev, S[j], d[j] + e[j]);
                 }
             }
-            if (ok && srow < D) store_half_row_mixed(sm + L::SB, srow, 4 * hf, S);
+            if (ok && srow < D) {
+                *reinterpret_cast<uint4*>(sm + L::SB + swz(srow, 2 * hf)) = pack8(S);
+                *reinterpret_cast<uint4*>(sm + L::SB + swz(srow, 2 * hf + 1)) = pack8_fma(S + 8);
+            }
             gprev = reinterpret_cast<const float*>(st + L::SC)[128];
             // M4 of this chunk may overwrite the output accumulators of chunk c - 2: the output
             // warps read them in iteration c - 1, before this arrival
@@ -988,13 +1000,14 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 if (ok) {
                     const int i = srow - 64;
                     const float us = reinterpret_cast<const float*>(st + L::SC)[i];
-                    float d[32];
-                    tmem_ld32(tmem + L::T_D4 + s * 64 + lane_base + col, d);
+                    float d[16];
+                    tmem_ld16(tmem + L::T_D4 + s * 64 + lane_base + col, d);
                     const uint8_t* urow = st + L::U + i * 256;
-                    uint32_t phi[16], plo[16], pub[16];
+                    const int ch0 = 8 * (jsl & 1) + 4 * hf;  // first 4-float chunk of these columns
+                    uint32_t phi[8], plo[8], pub[8];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 ut = *reinterpret_cast<const float4*>(urow + (((8 * hf + q) ^ (i & 7)) << 4));
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 ut = *reinterpret_cast<const float4*>(urow + (((ch0 + q) ^ (i & 7)) << 4));
                         const float u[4] = {ut.x + d[4 * q], ut.y + d[4 * q + 1], ut.z + d[4 * q + 2], ut.w + d[4 * q + 3]};
 #pragma unroll
                         for (int e = 0; e < 4; e += 2) {
@@ -1010,11 +1023,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                         }
                     }
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t off = swz(i, 4 * hf + q);
-                        *reinterpret_cast<uint4*>(sm + L::UHI + off) = make_uint4(phi[4 * q], phi[4 * q + 1], phi[4 * q + 2], phi[4 * q + 3]);
-                        *reinterpret_cast<uint4*>(sm + L::ULO + off) = make_uint4(plo[4 * q], plo[4 * q + 1], plo[4 * q + 2], plo[4 * q + 3]);
-                        *reinterpret_cast<uint4*>(sm + L::UB + off) = make_uint4(pub[4 * q], pub[4 * q + 1], pub[4 * q + 2], pub[4 * q + 3]);
+                    for (int q = 0; q < 2; ++q) {
+                        const uint4 vh = make_uint4(phi[4 * q], phi[4 * q + 1], phi[4 * q + 2], phi[4 * q + 3]);
+                        const uint4 vl = make_uint4(plo[4 * q], plo[4 * q + 1], plo[4 * q + 2], plo[4 * q + 3]);
+                        const uint4 vb = make_uint4(pub[4 * q], pub[4 * q + 1], pub[4 * q + 2], pub[4 * q + 3]);
+                        *reinterpret_cast<uint4*>(sm + L::UHL + swz(i, 2 * hf + q)) = vh;
+                        *reinterpret_cast<uint4*>(sm + L::UHL + swz(i, 4 + 2 * hf + q)) = vl;
+                        *reinterpret_cast<uint4*>(sm + L::UB + swz(i, 2 * hf + q)) = vb;
                     }
                 }
                 arrive(1, 4, c);
@@ -1027,15 +1042,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         ok = wwait(CB_M5, (nch - 1) & 1, nch) && ok;
         tc_fence_after();
         if (ok) {
-            float d[32], e[32];
-            tmem_ld32x2(tmem + L::T_S + lane_base + col, tmem + L::T_S + lane_base + kNV + col, d, e);
+            float d[16], e[16];
+            tmem_ld16x2(tmem + L::T_S + lane_base + col, tmem + L::T_S + lane_base + 32 + col, d, e);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) S[j] = fmaf(gprev, S[j], d[j] + e[j]);
+            for (int j = 0; j < 16; ++j) S[j] = fmaf(gprev, S[j], d[j] + e[j]);
             const size_t o = soff + (size_t)srow * p.DV + col;
-            if (p.s_final && srow < D && GUARD((long long)(o + 32) <= p.state_elems, DBG_GLOBAL_OOB, 4)) {
+            if (p.s_final && srow < D && GUARD((long long)(o + 16) <= p.state_elems, DBG_GLOBAL_OOB, 4)) {
                 float4* dst = reinterpret_cast<float4*>(p.s_final + o);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+                for (int q = 0; q < 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
             }
         }
         if (!uwarp) y_epilogue(nch - 1);
