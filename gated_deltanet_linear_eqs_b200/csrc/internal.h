@@ -39,7 +39,7 @@ struct PrefillArgs {
 // writes and the chain kernel reads, plus the chunk-record base of every packed document.
 struct PrefillWorkspace {
     int nrec_chunks;  // chunk records (an upper bound for packed documents)
-    size_t off_cb, off_map, off_w, off_p, off_u, off_s, total;
+    size_t off_cb, off_map, off_w, off_p, off_u, off_s, off_x, total;
 };
 PrefillWorkspace prefill_workspace(int num_seqs, int T, int H, int d, bool varlen);
 

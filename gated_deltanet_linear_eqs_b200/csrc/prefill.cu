@@ -19,16 +19,22 @@
 // alone; only U, Y and S' need the state.  The forward therefore runs as
 //   chunk-base scan (packed documents only): first record index of every document
 //   prep kernel   one CTA per (chunk, head), every chunk of every document at once: decay, norms,
-//                 A and P, the 64x64 triangular inverse, W and Ut, written to a workspace record
+//                 A and P, the 64x64 triangular inverse, W and Ut, and X = -W K_prev^T (the
+//                 chunk's -W against the previous chunk's keys), written to a workspace record
 //                 as ready-made tensor-core operand tiles
-//   chain kernel  one CTA per (document, head, 64-column slice of dv) walks its chunks in order
-//                 with the fp32 state in registers: U = Ut - W S, S' and Y on the tensor cores.
+//   chain kernel  one CTA per (document, head, 32-column slice of dv) walks its chunks in order
+//                 with the fp32 state in registers.  U_c = Ut_c - W_c S^c is formed from the
+//                 state one chunk back plus X_c U'_{c-1}, so that the state update runs a chunk
+//                 behind the pseudo-value recursion instead of inside it.
 // Only the chain kernel is sequential, and it does the state-dependent work alone.
 //
 // Workspace record of (chunk record g, head h), r = g * H + h:
 //   W  [r][dk/64][64 tokens][128 B]  -W, bf16, 128-byte swizzled rows (K-major MMA operand)
 //   P  [r][64 tokens][128 B]          P, bf16, 128-byte swizzled rows
-//   U  [r][dv/64][64 tokens][256 B]   Ut, fp32, 16-byte chunk q of row i at position q ^ (i % 8)
+//   U  [r][dv/32][64 tokens][128 B]   Ut, fp32, 32-column slices, 16-byte chunk q of row i at
+//                                     position q ^ (i % 8)
+//   X  [r][64 tokens][128 B]          -W K_prev^T (bf16, 128-byte swizzled rows): W of this chunk
+//                                     times the K tile of the previous chunk of the document
 //   SC [r][256] fp32                  [0,64) rk_i Gam_C/gamma_i (0 past the end), [64,128)
 //                                     scale gamma_i rq_i, [128] gamma_C
 #include <mutex>
@@ -52,6 +58,7 @@ constexpr int kLd = 72;  // bf16 row stride (elements) of the A / T scratch: 144
 constexpr int kNV = 32;  // dv columns per chain CTA (operand tiles stay 64 columns wide)
 constexpr uint32_t kRecP = 8192;
 constexpr uint32_t kRecS = 1024;
+constexpr uint32_t kRecX = 8192;
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -118,8 +125,9 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 // ============================================================================ chunk-base scan
 // cb[n] = sum over documents m < n of ceil(len_m / 64); cb[num_seqs] = total chunk records.
-// Then, for every record g < nrec, map[g] = (first token, valid tokens) of the chunk it holds
-// ((0, 0) past the last record), so that a prep CTA finds its chunk with one load.
+// Then, for every record g < nrec, map[g] = (first token, valid tokens + 65536 if the chunk is
+// not the first of its document) ((0, 0) past the last record), so that a prep CTA finds its
+// chunk with one load.
 constexpr int kMapSmem = 8192;  // documents whose bases are searched in shared memory
 __global__ void __launch_bounds__(1024) chunk_base_kernel(const int32_t* __restrict__ cu, int n,
                                                            int nrec, int32_t* __restrict__ cb,
@@ -176,8 +184,9 @@ __global__ void __launch_bounds__(1024) chunk_base_kernel(const int32_t* __restr
                 const int mid = (lo + hi + 1) >> 1;
                 if ((in_smem ? scb[mid] : cb[mid]) <= g) lo = mid; else hi = mid - 1;
             }
-            const int t0 = cu[lo] + (g - (in_smem ? scb[lo] : cb[lo])) * kChunk;
-            m = make_int2(t0, min(kChunk, cu[lo + 1] - t0));
+            const int c = g - (in_smem ? scb[lo] : cb[lo]);
+            const int t0 = cu[lo] + c * kChunk;
+            m = make_int2(t0, min(kChunk, cu[lo + 1] - t0) + (c > 0 ? 65536 : 0));
         }
         map[g] = m;
     }
@@ -189,7 +198,8 @@ struct PrepLayout {
     static constexpr int KB = D / 64;
     static constexpr int KQ = 0;                      // per dk block: K rows 0-63, Q rows 64-127
     static constexpr int V = KB * 16384;              // V: dv/64 blocks of 64 tokens x 64 columns
-    static constexpr int AF = V + KB * 8192;          // A, bf16 64 x kLd
+    static constexpr int KP = V + KB * 8192;          // K tile of the previous chunk, then X
+    static constexpr int AF = KP + KB * 8192;         // A, bf16 64 x kLd
     static constexpr int TF = AF + 64 * kLd * 2;      // T, bf16 64 x kLd
     static constexpr int TWN = AF;                    // 128 rows: T_w (0-63), N_b (64-127), written
                                                       // over A and T once T is in registers
@@ -198,17 +208,18 @@ struct PrepLayout {
     static constexpr int SC = AB + 512;               // scalar arrays, 64 floats each
     static constexpr int BAR = SC + 8 * 256;
     static constexpr int MISC = BAR + 8 * 8;          // tmem base, abort flag, zero word
-    static constexpr int BYTES = MISC + 16;
-    static constexpr int TX = KB * 16384 + KB * 8192;
+    // the X product reads 128 rows from the last -W block: 8 KB past it must be allocated
+    static constexpr int BYTES = MISC + 16 > TWN + (KB + 1) * 8192 ? MISC + 16 : TWN + (KB + 1) * 8192;
+    static constexpr int TX = KB * 16384 + KB * 8192;  // + KB * 8192 with the previous K tile
     static constexpr uint32_t T_D1 = 0;               // [K K^T | Q K^T] (64 columns), then
-    static constexpr uint32_t T_D3 = 0;               // W (D columns, lanes 0-63)
+    static constexpr uint32_t T_D3 = 0;               // W (D columns, lanes 0-63), then X
     static constexpr uint32_t T_DU = D;               // N_b V (D columns, lanes 64-127)
     static constexpr uint32_t T_COLS = 2 * D;
     static_assert(TWN % 1024 == 0 && TF + 64 * kLd * 2 >= TWN + 16384, "T_w / N_b tile");
-    static_assert(3 * (BYTES + 1024 + 1024) <= 233472, "three prep CTAs per SM");
+    static_assert(2 * (BYTES + 1024 + 1024) <= 233472, "two prep CTAs per SM");
 };
 enum { PS_G = 0, PS_GAM, PS_BETA, PS_RK, PS_RQ, PS_FTW, PS_CARRY, PS_COLF };
-enum { PB_FULL = 0, PB_TMEM, PB_M1, PB_RA1, PB_M3, PB_FIN, PB_COUNT };
+enum { PB_FULL = 0, PB_TMEM, PB_M1, PB_RA1, PB_M3, PB_RW, PB_MX, PB_FIN, PB_COUNT };
 
 struct PrepParams {
     const float* alpha;
@@ -224,6 +235,7 @@ struct PrepParams {
     uint8_t* ws_p;
     uint8_t* ws_u;
     float* ws_s;
+    uint8_t* ws_x;
     int* status;
     long long ab_elems;
 };
@@ -244,15 +256,18 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int g = bid / p.H;
     long base;
     int nvalid;
+    bool has_prev;  // the chunk has a predecessor in its document: X is computed
     if (p.map) {
         const int2 m = p.map[g];
-        if (m.y <= 0) return;  // grid sized for the worst case
+        nvalid = m.y & 0xffff;
+        if (nvalid <= 0) return;  // grid sized for the worst case
         base = m.x;
-        nvalid = m.y;
+        has_prev = (m.y >> 16) != 0;
     } else {
         const int n = g / p.nchunk_dense, c = g % p.nchunk_dense;
         base = (long)n * p.T + (long)c * kChunk;
         nvalid = min(kChunk, p.T - c * kChunk);
+        has_prev = c > 0;
     }
     const size_t rec = (size_t)g * p.H + h;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -290,13 +305,15 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // the tile copies first (lane 0's arrival carries the byte count), then alpha and beta;
         // the other 31 arrivals follow the alpha / beta stores of all lanes
         if (lane == 0) {
-            mbar_arrive_expect_tx(&bars[PB_FULL], L::TX);
+            mbar_arrive_expect_tx(&bars[PB_FULL], L::TX + (has_prev ? KB * 8192 : 0));
             const int z = (int)base;
 #pragma unroll
             for (int b = 0; b < KB; ++b) {
                 tma_load_3d(sm + L::KQ + b * 16384, &tm_k, 64 * b, h, z, &bars[PB_FULL]);
                 tma_load_3d(sm + L::KQ + b * 16384 + 8192, &tm_q, 64 * b, h, z, &bars[PB_FULL]);
                 tma_load_3d(sm + L::V + b * 8192, &tm_v, 64 * b, h, z, &bars[PB_FULL]);
+                if (has_prev)
+                    tma_load_3d(sm + L::KP + b * 8192, &tm_k, 64 * b, h, z - kChunk, &bars[PB_FULL]);
             }
         }
         float* ab = reinterpret_cast<float*>(sm + L::AB);
@@ -372,6 +389,23 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16(tmem + L::T_DU, dTWN + kk * KS, dVb + kk * MS, ID_N, kk != 0);
                 mma_commit(&bars[PB_M3]);
+            }
+            if (ok && has_prev) {
+                // X = -W K_prev^T from the -W image (rows 0-63 of each 64-column block; the
+                // 64 rows after it are read too and give unused accumulator rows)
+                ok = mbar_wait(&bars[PB_RW], 0, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    const uint64_t dWI = sdesc(s0 + L::TWN, 16, 1024);
+                    const uint64_t dKP = sdesc(s0 + L::KP, 16, 1024);
+#pragma unroll
+                    for (int b = 0; b < KB; ++b)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16(tmem + L::T_D3, dWI + b * (8192 >> 4) + kk * KS,
+                                     dKP + b * (8192 >> 4) + kk * KS, ID_M1, (b | kk) != 0);
+                    mma_commit(&bars[PB_MX]);
+                }
             }
             if (!ok && !*abort_flag) fail(PB_COUNT);
             // no MMA may still be writing TMEM or arriving on a barrier when the CTA ends
@@ -619,7 +653,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const int i = t - 64;
                 const bool valid = i < nvalid;
                 const float bi = sBeta[i];
-                uint8_t* urec = sm + L::KQ + (size_t)i * 256;
+                // 32-column slice (2 s + hf) of Ut: 64 rows x 128 bytes
+                uint8_t* urec = sm + L::KQ + (size_t)i * 128;
 #pragma unroll
                 for (int s = 0; s < KB; ++s) {
                     float d[32], vv[32];
@@ -632,8 +667,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         u.y = valid ? fmaf(bi, vv[4 * q + 1], d[4 * q + 1]) : 0.f;
                         u.z = valid ? fmaf(bi, vv[4 * q + 2], d[4 * q + 2]) : 0.f;
                         u.w = valid ? fmaf(bi, vv[4 * q + 3], d[4 * q + 3]) : 0.f;
-                        const int ch = hf * 8 + q;
-                        *reinterpret_cast<float4*>(urec + s * 16384 + ((ch ^ (i & 7)) << 4)) = u;
+                        *reinterpret_cast<float4*>(urec + (2 * s + hf) * 8192 + ((q ^ (i & 7)) << 4)) = u;
                     }
                 }
             }
@@ -642,11 +676,29 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         fence_proxy_async_smem();
         named_sync(1, 256);
         if (ok && t == 0 && hf == 0) {
+            if (has_prev) mbar_arrive(&bars[PB_RW]);  // the -W image is ready for X
             bulk_store(p.ws_w + rec * (size_t)(D * 128), sm + L::TWN, D * 128);
             bulk_store(p.ws_u + rec * (size_t)(D * 256), sm + L::KQ, D * 256);
             bulk_commit();
-            bulk_wait_read();  // the CTA's shared memory must outlive the copies' reads
         }
+        if (has_prev) {
+            // (6) X = -W K_prev^T (lanes 0-63) -> bf16 image over the previous K tile
+            ok = wwait(PB_MX, 0) && ok;
+            tc_fence_after();
+            if (ok && t < 64) {
+                float x[32];
+                tmem_ld32(tmem + L::T_D3 + lane_base + 32 * hf, x);
+                store_half_row_mixed(sm + L::KP, t, hf * 4, x);
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            named_sync(1, 256);
+            if (ok && t == 0 && hf == 0) {
+                bulk_store(p.ws_x + rec * (size_t)8192, sm + L::KP, 8192);
+                bulk_commit();
+            }
+        }
+        if (t == 0 && hf == 0) bulk_wait_read();  // shared memory must outlive the copies' reads
     }
 #undef GUARD
     __syncwarp();
@@ -658,35 +710,50 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 }
 
 // ============================================================================ chain kernel
+// Per chunk c of a document, with S^c the state at the chunk's start (S^0 = s0), gamma_c the
+// chunk's total decay and U'_c = diag(rk Gam_C / gamma) U_c:
+//   S^{c+1} = gamma_c S^c + K_c^T U'_c
+//   U_c     = Ut_c - W_c S^c
+//           = Ut_c + gamma_{c-1} (-W_c S^{c-1}) + X_c U'_{c-1}     (c >= 1, X_c = -W_c K_{c-1}^T)
+//   Y_c     = diag(scale gamma rq) Q_c S^c + P_c U_c
+// In the second form U_c needs the state one chunk back, and the step from U_{c-1} to U_c is a
+// single 64-token product X_c U'_{c-1}.  So the sequential loop per chunk is
+//   (B) pseudo-value epilogue -> M4b = X U' (4 MMAs) -> (B)
+// and the state update (M5 and its readout (A)) and the product -W S (M4a) run a chunk behind it:
+//   M4a(j)   = [Q_{j-1} ; -W_j] S^{max(j-1,0)}_bf16                 -> D4a[j & 1]
+//   M4b(c+1) = [P_c ; X_{c+1}] [U'_hi | U'_lo | U_bf16 | 0]_c        -> D4b[c & 1]
+//              rows 64-127, columns 0-63: X_{c+1} U'_c; rows 0-63, columns 64-95: P_c U_c
+//   M5(c)    = K_c^T [U'_hi | U'_lo]_c                              -> D5[c & 1]
+//   Y_c      = ysc (rows 0-63 of D4a[(c+1) & 1]) + (rows 0-63, columns 64-95 of D4b[c & 1])
+// Issuing a tensor-core instruction holds the issuing thread for about as long as the tensor
+// pipe takes to execute it, so the products are issued by two threads of their own (one for
+// M4a, one for M4b and M5) that wait on the epilogue warps' arrivals; the epilogue warps never
+// issue.
 template <int D>
 struct ChainLayout {
     static constexpr int KB = D / 64;
-    static constexpr int KQW_BLOCK = 192 * 128;   // per dk block: K rows 0-63, Q 64-127, -W 128-191
-    static constexpr int KQW = KB * KQW_BLOCK;
-    static constexpr int P = KQW;                 // P, 64 rows (read as 128 rows: then U)
-    static constexpr int U = P + 8192;            // Ut image of the 64-column slice: fp32, 64 x 256 B
-    static constexpr int SC = U + 16384;          // record scalars
-    static constexpr int STAGE = SC + 1024;
-    // The CTA's 32 state columns use the first half of 64-column operand tiles; an N = 64 MMA
-    // costs the tensor core what an N = 32 one does.
-    static constexpr int SB = 2 * STAGE;          // S in bf16: D rows x 64 columns (0-31 used)
-    static constexpr int UHL = SB + D * 128;      // [U'_hi (columns 0-31) | U'_lo (32-63)], 64 rows
-    static constexpr int UB = UHL + 8192;         // U in bf16, 64 rows (columns 0-31 used)
-    static constexpr int BAR = UB + 8192;
-    static constexpr int MISC = BAR + 16 * 8;     // tmem base, abort flag, zero word, 2 counters
-    static constexpr int BYTES = MISC + 32;
-    static constexpr int TX = KB * 16384 + KB * 8192 + 8192 + 16384 + 1024;
-    static constexpr uint32_t T_S = 0;            // [K^T U'_hi | K^T U'_lo] of the chunk, 64 columns
-    static constexpr uint32_t T_D4 = 64;          // [Q S ; -W S], 2 x 64 columns (0-31 used)
-    static constexpr uint32_t T_D6 = 192;         // P U, 2 x 64 columns (0-31 used)
+    // Each operand has a ring of two slots of its own, released by its last reader, so that the
+    // copy for chunk c + 2 starts as soon as chunk c no longer needs that operand.
+    static constexpr int QWR = 0;                   // slot j: per dk block [Q_{j-1} | -W_j], 16 KB
+    static constexpr int PXR = QWR + 2 * KB * 16384; // slot u: [P_u | X_{u+1}], 16 KB
+    static constexpr int KR = PXR + 32768;          // slot: K_c, KB x 8 KB
+    static constexpr int USR = KR + 2 * KB * 8192;  // slot: Ut slice 8 KB, then the scalars 1 KB
+    static constexpr int SB = USR + 2 * 9216;       // 2 buffers: S^c in bf16, D rows x 64 cols
+    static constexpr int UU = SB + 2 * D * 128;     // 2 buffers: [U'_hi | U'_lo] then [U_bf16 | 0]
+    static constexpr int BAR = UU + 2 * 16384;
+    static constexpr int MISC = BAR + 32 * 8;       // tmem base, abort flag, zero word
+    static constexpr int BYTES = MISC + 16;
+    static constexpr uint32_t T_D4A = 0;            // 2 x 64 columns
+    static constexpr uint32_t T_D4B = 128;          // 2 x 128 columns
+    static constexpr uint32_t T_D5 = 384;           // 2 x 64 columns
     static constexpr uint32_t T_COLS = 512;
-    static_assert(STAGE % 1024 == 0, "stage tiles stay 1024-byte aligned");
-    static_assert(BYTES + 1024 <= 232448 - 1024, "shared memory budget");
+    static_assert(SB % 1024 == 0 && UU % 1024 == 0 && KR % 1024 == 0, "tile alignment");
+    static_assert(BYTES + 1024 <= 232448, "shared memory budget");
 };
+// ring barriers (full / empty per slot), then per-step arrivals and tensor-core completions
 enum {
-    CB_FULL0 = 0, CB_FULL1, CB_EMPTY0, CB_EMPTY1,  // input ring
-    CB_M4, CB_M5, CB_M6_0, CB_M6_1,                // tensor-core completions
-    CB_COUNT
+    CB_QWF = 0, CB_QWE = 2, CB_PXF = 4, CB_PXE = 6, CB_KF = 8, CB_KE = 10, CB_UF = 12, CB_UE = 14,
+    CB_AD = 16, CB_BD = 18, CB_YD = 20, CB_M4A = 22, CB_M4B = 24, CB_M5 = 26, CB_COUNT = 28
 };
 
 struct ChainParams {
@@ -701,19 +768,18 @@ struct ChainParams {
     const uint8_t* ws_p;
     const uint8_t* ws_u;
     const float* ws_s;
+    const uint8_t* ws_x;
     int* status;
     long long y_elems, state_elems;
 };
 
-constexpr int kChainThreads = 384;
+constexpr int kChainThreads = 512;
 
-// Warp roles: 0 loads (TMA for K and Q, bulk copies for the workspace record), 1 owns the TMEM
-// allocation and issues the output product, 4..11 are the epilogue warps.  Epilogue warp w reads
-// TMEM lanes 32 (w % 4) .. +31 and columns 16 ((w - 4) / 4) .. +15 of the CTA's 32; lanes 0-63
-// carry the output rows (Y) and lanes 64-127 the pseudo-value rows (U); all eight hold a
-// 16-column strip of S.  There is no separate MMA warp:
-// the last epilogue warp to finish a step (found with a shared-memory arrival counter) issues the
-// tensor-core products that depend on it, which saves a wake-up on the sequential path.
+// Warp roles: 0 loads the [Q; -W] and [P; X] rings, 1 owns the TMEM allocation and loads the
+// Ut / scalar and K rings; 2, 3, 4, 5, 8, 9, 14, 15 hold the state (16 columns each: rows
+// 32 (w % 4) .. +31, columns 0-15 for w < 8, 16-31 otherwise) for the readout (A), warps 4, 5,
+// 8, 9 also write Y; 6, 7, 10, 11 run the pseudo-value epilogue (B) on rows 64-127 (16 columns
+// each); 12 issues M4a, 13 issues M4b and M5.  Warp w reads TMEM lanes 32 (w % 4) .. +31.
 template <int D>
 __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -763,19 +829,23 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
     volatile int* never = reinterpret_cast<volatile int*>(sm + L::MISC + 8);
-    int* arrivals = reinterpret_cast<int*>(sm + L::MISC + 16);  // (A) and (B) completions
     if (tid == 0) {
-        mbar_init(&bars[CB_FULL0], 1);
-        mbar_init(&bars[CB_FULL1], 1);
-        mbar_init(&bars[CB_EMPTY0], 5);  // MMA commit + 4 output warps
-        mbar_init(&bars[CB_EMPTY1], 5);
-        for (int b = CB_M4; b < CB_COUNT; ++b) mbar_init(&bars[b], 1);
+        for (int b = 0; b < CB_COUNT; ++b) {
+            int cnt = 1;
+            if (b == CB_UE || b == CB_UE + 1) cnt = 12;  // 8 readout warps + 4 pseudo-value warps
+            if (b == CB_AD || b == CB_AD + 1) cnt = 8;
+            if (b == CB_BD || b == CB_BD + 1 || b == CB_YD || b == CB_YD + 1) cnt = 4;
+            mbar_init(&bars[b], cnt);
+        }
         *abort_flag = 0;
         *never = 0;
-        arrivals[0] = 0;
-        arrivals[1] = 0;
         fence_mbar_init();
     }
+    // the unused columns of the 64-column operand tiles feed only unused accumulator columns;
+    // zero them (and the rest of those tiles) once so that they hold finite values
+    for (int e = tid; e < (2 * D * 128 + 2 * 16384) / 16; e += kChainThreads)
+        reinterpret_cast<uint4*>(sm + L::SB)[e] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
     if (warp == 1) tmem_alloc(tmem_slot, L::T_COLS);
     tc_fence_before();
     __syncthreads();
@@ -792,268 +862,326 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (!ok && lane == 0) fail(bar, c);
         return ok;
     };
+    // single-thread wait for use `u` of a two-buffer barrier pair: its completion (or, with
+    // `empty`, the completion of use u - 2, which frees the slot)
+    auto slot_wait = [&](int bar0, int u, bool empty) {
+        const uint32_t par = ((u >> 1) & 1) ^ (empty ? 1u : 0u);
+        if (mbar_wait(&bars[bar0 + (u & 1)], par, abort_flag)) return true;
+        if (!*abort_flag) fail(bar0 + (u & 1), u);
+        return false;
+    };
+    auto spin_done = [&](int bar0, int u) {
+        if (mbar_spin(&bars[bar0 + (u & 1)], (u >> 1) & 1, abort_flag)) return true;
+        if (!*abort_flag) fail(bar0 + (u & 1), u);
+        return false;
+    };
     constexpr uint32_t kRecW = D * 128, kRecU = D * 256;
+    auto recof = [&](int c) { return (size_t)(cbase + c) * p.H + h; };
+    auto zof = [&](int c) { return (int)(t0 + (long)c * kChunk); };
+    auto usc_of = [&](int s) { return reinterpret_cast<const float*>(sm + L::USR + s * 9216 + 8192); };
+    constexpr uint32_t ID_KN = idesc_bf16(128, 64, false, true);
+    constexpr uint32_t ID_KN128 = idesc_bf16(128, 128, false, true);
+    constexpr uint32_t ID_M5 = idesc_bf16(128, 64, true, true);
+    constexpr uint64_t KS = 32 >> 4, MS = 2048 >> 4;
 
     if (warp == 0) {
-        // ---------------------------------------------------------------- loads
+        // ---------------------------------------------------------------- loads: [Q; -W], [P; X]
         if (lane == 0) {
             prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_k);
-            int issued = 0;
-            for (int c = 0; c < nch; ++c) {
-                const int s = c & 1;
-                if (!mbar_wait(&bars[CB_EMPTY0 + s], ((c >> 1) & 1) ^ 1, abort_flag)) {
-                    if (!*abort_flag) fail(CB_EMPTY0 + s, c);
-                    break;
-                }
-                uint8_t* st = sm + s * L::STAGE;
-                const size_t rec = (size_t)(cbase + c) * p.H + h;
-                uint64_t* full = &bars[CB_FULL0 + s];
-                mbar_arrive_expect_tx(full, L::TX);
-                const int z = (int)(t0 + (long)c * kChunk);
+            int nq = 0, npx = 0;  // uses issued
+            for (int j = 0; j <= nch; ++j) {
+                // slot j of the [Q; -W] ring: Q of chunk j - 1, -W of chunk j
+                if (!slot_wait(CB_QWE, j, true)) break;
+                uint64_t* full = &bars[CB_QWF + (j & 1)];
+                mbar_arrive_expect_tx(full, (j >= 1 ? KB * 8192 : 0) + (j < nch ? KB * 8192 : 0));
 #pragma unroll
                 for (int b = 0; b < KB; ++b) {
-                    tma_load_3d(st + b * L::KQW_BLOCK, &tm_k, 64 * b, h, z, full);
-                    tma_load_3d(st + b * L::KQW_BLOCK + 8192, &tm_q, 64 * b, h, z, full);
-                    bulk_load(st + b * L::KQW_BLOCK + 16384, p.ws_w + rec * kRecW + b * 8192, 8192, full);
+                    uint8_t* blk = sm + L::QWR + ((j & 1) * KB + b) * 16384;
+                    if (j >= 1) tma_load_3d(blk, &tm_q, 64 * b, h, zof(j - 1), full);
+                    if (j < nch) bulk_load(blk + 8192, p.ws_w + recof(j) * kRecW + b * 8192, 8192, full);
                 }
-                bulk_load(st + L::P, p.ws_p + rec * kRecP, kRecP, full);
-                bulk_load(st + L::U, p.ws_u + rec * kRecU + (size_t)(jsl >> 1) * 16384, 16384, full);
-                bulk_load(st + L::SC, p.ws_s + rec * (kRecS / 4), kRecS, full);
-                if (c + 2 < nch) {  // warm L2 for the chunk that will reuse this stage
-                    const size_t rec2 = rec + 2 * (size_t)p.H;
+                ++nq;
+                // use j of the [P; X] ring: P of chunk j, X of chunk j + 1 (the last has none)
+                if (j < nch) {
+                    if (!slot_wait(CB_PXE, j, true)) break;
+                    uint64_t* pf = &bars[CB_PXF + (j & 1)];
+                    uint8_t* slot = sm + L::PXR + (j & 1) * 16384;
+                    mbar_arrive_expect_tx(pf, kRecP + (j + 1 < nch ? kRecX : 0));
+                    bulk_load(slot, p.ws_p + recof(j) * kRecP, kRecP, pf);
+                    if (j + 1 < nch) bulk_load(slot + 8192, p.ws_x + recof(j + 1) * kRecX, kRecX, pf);
+                    ++npx;
+                }
+                if (j + 2 < nch) {  // warm L2 for the use that will follow in this slot
 #pragma unroll
-                    for (int b = 0; b < KB; ++b) {
-                        tma_prefetch_3d(&tm_k, 64 * b, h, z + 2 * kChunk);
-                        tma_prefetch_3d(&tm_q, 64 * b, h, z + 2 * kChunk);
-                    }
-                    bulk_prefetch_l2(p.ws_w + rec2 * kRecW, kRecW);
-                    bulk_prefetch_l2(p.ws_p + rec2 * kRecP, kRecP);
-                    bulk_prefetch_l2(p.ws_u + rec2 * kRecU + (size_t)(jsl >> 1) * 16384, 16384);
-                    bulk_prefetch_l2(p.ws_s + rec2 * (kRecS / 4), kRecS);
+                    for (int b = 0; b < KB; ++b) tma_prefetch_3d(&tm_q, 64 * b, h, zof(j + 1));
+                    bulk_prefetch_l2(p.ws_w + recof(j + 2) * kRecW, kRecW);
+                    bulk_prefetch_l2(p.ws_p + recof(j + 2) * kRecP, kRecP);
+                    if (j + 3 < nch) bulk_prefetch_l2(p.ws_x + recof(j + 3) * kRecX, kRecX);
                 }
-                ++issued;
             }
-            // Tail of the ring: do not exit while a copy or a commit-arrive on this CTA's shared
-            // memory is still pending.
-            for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c) {
-                mbar_wait(&bars[CB_FULL0 + (c & 1)], (c >> 1) & 1, never, 100000000ull);
-                mbar_wait(&bars[CB_EMPTY0 + (c & 1)], (c >> 1) & 1, abort_flag);
+            // do not exit while a copy or a commit-arrive on this CTA's shared memory is pending
+            for (int u = nq - 2 < 0 ? 0 : nq - 2; u < nq; ++u) {
+                mbar_wait(&bars[CB_QWF + (u & 1)], (u >> 1) & 1, never, 100000000ull);
+                mbar_wait(&bars[CB_QWE + (u & 1)], (u >> 1) & 1, abort_flag);
+            }
+            for (int u = npx - 2 < 0 ? 0 : npx - 2; u < npx; ++u) {
+                mbar_wait(&bars[CB_PXF + (u & 1)], (u >> 1) & 1, never, 100000000ull);
+                mbar_wait(&bars[CB_PXE + (u & 1)], (u >> 1) & 1, abort_flag);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- output product M6
+        // ---------------------------------------------------------------- loads: Ut / scalars, K
         if (lane == 0) {
-            constexpr uint32_t ID_KN = idesc_bf16(128, 64, false, true);  // U_bf16 tile is 64 wide
-            constexpr uint64_t KS = 32 >> 4, MS = 2048 >> 4;
-            const uint64_t dUB = sdesc(smem_u32(sm + L::UB), 8192, 1024);
+            prefetch_tmap(&tm_k);
+            int nl = 0;
             for (int c = 0; c < nch; ++c) {
+                const size_t rec = recof(c);
                 const int s = c & 1;
-                // U_bf16 of chunk c is complete once M5(c) is (M5 is issued after it is written)
-                if (!mbar_wait(&bars[CB_M5], c & 1, abort_flag)) {
-                    if (!*abort_flag) fail(CB_M5, c);
-                    break;
-                }
-                tc_fence_after();
-                const uint64_t dP = sdesc(smem_u32(sm + s * L::STAGE + L::P), 16, 1024);
+                if (!slot_wait(CB_UE, c, true)) break;
+                uint64_t* uf = &bars[CB_UF + s];
+                mbar_arrive_expect_tx(uf, 8192 + kRecS);
+                bulk_load(sm + L::USR + s * 9216, p.ws_u + rec * kRecU + (size_t)jsl * 8192, 8192, uf);
+                bulk_load(sm + L::USR + s * 9216 + 8192, p.ws_s + rec * (kRecS / 4), kRecS, uf);
+                if (!slot_wait(CB_KE, c, true)) break;
+                uint64_t* kf = &bars[CB_KF + s];
+                mbar_arrive_expect_tx(kf, KB * 8192);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + L::T_D6 + s * 64, dP + kk * KS, dUB + kk * MS, ID_KN, kk != 0);
-                mma_commit(&bars[CB_M6_0 + s]);
-                mma_commit(&bars[CB_EMPTY0 + s]);
+                for (int b = 0; b < KB; ++b)
+                    tma_load_3d(sm + L::KR + (s * KB + b) * 8192, &tm_k, 64 * b, h, zof(c), kf);
+                ++nl;
+                if (c + 2 < nch) {
+                    const size_t rec2 = recof(c + 2);
+#pragma unroll
+                    for (int b = 0; b < KB; ++b) tma_prefetch_3d(&tm_k, 64 * b, h, zof(c + 2));
+                    bulk_prefetch_l2(p.ws_u + rec2 * kRecU + (size_t)jsl * 8192, 8192);
+                    bulk_prefetch_l2(p.ws_s + rec2 * (kRecS / 4), kRecS);
+                }
+            }
+            for (int u = nl - 2 < 0 ? 0 : nl - 2; u < nl; ++u) {
+                mbar_wait(&bars[CB_UF + (u & 1)], (u >> 1) & 1, never, 100000000ull);
+                mbar_wait(&bars[CB_KF + (u & 1)], (u >> 1) & 1, never, 100000000ull);
+                mbar_wait(&bars[CB_KE + (u & 1)], (u >> 1) & 1, abort_flag);
             }
         }
         __syncwarp();
-    } else if (warp >= 4) {
-        // ---------------------------------------------------------------- epilogue warps
-        const int qd = warp & 3, hf = (warp - 4) >> 2;
-        const int srow = qd * 32 + lane;               // TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
-        const uint32_t col = 16 * hf;
-        const bool uwarp = qd >= 2;                    // U rows; the others write Y
-        float S[16];
-        {
-            // D = 64: lanes 64-127 of the state product mirror rows 0-63
-            const size_t o = soff + (size_t)(srow % D) * p.DV + col;
-            const bool in = p.s0 && GUARD((long long)(o + 16) <= p.state_elems, DBG_GLOBAL_OOB, 2);
+    } else if (warp == 12) {
+        // ---------------------------------------------------------------- issue M4a
+        // M4a(j) reads S^{max(j-1,0)} (written by the readout of that step, which also implies
+        // that the readers of D4a[j & 1] from step j - 2 are done) and slot j of the [Q; -W] ring
+        if (lane == 0) {
+            for (int j = 0; j <= nch; ++j) {
+                if ((j != 1 && !spin_done(CB_AD, j >= 1 ? j - 1 : 0)) || !spin_done(CB_QWF, j)) break;
+                tc_fence_after();
+                const int sbuf = (j >= 1 ? j - 1 : 0) & 1;
+                const uint64_t dA = sdesc(smem_u32(sm + L::QWR + (j & 1) * KB * 16384), 16, 1024);
+                const uint64_t dSB = sdesc(smem_u32(sm + L::SB + sbuf * D * 128), D * 128, 1024);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v = in ? *reinterpret_cast<const float4*>(p.s0 + o + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
-                S[4 * q] = v.x; S[4 * q + 1] = v.y; S[4 * q + 2] = v.z; S[4 * q + 3] = v.w;
+                for (int b = 0; b < KB; ++b)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem + L::T_D4A + (j & 1) * 64, dA + b * (16384 >> 4) + kk * KS,
+                                 dSB + (b * 4 + kk) * MS, ID_KN, (b | kk) != 0);
+                mma_commit(&bars[CB_M4A + (j & 1)]);
+                mma_commit(&bars[CB_QWE + (j & 1)]);
             }
-            // the unused halves of the operand tiles feed only unused accumulator columns;
-            // zero them once so that they hold finite values
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            for (int e = tid - 128; e < (D * 128 + 16384) / 16; e += 256)
-                reinterpret_cast<uint4*>(sm + L::SB)[e] = z;
-            fence_proxy_async_smem();
-            named_sync(1, 256);
         }
-        float gprev = 1.f;
-        bool ok = true;
-
-        constexpr uint32_t ID_KN = idesc_bf16(128, 64, false, true);
-        constexpr uint32_t ID_M5 = idesc_bf16(128, 64, true, true);  // B = [U'_hi | U'_lo]
-        constexpr uint64_t KS = 32 >> 4, MS = 2048 >> 4, BLK = L::KQW_BLOCK >> 4;
-        static_assert(L::SB + D * 128 + 16384 == L::UB + 8192, "tiles zeroed at start");
-        // M4: [Q; -W] S_bf16  ->  Q S (lanes 0-63), -W S (lanes 64-127)
-        auto issue_m4 = [&](int c) {
-            const int s = c & 1;
-            const uint64_t dQW = sdesc(smem_u32(sm + s * L::STAGE + 8192), 16, 1024);
-            const uint64_t dSB = sdesc(smem_u32(sm + L::SB), D * 128, 1024);
-            const uint32_t d4 = tmem + L::T_D4 + s * 64;
-#pragma unroll
-            for (int b = 0; b < KB; ++b)
+        __syncwarp();
+    } else if (warp == 13) {
+        // ---------------------------------------------------------------- issue M4b and M5
+        if (lane == 0) {
+            for (int c = 0; c < nch; ++c) {
+                const int s = c & 1;
+                // U'_c and U_c are written; the [P; X] slot c has landed; the output warps have
+                // read D4b[c & 1] from chunk c - 2
+                if (!spin_done(CB_BD, c) || !spin_done(CB_PXF, c) || (c >= 2 && !spin_done(CB_YD, c - 2))) break;
+                tc_fence_after();
+                const uint64_t dPX = sdesc(smem_u32(sm + L::PXR + s * 16384), 16, 1024);
+                const uint64_t dUU = sdesc(smem_u32(sm + L::UU + s * 16384), 8192, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(d4, dQW + b * BLK + kk * KS, dSB + (b * 4 + kk) * MS, ID_KN, (b | kk) != 0);
-            mma_commit(&bars[CB_M4]);
-        };
-        // M5: K^T [U'_hi | U'_lo] (U' = diag(Gam_C,. rk) U in two bf16 terms, side by side in one
-        // 64-column tile).  The output product M6 is issued by warp 1 once M5 is done, so that it
-        // does not delay M5's completion.
-        auto issue_m56 = [&](int c) {
-            const int s = c & 1;
-            const uint64_t dKt = sdesc(smem_u32(sm + s * L::STAGE), D == 128 ? L::KQW_BLOCK : 0, 1024);
-            const uint64_t dUHL = sdesc(smem_u32(sm + L::UHL), 8192, 1024);
+                    mma_bf16(tmem + L::T_D4B + s * 128, dPX + kk * KS, dUU + kk * MS, ID_KN128, kk != 0);
+                mma_commit(&bars[CB_M4B + s]);
+                mma_commit(&bars[CB_PXE + s]);
+                if (!spin_done(CB_KF, c)) break;
+                tc_fence_after();
+                const uint64_t dKt = sdesc(smem_u32(sm + L::KR + s * KB * 8192), D == 128 ? 8192 : 0, 1024);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + L::T_S, dKt + kk * MS, dUHL + kk * MS, ID_M5, kk != 0);
-            mma_commit(&bars[CB_M5]);
-        };
-        // Arrival of this warp at the end of a step; the last of `n` arrivals for chunk c issues
-        // the dependent products.  The warp's shared-memory and TMEM accesses are ordered before
-        // the counter update (proxy and tcgen05 fences, then a CTA-scope fence), and the issuing
-        // thread orders the counter read before its tcgen05 operations the same way.
-        auto arrive = [&](int which, int n, int c) {
-            tc_fence_before();
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + L::T_D5 + s * 64, dKt + kk * MS, dUU + kk * MS, ID_M5, kk != 0);
+                mma_commit(&bars[CB_M5 + s]);
+                mma_commit(&bars[CB_KE + s]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- epilogue warps
+        const int qd = warp & 3;
+        const int srow = qd * 32 + lane;               // TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
+        const bool uwarp = warp == 6 || warp == 7 || warp == 10 || warp == 11;
+        const bool ywarp = warp == 4 || warp == 5 || warp == 8 || warp == 9;
+        const int hf = warp >= 8 ? 1 : 0;              // column half (16 columns) of the warp
+        bool ok = true;
+        // end of a step: order this warp's shared-memory writes (for the tensor cores) and TMEM
+        // reads before the arrival
+        auto signal = [&](int bar) {
             fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                __threadfence_block();
-                const int old = atomicAdd(arrivals + which, 1);
-                if (old == n * c + n - 1) {
-                    __threadfence_block();
-                    tc_fence_after();
-                    if (which == 0) issue_m4(c); else issue_m56(c);
-                }
-            }
-            __syncwarp();
-        };
-
-        auto y_epilogue = [&](int cy) {
-            const int s = cy & 1;
-            ok = wwait(CB_M6_0 + s, (cy >> 1) & 1, cy) && ok;
-            tc_fence_after();
-            if (ok) {
-                const uint8_t* st = sm + s * L::STAGE;
-                const int nv = min(kChunk, len - cy * kChunk);
-                float a[16], b[16];
-                tmem_ld16x2(tmem + L::T_D4 + s * 64 + lane_base + col, tmem + L::T_D6 + s * 64 + lane_base + col, a, b);
-                const float ys = reinterpret_cast<const float*>(st + L::SC)[64 + srow];
-                const size_t yoff = ((size_t)(t0 + (long)cy * kChunk + srow) * p.H + h) * p.DV + jsl * kNV + col;
-                if (srow < nv && GUARD((long long)(yoff + 16) <= p.y_elems, DBG_GLOBAL_OOB, 3)) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) a[j] = fmaf(ys, a[j], b[j]);
-                    uint4* dst = reinterpret_cast<uint4*>(p.y + yoff);
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) dst[q] = pack8(a + 8 * q);
-                }
-            }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[CB_EMPTY0 + s]);
+            if (lane == 0) mbar_arrive(&bars[bar]);
         };
 
-        for (int c = 0; c < nch; ++c) {
-            const int s = c & 1;
-            const uint8_t* st = sm + s * L::STAGE;
-            // (A) S_c = gamma_C S_{c-1} + K^T U'  ->  bf16 operand rows
-            ok = wwait(CB_FULL0 + s, (c >> 1) & 1, c) && ok;
-            if (c >= 1) {
-                ok = wwait(CB_M5, (c - 1) & 1, c) && ok;
-                tc_fence_after();
-                if (ok) {
-                    float d[16], e[16];
-                    tmem_ld16x2(tmem + L::T_S + lane_base + col, tmem + L::T_S + lane_base + 32 + col, d, e);
+        if (!uwarp) {
+            // ------------------------------------------------ (A): state readout, and Y
+            const int col0 = 16 * hf;
+            float S[16], pu[16];
+            {
+                const size_t o = soff + (size_t)(srow % D) * p.DV + col0;  // D = 64: mirror rows
+                const bool in = p.s0 && GUARD((long long)(o + 16) <= p.state_elems, DBG_GLOBAL_OOB, 2);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) S[j] = fmaf(gprev, S[j], d[j] + e[j]);
+                for (int q = 0; q < 4; ++q) {
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (in) v = *reinterpret_cast<const float4*>(p.s0 + o + 4 * q);
+                    S[4 * q] = v.x; S[4 * q + 1] = v.y; S[4 * q + 2] = v.z; S[4 * q + 3] = v.w;
                 }
             }
-            if (ok && srow < D) {
-                *reinterpret_cast<uint4*>(sm + L::SB + swz(srow, 2 * hf)) = pack8(S);
-                *reinterpret_cast<uint4*>(sm + L::SB + swz(srow, 2 * hf + 1)) = pack8_fma(S + 8);
+            // gamma of the previous chunk; the output scale of the previous chunk's rows, read
+            // while its slot is held
+            float gprev = 1.f, ysprev = 0.f;
+            for (int a = 0; a <= nch; ++a) {
+                float g_a = 1.f, ys_a = 0.f;
+                if (a < nch) {
+                    ok = wwait(CB_UF + (a & 1), (a >> 1) & 1, a) && ok;
+                    const float* sc = usc_of(a & 1);
+                    g_a = sc[128];
+                    if (ywarp) ys_a = sc[64 + srow];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[CB_UE + (a & 1)]);
+                }
+                if (a >= 1) {
+                    ok = wwait(CB_M5 + ((a - 1) & 1), ((a - 1) >> 1) & 1, a) && ok;
+                    tc_fence_after();
+                    if (ok) {
+                        const uint32_t t5 = tmem + L::T_D5 + ((a - 1) & 1) * 64 + lane_base + col0;
+                        float d[16], e[16];
+                        tmem_ld16x2(t5, t5 + 32, d, e);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) S[j] = fmaf(gprev, S[j], d[j] + e[j]);
+                    }
+                    if (ywarp) {
+                        // P_{a-1} U_{a-1} (M4b(a), complete before M5(a-1) is): into registers,
+                        // so that the accumulator is released at once
+                        const int cy = a - 1;
+                        ok = wwait(CB_M4B + (cy & 1), (cy >> 1) & 1, cy) && ok;
+                        tc_fence_after();
+                        if (ok) tmem_ld16(tmem + L::T_D4B + (cy & 1) * 128 + 64 + lane_base + col0, pu);
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars[CB_YD + (cy & 1)]);
+                    }
+                }
+                if (a < nch) {
+                    // S^a -> bf16 operand rows (columns col0 .. col0 + 15 of the 64-wide tile)
+                    if (ok && srow < D) {
+                        uint8_t* sb = sm + L::SB + (a & 1) * D * 128;
+                        *reinterpret_cast<uint4*>(sb + swz(srow, col0 / 8)) = pack8(S);
+                        *reinterpret_cast<uint4*>(sb + swz(srow, col0 / 8 + 1)) = pack8_fma(S + 8);
+                    }
+                    signal(CB_AD + (a & 1));
+                    gprev = g_a;
+                } else if (ok && p.s_final && srow < D) {
+                    const size_t o = soff + (size_t)srow * p.DV + col0;
+                    if (GUARD((long long)(o + 16) <= p.state_elems, DBG_GLOBAL_OOB, 4)) {
+                        float4* dst = reinterpret_cast<float4*>(p.s_final + o);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+                    }
+                }
+                if (ywarp && a >= 1) {
+                    // Y_{a-1} = ysc (Q_{a-1} S^{a-1}) + P_{a-1} U_{a-1}: rows 0-63 of M4a(a), M4b(a)
+                    const int cy = a - 1;
+                    ok = wwait(CB_M4A + (a & 1), (a >> 1) & 1, a) && ok;
+                    tc_fence_after();
+                    if (ok) {
+                        const int nv = min(kChunk, len - cy * kChunk);
+                        float qs[16];
+                        tmem_ld16(tmem + L::T_D4A + (a & 1) * 64 + lane_base + col0, qs);
+                        const size_t yoff = ((size_t)(t0 + (long)cy * kChunk + srow) * p.H + h) * p.DV + jsl * kNV + col0;
+                        if (srow < nv && GUARD((long long)(yoff + 16) <= p.y_elems, DBG_GLOBAL_OOB, 3)) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) qs[j] = fmaf(ysprev, qs[j], pu[j]);
+                            uint4* dst = reinterpret_cast<uint4*>(p.y + yoff);
+                            dst[0] = pack8(qs);
+                            dst[1] = pack8(qs + 8);
+                        }
+                    }
+                    tc_fence_before();
+                }
+                ysprev = ys_a;
             }
-            gprev = reinterpret_cast<const float*>(st + L::SC)[128];
-            // M4 of this chunk may overwrite the output accumulators of chunk c - 2: the output
-            // warps read them in iteration c - 1, before this arrival
-            arrive(0, 8, c);
-
-            if (uwarp) {
-                // (B) U = Ut + (-W S) -> U'_hi, U'_lo (scaled for the state update), U_bf16.
-                // M6 of the previous chunk (issued by another thread, so not covered by this
-                // chunk's M4 commit) must have finished reading U_bf16.
-                ok = wwait(CB_M4, c & 1, c) && ok;
-                if (c >= 1) ok = wwait(CB_M6_0 + ((c - 1) & 1), ((c - 1) >> 1) & 1, c) && ok;
+        } else {
+            // ------------------------------------------------ (B): pseudo-values, rows 64-127
+            const int col0 = 16 * hf;
+            const int i = srow - 64;
+            float gprev = 1.f;
+            for (int c = 0; c < nch; ++c) {
+                const int s = c & 1;
+                ok = wwait(CB_UF + s, (c >> 1) & 1, c) && ok;
+                ok = wwait(CB_M4A + s, (c >> 1) & 1, c) && ok;
+                if (c >= 1) ok = wwait(CB_M4B + ((c - 1) & 1), ((c - 1) >> 1) & 1, c) && ok;
                 tc_fence_after();
+                const float* sc = usc_of(s);
                 if (ok) {
-                    const int i = srow - 64;
-                    const float us = reinterpret_cast<const float*>(st + L::SC)[i];
-                    float d[16];
-                    tmem_ld16(tmem + L::T_D4 + s * 64 + lane_base + col, d);
-                    const uint8_t* urow = st + L::U + i * 256;
-                    const int ch0 = 8 * (jsl & 1) + 4 * hf;  // first 4-float chunk of these columns
+                    const float us = sc[i];
+                    float d[16], e[16], f[16];
+                    tmem_ld16(tmem + L::T_D4A + s * 64 + lane_base + col0, d);
+                    if (c >= 1) {
+                        const uint32_t t4 = tmem + L::T_D4B + ((c - 1) & 1) * 128 + lane_base + col0;
+                        tmem_ld16x2(t4, t4 + 32, e, f);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) e[j] = f[j] = 0.f;
+                    }
+                    const uint8_t* urow = sm + L::USR + s * 9216 + i * 128;
                     uint32_t phi[8], plo[8], pub[8];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const float4 ut = *reinterpret_cast<const float4*>(urow + (((ch0 + q) ^ (i & 7)) << 4));
-                        const float u[4] = {ut.x + d[4 * q], ut.y + d[4 * q + 1], ut.z + d[4 * q + 2], ut.w + d[4 * q + 3]};
+                        const float4 ut = *reinterpret_cast<const float4*>(urow + (((4 * hf + q) ^ (i & 7)) << 4));
+                        const float utv[4] = {ut.x, ut.y, ut.z, ut.w};
+                        float u[4];
 #pragma unroll
-                        for (int e = 0; e < 4; e += 2) {
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int j = 4 * q + e2;
+                            u[e2] = fmaf(gprev, d[j], utv[e2] + (e[j] + f[j]));
+                        }
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; e2 += 2) {
                             // U' = hi + lo with hi = U' truncated to bf16 and lo = the exact fp32
-                            // rest, itself truncated: |U' - hi - lo| < 2^-14 |U'|.  Bit operations
-                            // only, no conversion instructions.
-                            const uint32_t b0 = __float_as_uint(u[e] * us), b1 = __float_as_uint(u[e + 1] * us);
+                            // rest, itself truncated: |U' - hi - lo| < 2^-14 |U'|
+                            const uint32_t b0 = __float_as_uint(u[e2] * us), b1 = __float_as_uint(u[e2 + 1] * us);
                             const float l0 = __uint_as_float(b0) - __uint_as_float(b0 & 0xffff0000u);
                             const float l1 = __uint_as_float(b1) - __uint_as_float(b1 & 0xffff0000u);
-                            phi[2 * q + e / 2] = __byte_perm(b0, b1, 0x7632);
-                            plo[2 * q + e / 2] = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
-                            pub[2 * q + e / 2] = pack_bf16(u[e], u[e + 1]);
+                            phi[2 * q + e2 / 2] = __byte_perm(b0, b1, 0x7632);
+                            plo[2 * q + e2 / 2] = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
+                            pub[2 * q + e2 / 2] = pack_bf16(u[e2], u[e2 + 1]);
                         }
                     }
+                    uint8_t* uhl = sm + L::UU + s * 16384;
+                    uint8_t* ub = uhl + 8192;
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
-                        const uint4 vh = make_uint4(phi[4 * q], phi[4 * q + 1], phi[4 * q + 2], phi[4 * q + 3]);
-                        const uint4 vl = make_uint4(plo[4 * q], plo[4 * q + 1], plo[4 * q + 2], plo[4 * q + 3]);
-                        const uint4 vb = make_uint4(pub[4 * q], pub[4 * q + 1], pub[4 * q + 2], pub[4 * q + 3]);
-                        *reinterpret_cast<uint4*>(sm + L::UHL + swz(i, 2 * hf + q)) = vh;
-                        *reinterpret_cast<uint4*>(sm + L::UHL + swz(i, 4 + 2 * hf + q)) = vl;
-                        *reinterpret_cast<uint4*>(sm + L::UB + swz(i, 2 * hf + q)) = vb;
+                        *reinterpret_cast<uint4*>(uhl + swz(i, 2 * hf + q)) = make_uint4(phi[4 * q], phi[4 * q + 1], phi[4 * q + 2], phi[4 * q + 3]);
+                        *reinterpret_cast<uint4*>(uhl + swz(i, 4 + 2 * hf + q)) = make_uint4(plo[4 * q], plo[4 * q + 1], plo[4 * q + 2], plo[4 * q + 3]);
+                        *reinterpret_cast<uint4*>(ub + swz(i, 2 * hf + q)) = make_uint4(pub[4 * q], pub[4 * q + 1], pub[4 * q + 2], pub[4 * q + 3]);
                     }
                 }
-                arrive(1, 4, c);
-            } else if (c >= 1) {
-                // (C) outputs of the previous chunk, while this chunk's M4 runs
-                y_epilogue(c - 1);
+                gprev = sc[128];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[CB_UE + s]);
+                signal(CB_BD + s);
             }
         }
-        // the final state and the outputs of the last chunk
-        ok = wwait(CB_M5, (nch - 1) & 1, nch) && ok;
-        tc_fence_after();
-        if (ok) {
-            float d[16], e[16];
-            tmem_ld16x2(tmem + L::T_S + lane_base + col, tmem + L::T_S + lane_base + 32 + col, d, e);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) S[j] = fmaf(gprev, S[j], d[j] + e[j]);
-            const size_t o = soff + (size_t)srow * p.DV + col;
-            if (p.s_final && srow < D && GUARD((long long)(o + 16) <= p.state_elems, DBG_GLOBAL_OOB, 4)) {
-                float4* dst = reinterpret_cast<float4*>(p.s_final + o);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
-            }
-        }
-        if (!uwarp) y_epilogue(nch - 1);
         tc_fence_before();
     }
 #undef GUARD
@@ -1135,7 +1263,7 @@ cudaError_t launch_prep(const PrefillArgs& a, cudaStream_t st) {
     const int ntask = w.nrec_chunks * a.H;
     PrepParams pp{a.alpha, a.beta, varlen ? map : nullptr, a.num_seqs, a.T, a.H,
                   nchunk_dense, ntask, 2 * nsm, a.scale, a.l2norm, ws + w.off_w, ws + w.off_p,
-                  ws + w.off_u, reinterpret_cast<float*>(ws + w.off_s), a.status,
+                  ws + w.off_u, reinterpret_cast<float*>(ws + w.off_s), ws + w.off_x, a.status,
                   (long long)tokens * a.H};
     const int smem1 = PrepLayout<D>::BYTES + 1024;
     if ((e = cudaFuncSetAttribute(prep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1160,7 +1288,7 @@ cudaError_t launch_chain(const PrefillArgs& a, cudaStream_t st) {
     ChainParams cp{a.s0, static_cast<__nv_bfloat16*>(a.y), a.s_final, a.cu_seqlens,
                    varlen ? cb : nullptr, a.num_seqs, a.T, a.H, a.dv, nchunk_dense,
                    w.nrec_chunks, ws + w.off_w, ws + w.off_p, ws + w.off_u,
-                   reinterpret_cast<const float*>(ws + w.off_s), a.status,
+                   reinterpret_cast<const float*>(ws + w.off_s), ws + w.off_x, a.status,
                    (long long)tokens * a.H * a.dv, (long long)a.num_seqs * a.H * a.dk * a.dv};
     const int smem2 = ChainLayout<D>::BYTES + 1024;
     cudaError_t e;
@@ -1194,6 +1322,8 @@ PrefillWorkspace prefill_workspace(int num_seqs, int T, int H, int d, bool varle
     off += up(R * (size_t)d * 256);
     w.off_s = off;
     off += up(R * kRecS);
+    w.off_x = off;
+    off += up(R * kRecX);
     w.total = off;
     return w;
 }

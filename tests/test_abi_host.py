@@ -47,9 +47,9 @@ def test_status_strings(lib):
 
 def test_workspace_bytes(lib):
     n = ctypes.c_size_t(7)
-    # prefill: per (chunk record, head) -W (d*64 bf16), P (64*64 bf16), Ut (64*d fp32) and
-    # 256 fp32 scalars; packed documents add the chunk-record base array
-    rec = lambda d: d * 128 + 8192 + d * 256 + 1024
+    # prefill: per (chunk record, head) -W (d*64 bf16), P (64*64 bf16), Ut (64*d fp32),
+    # 256 fp32 scalars and X (64*64 bf16); packed documents add the chunk-record base array
+    rec = lambda d: d * 128 + 8192 + d * 256 + 1024 + 8192
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL, 1, 4096, 16, 128, 128, 0,
                                    ctypes.byref(n)) == 0
     assert n.value == 64 * 16 * rec(128)
