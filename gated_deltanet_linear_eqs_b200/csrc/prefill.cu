@@ -858,7 +858,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         record_status(p.status, GDN_ERR_TIMEOUT);
     };
     auto wwait = [&](int bar, uint32_t parity, int c) {
-        const bool ok = mbar_spin_warp(&bars[bar], parity, abort_flag);
+        const bool ok = mbar_wait_warp(&bars[bar], parity, abort_flag);
         if (!ok && lane == 0) fail(bar, c);
         return ok;
     };
@@ -1127,27 +1127,32 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             float gprev = 1.f;
             for (int c = 0; c < nch; ++c) {
                 const int s = c & 1;
+                // this chunk's Ut row and scalars first: their loads overlap the product waits
                 ok = wwait(CB_UF + s, (c >> 1) & 1, c) && ok;
+                const float* sc = usc_of(s);
+                const float us = sc[i], gnext = sc[128];
+                const uint8_t* urow = sm + L::USR + s * 9216 + i * 128;
+                float4 utq[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    utq[q] = *reinterpret_cast<const float4*>(urow + (((4 * hf + q) ^ (i & 7)) << 4));
                 ok = wwait(CB_M4A + s, (c >> 1) & 1, c) && ok;
                 if (c >= 1) ok = wwait(CB_M4B + ((c - 1) & 1), ((c - 1) >> 1) & 1, c) && ok;
                 tc_fence_after();
-                const float* sc = usc_of(s);
                 if (ok) {
-                    const float us = sc[i];
                     float d[16], e[16], f[16];
-                    tmem_ld16(tmem + L::T_D4A + s * 64 + lane_base + col0, d);
                     if (c >= 1) {
                         const uint32_t t4 = tmem + L::T_D4B + ((c - 1) & 1) * 128 + lane_base + col0;
-                        tmem_ld16x2(t4, t4 + 32, e, f);
+                        tmem_ld16x3(tmem + L::T_D4A + s * 64 + lane_base + col0, t4, t4 + 32, d, e, f);
                     } else {
+                        tmem_ld16(tmem + L::T_D4A + s * 64 + lane_base + col0, d);
 #pragma unroll
                         for (int j = 0; j < 16; ++j) e[j] = f[j] = 0.f;
                     }
-                    const uint8_t* urow = sm + L::USR + s * 9216 + i * 128;
                     uint32_t phi[8], plo[8], pub[8];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const float4 ut = *reinterpret_cast<const float4*>(urow + (((4 * hf + q) ^ (i & 7)) << 4));
+                        const float4 ut = utq[q];
                         const float utv[4] = {ut.x, ut.y, ut.z, ut.w};
                         float u[4];
 #pragma unroll
@@ -1176,7 +1181,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                         *reinterpret_cast<uint4*>(ub + swz(i, 2 * hf + q)) = make_uint4(pub[4 * q], pub[4 * q + 1], pub[4 * q + 2], pub[4 * q + 3]);
                     }
                 }
-                gprev = sc[128];
+                gprev = gnext;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[CB_UE + s]);
                 signal(CB_BD + s);
