@@ -971,7 +971,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // that the readers of D4a[j & 1] from step j - 2 are done) and slot j of the [Q; -W] ring
         if (lane == 0) {
             for (int j = 0; j <= nch; ++j) {
-                if ((j != 1 && !spin_done(CB_AD, j >= 1 ? j - 1 : 0)) || !spin_done(CB_QWF, j)) break;
+                // the copy normally landed long before the readout ends: check it first, so that
+                // the readout's arrival is the last wait before the issue
+                if (!spin_done(CB_QWF, j) || (j != 1 && !spin_done(CB_AD, j >= 1 ? j - 1 : 0))) break;
                 tc_fence_after();
                 const int sbuf = (j >= 1 ? j - 1 : 0) & 1;
                 const uint64_t dA = sdesc(smem_u32(sm + L::QWR + (j & 1) * KB * 16384), 16, 1024);
@@ -994,7 +996,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 const int s = c & 1;
                 // U'_c and U_c are written; the [P; X] slot c has landed; the output warps have
                 // read D4b[c & 1] from chunk c - 2
-                if (!spin_done(CB_BD, c) || !spin_done(CB_PXF, c) || (c >= 2 && !spin_done(CB_YD, c - 2))) break;
+                // (the copy and the output reads normally completed long before the epilogue ends:
+                // checked first, so that the epilogue's arrival is the last wait before the issue)
+                if (!spin_done(CB_PXF, c) || (c >= 2 && !spin_done(CB_YD, c - 2)) || !spin_done(CB_BD, c)) break;
                 tc_fence_after();
                 const uint64_t dPX = sdesc(smem_u32(sm + L::PXR + s * 16384), 16, 1024);
                 const uint64_t dUU = sdesc(smem_u32(sm + L::UU + s * 16384), 8192, 1024);
