@@ -276,7 +276,8 @@ def train_inputs(dev, seed=0):
 
 
 def run_train(args, dev, uuid, max_over_ranks, barrier, rank):
-    """Training shape: forward (gdn_prefill) + backward (gdn_backward) per step."""
+    """Training shape: forward (gdn_prefill: prep and chain kernels) + backward (gdn_backward:
+    chunk-matrix, forward-chain, reverse-chain and local-gradient kernels) per step."""
     import torch
     from gated_deltanet_linear_eqs_b200 import api
     from gated_deltanet_linear_eqs_b200._abi import GDN_OP_BACKWARD, GDN_OP_PREFILL
@@ -312,7 +313,7 @@ def run_train(args, dev, uuid, max_over_ranks, barrier, rank):
     tokens = TRAIN_B * TRAIN_T
     return {"metric": "GDN fwd+bwd tokens/s (training shape)", "unit": "tokens/s",
             "value": tokens / ((f_ms + b_ms) / 1e3), "ms_per_step": f_ms + b_ms,
-            "fwd_ms": f_ms, "bwd_ms": b_ms, "steps": steps, "gpu_launches": 4 * steps,
+            "fwd_ms": f_ms, "bwd_ms": b_ms, "steps": steps, "gpu_launches": 6 * steps,
             "config": {"workload": f"train: B={TRAIN_B}, T={TRAIN_T}, H={TRAIN_H}, dk=dv={D}, "
                                    "bf16, dy ~ N(0,1), S0 = 0"},
             "clocks": clk.summary()}

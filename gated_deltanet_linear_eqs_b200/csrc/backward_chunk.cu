@@ -1,0 +1,900 @@
+// backward_chunk.cu -- the backward pass of eqs. (1)-(4) (Qwen3.8-Flash-Next summary, picx.dev,
+// "Theoretical foundations"; the reverse recurrence of its Appendix B) in the chunked WY form of
+// the forward, on 64-token chunks, in fp32.
+//
+// Per chunk, with q^ = rq q, k^ = rk k the normalised rows, Lg the inclusive cumsum of ln(alpha),
+// gam = e^Lg, gC = gam of the chunk's last token, Gam_ij = e^(Lg_i - Lg_j), S = S^c the state at
+// the chunk's start and dS' the gradient of the state at its end:
+//   A = strictLower(diag(beta) (K^ K^T * Gam)),  T = (I + A)^-1
+//   W = T diag(beta gam) K^,  Ut = T diag(beta) V,  U = Ut - W S
+//   P = scale (Q^ K^T * Gam * lower-incl)
+//   Y = scale diag(gam) Q^ S + P U,   S' = gC S + K^T diag(gC / gam) U
+// The reverse chain is the transpose of the forward one:
+//   dU = diag(gC / gam) K^ dS' + P^T dY
+//   dS = gC dS' + scale Q^T diag(gam) dY - W^T dU
+// and every other gradient is local to the chunk once S, dS' and dU are known:
+//   dV = diag(beta) T^T dU,  dW = -dU S^T,  dT = dU (diag(beta) V)^T + dW (diag(beta gam) K^)^T,
+//   dA = -T^T dT T^T (strictly lower),  dP = dY U^T (lower-incl),
+//   dq^ = scale diag(gam) dY S^T + (scale dP * Gam) K^,
+//   dk^ = diag(beta gam) T^T dW + diag(gC / gam) U dS'^T + E K^ + E^T K^ + (scale dP * Gam)^T Q^
+//         with E = dA * beta_i Gam_ij,
+//   dbeta, d ln(alpha) (through gam, gC and Gam: d Lg_i collects (dA * A + dP * P) row i minus
+//   column i, and the gam / gC terms; d ln alpha is its reverse cumsum), and the L2-norm
+//   backward dq = rq (dq^ - q^ (q^ . dq^)).
+// Tokens past the end of a sequence are zero rows with alpha = 1, beta = 0, which makes them exact
+// identity steps, so no masks are needed.  gam can be far below 1 (it decays over the whole
+// chunk): the decay gradients are carried as gam_i d gam_i and gC d gC, and gC / gam_i as
+// e^(Lg_last - Lg_i), so that no term divides by gam.
+//
+// Kernels (one launch each, in stream order):
+//   bwdc_prep   one CTA per (chunk, head): norms, Lg, A / beta (kept for dbeta), P, T, W, Ut
+//   bwdc_fwd    one CTA per (sequence, head, 32 state columns): S^c and U of every chunk
+//   bwdc_rev    one CTA per (sequence, head, 32 state columns): dS' and dU of every chunk, dS0
+//   bwdc_local  one CTA per (chunk, head): all gradients of the chunk's tokens
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr int kCB = 64;   // chunk length
+constexpr int kNVB = 32;  // state columns per chain CTA
+constexpr int kL64 = 68;  // row stride (floats) of 64 x 64 shared matrices
+
+// Workspace arrays (float offsets); one record per (sequence, chunk, head), r = (b nch + c) H + h.
+struct BwdChunkWs {
+    size_t W, Ut, P, Tm, At, SC, S, U, dSp, dU, total;
+};
+BwdChunkWs bwdc_ws(int B, int T, int H, int D) {
+    const size_t nch = (size_t)(T + kCB - 1) / kCB, R = (size_t)B * nch * H;
+    BwdChunkWs w{};
+    size_t o = 0;
+    w.W = o;   o += R * kCB * D;
+    w.Ut = o;  o += R * kCB * D;
+    w.P = o;   o += R * kCB * kCB;
+    w.Tm = o;  o += R * kCB * kCB;
+    w.At = o;  o += R * kCB * kCB;
+    w.SC = o;  o += R * 256;  // rq[64], rk[64], Lg[64], beta[64]
+    w.S = o;   o += R * D * D;
+    w.U = o;   o += R * kCB * D;
+    w.dSp = o; o += R * D * D;
+    w.dU = o;  o += R * kCB * D;
+    w.total = o;
+    return w;
+}
+
+// acc[n] += sum_k a[k * as] * b[k * bs + n], n < NC (rows of b 16-byte aligned)
+template <int NC>
+__device__ __forceinline__ void mm_nn(float* acc, const float* a, int as, const float* b, int bs, int K) {
+#pragma unroll 2
+    for (int k = 0; k < K; ++k) {
+        const float x = a[k * as];
+        const float4* br = reinterpret_cast<const float4*>(b + (size_t)k * bs);
+#pragma unroll
+        for (int n = 0; n < NC / 4; ++n) {
+            const float4 y = br[n];
+            acc[4 * n + 0] = fmaf(x, y.x, acc[4 * n + 0]);
+            acc[4 * n + 1] = fmaf(x, y.y, acc[4 * n + 1]);
+            acc[4 * n + 2] = fmaf(x, y.z, acc[4 * n + 2]);
+            acc[4 * n + 3] = fmaf(x, y.w, acc[4 * n + 3]);
+        }
+    }
+}
+
+// acc[4u + e] += sum_k a[k * as] * b[k * bs + cs * u + e]: NC / 4 column chunks of 4, cs apart
+template <int NC>
+__device__ __forceinline__ void mm_nn_il(float* acc, const float* a, int as, const float* b, int bs, int cs, int K) {
+#pragma unroll 2
+    for (int k = 0; k < K; ++k) {
+        const float x = a[k * as];
+#pragma unroll
+        for (int u = 0; u < NC / 4; ++u) {
+            const float4 y = *reinterpret_cast<const float4*>(b + (size_t)k * bs + cs * u);
+            acc[4 * u + 0] = fmaf(x, y.x, acc[4 * u + 0]);
+            acc[4 * u + 1] = fmaf(x, y.y, acc[4 * u + 1]);
+            acc[4 * u + 2] = fmaf(x, y.z, acc[4 * u + 2]);
+            acc[4 * u + 3] = fmaf(x, y.w, acc[4 * u + 3]);
+        }
+    }
+}
+// acc[n] += sum_k a[k * as] * b[k * bs + n * step]
+template <int NC>
+__device__ __forceinline__ void mm_nn_str(float* acc, const float* a, int as, const float* b, int bs, int step, int K) {
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        const float x = a[k * as];
+#pragma unroll
+        for (int n = 0; n < NC; ++n) acc[n] = fmaf(x, b[(size_t)k * bs + n * step], acc[n]);
+    }
+}
+
+// acc[n] += sum_k a[k] * b[n * bs + k], k contiguous in both (16-byte aligned), K % 4 == 0.
+// GLOBAL: b is read-only global memory (read through the non-coherent cache).
+template <int NC, bool GLOBAL>
+__device__ __forceinline__ void mm_nt(float* acc, const float* a, const float* b, int bs, int K) {
+#pragma unroll 2
+    for (int k = 0; k < K; k += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(a + k);
+#pragma unroll
+        for (int n = 0; n < NC; ++n) {
+            const float4* p = reinterpret_cast<const float4*>(b + (size_t)n * bs + k);
+            const float4 y = GLOBAL ? __ldg(p) : *p;
+            acc[n] = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc[n]))));
+        }
+    }
+}
+
+__device__ __forceinline__ size_t tok_off(int b, int t, int h, int T, int H) {
+    return ((size_t)b * T + t) * H + h;
+}
+
+// 8 consecutive elements (16-byte aligned) -> fp32
+__device__ __forceinline__ void ld8(const __nv_bfloat16* p, float* o) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        o[2 * j] = __uint_as_float(w[j] << 16);
+        o[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void ld8(const float* p, float* o) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+__device__ __forceinline__ void st8(float* p, const float* x, float s) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(x[0] * s, x[1] * s, x[2] * s, x[3] * s);
+    reinterpret_cast<float4*>(p)[1] = make_float4(x[4] * s, x[5] * s, x[6] * s, x[7] * s);
+}
+
+// Rows t0 .. t0 + 63 of a [B, T, H, D] tensor (zero past nv) -> 64 x D fp32 shared tile of row
+// stride LD, each row scaled by scl[i] (nullptr: 1); NT threads, all loads issued before any store.
+template <int D, int LD, int NT, typename Tin>
+__device__ __forceinline__ void load_rows(float* dst, const Tin* src, int b, int t0, int nv, int h, int T,
+                                          int H, const float* scl, int tid) {
+    constexpr int PER = kCB * D / 8 / NT;  // 8-element groups per thread
+    static_assert(PER * NT * 8 == kCB * D, "tile split");
+    float x[PER][8];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int e = (tid + u * NT) * 8, i = e / D, m = e % D;
+        if (i < nv) ld8(src + tok_off(b, t0 + i, h, T, H) * D + m, x[u]);
+        else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[u][j] = 0.f;
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int e = (tid + u * NT) * 8, i = e / D, m = e % D;
+        st8(dst + i * LD + m, x[u], scl ? scl[i] : 1.f);
+    }
+}
+// 64 x D fp32 record array (row-major) -> shared tile of row stride LD
+template <int D, int LD, int NT>
+__device__ __forceinline__ void load_rec(float* dst, const float* src, int tid) {
+    constexpr int PER = kCB * D / 4 / NT;
+    float4 x[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) x[u] = reinterpret_cast<const float4*>(src)[tid + u * NT];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int e = (tid + u * NT) * 4;
+        *reinterpret_cast<float4*>(dst + (e / D) * LD + e % D) = x[u];
+    }
+}
+
+// fp32 -> tf32 (round to nearest, ties away), for the tensor-core products
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// C[64][D] (shared, row stride ldc) = s * A G^T with A [64][D] shared (row stride lda) and G [D][D]
+// row-major global: one 16 x (D/4) block of C per warp (16 warps), tf32 MMAs, fp32 accumulation.
+template <int D>
+__device__ __forceinline__ void gemm_nt_glob(float* C, int ldc, const float* A, int lda,
+                                             const float* __restrict__ G, float s, int warp, int lane) {
+    constexpr int CT = D / 32;  // 8-column tiles per warp
+    const int rt = warp & 3, ct0 = (warp >> 2) * CT;
+    const int gid = lane >> 2, tig = lane & 3;
+    float acc[CT][4];
+#pragma unroll
+    for (int t = 0; t < CT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+    const float* alo = A + (rt * 16 + gid) * lda + tig;
+    const float* ahi = alo + 8 * lda;
+#pragma unroll 2
+    for (int k0 = 0; k0 < D; k0 += 8) {
+        const uint32_t a0 = to_tf32(alo[k0]), a1 = to_tf32(ahi[k0]);
+        const uint32_t a2 = to_tf32(alo[k0 + 4]), a3 = to_tf32(ahi[k0 + 4]);
+#pragma unroll
+        for (int t = 0; t < CT; ++t) {
+            const float* g = G + (size_t)((ct0 + t) * 8 + gid) * D + k0 + tig;
+            mma_tf32(acc[t], a0, a1, a2, a3, to_tf32(__ldg(g)), to_tf32(__ldg(g + 4)));
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < CT; ++t) {
+        float* c = C + (rt * 16 + gid) * ldc + (ct0 + t) * 8 + 2 * tig;
+        c[0] = s * acc[t][0];
+        c[1] = s * acc[t][1];
+        c[8 * ldc] = s * acc[t][2];
+        c[8 * ldc + 1] = s * acc[t][3];
+    }
+}
+
+// sum over the 8 consecutive lanes that share a row
+__device__ __forceinline__ float row8_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    return x;
+}
+
+// ============================================================================ bwdc_prep
+template <int D>
+struct PrepB {
+    static constexpr int LD = D + 4;
+    static constexpr int BYTES = (3 * kCB * LD + 2 * kCB * kL64 + 5 * kCB + 768) * 4;
+};
+
+template <int D, typename Tin>
+__global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                                 const Tin* __restrict__ v, const float* __restrict__ alpha,
+                                                 const float* __restrict__ beta, float* __restrict__ ws,
+                                                 const BwdChunkWs w, int T, int H, int nch, float scale,
+                                                 int l2norm) {
+    constexpr int LD = PrepB<D>::LD;
+    extern __shared__ float smf[];
+    float* qh = smf;
+    float* kh = qh + kCB * LD;
+    float* vs = kh + kCB * LD;
+    float* Am = vs + kCB * LD;
+    float* Tm = Am + kCB * kL64;
+    float* rq = Tm + kCB * kL64;
+    float* rk = rq + kCB;
+    float* Lg = rk + kCB;
+    float* be = Lg + kCB;
+    float* gam = be + kCB;
+    float* Xs = gam + kCB;  // 3 x 16 x 16 block products
+    const size_t r = blockIdx.x;
+    const int h = (int)(r % H);
+    const int gr = (int)(r / H);
+    const int c = gr % nch, b = gr / nch;
+    const int t0 = c * kCB, nv = min(kCB, T - t0);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    load_rows<D, LD, 256>(qh, q, b, t0, nv, h, T, H, nullptr, tid);
+    load_rows<D, LD, 256>(kh, k, b, t0, nv, h, T, H, nullptr, tid);
+    load_rows<D, LD, 256>(vs, v, b, t0, nv, h, T, H, nullptr, tid);
+    if (tid < kCB) {
+        const size_t o = tok_off(b, t0 + tid, h, T, H);
+        be[tid] = tid < nv ? beta[o] : 0.f;
+        Lg[tid] = tid < nv ? logf(alpha[o]) : 0.f;
+    }
+    __syncthreads();
+    for (int rr = 0; rr < 16; ++rr) {  // warp w: rows 16 w .. 16 w + 15 of [q; k]
+        const int row = warp * 16 + rr;
+        const float* x = row < kCB ? qh + row * LD : kh + (row - kCB) * LD;
+        float s = 0.f;
+        for (int m = lane; m < D; m += 32) s = fmaf(x[m], x[m], s);
+        s = warp_sum(s);
+        if (lane == 0) {
+            const float rn = l2norm ? 1.0f / sqrtf(s + kNormEps) : 1.0f;
+            if (row < kCB) rq[row] = rn; else rk[row - kCB] = rn;
+        }
+    }
+    if (tid == 0) {
+        float acc = 0.f;
+        for (int i = 0; i < kCB; ++i) { acc += Lg[i]; Lg[i] = acc; }
+    }
+    __syncthreads();
+    if (tid < kCB) gam[tid] = expf(Lg[tid]);
+    for (int e = tid; e < kCB * D; e += 256) {
+        const int i = e / D, m = e % D;
+        qh[i * LD + m] *= rq[i];
+        kh[i * LD + m] *= rk[i];
+    }
+    __syncthreads();
+    // A / beta and P
+    {  // thread: row i, columns j = g + 4 n (rows g + 4 n of K^ sit in distinct banks)
+        const int i = tid >> 2, g = tid & 3;
+        float kk[16], qk[16];
+#pragma unroll
+        for (int n = 0; n < 16; ++n) kk[n] = qk[n] = 0.f;
+        mm_nt<16, false>(kk, kh + i * LD, kh + g * LD, 4 * LD, D);
+        mm_nt<16, false>(qk, qh + i * LD, kh + g * LD, 4 * LD, D);
+        float* Atg = ws + w.At + r * kCB * kCB + i * kCB;
+        float* Pg = ws + w.P + r * kCB * kCB + i * kCB;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+            const int j = g + 4 * n;
+            const float gm = expf(fminf(Lg[i] - Lg[j], 0.f));
+            const float at = j < i ? kk[n] * gm : 0.f;
+            Atg[j] = at;
+            Am[i * kL64 + j] = be[i] * at;
+            Pg[j] = j <= i ? scale * qk[n] * gm : 0.f;
+        }
+    }
+    __syncthreads();
+    // T = (I + A)^-1 by 16 x 16 blocks: the diagonal blocks by forward substitution (one column
+    // per thread), then T_ij = -T_ii sum_{j <= m < i} A_im T_mj for block distance 1, 2, 3
+    if (tid < kCB) {
+        const int bb = tid >> 4, m = tid & 15, o = 16 * bb;
+        for (int ii = 0; ii < 16; ++ii) {
+            float acc = 0.f;
+            for (int j = 0; j < ii; ++j) acc = fmaf(Am[(o + ii) * kL64 + o + j], Tm[(o + j) * kL64 + o + m], acc);
+            Tm[(o + ii) * kL64 + o + m] = ii < m ? 0.f : (ii == m ? 1.f : -acc);
+        }
+    }
+    for (int e = tid; e < kCB * kCB; e += 256) {  // zero the blocks above the diagonal
+        const int ii = e / kCB, j = e % kCB;
+        if ((j >> 4) > (ii >> 4)) Tm[ii * kL64 + j] = 0.f;
+    }
+    __syncthreads();
+    for (int dd = 1; dd < 4; ++dd) {
+        const int npair = 4 - dd;
+        for (int e = tid; e < npair * 256; e += 256) {  // X = sum_m A_im T_mj
+            const int pb = e >> 8, ii = (e >> 4) & 15, j = e & 15;
+            const int bi = pb + dd, bj = pb;
+            float acc = 0.f;
+            for (int m = 16 * bj; m < 16 * bi; ++m)
+                acc = fmaf(Am[(16 * bi + ii) * kL64 + m], Tm[m * kL64 + 16 * bj + j], acc);
+            Xs[e] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < npair * 256; e += 256) {  // T_ij = -T_ii X
+            const int pb = e >> 8, ii = (e >> 4) & 15, j = e & 15;
+            const int bi = pb + dd, bj = pb;
+            float acc = 0.f;
+            for (int m = 0; m < 16; ++m) acc = fmaf(Tm[(16 * bi + ii) * kL64 + 16 * bi + m], Xs[(pb << 8) + (m << 4) + j], acc);
+            Tm[(16 * bi + ii) * kL64 + 16 * bj + j] = -acc;
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < kCB * kCB; e += 256) ws[w.Tm + r * kCB * kCB + e] = Tm[(e / kCB) * kL64 + e % kCB];
+    // W = T diag(beta gam) K^, Ut = T diag(beta) V
+    {  // thread: row i, column chunks 4 g + 16 u
+        constexpr int NC = D / 4;
+        const int i = tid >> 2, g = tid & 3;
+        float wa[NC], ua[NC];
+#pragma unroll
+        for (int n = 0; n < NC; ++n) wa[n] = ua[n] = 0.f;
+        for (int j = 0; j < kCB; ++j) {
+            const float tij = Tm[i * kL64 + j];
+            const float fw = tij * be[j] * gam[j], fu = tij * be[j];
+            const float* kr = kh + j * LD + 4 * g;
+            const float* vr = vs + j * LD + 4 * g;
+#pragma unroll
+            for (int n = 0; n < NC / 4; ++n) {
+                const float4 y = *reinterpret_cast<const float4*>(kr + 16 * n);
+                const float4 z = *reinterpret_cast<const float4*>(vr + 16 * n);
+                wa[4 * n] = fmaf(fw, y.x, wa[4 * n]); wa[4 * n + 1] = fmaf(fw, y.y, wa[4 * n + 1]);
+                wa[4 * n + 2] = fmaf(fw, y.z, wa[4 * n + 2]); wa[4 * n + 3] = fmaf(fw, y.w, wa[4 * n + 3]);
+                ua[4 * n] = fmaf(fu, z.x, ua[4 * n]); ua[4 * n + 1] = fmaf(fu, z.y, ua[4 * n + 1]);
+                ua[4 * n + 2] = fmaf(fu, z.z, ua[4 * n + 2]); ua[4 * n + 3] = fmaf(fu, z.w, ua[4 * n + 3]);
+            }
+        }
+        float* Wg = ws + w.W + r * kCB * D + (size_t)i * D + 4 * g;
+        float* Ug = ws + w.Ut + r * kCB * D + (size_t)i * D + 4 * g;
+#pragma unroll
+        for (int n = 0; n < NC / 4; ++n) {
+            *reinterpret_cast<float4*>(Wg + 16 * n) = make_float4(wa[4 * n], wa[4 * n + 1], wa[4 * n + 2], wa[4 * n + 3]);
+            *reinterpret_cast<float4*>(Ug + 16 * n) = make_float4(ua[4 * n], ua[4 * n + 1], ua[4 * n + 2], ua[4 * n + 3]);
+        }
+    }
+    if (tid < kCB) {
+        float* sc = ws + w.SC + r * 256;
+        sc[tid] = rq[tid]; sc[64 + tid] = rk[tid]; sc[128 + tid] = Lg[tid]; sc[192 + tid] = be[tid];
+    }
+}
+
+// ============================================================================ chains
+template <int D>
+struct ChainB {
+    static constexpr int LDS = kNVB + 4;
+    static constexpr int LD = D + 4;
+    static constexpr int FWD_BYTES = (D * LDS + 2 * kCB * LD + kCB * LDS + 2 * kCB) * 4;
+    static constexpr int REV_BYTES = (D * LDS + 3 * kCB * LD + kCB * kL64 + 2 * kCB * LDS + 3 * kCB) * 4;
+};
+
+// Forward: S^c and U of every chunk, 32 state columns per CTA.
+template <int D, typename Tin>
+__global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const float* __restrict__ s0,
+                                                float* __restrict__ ws, const BwdChunkWs w, int T, int H,
+                                                int nch) {
+    using L = ChainB<D>;
+    constexpr int LDS = L::LDS, LD = L::LD;
+    extern __shared__ float smf[];
+    float* Ss = smf;
+    float* Wt = Ss + D * LDS;
+    float* Kt = Wt + kCB * LD;
+    float* Us = Kt + kCB * LD;
+    float* dec = Us + kCB * LDS;  // gC / gam
+    float* rks = dec + kCB;
+    constexpr int nsl = D / kNVB;
+    const int jsl = blockIdx.x % nsl, h = (blockIdx.x / nsl) % H, b = blockIdx.x / (nsl * H);
+    const int col0 = jsl * kNVB, tid = threadIdx.x;
+    for (int e = tid; e < D * kNVB; e += 256) {
+        const int m = e / kNVB, n = e % kNVB;
+        Ss[m * LDS + n] = s0 ? s0[(((size_t)b * H + h) * D + m) * D + col0 + n] : 0.f;
+    }
+    for (int c = 0; c < nch; ++c) {
+        const size_t r = ((size_t)b * nch + c) * H + h;
+        __syncthreads();
+        float* Sg = ws + w.S + r * D * D;
+        for (int e = tid; e < D * kNVB; e += 256) {
+            const int m = e / kNVB, n = e % kNVB;
+            Sg[(size_t)m * D + col0 + n] = Ss[m * LDS + n];
+        }
+        const float* SCg = ws + w.SC + r * 256;
+        if (tid < kCB) {
+            dec[tid] = expf(SCg[128 + kCB - 1] - SCg[128 + tid]);
+            rks[tid] = SCg[64 + tid];
+        }
+        const float gC = expf(SCg[128 + kCB - 1]);
+        load_rec<D, LD, 256>(Wt, ws + w.W + r * kCB * D, tid);
+        __syncthreads();
+        load_rows<D, LD, 256>(Kt, k, b, c * kCB, min(kCB, T - c * kCB), h, T, H, rks, tid);
+        {  // U = Ut - W S: row i, 8 columns
+            const int i = tid >> 2, n0 = (tid & 3) * 8;
+            float acc[8];
+#pragma unroll
+            for (int n = 0; n < 8; ++n) acc[n] = 0.f;
+            mm_nn<8>(acc, Wt + i * LD, 1, Ss + n0, LDS, D);
+            const float* Utg = ws + w.Ut + r * kCB * D + (size_t)i * D + col0 + n0;
+            float* Ug = ws + w.U + r * kCB * D + (size_t)i * D + col0 + n0;
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                const float u = Utg[n] - acc[n];
+                Us[i * LDS + n0 + n] = u;
+                Ug[n] = u;
+            }
+        }
+        __syncthreads();
+        {  // S = gC S + K^T diag(gC / gam) U
+            constexpr int TPR = 256 / D, NC = kNVB / TPR;
+            const int m = tid / TPR, n0 = (tid % TPR) * NC;
+            float acc[NC];
+#pragma unroll
+            for (int n = 0; n < NC; ++n) acc[n] = 0.f;
+            for (int i = 0; i < kCB; ++i) {
+                const float x = Kt[i * LD + m] * dec[i];
+                const float4* ur = reinterpret_cast<const float4*>(Us + i * LDS + n0);
+#pragma unroll
+                for (int n = 0; n < NC / 4; ++n) {
+                    const float4 y = ur[n];
+                    acc[4 * n] = fmaf(x, y.x, acc[4 * n]); acc[4 * n + 1] = fmaf(x, y.y, acc[4 * n + 1]);
+                    acc[4 * n + 2] = fmaf(x, y.z, acc[4 * n + 2]); acc[4 * n + 3] = fmaf(x, y.w, acc[4 * n + 3]);
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < NC; ++n) Ss[m * LDS + n0 + n] = fmaf(gC, Ss[m * LDS + n0 + n], acc[n]);
+        }
+    }
+}
+
+// Reverse: dS' and dU of every chunk, and dS0, 32 state columns per CTA.
+template <int D, typename Tin>
+__global__ void __launch_bounds__(256) bwdc_rev(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                                const Tin* __restrict__ dy, const float* __restrict__ ds_final,
+                                                float* __restrict__ ds0, float* __restrict__ ws,
+                                                const BwdChunkWs w, int T, int H, int nch, float scale) {
+    using L = ChainB<D>;
+    constexpr int LDS = L::LDS, LD = L::LD;
+    extern __shared__ float smf[];
+    float* Ss = smf;                 // dS slice
+    float* Kt = Ss + D * LDS;        // K^
+    float* Qt = Kt + kCB * LD;       // scale gam Q^
+    float* Wt = Qt + kCB * LD;
+    float* Pm = Wt + kCB * LD;
+    float* dYs = Pm + kCB * kL64;
+    float* dUs = dYs + kCB * LDS;
+    float* dec = dUs + kCB * LDS;    // gC / gam
+    float* ysc = dec + kCB;          // scale gam rq
+    float* rks = ysc + kCB;
+    constexpr int nsl = D / kNVB;
+    const int jsl = blockIdx.x % nsl, h = (blockIdx.x / nsl) % H, b = blockIdx.x / (nsl * H);
+    const int col0 = jsl * kNVB, tid = threadIdx.x;
+    for (int e = tid; e < D * kNVB; e += 256) {
+        const int m = e / kNVB, n = e % kNVB;
+        Ss[m * LDS + n] = ds_final ? ds_final[(((size_t)b * H + h) * D + m) * D + col0 + n] : 0.f;
+    }
+    for (int c = nch - 1; c >= 0; --c) {
+        const size_t r = ((size_t)b * nch + c) * H + h;
+        __syncthreads();
+        float* dSg = ws + w.dSp + r * D * D;
+        for (int e = tid; e < D * kNVB; e += 256) {
+            const int m = e / kNVB, n = e % kNVB;
+            dSg[(size_t)m * D + col0 + n] = Ss[m * LDS + n];
+        }
+        const float* SCg = ws + w.SC + r * 256;
+        if (tid < kCB) {
+            dec[tid] = expf(SCg[128 + kCB - 1] - SCg[128 + tid]);
+            ysc[tid] = scale * expf(SCg[128 + tid]) * SCg[tid];
+            rks[tid] = SCg[64 + tid];
+        }
+        const float gC = expf(SCg[128 + kCB - 1]);
+        load_rec<D, LD, 256>(Wt, ws + w.W + r * kCB * D, tid);
+        load_rec<kCB, kL64, 256>(Pm, ws + w.P + r * kCB * kCB, tid);
+        {  // dY slice: 64 rows x 32 columns, one 8-element group per thread
+            const int i = tid >> 2, n = (tid & 3) * 8, t = c * kCB + i;
+            float x[8];
+            if (t < T) ld8(dy + tok_off(b, t, h, T, H) * D + col0 + n, x);
+            else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) x[j] = 0.f;
+            }
+            st8(dYs + i * LDS + n, x, 1.f);
+        }
+        __syncthreads();
+        const int nvc = min(kCB, T - c * kCB);
+        load_rows<D, LD, 256>(Kt, k, b, c * kCB, nvc, h, T, H, rks, tid);
+        load_rows<D, LD, 256>(Qt, q, b, c * kCB, nvc, h, T, H, ysc, tid);
+        __syncthreads();
+        {  // dU = diag(gC / gam) K^ dS + P^T dY
+            const int i = tid >> 2, n0 = (tid & 3) * 8;
+            float a1[8], a2[8];
+#pragma unroll
+            for (int n = 0; n < 8; ++n) a1[n] = a2[n] = 0.f;
+            mm_nn<8>(a1, Kt + i * LD, 1, Ss + n0, LDS, D);
+            mm_nn<8>(a2, Pm + i, kL64, dYs + n0, LDS, kCB);
+            float* dUg = ws + w.dU + r * kCB * D + (size_t)i * D + col0 + n0;
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                const float du = fmaf(dec[i], a1[n], a2[n]);
+                dUs[i * LDS + n0 + n] = du;
+                dUg[n] = du;
+            }
+        }
+        __syncthreads();
+        {  // dS = gC dS + (scale gam Q^)^T dY - W^T dU
+            constexpr int TPR = 256 / D, NC = kNVB / TPR;
+            const int m = tid / TPR, n0 = (tid % TPR) * NC;
+            float acc[NC];
+#pragma unroll
+            for (int n = 0; n < NC; ++n) acc[n] = 0.f;
+            for (int i = 0; i < kCB; ++i) {
+                const float xq = Qt[i * LD + m], xw = Wt[i * LD + m];
+                const float4* yr = reinterpret_cast<const float4*>(dYs + i * LDS + n0);
+                const float4* ur = reinterpret_cast<const float4*>(dUs + i * LDS + n0);
+#pragma unroll
+                for (int n = 0; n < NC / 4; ++n) {
+                    const float4 y = yr[n], u = ur[n];
+                    acc[4 * n] = fmaf(xq, y.x, fmaf(-xw, u.x, acc[4 * n]));
+                    acc[4 * n + 1] = fmaf(xq, y.y, fmaf(-xw, u.y, acc[4 * n + 1]));
+                    acc[4 * n + 2] = fmaf(xq, y.z, fmaf(-xw, u.z, acc[4 * n + 2]));
+                    acc[4 * n + 3] = fmaf(xq, y.w, fmaf(-xw, u.w, acc[4 * n + 3]));
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < NC; ++n) Ss[m * LDS + n0 + n] = fmaf(gC, Ss[m * LDS + n0 + n], acc[n]);
+        }
+    }
+    __syncthreads();
+    if (ds0)
+        for (int e = tid; e < D * kNVB; e += 256) {
+            const int m = e / kNVB, n = e % kNVB;
+            ds0[(((size_t)b * H + h) * D + m) * D + col0 + n] = Ss[m * LDS + n];
+        }
+}
+
+// ============================================================================ bwdc_local
+template <int D>
+struct LocalB {
+    static constexpr int LD = D + 4;
+    static constexpr int BYTES = (5 * kCB * LD + 3 * kCB * kL64 + 10 * kCB + 32) * 4;
+};
+
+template <int D, typename Tin>
+__global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                                     const Tin* __restrict__ v, const Tin* __restrict__ dy,
+                                                     const float* __restrict__ alpha, Tin* __restrict__ dq,
+                                                     Tin* __restrict__ dk, Tin* __restrict__ dv,
+                                                     float* __restrict__ dalpha, float* __restrict__ dbeta,
+                                                     const float* __restrict__ ws, const BwdChunkWs w, int T,
+                                                     int H, int nch, float scale, int l2norm) {
+    constexpr int LD = LocalB<D>::LD;
+    constexpr int NC = D / 8;  // columns per thread in 64 x D results
+    extern __shared__ float smf[];
+    float* KH = smf;
+    float* QH = KH + kCB * LD;
+    float* B1 = QH + kCB * LD;   // dU, later dY
+    float* B2 = B1 + kCB * LD;   // V, later U
+    float* B3 = B2 + kCB * LD;   // dW
+    float* Tm = B3 + kCB * LD;
+    float* M1 = Tm + kCB * kL64;  // dT, then dA, then E
+    float* M2 = M1 + kCB * kL64;  // T^T dT, then dP, then F
+    float* rq = M2 + kCB * kL64;
+    float* rk = rq + kCB;
+    float* Lg = rk + kCB;
+    float* be = Lg + kCB;
+    float* gam = be + kCB;
+    float* colM = gam + kCB;      // column sums of dA * A + dP * P
+    float* dLg = colM + kCB;
+    float* red = dLg + kCB;       // [0]: d gC
+    const size_t r = blockIdx.x;
+    const int h = (int)(r % H);
+    const int gr = (int)(r / H);
+    const int c = gr % nch, b = gr / nch;
+    const int t0 = c * kCB, nv = min(kCB, T - t0);
+    const int tid = threadIdx.x, lane = tid & 31;
+    // thread: row i; in 64 x D results the column chunks 4 g + 32 u, in 64 x 64 results the
+    // columns g + 8 n (both spread a warp's shared-memory accesses over distinct banks)
+    const int i = tid >> 3, g = tid & 7;
+    auto col = [&](int n) { return 4 * g + 32 * (n >> 2) + (n & 3); };
+    const float* Sg = ws + w.S + r * D * D;
+    const float* dSg = ws + w.dSp + r * D * D;
+
+    const float* SCg = ws + w.SC + r * 256;
+    if (tid < kCB) {
+        rq[tid] = SCg[tid]; rk[tid] = SCg[64 + tid]; Lg[tid] = SCg[128 + tid]; be[tid] = SCg[192 + tid];
+        gam[tid] = expf(SCg[128 + tid]);
+        colM[tid] = 0.f;
+    }
+    if (tid == 0) red[0] = 0.f;
+    __syncthreads();
+    load_rows<D, LD, 512>(QH, q, b, t0, nv, h, T, H, rq, tid);
+    load_rows<D, LD, 512>(KH, k, b, t0, nv, h, T, H, rk, tid);
+    load_rows<D, LD, 512>(B2, v, b, t0, nv, h, T, H, nullptr, tid);
+    load_rec<D, LD, 512>(B1, ws + w.dU + r * kCB * D, tid);
+    load_rec<kCB, kL64, 512>(Tm, ws + w.Tm + r * kCB * kCB, tid);
+    __syncthreads();
+    const float gC = expf(Lg[kCB - 1]);
+    const float bi = be[i], gi = gam[i];
+    const float dec = expf(Lg[kCB - 1] - Lg[i]);  // gC / gam_i
+    float dbe = 0.f, dlg = 0.f;  // dlg = gam_i * d gam_i
+    float dqh[NC], dkh[NC];
+    // 1. Z1 = T^T dU: dV = diag(beta) Z1, dbeta += v . Z1
+    {
+        float z[NC];
+#pragma unroll
+        for (int n = 0; n < NC; ++n) z[n] = 0.f;
+        mm_nn_il<NC>(z, Tm + i, kL64, B1 + 4 * g, LD, 32, kCB);
+        float p = 0.f;
+#pragma unroll
+        for (int n = 0; n < NC; ++n) p = fmaf(B2[i * LD + col(n)], z[n], p);
+        dbe += row8_sum(p);
+        if (i < nv) {
+            Tin* dst = dv + tok_off(b, t0 + i, h, T, H) * D;
+#pragma unroll
+            for (int n = 0; n < NC; ++n) dst[col(n)] = from_f32<Tin>(bi * z[n]);
+        }
+    }
+    // 2. dW = -dU S^T
+    __syncthreads();
+    gemm_nt_glob<D>(B3, LD, B1, LD, Sg, -1.f, tid >> 5, lane);
+    __syncthreads();
+    // 3. Z2 = T^T dW: dk^ = diag(beta gam) Z2, d(beta gam) = k^ . Z2
+    {
+        float z[NC];
+#pragma unroll
+        for (int n = 0; n < NC; ++n) z[n] = 0.f;
+        mm_nn_il<NC>(z, Tm + i, kL64, B3 + 4 * g, LD, 32, kCB);
+        float p = 0.f;
+#pragma unroll
+        for (int n = 0; n < NC; ++n) {
+            dkh[n] = bi * gi * z[n];
+            p = fmaf(KH[i * LD + col(n)], z[n], p);
+        }
+        const float dbg = row8_sum(p);
+        dbe += dbg * gi;
+        dlg += dbg * bi * gi;
+    }
+    // 4. dT = dU (diag(beta) V)^T + dW (diag(beta gam) K^)^T  -> M1
+    {
+        float t1[8], t2[8];
+#pragma unroll
+        for (int n = 0; n < 8; ++n) t1[n] = t2[n] = 0.f;
+        mm_nt<8, false>(t1, B1 + i * LD, B2 + g * LD, 8 * LD, D);
+        mm_nt<8, false>(t2, B3 + i * LD, KH + g * LD, 8 * LD, D);
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            const int j = g + 8 * n;
+            M1[i * kL64 + j] = be[j] * (t1[n] + gam[j] * t2[n]);
+        }
+    }
+    __syncthreads();
+    // B1 <- dY, B2 <- U for the second half
+    load_rows<D, LD, 512>(B1, dy, b, t0, nv, h, T, H, nullptr, tid);
+    load_rec<D, LD, 512>(B2, ws + w.U + r * kCB * D, tid);
+    // 5. dA = -T^T dT T^T (strictly lower) -> M1
+    {
+        float x[8];
+#pragma unroll
+        for (int n = 0; n < 8; ++n) x[n] = 0.f;
+        mm_nn_str<8>(x, Tm + i, kL64, M1 + g, kL64, 8, kCB);
+#pragma unroll
+        for (int n = 0; n < 8; ++n) M2[i * kL64 + g + 8 * n] = x[n];
+    }
+    __syncthreads();
+    {
+        float x[8];
+#pragma unroll
+        for (int n = 0; n < 8; ++n) x[n] = 0.f;
+        mm_nt<8, false>(x, M2 + i * kL64, Tm + g * kL64, 8 * kL64, kCB);
+#pragma unroll
+        for (int n = 0; n < 8; ++n) M1[i * kL64 + g + 8 * n] = (g + 8 * n < i) ? -x[n] : 0.f;
+    }
+    // 6. G1 = dY S^T: dq^ = scale gam G1, gam d gam += scale gam q^ . G1
+    __syncthreads();  // B1, B2 = dY, U; B3 free
+    gemm_nt_glob<D>(B3, LD, B1, LD, Sg, 1.f, tid >> 5, lane);
+    __syncthreads();
+    {
+        float x[NC];
+#pragma unroll
+        for (int n = 0; n < NC; ++n) x[n] = B3[i * LD + col(n)];
+        float p = 0.f;
+#pragma unroll
+        for (int n = 0; n < NC; ++n) {
+            dqh[n] = scale * gi * x[n];
+            p = fmaf(QH[i * LD + col(n)], x[n], p);
+        }
+        dlg += scale * gi * row8_sum(p);
+    }
+    // 7. G2 = U dS'^T: dk^ += (gC / gam) G2; dr = k^ . G2 = d(gC / gam_i)
+    __syncthreads();
+    gemm_nt_glob<D>(B3, LD, B2, LD, dSg, 1.f, tid >> 5, lane);
+    __syncthreads();
+    {
+        float x[NC];
+#pragma unroll
+        for (int n = 0; n < NC; ++n) x[n] = B3[i * LD + col(n)];
+        float p = 0.f;
+#pragma unroll
+        for (int n = 0; n < NC; ++n) {
+            dkh[n] = fmaf(dec, x[n], dkh[n]);
+            p = fmaf(KH[i * LD + col(n)], x[n], p);
+        }
+        const float dr = row8_sum(p);  // d (gC / gam_i)
+        dlg -= dr * dec;
+        // gC d gC: sum over rows of dr gC / gam_i, plus gC <S, dS'>
+        float s = 0.f;
+        for (int e = tid; e < D * D / 4; e += 512) {
+            const float4 a = __ldg(reinterpret_cast<const float4*>(Sg) + e);
+            const float4 d = __ldg(reinterpret_cast<const float4*>(dSg) + e);
+            s = fmaf(a.x, d.x, fmaf(a.y, d.y, fmaf(a.z, d.z, fmaf(a.w, d.w, s))));
+        }
+        s = s * gC + ((tid & 7) == 0 ? dr * dec : 0.f);
+        s = warp_sum(s);
+        if (lane == 0) atomicAdd(red, s);
+    }
+    __syncthreads();  // M1 = dA complete; B1, B2 = dY, U
+    // 8. dP = dY U^T (lower-incl); the scalar terms of dA and dP; E and F in place
+    float rowM = 0.f;
+    {
+        float x[8];
+#pragma unroll
+        for (int n = 0; n < 8; ++n) x[n] = 0.f;
+        mm_nt<8, false>(x, B1 + i * LD, B2 + g * LD, 8 * LD, D);
+        const float* Atg = ws + w.At + r * kCB * kCB + i * kCB;
+        const float* Pg = ws + w.P + r * kCB * kCB + i * kCB;
+        float pbe = 0.f;
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            const int j = g + 8 * n;
+            const float dp = j <= i ? x[n] : 0.f;
+            const float da = M1[i * kL64 + j];
+            const float at = Atg[j];
+            const float mij = da * bi * at + dp * Pg[j];
+            pbe = fmaf(da, at, pbe);
+            rowM += mij;
+            atomicAdd(&colM[j], mij);
+            const float gm = j <= i ? expf(fminf(Lg[i] - Lg[j], 0.f)) : 0.f;
+            M1[i * kL64 + j] = da * bi * gm;        // E
+            M2[i * kL64 + j] = scale * dp * gm;     // F
+        }
+        dbe += row8_sum(pbe);
+        rowM = row8_sum(rowM);
+    }
+    __syncthreads();
+    // 9. dk^ += E K^ + E^T K^ + F^T Q^;  dq^ += F K^
+    mm_nn_il<NC>(dkh, M1 + i * kL64, 1, KH + 4 * g, LD, 32, kCB);
+    mm_nn_il<NC>(dkh, M1 + i, kL64, KH + 4 * g, LD, 32, kCB);
+    mm_nn_il<NC>(dkh, M2 + i, kL64, QH + 4 * g, LD, 32, kCB);
+    mm_nn_il<NC>(dqh, M2 + i * kL64, 1, KH + 4 * g, LD, 32, kCB);
+    // 10. d Lg_i = gam_i d gam_i + rowM_i - colM_i (+ gC d gC for the last token); reverse cumsum
+    if ((tid & 7) == 0) dLg[i] = dlg + rowM - colM[i];
+    __syncthreads();
+    if (tid == 0) {
+        float acc = red[0];  // gC d gC enters at the last token
+        for (int ii = kCB - 1; ii >= 0; --ii) {
+            acc += dLg[ii];
+            dLg[ii] = acc;  // d ln(alpha_ii)
+        }
+    }
+    __syncthreads();
+    if ((tid & 7) == 0 && i < nv) {
+        const size_t o = tok_off(b, t0 + i, h, T, H);
+        dalpha[o] = dLg[i] / alpha[o];
+        dbeta[o] = dbe;
+    }
+    // 11. norm backward: dx = r (dx^ - x^ (x^ . dx^))
+    {
+        float pq = 0.f, pk = 0.f;
+#pragma unroll
+        for (int n = 0; n < NC; ++n) {
+            pq = fmaf(QH[i * LD + col(n)], dqh[n], pq);
+            pk = fmaf(KH[i * LD + col(n)], dkh[n], pk);
+        }
+        pq = row8_sum(pq);
+        pk = row8_sum(pk);
+        if (i < nv) {
+            const size_t o = tok_off(b, t0 + i, h, T, H) * D;
+            const float rqi = l2norm ? rq[i] : 1.f, rki = l2norm ? rk[i] : 1.f;
+#pragma unroll
+            for (int n = 0; n < NC; ++n) {
+                const float gq = l2norm ? rqi * (dqh[n] - QH[i * LD + col(n)] * pq) : dqh[n];
+                const float gk = l2norm ? rki * (dkh[n] - KH[i * LD + col(n)] * pk) : dkh[n];
+                dq[o + col(n)] = from_f32<Tin>(gq);
+                dk[o + col(n)] = from_f32<Tin>(gk);
+            }
+        }
+    }
+}
+
+template <int D, typename Tin>
+cudaError_t launch_chunked(const BackwardArgs& a, cudaStream_t st) {
+    const int nch = (a.T + kCB - 1) / kCB;
+    const BwdChunkWs w = bwdc_ws(a.B, a.T, a.H, D);
+    if (a.ws == nullptr || a.ws_bytes < w.total * sizeof(float)) return cudaErrorInvalidValue;
+    float* ws = static_cast<float*>(a.ws);
+    const Tin* q = static_cast<const Tin*>(a.q);
+    const Tin* k = static_cast<const Tin*>(a.k);
+    const Tin* v = static_cast<const Tin*>(a.v);
+    const Tin* dy = static_cast<const Tin*>(a.dy);
+    const unsigned R = (unsigned)((size_t)a.B * nch * a.H);
+    const unsigned chains = (unsigned)(a.B * a.H * (D / kNVB));
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(bwdc_prep<D, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  PrepB<D>::BYTES)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwdc_fwd<D, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  ChainB<D>::FWD_BYTES)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwdc_rev<D, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  ChainB<D>::REV_BYTES)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwdc_local<D, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  LocalB<D>::BYTES)) != cudaSuccess)
+        return e;
+    bwdc_prep<D, Tin><<<R, 256, PrepB<D>::BYTES, st>>>(q, k, v, a.alpha, a.beta, ws, w, a.T, a.H, nch,
+                                                        a.scale, a.l2norm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwdc_fwd<D, Tin><<<chains, 256, ChainB<D>::FWD_BYTES, st>>>(k, a.s0, ws, w, a.T, a.H, nch);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwdc_rev<D, Tin><<<chains, 256, ChainB<D>::REV_BYTES, st>>>(q, k, dy, a.ds_final, a.ds0, ws, w, a.T,
+                                                                 a.H, nch, a.scale);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwdc_local<D, Tin><<<R, 512, LocalB<D>::BYTES, st>>>(
+        q, k, v, dy, a.alpha, static_cast<Tin*>(a.dq), static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv),
+        a.dalpha, a.dbeta, ws, w, a.T, a.H, nch, a.scale, a.l2norm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t backward_chunked_workspace_bytes(int B, int T, int H, int dk, int dv) {
+    (void)dv;
+    return bwdc_ws(B, T, H, dk).total * sizeof(float);
+}
+
+cudaError_t launch_backward_chunked(const BackwardArgs& a, cudaStream_t st) {
+    if (a.dtype == GDN_BF16)
+        return a.dkdim == 128 ? launch_chunked<128, __nv_bfloat16>(a, st)
+                              : launch_chunked<64, __nv_bfloat16>(a, st);
+    return a.dkdim == 128 ? launch_chunked<128, float>(a, st) : launch_chunked<64, float>(a, st);
+}
+
+}  // namespace gdn

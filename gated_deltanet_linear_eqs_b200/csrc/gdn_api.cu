@@ -102,7 +102,7 @@ int gdn_workspace_bytes(int op, int B, int T, int H, int dk, int dv, int num_seq
             return GDN_OK;
         case GDN_OP_BACKWARD:
             if (B < 1) return GDN_ERR_INVALID_ARG;
-            *bytes = gdn::backward_workspace_bytes(B, T, H, dk, dv);
+            *bytes = gdn::backward_chunked_workspace_bytes(B, T, H, dk, dv);
             return GDN_OK;
         default:
             return GDN_ERR_INVALID_ARG;
@@ -214,14 +214,14 @@ int gdn_backward(const void* q, const void* k, const void* v, const float* alpha
         return GDN_ERR_INVALID_ARG;
     if (B < 1 || T < 1 || H < 1) return GDN_ERR_INVALID_ARG;
     if (int rc = check_dims(dk, dv, dtype)) return rc;
-    const size_t need = gdn::backward_workspace_bytes(B, T, H, dk, dv);
+    const size_t need = gdn::backward_chunked_workspace_bytes(B, T, H, dk, dv);
     if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return GDN_ERR_WORKSPACE;
     DeviceInfo dev;
     if (int rc = current_device_info(&dev)) return rc;
     gdn::BackwardArgs a{q, k, v, alpha, beta, s0, dy, ds_final, dq, dk_out, dv_out, dalpha,
                         dbeta, ds0, B, T, H, dk, dv, dtype, scale, l2norm_qk ? 1 : 0, ws,
                         ws_bytes, dev.status};
-    return map_cuda(gdn::launch_backward(a, static_cast<cudaStream_t>(stream)));
+    return map_cuda(gdn::launch_backward_chunked(a, static_cast<cudaStream_t>(stream)));
 }
 
 int gdn_backward_noalloc(const void* q, const void* k, const void* v, const float* alpha,

@@ -67,8 +67,13 @@ cudaError_t launch_prefill_phase(const PrefillArgs& a, int phase, cudaStream_t s
 cudaError_t launch_prefill_seq(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st);
 
-// Workspace the backward pass needs (chunk-start states), bytes.
+// Workspace of the token-loop backward (chunk-start states), bytes; the fixed-scratch entry point
+// runs that path.
 size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv);
+
+// The chunked backward (gdn_backward): per-chunk fp32 records (chunk matrices, S^c, dS', U, dU).
+size_t backward_chunked_workspace_bytes(int B, int T, int H, int dk, int dv);
+cudaError_t launch_backward_chunked(const BackwardArgs& a, cudaStream_t st);
 
 // Size of the fixed device scratch array behind gdn_backward_noalloc.
 constexpr size_t kBackwardFixedScratchBytes = size_t(32) << 20;

@@ -152,7 +152,13 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* al
  * alpha (d/d alpha itself), beta and s0 (ds0 may be NULL if not wanted).
  * Dense layout as gdn_prefill.  dq, dk_out, dv_out have q/k/v's dtype; dalpha,
  * dbeta [B,T,H] fp32; ds0 [B,H,dk,dv] fp32.
- *   ws/ws_bytes: see gdn_workspace_bytes(GDN_OP_BACKWARD, ...).
+ *   ws/ws_bytes: see gdn_workspace_bytes(GDN_OP_BACKWARD, ...): per (sequence, 64-token
+ *   chunk, head) the chunk's fp32 matrices (W, Ut, P, T, A/beta; 4 * (2*64*dk + 3*64*64)
+ *   bytes), 1 KB of scalars, its start state and end-state gradient (2 * 4*dk*dv bytes) and
+ *   its pseudo-values and their gradient (2 * 4*64*dv bytes).
+ * Runs the chunked form: a chunk-parallel pass (the chunk matrices), a forward and a reverse
+ * pass over the chunks (states and state gradients), and a chunk-parallel pass for every
+ * token's gradients, all in fp32.
  */
 int gdn_backward(const void* q, const void* k, const void* v, const float* alpha,
                  const float* beta, const float* s0, const void* dy, const float* ds_final,
@@ -172,9 +178,12 @@ int gdn_backward(const void* q, const void* k, const void* v, const float* alpha
  * process exits.  It allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
  *   - Arguments, layouts, results and error codes are those of gdn_backward; inputs and
  *     outputs are still the caller's buffers.
- *   - Sizes whose workspace (gdn_workspace_bytes(GDN_OP_BACKWARD, ...)) exceeds
+ *   - It runs the token-loop form of the backward (one fp32 state checkpoint per 64-token
+ *     chunk, each chunk replayed token by token), whose scratch is
+ *     (ceil(T/64) + 64) * B*H*dk*dv*4 bytes; sizes where that exceeds
  *     gdn_backward_noalloc_max_workspace() are rejected with GDN_ERR_WORKSPACE before any
- *     launch.  At dk = dv = 128 that is B*H*(ceil(T/64) + 64) <= 512.
+ *     launch.  At dk = dv = 128 that is B*H*(ceil(T/64) + 64) <= 512.  Its results agree with
+ *     gdn_backward's to rounding (both are fp32).
  *   - The first call on each device looks up the scratch array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call before any
  *     stream capture.

@@ -65,13 +65,15 @@ def test_workspace_bytes(lib):
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_DECODE, 4, 1, 2, 128, 128, 0,
                                    ctypes.byref(n)) == 0
     assert n.value == 0
+    # chunked backward: per (sequence, chunk, head) record, fp32: W, Ut, U, dU (64 x d each),
+    # P, T, A/beta (64 x 64 each), 256 scalars, S^c and dS' (d x d each)
+    brec = lambda d: 4 * (4 * 64 * d + 3 * 64 * 64 + 256 + 2 * d * d)
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_BACKWARD, 8, 4096, 32, 128, 128, 0,
                                    ctypes.byref(n)) == 0
-    # one fp32 state per 64-token chunk (checkpoints) + 64 per chain (replayed chunk)
-    assert n.value == (64 + 64) * 8 * 32 * 128 * 128 * 4
+    assert n.value == 8 * 64 * 32 * brec(128)
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_BACKWARD, 1, 65, 1, 64, 64, 0,
                                    ctypes.byref(n)) == 0
-    assert n.value == (2 + 64) * 64 * 64 * 4
+    assert n.value == 2 * brec(64)
     assert lib.gdn_workspace_bytes(42, 1, 1, 1, 64, 64, 0, ctypes.byref(n)) == \
         _abi.GDN_ERR_INVALID_ARG
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL_VARLEN, 1, 10, 1, 64, 64, 0,
