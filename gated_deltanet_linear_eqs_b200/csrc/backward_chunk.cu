@@ -594,11 +594,43 @@ __global__ void __launch_bounds__(256) bwdc_rev(const Tin* __restrict__ q, const
 }
 
 // ============================================================================ bwdc_local
+// Every product runs as warp-level tf32 MMA tiles (m16n8k8, fp32 accumulation).  Warp w owns rows
+// 16 (w % 4) .. +15 and, in 64 x D results, columns (w / 4) D/4 .. +D/4 - 1 (in 64 x 64 results
+// columns 16 (w / 4) .. +15); lane (gid, tig) holds rows gid, gid + 8 and columns 2 tig, 2 tig + 1
+// of each 16 x 8 tile.  dq^ and dk^ stay in registers in that layout across the products.
 template <int D>
 struct LocalB {
     static constexpr int LD = D + 4;
-    static constexpr int BYTES = (5 * kCB * LD + 3 * kCB * kL64 + 10 * kCB + 32) * 4;
+    static constexpr int NROW = 10;  // row accumulators
+    static constexpr int BYTES = (5 * kCB * LD + 3 * kCB * kL64 + (5 + NROW + 1) * kCB + 32) * 4;
 };
+
+// acc[t] (16 x 8 tile t at rows r0.., columns c0 + 8 t ..) += A B over k < K, tf32
+template <int CT, typename FA, typename FB>
+__device__ __forceinline__ void wmma_acc(float (&acc)[CT][4], int K, int r0, int c0, FA a, FB b, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = to_tf32(a(r0 + gid, k0 + tig)), a1 = to_tf32(a(r0 + gid + 8, k0 + tig));
+        const uint32_t a2 = to_tf32(a(r0 + gid, k0 + tig + 4)), a3 = to_tf32(a(r0 + gid + 8, k0 + tig + 4));
+#pragma unroll
+        for (int t = 0; t < CT; ++t) {
+            const int n = c0 + 8 * t + gid;
+            mma_tf32(acc[t], a0, a1, a2, a3, to_tf32(b(k0 + tig, n)), to_tf32(b(k0 + tig + 4, n)));
+        }
+    }
+}
+template <int CT>
+__device__ __forceinline__ void zero_acc(float (&acc)[CT][4]) {
+#pragma unroll
+    for (int t = 0; t < CT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+}
+// sum over the 4 lanes of a quad (the lanes that share a tile row)
+__device__ __forceinline__ float quad_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    return x;
+}
 
 template <int D, typename Tin>
 __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, const Tin* __restrict__ k,
@@ -609,7 +641,7 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
                                                      const float* __restrict__ ws, const BwdChunkWs w, int T,
                                                      int H, int nch, float scale, int l2norm) {
     constexpr int LD = LocalB<D>::LD;
-    constexpr int NC = D / 8;  // columns per thread in 64 x D results
+    constexpr int CT = D / 32;  // 8-column tiles per warp in 64 x D results
     extern __shared__ float smf[];
     float* KH = smf;
     float* QH = KH + kCB * LD;
@@ -618,25 +650,33 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
     float* B3 = B2 + kCB * LD;   // dW
     float* Tm = B3 + kCB * LD;
     float* M1 = Tm + kCB * kL64;  // dT, then dA, then E
-    float* M2 = M1 + kCB * kL64;  // T^T dT, then dP, then F
+    float* M2 = M1 + kCB * kL64;  // T^T dT, then F
     float* rq = M2 + kCB * kL64;
     float* rk = rq + kCB;
     float* Lg = rk + kCB;
     float* be = Lg + kCB;
     float* gam = be + kCB;
-    float* colM = gam + kCB;      // column sums of dA * A + dP * P
-    float* dLg = colM + kCB;
-    float* red = dLg + kCB;       // [0]: d gC
+    float* racc = gam + kCB;      // NROW row accumulators of 64
+    float* r_dbe = racc;          // v . T^T dU  + sum_j dA_ij At_ij
+    float* r_dbg = racc + 64;     // k^ . T^T dW  (d (beta gam))
+    float* r_g1 = racc + 128;     // q^ . dY S^T
+    float* r_dr = racc + 192;     // k^ . U dS'^T  (d (gC / gam))
+    float* rowM = racc + 256;     // row sums of dA * A + dP * P
+    float* colM = racc + 320;     // column sums
+    float* r_pq = racc + 384;     // q^ . dq^
+    float* r_pk = racc + 448;     // k^ . dk^
+    float* dLg = racc + 512;
+    float* red = racc + 640;      // [0]: gC d gC
     const size_t r = blockIdx.x;
     const int h = (int)(r % H);
     const int gr = (int)(r / H);
     const int c = gr % nch, b = gr / nch;
     const int t0 = c * kCB, nv = min(kCB, T - t0);
-    const int tid = threadIdx.x, lane = tid & 31;
-    // thread: row i; in 64 x D results the column chunks 4 g + 32 u, in 64 x 64 results the
-    // columns g + 8 n (both spread a warp's shared-memory accesses over distinct banks)
-    const int i = tid >> 3, g = tid & 7;
-    auto col = [&](int n) { return 4 * g + 32 * (n >> 2) + (n & 3); };
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int r0 = (warp & 3) * 16;             // tile rows of this warp
+    const int cD = (warp >> 2) * (D / 4);       // first column in 64 x D results
+    const int c64 = (warp >> 2) * 16;           // first column in 64 x 64 results
     const float* Sg = ws + w.S + r * D * D;
     const float* dSg = ws + w.dSp + r * D * D;
 
@@ -644,9 +684,8 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
     if (tid < kCB) {
         rq[tid] = SCg[tid]; rk[tid] = SCg[64 + tid]; Lg[tid] = SCg[128 + tid]; be[tid] = SCg[192 + tid];
         gam[tid] = expf(SCg[128 + tid]);
-        colM[tid] = 0.f;
     }
-    if (tid == 0) red[0] = 0.f;
+    for (int e = tid; e < LocalB<D>::NROW * kCB + 32; e += 512) racc[e] = 0.f;
     __syncthreads();
     load_rows<D, LD, 512>(QH, q, b, t0, nv, h, T, H, rq, tid);
     load_rows<D, LD, 512>(KH, k, b, t0, nv, h, T, H, rk, tid);
@@ -655,196 +694,246 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
     load_rec<kCB, kL64, 512>(Tm, ws + w.Tm + r * kCB * kCB, tid);
     __syncthreads();
     const float gC = expf(Lg[kCB - 1]);
-    const float bi = be[i], gi = gam[i];
-    const float dec = expf(Lg[kCB - 1] - Lg[i]);  // gC / gam_i
-    float dbe = 0.f, dlg = 0.f;  // dlg = gam_i * d gam_i
-    float dqh[NC], dkh[NC];
+    // row of element e (0..3) of a tile
+    auto rowof = [&](int e) { return r0 + gid + (e >> 1) * 8; };
+    // add a per-lane value for each of the lane's two rows into a row accumulator (quad sum first)
+    auto row_add = [&](float* acc, float lo, float hi) {
+        lo = quad_sum(lo);
+        hi = quad_sum(hi);
+        if (tig == 0) {
+            atomicAdd(&acc[r0 + gid], lo);
+            atomicAdd(&acc[r0 + gid + 8], hi);
+        }
+    };
+    auto aT = [&](const float* M) { return [M](int i, int kk) { return M[kk * kL64 + i]; }; };
+    auto aR = [&](const float* M, int ld) { return [M, ld](int i, int kk) { return M[i * ld + kk]; }; };
+    auto bR = [&](const float* M, int ld) { return [M, ld](int kk, int n) { return M[kk * ld + n]; }; };
+    auto bT = [&](const float* M, int ld) { return [M, ld](int kk, int n) { return M[n * ld + kk]; }; };
+
+    float dqa[CT][4], dka[CT][4];
+    zero_acc(dqa);
+    zero_acc(dka);
     // 1. Z1 = T^T dU: dV = diag(beta) Z1, dbeta += v . Z1
     {
-        float z[NC];
+        float z[CT][4];
+        zero_acc(z);
+        wmma_acc(z, kCB, r0, cD, aT(Tm), bR(B1, LD), lane);
+        float lo = 0.f, hi = 0.f;
 #pragma unroll
-        for (int n = 0; n < NC; ++n) z[n] = 0.f;
-        mm_nn_il<NC>(z, Tm + i, kL64, B1 + 4 * g, LD, 32, kCB);
-        float p = 0.f;
+        for (int t = 0; t < CT; ++t)
 #pragma unroll
-        for (int n = 0; n < NC; ++n) p = fmaf(B2[i * LD + col(n)], z[n], p);
-        dbe += row8_sum(p);
-        if (i < nv) {
-            Tin* dst = dv + tok_off(b, t0 + i, h, T, H) * D;
-#pragma unroll
-            for (int n = 0; n < NC; ++n) dst[col(n)] = from_f32<Tin>(bi * z[n]);
-        }
+            for (int e = 0; e < 4; ++e) {
+                const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
+                const float pv = B2[i * LD + n] * z[t][e];
+                if (e < 2) lo += pv; else hi += pv;
+                if (i < nv) dv[tok_off(b, t0 + i, h, T, H) * D + n] = from_f32<Tin>(be[i] * z[t][e]);
+            }
+        row_add(r_dbe, lo, hi);
     }
     // 2. dW = -dU S^T
-    __syncthreads();
-    gemm_nt_glob<D>(B3, LD, B1, LD, Sg, -1.f, tid >> 5, lane);
+    gemm_nt_glob<D>(B3, LD, B1, LD, Sg, -1.f, warp, lane);
     __syncthreads();
     // 3. Z2 = T^T dW: dk^ = diag(beta gam) Z2, d(beta gam) = k^ . Z2
     {
-        float z[NC];
+        float z[CT][4];
+        zero_acc(z);
+        wmma_acc(z, kCB, r0, cD, aT(Tm), bR(B3, LD), lane);
+        float lo = 0.f, hi = 0.f;
 #pragma unroll
-        for (int n = 0; n < NC; ++n) z[n] = 0.f;
-        mm_nn_il<NC>(z, Tm + i, kL64, B3 + 4 * g, LD, 32, kCB);
-        float p = 0.f;
+        for (int t = 0; t < CT; ++t)
 #pragma unroll
-        for (int n = 0; n < NC; ++n) {
-            dkh[n] = bi * gi * z[n];
-            p = fmaf(KH[i * LD + col(n)], z[n], p);
-        }
-        const float dbg = row8_sum(p);
-        dbe += dbg * gi;
-        dlg += dbg * bi * gi;
+            for (int e = 0; e < 4; ++e) {
+                const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
+                dka[t][e] = be[i] * gam[i] * z[t][e];
+                const float pv = KH[i * LD + n] * z[t][e];
+                if (e < 2) lo += pv; else hi += pv;
+            }
+        row_add(r_dbg, lo, hi);
     }
-    // 4. dT = dU (diag(beta) V)^T + dW (diag(beta gam) K^)^T  -> M1
+    // 4. dT = (dU V^T + dW (gam K^)^T) diag(beta) -> M1
     {
-        float t1[8], t2[8];
+        float x[2][4];
+        zero_acc(x);
+        wmma_acc(x, D, r0, c64, aR(B1, LD), bT(B2, LD), lane);
+        const float* gm = gam;
+        const float* kh = KH;
+        wmma_acc(x, D, r0, c64, aR(B3, LD), [kh, gm](int kk, int j) { return kh[j * LD + kk] * gm[j]; }, lane);
 #pragma unroll
-        for (int n = 0; n < 8; ++n) t1[n] = t2[n] = 0.f;
-        mm_nt<8, false>(t1, B1 + i * LD, B2 + g * LD, 8 * LD, D);
-        mm_nt<8, false>(t2, B3 + i * LD, KH + g * LD, 8 * LD, D);
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int n = 0; n < 8; ++n) {
-            const int j = g + 8 * n;
-            M1[i * kL64 + j] = be[j] * (t1[n] + gam[j] * t2[n]);
-        }
+            for (int e = 0; e < 4; ++e) {
+                const int i = rowof(e), j = c64 + 8 * t + 2 * tig + (e & 1);
+                M1[i * kL64 + j] = be[j] * x[t][e];
+            }
     }
     __syncthreads();
     // B1 <- dY, B2 <- U for the second half
     load_rows<D, LD, 512>(B1, dy, b, t0, nv, h, T, H, nullptr, tid);
     load_rec<D, LD, 512>(B2, ws + w.U + r * kCB * D, tid);
-    // 5. dA = -T^T dT T^T (strictly lower) -> M1
+    // 5. dA = -(T^T dT) T^T, strictly lower -> M1
     {
-        float x[8];
+        float x[2][4];
+        zero_acc(x);
+        wmma_acc(x, kCB, r0, c64, aT(Tm), bR(M1, kL64), lane);
 #pragma unroll
-        for (int n = 0; n < 8; ++n) x[n] = 0.f;
-        mm_nn_str<8>(x, Tm + i, kL64, M1 + g, kL64, 8, kCB);
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int n = 0; n < 8; ++n) M2[i * kL64 + g + 8 * n] = x[n];
+            for (int e = 0; e < 4; ++e) M2[rowof(e) * kL64 + c64 + 8 * t + 2 * tig + (e & 1)] = x[t][e];
     }
     __syncthreads();
     {
-        float x[8];
+        float x[2][4];
+        zero_acc(x);
+        wmma_acc(x, kCB, r0, c64, aR(M2, kL64), bT(Tm, kL64), lane);
 #pragma unroll
-        for (int n = 0; n < 8; ++n) x[n] = 0.f;
-        mm_nt<8, false>(x, M2 + i * kL64, Tm + g * kL64, 8 * kL64, kCB);
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int n = 0; n < 8; ++n) M1[i * kL64 + g + 8 * n] = (g + 8 * n < i) ? -x[n] : 0.f;
+            for (int e = 0; e < 4; ++e) {
+                const int i = rowof(e), j = c64 + 8 * t + 2 * tig + (e & 1);
+                M1[i * kL64 + j] = j < i ? -x[t][e] : 0.f;
+            }
     }
-    // 6. G1 = dY S^T: dq^ = scale gam G1, gam d gam += scale gam q^ . G1
-    __syncthreads();  // B1, B2 = dY, U; B3 free
-    gemm_nt_glob<D>(B3, LD, B1, LD, Sg, 1.f, tid >> 5, lane);
-    __syncthreads();
+    // 6. G1 = dY S^T: dq^ = scale gam G1, q^ . G1 for d gam
     {
-        float x[NC];
+        float x[CT][4];
+        zero_acc(x);
+        const float* sg = Sg;
+        wmma_acc(x, D, r0, cD, aR(B1, LD), [sg](int kk, int n) { return __ldg(sg + (size_t)n * D + kk); }, lane);
+        float lo = 0.f, hi = 0.f;
 #pragma unroll
-        for (int n = 0; n < NC; ++n) x[n] = B3[i * LD + col(n)];
-        float p = 0.f;
+        for (int t = 0; t < CT; ++t)
 #pragma unroll
-        for (int n = 0; n < NC; ++n) {
-            dqh[n] = scale * gi * x[n];
-            p = fmaf(QH[i * LD + col(n)], x[n], p);
-        }
-        dlg += scale * gi * row8_sum(p);
+            for (int e = 0; e < 4; ++e) {
+                const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
+                dqa[t][e] = scale * gam[i] * x[t][e];
+                const float pv = QH[i * LD + n] * x[t][e];
+                if (e < 2) lo += pv; else hi += pv;
+            }
+        row_add(r_g1, lo, hi);
     }
-    // 7. G2 = U dS'^T: dk^ += (gC / gam) G2; dr = k^ . G2 = d(gC / gam_i)
-    __syncthreads();
-    gemm_nt_glob<D>(B3, LD, B2, LD, dSg, 1.f, tid >> 5, lane);
-    __syncthreads();
+    // 7. G2 = U dS'^T: dk^ += (gC / gam) G2, k^ . G2 = d (gC / gam_i); gC <S, dS'>
     {
-        float x[NC];
+        float x[CT][4];
+        zero_acc(x);
+        const float* dsg = dSg;
+        wmma_acc(x, D, r0, cD, aR(B2, LD), [dsg](int kk, int n) { return __ldg(dsg + (size_t)n * D + kk); }, lane);
+        float lo = 0.f, hi = 0.f;
 #pragma unroll
-        for (int n = 0; n < NC; ++n) x[n] = B3[i * LD + col(n)];
-        float p = 0.f;
+        for (int t = 0; t < CT; ++t)
 #pragma unroll
-        for (int n = 0; n < NC; ++n) {
-            dkh[n] = fmaf(dec, x[n], dkh[n]);
-            p = fmaf(KH[i * LD + col(n)], x[n], p);
-        }
-        const float dr = row8_sum(p);  // d (gC / gam_i)
-        dlg -= dr * dec;
-        // gC d gC: sum over rows of dr gC / gam_i, plus gC <S, dS'>
+            for (int e = 0; e < 4; ++e) {
+                const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
+                dka[t][e] = fmaf(expf(Lg[kCB - 1] - Lg[i]), x[t][e], dka[t][e]);
+                const float pv = KH[i * LD + n] * x[t][e];
+                if (e < 2) lo += pv; else hi += pv;
+            }
+        row_add(r_dr, lo, hi);
         float s = 0.f;
         for (int e = tid; e < D * D / 4; e += 512) {
-            const float4 a = __ldg(reinterpret_cast<const float4*>(Sg) + e);
-            const float4 d = __ldg(reinterpret_cast<const float4*>(dSg) + e);
-            s = fmaf(a.x, d.x, fmaf(a.y, d.y, fmaf(a.z, d.z, fmaf(a.w, d.w, s))));
+            const float4 a4 = __ldg(reinterpret_cast<const float4*>(Sg) + e);
+            const float4 d4 = __ldg(reinterpret_cast<const float4*>(dSg) + e);
+            s = fmaf(a4.x, d4.x, fmaf(a4.y, d4.y, fmaf(a4.z, d4.z, fmaf(a4.w, d4.w, s))));
         }
-        s = s * gC + ((tid & 7) == 0 ? dr * dec : 0.f);
         s = warp_sum(s);
-        if (lane == 0) atomicAdd(red, s);
+        if (lane == 0) atomicAdd(red, s * gC);
     }
-    __syncthreads();  // M1 = dA complete; B1, B2 = dY, U
+    __syncthreads();  // M1 = dA
     // 8. dP = dY U^T (lower-incl); the scalar terms of dA and dP; E and F in place
-    float rowM = 0.f;
     {
-        float x[8];
+        float x[2][4];
+        zero_acc(x);
+        wmma_acc(x, D, r0, c64, aR(B1, LD), bT(B2, LD), lane);
+        const float* Atg = ws + w.At + r * kCB * kCB;
+        const float* Pg = ws + w.P + r * kCB * kCB;
+        float mlo = 0.f, mhi = 0.f, plo = 0.f, phi = 0.f;
+        float cs[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-        for (int n = 0; n < 8; ++n) x[n] = 0.f;
-        mm_nt<8, false>(x, B1 + i * LD, B2 + g * LD, 8 * LD, D);
-        const float* Atg = ws + w.At + r * kCB * kCB + i * kCB;
-        const float* Pg = ws + w.P + r * kCB * kCB + i * kCB;
-        float pbe = 0.f;
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int n = 0; n < 8; ++n) {
-            const int j = g + 8 * n;
-            const float dp = j <= i ? x[n] : 0.f;
-            const float da = M1[i * kL64 + j];
-            const float at = Atg[j];
-            const float mij = da * bi * at + dp * Pg[j];
-            pbe = fmaf(da, at, pbe);
-            rowM += mij;
-            atomicAdd(&colM[j], mij);
-            const float gm = j <= i ? expf(fminf(Lg[i] - Lg[j], 0.f)) : 0.f;
-            M1[i * kL64 + j] = da * bi * gm;        // E
-            M2[i * kL64 + j] = scale * dp * gm;     // F
-        }
-        dbe += row8_sum(pbe);
-        rowM = row8_sum(rowM);
+            for (int e = 0; e < 4; ++e) {
+                const int i = rowof(e), j = c64 + 8 * t + 2 * tig + (e & 1);
+                const float dp = j <= i ? x[t][e] : 0.f;
+                const float da = M1[i * kL64 + j];
+                const float at = Atg[i * kCB + j];
+                const float mij = da * be[i] * at + dp * Pg[i * kCB + j];
+                if (e < 2) { mlo += mij; plo += da * at; } else { mhi += mij; phi += da * at; }
+                cs[t][e & 1] += mij;
+                const float gm = j <= i ? expf(fminf(Lg[i] - Lg[j], 0.f)) : 0.f;
+                M1[i * kL64 + j] = da * be[i] * gm;     // E
+                M2[i * kL64 + j] = scale * dp * gm;     // F
+            }
+        row_add(rowM, mlo, mhi);
+        row_add(r_dbe, plo, phi);
+        // column sums: over the 8 rows-pairs of the quad column (lanes with equal tig)
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                float v0 = cs[t][u];
+                v0 += __shfl_xor_sync(0xffffffffu, v0, 4);
+                v0 += __shfl_xor_sync(0xffffffffu, v0, 8);
+                v0 += __shfl_xor_sync(0xffffffffu, v0, 16);
+                if (gid == 0) atomicAdd(&colM[c64 + 8 * t + 2 * tig + u], v0);
+            }
     }
     __syncthreads();
     // 9. dk^ += E K^ + E^T K^ + F^T Q^;  dq^ += F K^
-    mm_nn_il<NC>(dkh, M1 + i * kL64, 1, KH + 4 * g, LD, 32, kCB);
-    mm_nn_il<NC>(dkh, M1 + i, kL64, KH + 4 * g, LD, 32, kCB);
-    mm_nn_il<NC>(dkh, M2 + i, kL64, QH + 4 * g, LD, 32, kCB);
-    mm_nn_il<NC>(dqh, M2 + i * kL64, 1, KH + 4 * g, LD, 32, kCB);
+    wmma_acc(dka, kCB, r0, cD, aR(M1, kL64), bR(KH, LD), lane);
+    wmma_acc(dka, kCB, r0, cD, aT(M1), bR(KH, LD), lane);
+    wmma_acc(dka, kCB, r0, cD, aT(M2), bR(QH, LD), lane);
+    wmma_acc(dqa, kCB, r0, cD, aR(M2, kL64), bR(KH, LD), lane);
+    // 11a. row dots for the norm backward
+    {
+        float ql = 0.f, qh2 = 0.f, kl = 0.f, kh2 = 0.f;
+#pragma unroll
+        for (int t = 0; t < CT; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
+                const float pq = QH[i * LD + n] * dqa[t][e], pk = KH[i * LD + n] * dka[t][e];
+                if (e < 2) { ql += pq; kl += pk; } else { qh2 += pq; kh2 += pk; }
+            }
+        row_add(r_pq, ql, qh2);
+        row_add(r_pk, kl, kh2);
+    }
+    __syncthreads();
     // 10. d Lg_i = gam_i d gam_i + rowM_i - colM_i (+ gC d gC for the last token); reverse cumsum
-    if ((tid & 7) == 0) dLg[i] = dlg + rowM - colM[i];
+    if (tid < kCB) {
+        const int i = tid;
+        const float dec = expf(Lg[kCB - 1] - Lg[i]);
+        const float dlg = r_dbg[i] * be[i] * gam[i] + scale * gam[i] * r_g1[i] - r_dr[i] * dec;
+        dLg[i] = dlg + rowM[i] - colM[i];
+        atomicAdd(red, r_dr[i] * dec);
+    }
     __syncthreads();
     if (tid == 0) {
-        float acc = red[0];  // gC d gC enters at the last token
+        float acc = red[0];
         for (int ii = kCB - 1; ii >= 0; --ii) {
             acc += dLg[ii];
             dLg[ii] = acc;  // d ln(alpha_ii)
         }
     }
     __syncthreads();
-    if ((tid & 7) == 0 && i < nv) {
+    if (tid < nv) {
+        const int i = tid;
         const size_t o = tok_off(b, t0 + i, h, T, H);
         dalpha[o] = dLg[i] / alpha[o];
-        dbeta[o] = dbe;
+        dbeta[o] = r_dbe[i] + r_dbg[i] * gam[i];
     }
-    // 11. norm backward: dx = r (dx^ - x^ (x^ . dx^))
-    {
-        float pq = 0.f, pk = 0.f;
+    // 11b. dx = r (dx^ - x^ (x^ . dx^))
 #pragma unroll
-        for (int n = 0; n < NC; ++n) {
-            pq = fmaf(QH[i * LD + col(n)], dqh[n], pq);
-            pk = fmaf(KH[i * LD + col(n)], dkh[n], pk);
-        }
-        pq = row8_sum(pq);
-        pk = row8_sum(pk);
-        if (i < nv) {
-            const size_t o = tok_off(b, t0 + i, h, T, H) * D;
-            const float rqi = l2norm ? rq[i] : 1.f, rki = l2norm ? rk[i] : 1.f;
+    for (int t = 0; t < CT; ++t)
 #pragma unroll
-            for (int n = 0; n < NC; ++n) {
-                const float gq = l2norm ? rqi * (dqh[n] - QH[i * LD + col(n)] * pq) : dqh[n];
-                const float gk = l2norm ? rki * (dkh[n] - KH[i * LD + col(n)] * pk) : dkh[n];
-                dq[o + col(n)] = from_f32<Tin>(gq);
-                dk[o + col(n)] = from_f32<Tin>(gk);
+        for (int e = 0; e < 4; ++e) {
+            const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
+            if (i < nv) {
+                const size_t o = tok_off(b, t0 + i, h, T, H) * D + n;
+                const float gq = l2norm ? rq[i] * (dqa[t][e] - QH[i * LD + n] * r_pq[i]) : dqa[t][e];
+                const float gk = l2norm ? rk[i] * (dka[t][e] - KH[i * LD + n] * r_pk[i]) : dka[t][e];
+                dq[o] = from_f32<Tin>(gq);
+                dk[o] = from_f32<Tin>(gk);
             }
         }
-    }
 }
 
 template <int D, typename Tin>
