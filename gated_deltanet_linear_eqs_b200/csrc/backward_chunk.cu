@@ -249,7 +249,7 @@ __device__ __forceinline__ float row8_sum(float x) {
 template <int D>
 struct PrepB {
     static constexpr int LD = D + 4;
-    static constexpr int BYTES = (3 * kCB * LD + 2 * kCB * kL64 + 5 * kCB + 768) * 4;
+    static constexpr int BYTES = (2 * kCB * LD + 2 * kCB * kL64 + 5 * kCB + 768) * 4;  // two CTAs per SM
 };
 
 template <int D, typename Tin>
@@ -262,8 +262,8 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
     extern __shared__ float smf[];
     float* qh = smf;
     float* kh = qh + kCB * LD;
-    float* vs = kh + kCB * LD;
-    float* Am = vs + kCB * LD;
+    float* vs = qh;  // V takes Q's place once the Gram products are done
+    float* Am = kh + kCB * LD;
     float* Tm = Am + kCB * kL64;
     float* rq = Tm + kCB * kL64;
     float* rk = rq + kCB;
@@ -280,7 +280,6 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
 
     load_rows<D, LD, 256>(qh, q, b, t0, nv, h, T, H, nullptr, tid);
     load_rows<D, LD, 256>(kh, k, b, t0, nv, h, T, H, nullptr, tid);
-    load_rows<D, LD, 256>(vs, v, b, t0, nv, h, T, H, nullptr, tid);
     if (tid < kCB) {
         const size_t o = tok_off(b, t0 + tid, h, T, H);
         be[tid] = tid < nv ? beta[o] : 0.f;
@@ -331,6 +330,7 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
         }
     }
     __syncthreads();
+    load_rows<D, LD, 256>(vs, v, b, t0, nv, h, T, H, nullptr, tid);  // Q is no longer read
     // T = (I + A)^-1 by 16 x 16 blocks: the diagonal blocks by forward substitution (one column
     // per thread), then T_ij = -T_ii sum_{j <= m < i} A_im T_mj for block distance 1, 2, 3
     if (tid < kCB) {
@@ -412,27 +412,59 @@ struct ChainB {
     static constexpr int REV_BYTES = (D * LDS + 3 * kCB * LD + kCB * kL64 + 2 * kCB * LDS + 3 * kCB) * 4;
 };
 
+// Per-thread registers holding one chunk's operands between their load and their store to shared
+// memory: the copy for the next chunk is issued before the current chunk's arithmetic.
+template <int D>
+struct ChunkRegs {
+    static constexpr int PW = kCB * D / 4 / 256;    // float4 of W
+    static constexpr int PP = kCB * kCB / 4 / 256;  // float4 of P
+    static constexpr int PR = kCB * D / 8 / 256;    // 8-element groups of a token tile
+    float4 w[PW], pm[PP];
+    float k[PR][8], q[PR][8], y[8];
+};
+
 // Forward: S^c and U of every chunk, 32 state columns per CTA.
 template <int D, typename Tin>
 __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const float* __restrict__ s0,
                                                 float* __restrict__ ws, const BwdChunkWs w, int T, int H,
                                                 int nch) {
     using L = ChainB<D>;
+    using R = ChunkRegs<D>;
     constexpr int LDS = L::LDS, LD = L::LD;
     extern __shared__ float smf[];
     float* Ss = smf;
     float* Wt = Ss + D * LDS;
-    float* Kt = Wt + kCB * LD;
+    float* Kt = Wt + kCB * LD;   // raw K rows
     float* Us = Kt + kCB * LD;
     float* dec = Us + kCB * LDS;  // gC / gam
     float* rks = dec + kCB;
     constexpr int nsl = D / kNVB;
     const int jsl = blockIdx.x % nsl, h = (blockIdx.x / nsl) % H, b = blockIdx.x / (nsl * H);
     const int col0 = jsl * kNVB, tid = threadIdx.x;
+    const int iu = tid >> 2, nu = (tid & 3) * 8;  // U element block of this thread
+    R rg;
+    auto fetch = [&](int c) {
+        const size_t r = ((size_t)b * nch + c) * H + h;
+        const float4* Wg = reinterpret_cast<const float4*>(ws + w.W + r * kCB * D);
+#pragma unroll
+        for (int u = 0; u < R::PW; ++u) rg.w[u] = Wg[tid + u * 256];
+        const int t0c = c * kCB, nvc = min(kCB, T - t0c);
+#pragma unroll
+        for (int u = 0; u < R::PR; ++u) {
+            const int e = (tid + u * 256) * 8, i = e / D, m = e % D;
+            if (i < nvc) ld8(k + tok_off(b, t0c + i, h, T, H) * D + m, rg.k[u]);
+            else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) rg.k[u][j] = 0.f;
+            }
+        }
+        ld8(ws + w.Ut + r * kCB * D + (size_t)iu * D + col0 + nu, rg.y);  // Ut of this thread's U block
+    };
     for (int e = tid; e < D * kNVB; e += 256) {
         const int m = e / kNVB, n = e % kNVB;
         Ss[m * LDS + n] = s0 ? s0[(((size_t)b * H + h) * D + m) * D + col0 + n] : 0.f;
     }
+    fetch(0);
     for (int c = 0; c < nch; ++c) {
         const size_t r = ((size_t)b * nch + c) * H + h;
         __syncthreads();
@@ -441,39 +473,49 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
             const int m = e / kNVB, n = e % kNVB;
             Sg[(size_t)m * D + col0 + n] = Ss[m * LDS + n];
         }
+#pragma unroll
+        for (int u = 0; u < R::PW; ++u) {
+            const int e = (tid + u * 256) * 4;
+            *reinterpret_cast<float4*>(Wt + (e / D) * LD + e % D) = rg.w[u];
+        }
+#pragma unroll
+        for (int u = 0; u < R::PR; ++u) {
+            const int e = (tid + u * 256) * 8;
+            st8(Kt + (e / D) * LD + e % D, rg.k[u], 1.f);
+        }
+        float ut[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ut[j] = rg.y[j];
         const float* SCg = ws + w.SC + r * 256;
         if (tid < kCB) {
             dec[tid] = expf(SCg[128 + kCB - 1] - SCg[128 + tid]);
             rks[tid] = SCg[64 + tid];
         }
         const float gC = expf(SCg[128 + kCB - 1]);
-        load_rec<D, LD, 256>(Wt, ws + w.W + r * kCB * D, tid);
         __syncthreads();
-        load_rows<D, LD, 256>(Kt, k, b, c * kCB, min(kCB, T - c * kCB), h, T, H, rks, tid);
-        {  // U = Ut - W S: row i, 8 columns
-            const int i = tid >> 2, n0 = (tid & 3) * 8;
+        if (c + 1 < nch) fetch(c + 1);
+        {  // U = Ut - W S: row iu, 8 columns
             float acc[8];
 #pragma unroll
             for (int n = 0; n < 8; ++n) acc[n] = 0.f;
-            mm_nn<8>(acc, Wt + i * LD, 1, Ss + n0, LDS, D);
-            const float* Utg = ws + w.Ut + r * kCB * D + (size_t)i * D + col0 + n0;
-            float* Ug = ws + w.U + r * kCB * D + (size_t)i * D + col0 + n0;
+            mm_nn<8>(acc, Wt + iu * LD, 1, Ss + nu, LDS, D);
+            float* Ug = ws + w.U + r * kCB * D + (size_t)iu * D + col0 + nu;
 #pragma unroll
             for (int n = 0; n < 8; ++n) {
-                const float u = Utg[n] - acc[n];
-                Us[i * LDS + n0 + n] = u;
+                const float u = ut[n] - acc[n];
+                Us[iu * LDS + nu + n] = u;
                 Ug[n] = u;
             }
         }
         __syncthreads();
-        {  // S = gC S + K^T diag(gC / gam) U
+        {  // S = gC S + K^T diag(rk gC / gam) U
             constexpr int TPR = 256 / D, NC = kNVB / TPR;
             const int m = tid / TPR, n0 = (tid % TPR) * NC;
             float acc[NC];
 #pragma unroll
             for (int n = 0; n < NC; ++n) acc[n] = 0.f;
             for (int i = 0; i < kCB; ++i) {
-                const float x = Kt[i * LD + m] * dec[i];
+                const float x = Kt[i * LD + m] * (dec[i] * rks[i]);
                 const float4* ur = reinterpret_cast<const float4*>(Us + i * LDS + n0);
 #pragma unroll
                 for (int n = 0; n < NC / 4; ++n) {
