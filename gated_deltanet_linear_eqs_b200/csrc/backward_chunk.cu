@@ -409,7 +409,7 @@ struct ChainB {
     static constexpr int LDS = kNVB + 4;
     static constexpr int LD = D + 4;
     static constexpr int FWD_BYTES = (D * LDS + 2 * kCB * LD + kCB * LDS + 2 * kCB) * 4;
-    static constexpr int REV_BYTES = (D * LDS + 3 * kCB * LD + kCB * kL64 + 2 * kCB * LDS + 3 * kCB) * 4;
+    static constexpr int REV_BYTES = (D * LDS + 2 * kCB * LD + 2 * kCB * LDS + 3 * kCB) * 4;
 };
 
 // Per-thread registers holding one chunk's operands between their load and their store to shared
@@ -530,21 +530,20 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
     }
 }
 
-// Reverse: dS' and dU of every chunk, and dS0, 32 state columns per CTA.
+// Reverse: dS' and dU of every chunk, and dS0, 32 state columns per CTA.  The dU step reads K and
+// P, the dS step Q and W: the two pairs take turns in the same two tiles (two CTAs per SM).
 template <int D, typename Tin>
-__global__ void __launch_bounds__(256) bwdc_rev(const Tin* __restrict__ q, const Tin* __restrict__ k,
-                                                const Tin* __restrict__ dy, const float* __restrict__ ds_final,
-                                                float* __restrict__ ds0, float* __restrict__ ws,
-                                                const BwdChunkWs w, int T, int H, int nch, float scale) {
+__global__ void __launch_bounds__(256, 2) bwdc_rev(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                                   const Tin* __restrict__ dy, const float* __restrict__ ds_final,
+                                                   float* __restrict__ ds0, float* __restrict__ ws,
+                                                   const BwdChunkWs w, int T, int H, int nch, float scale) {
     using L = ChainB<D>;
     constexpr int LDS = L::LDS, LD = L::LD;
     extern __shared__ float smf[];
     float* Ss = smf;                 // dS slice
-    float* Kt = Ss + D * LDS;        // K^
-    float* Qt = Kt + kCB * LD;       // scale gam Q^
-    float* Wt = Qt + kCB * LD;
-    float* Pm = Wt + kCB * LD;
-    float* dYs = Pm + kCB * kL64;
+    float* X1 = Ss + D * LDS;        // K^ (dU step), then scale gam Q^ (dS step)
+    float* X2 = X1 + kCB * LD;       // P (dU step, row stride kL64), then W (dS step)
+    float* dYs = X2 + kCB * LD;
     float* dUs = dYs + kCB * LDS;
     float* dec = dUs + kCB * LDS;    // gC / gam
     float* ysc = dec + kCB;          // scale gam rq
@@ -571,8 +570,7 @@ __global__ void __launch_bounds__(256) bwdc_rev(const Tin* __restrict__ q, const
             rks[tid] = SCg[64 + tid];
         }
         const float gC = expf(SCg[128 + kCB - 1]);
-        load_rec<D, LD, 256>(Wt, ws + w.W + r * kCB * D, tid);
-        load_rec<kCB, kL64, 256>(Pm, ws + w.P + r * kCB * kCB, tid);
+        load_rec<kCB, kL64, 256>(X2, ws + w.P + r * kCB * kCB, tid);
         {  // dY slice: 64 rows x 32 columns, one 8-element group per thread
             const int i = tid >> 2, n = (tid & 3) * 8, t = c * kCB + i;
             float x[8];
@@ -585,16 +583,15 @@ __global__ void __launch_bounds__(256) bwdc_rev(const Tin* __restrict__ q, const
         }
         __syncthreads();
         const int nvc = min(kCB, T - c * kCB);
-        load_rows<D, LD, 256>(Kt, k, b, c * kCB, nvc, h, T, H, rks, tid);
-        load_rows<D, LD, 256>(Qt, q, b, c * kCB, nvc, h, T, H, ysc, tid);
+        load_rows<D, LD, 256>(X1, k, b, c * kCB, nvc, h, T, H, rks, tid);
         __syncthreads();
         {  // dU = diag(gC / gam) K^ dS + P^T dY
             const int i = tid >> 2, n0 = (tid & 3) * 8;
             float a1[8], a2[8];
 #pragma unroll
             for (int n = 0; n < 8; ++n) a1[n] = a2[n] = 0.f;
-            mm_nn<8>(a1, Kt + i * LD, 1, Ss + n0, LDS, D);
-            mm_nn<8>(a2, Pm + i, kL64, dYs + n0, LDS, kCB);
+            mm_nn<8>(a1, X1 + i * LD, 1, Ss + n0, LDS, D);
+            mm_nn<8>(a2, X2 + i, kL64, dYs + n0, LDS, kCB);
             float* dUg = ws + w.dU + r * kCB * D + (size_t)i * D + col0 + n0;
 #pragma unroll
             for (int n = 0; n < 8; ++n) {
@@ -604,6 +601,9 @@ __global__ void __launch_bounds__(256) bwdc_rev(const Tin* __restrict__ q, const
             }
         }
         __syncthreads();
+        load_rows<D, LD, 256>(X1, q, b, c * kCB, nvc, h, T, H, ysc, tid);
+        load_rec<D, LD, 256>(X2, ws + w.W + r * kCB * D, tid);
+        __syncthreads();
         {  // dS = gC dS + (scale gam Q^)^T dY - W^T dU
             constexpr int TPR = 256 / D, NC = kNVB / TPR;
             const int m = tid / TPR, n0 = (tid % TPR) * NC;
@@ -611,7 +611,7 @@ __global__ void __launch_bounds__(256) bwdc_rev(const Tin* __restrict__ q, const
 #pragma unroll
             for (int n = 0; n < NC; ++n) acc[n] = 0.f;
             for (int i = 0; i < kCB; ++i) {
-                const float xq = Qt[i * LD + m], xw = Wt[i * LD + m];
+                const float xq = X1[i * LD + m], xw = X2[i * LD + m];
                 const float4* yr = reinterpret_cast<const float4*>(dYs + i * LDS + n0);
                 const float4* ur = reinterpret_cast<const float4*>(dUs + i * LDS + n0);
 #pragma unroll
