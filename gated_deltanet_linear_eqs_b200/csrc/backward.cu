@@ -1,4 +1,6 @@
-// backward.cu -- reverse-mode gradients of the gated delta rule.
+// backward.cu -- reverse-mode gradients of the gated delta rule, token-loop form: the path of
+// gdn_backward_noalloc, whose scratch is a fixed array (gdn_backward runs the chunked form in
+// backward_chunk.cu).
 //
 // Forward (Qwen3.8-Flash-Next summary, picx.dev, "Theoretical foundations", eqs. (1)-(4)), per
 // head with normalised kh, qh:  St = a S;  e = v - St^T kh;  S' = St + b kh e^T;  y = scale S'^T qh.
@@ -483,7 +485,7 @@ size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv) {
     return (chunks + kC) * (size_t)B * H * dk * dv * sizeof(float);
 }
 
-cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st) {
+cudaError_t launch_backward_tokenloop(const BackwardArgs& a, cudaStream_t st) {
     if (a.dtype == GDN_BF16)
         return a.dkdim == 128 ? launch_t<128, __nv_bfloat16>(a, st) : launch_t<64, __nv_bfloat16>(a, st);
     return a.dkdim == 128 ? launch_t<128, float>(a, st) : launch_t<64, float>(a, st);

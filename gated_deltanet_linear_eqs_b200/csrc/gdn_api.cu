@@ -244,7 +244,7 @@ int gdn_backward_noalloc(const void* q, const void* k, const void* v, const floa
     gdn::BackwardArgs a{q, k, v, alpha, beta, s0, dy, ds_final, dq, dk_out, dv_out, dalpha,
                         dbeta, ds0, B, T, H, dk, dv, dtype, scale, l2norm_qk ? 1 : 0, scratch,
                         gdn::kBackwardFixedScratchBytes, dev.status};
-    return map_cuda(gdn::launch_backward(a, static_cast<cudaStream_t>(stream)));
+    return map_cuda(gdn::launch_backward_tokenloop(a, static_cast<cudaStream_t>(stream)));
 }
 
 size_t gdn_backward_noalloc_max_workspace(void) { return gdn::kBackwardFixedScratchBytes; }

@@ -65,7 +65,8 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_prefill_phase(const PrefillArgs& a, int phase, cudaStream_t st);
 // Token-by-token prefill on CUDA cores (used for fp32 inputs).
 cudaError_t launch_prefill_seq(const PrefillArgs& a, cudaStream_t st);
-cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t st);
+// The token-loop backward (one fp32 checkpoint per chunk, each chunk replayed token by token).
+cudaError_t launch_backward_tokenloop(const BackwardArgs& a, cudaStream_t st);
 
 // Workspace of the token-loop backward (chunk-start states), bytes; the fixed-scratch entry point
 // runs that path.
