@@ -86,33 +86,6 @@ __device__ __forceinline__ void mm_nn(float* acc, const float* a, int as, const 
     }
 }
 
-// acc[4u + e] += sum_k a[k * as] * b[k * bs + cs * u + e]: NC / 4 column chunks of 4, cs apart
-template <int NC>
-__device__ __forceinline__ void mm_nn_il(float* acc, const float* a, int as, const float* b, int bs, int cs, int K) {
-#pragma unroll 2
-    for (int k = 0; k < K; ++k) {
-        const float x = a[k * as];
-#pragma unroll
-        for (int u = 0; u < NC / 4; ++u) {
-            const float4 y = *reinterpret_cast<const float4*>(b + (size_t)k * bs + cs * u);
-            acc[4 * u + 0] = fmaf(x, y.x, acc[4 * u + 0]);
-            acc[4 * u + 1] = fmaf(x, y.y, acc[4 * u + 1]);
-            acc[4 * u + 2] = fmaf(x, y.z, acc[4 * u + 2]);
-            acc[4 * u + 3] = fmaf(x, y.w, acc[4 * u + 3]);
-        }
-    }
-}
-// acc[n] += sum_k a[k * as] * b[k * bs + n * step]
-template <int NC>
-__device__ __forceinline__ void mm_nn_str(float* acc, const float* a, int as, const float* b, int bs, int step, int K) {
-#pragma unroll 4
-    for (int k = 0; k < K; ++k) {
-        const float x = a[k * as];
-#pragma unroll
-        for (int n = 0; n < NC; ++n) acc[n] = fmaf(x, b[(size_t)k * bs + n * step], acc[n]);
-    }
-}
-
 // acc[n] += sum_k a[k] * b[n * bs + k], k contiguous in both (16-byte aligned), K % 4 == 0.
 // GLOBAL: b is read-only global memory (read through the non-coherent cache).
 template <int NC, bool GLOBAL>
@@ -235,14 +208,6 @@ __device__ __forceinline__ void gemm_nt_glob(float* C, int ldc, const float* A, 
         c[8 * ldc] = s * acc[t][2];
         c[8 * ldc + 1] = s * acc[t][3];
     }
-}
-
-// sum over the 8 consecutive lanes that share a row
-__device__ __forceinline__ float row8_sum(float x) {
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
-    x += __shfl_xor_sync(0xffffffffu, x, 4);
-    return x;
 }
 
 // ============================================================================ bwdc_prep
