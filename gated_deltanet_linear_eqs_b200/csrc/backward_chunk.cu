@@ -177,39 +177,6 @@ __device__ __forceinline__ void mma_tf32(float* c, uint32_t a0, uint32_t a1, uin
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// C[64][D] (shared, row stride ldc) = s * A G^T with A [64][D] shared (row stride lda) and G [D][D]
-// row-major global: one 16 x (D/4) block of C per warp (16 warps), tf32 MMAs, fp32 accumulation.
-template <int D>
-__device__ __forceinline__ void gemm_nt_glob(float* C, int ldc, const float* A, int lda,
-                                             const float* __restrict__ G, float s, int warp, int lane) {
-    constexpr int CT = D / 32;  // 8-column tiles per warp
-    const int rt = warp & 3, ct0 = (warp >> 2) * CT;
-    const int gid = lane >> 2, tig = lane & 3;
-    float acc[CT][4];
-#pragma unroll
-    for (int t = 0; t < CT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-    const float* alo = A + (rt * 16 + gid) * lda + tig;
-    const float* ahi = alo + 8 * lda;
-#pragma unroll 2
-    for (int k0 = 0; k0 < D; k0 += 8) {
-        const uint32_t a0 = to_tf32(alo[k0]), a1 = to_tf32(ahi[k0]);
-        const uint32_t a2 = to_tf32(alo[k0 + 4]), a3 = to_tf32(ahi[k0 + 4]);
-#pragma unroll
-        for (int t = 0; t < CT; ++t) {
-            const float* g = G + (size_t)((ct0 + t) * 8 + gid) * D + k0 + tig;
-            mma_tf32(acc[t], a0, a1, a2, a3, to_tf32(__ldg(g)), to_tf32(__ldg(g + 4)));
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < CT; ++t) {
-        float* c = C + (rt * 16 + gid) * ldc + (ct0 + t) * 8 + 2 * tig;
-        c[0] = s * acc[t][0];
-        c[1] = s * acc[t][1];
-        c[8 * ldc] = s * acc[t][2];
-        c[8 * ldc + 1] = s * acc[t][3];
-    }
-}
-
 // ============================================================================ bwdc_prep
 template <int D>
 struct PrepB {
@@ -639,6 +606,24 @@ __device__ __forceinline__ float quad_sum(float x) {
     return x;
 }
 
+// acc += A G^T for the warp's tiles, G [D][D] fp32 in global memory, staged in `buf` (row stride
+// LD) 64 rows at a time: the warps whose output columns fall in the staged rows compute.  Every
+// thread of the CTA calls it.
+template <int D, int LD, int CT, typename FA>
+__device__ __forceinline__ void gemm_staged(float (&acc)[CT][4], FA a, const float* G, float* buf, int r0,
+                                            int cD, int tid, int lane) {
+    for (int hh = 0; hh < D / 64; ++hh) {
+        __syncthreads();
+        load_rec<D, LD, 512>(buf, G + (size_t)hh * 64 * D, tid);
+        __syncthreads();
+        if (cD / 64 == hh) {
+            const float* bb = buf;
+            const int off = hh * 64;
+            wmma_acc(acc, D, r0, cD, a, [bb, off](int kk, int n) { return bb[(n - off) * LD + kk]; }, lane);
+        }
+    }
+}
+
 template <int D, typename Tin>
 __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                      const Tin* __restrict__ v, const Tin* __restrict__ dy,
@@ -737,8 +722,17 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
             }
         row_add(r_dbe, lo, hi);
     }
-    // 2. dW = -dU S^T
-    gemm_nt_glob<D>(B3, LD, B1, LD, Sg, -1.f, warp, lane);
+    // 2. dW = -dU S^T (S staged through M1..M2, free until step 4)
+    {
+        static_assert(2 * kCB * kL64 >= kCB * LD, "staging space");
+        float x[CT][4];
+        zero_acc(x);
+        gemm_staged<D, LD>(x, aR(B1, LD), Sg, M1, r0, cD, tid, lane);
+#pragma unroll
+        for (int t = 0; t < CT; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) B3[rowof(e) * LD + cD + 8 * t + 2 * tig + (e & 1)] = -x[t][e];
+    }
     __syncthreads();
     // 3. Z2 = T^T dW: dk^ = diag(beta gam) Z2, d(beta gam) = k^ . Z2
     {
@@ -804,8 +798,7 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
     {
         float x[CT][4];
         zero_acc(x);
-        const float* sg = Sg;
-        wmma_acc(x, D, r0, cD, aR(B1, LD), [sg](int kk, int n) { return __ldg(sg + (size_t)n * D + kk); }, lane);
+        gemm_staged<D, LD>(x, aR(B1, LD), Sg, B3, r0, cD, tid, lane);  // S through B3 (free)
         float lo = 0.f, hi = 0.f;
 #pragma unroll
         for (int t = 0; t < CT; ++t)
@@ -822,8 +815,7 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
     {
         float x[CT][4];
         zero_acc(x);
-        const float* dsg = dSg;
-        wmma_acc(x, D, r0, cD, aR(B2, LD), [dsg](int kk, int n) { return __ldg(dsg + (size_t)n * D + kk); }, lane);
+        gemm_staged<D, LD>(x, aR(B2, LD), dSg, B3, r0, cD, tid, lane);  // dS' through B3
         float lo = 0.f, hi = 0.f;
 #pragma unroll
         for (int t = 0; t < CT; ++t)
