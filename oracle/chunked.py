@@ -66,3 +66,117 @@ def forward_chunked(q, k, v, alpha, beta, s0=None, C=64, scale=1.0, l2norm=True,
                 S = gam[-1] * S + (Gam[-1][:, None] * K).T @ U
             sf[b, h] = S
     return y, sf
+
+
+def backward_chunked(q, k, v, alpha, beta, s0=None, dy=None, ds_final=None, C=64, scale=1.0,
+                     l2norm=True, eps=EPS):
+    """Gradients of L = <dy, y> + <ds_final, S_T> in the chunked form; same contract as
+    ``oracle.backward`` (dict of dq, dk, dv, dalpha, dbeta, ds0).
+
+    Per chunk, with the forward above written as U = Ut - W S,
+    Y = scale (diag(gamma) Qh S + P U) (P = Qh Kh^T * Gam, lower incl.) and
+    S' = gamma_n S + Kh^T diag(gamma_n / gamma) U, the reverse pass is:
+      - a chain over the chunks in reverse (the forward chain transposed):
+            dU = diag(gamma_n / gamma) Kh dS' + scale P^T dY
+            dS = gamma_n dS' + scale Qh^T diag(gamma) dY - W^T dU
+      - then, per chunk, from S, dS', U and dU alone:
+            dV = diag(beta) T^T dU,  dW = -dU S^T,
+            dT = dU (diag(beta) V)^T + dW (diag(beta gamma) Kh)^T,
+            dA = -T^T dT T^T restricted to A's strictly lower support,
+            dP = scale dY U^T on the lower triangle (diagonal included),
+            dQh = scale diag(gamma) dY S^T + (dP * Gam) Kh,
+            dKh = diag(beta gamma) T^T dW + diag(gamma_n / gamma) U dS'^T + E Kh + E^T Kh
+                  + (dP * Gam)^T Qh,   E = dA * beta_i Gam_ij,
+            dbeta and d ln(alpha) through gamma, gamma_n and Gam (d G_i collects row i minus
+            column i of dA * A + dP * (Qh Kh^T * Gam), and d ln(alpha) is the reverse cumsum
+            of d G), and the L2-norm backward dx = (dxh - xh <xh, dxh>) / sqrt(|x|^2 + eps).
+    """
+    q, k, v, alpha, beta = (np.asarray(x, dtype=np.float64) for x in (q, k, v, alpha, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dy = np.zeros((B, T, H, dv)) if dy is None else np.asarray(dy, dtype=np.float64)
+    dsf = np.zeros((B, H, dk, dv)) if ds_final is None else np.asarray(ds_final, dtype=np.float64)
+    out = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v),
+               dalpha=np.zeros_like(alpha), dbeta=np.zeros_like(beta), ds0=np.zeros((B, H, dk, dv)))
+    for b in range(B):
+        for h in range(H):
+            chunks = []
+            for t0 in range(0, T, C):
+                t1 = min(T, t0 + C)
+                n = t1 - t0
+                qr, kr = q[b, t0:t1, h], k[b, t0:t1, h]
+                rq = 1 / np.sqrt(np.sum(qr * qr, axis=-1) + eps) if l2norm else np.ones(n)
+                rk = 1 / np.sqrt(np.sum(kr * kr, axis=-1) + eps) if l2norm else np.ones(n)
+                Qh, Kh = rq[:, None] * qr, rk[:, None] * kr
+                G = np.cumsum(np.log(alpha[b, t0:t1, h]))
+                diff = G[:, None] - G[None, :]
+                lower_incl = np.tril(np.ones((n, n), dtype=bool))
+                Gam = np.where(lower_incl, np.exp(np.where(lower_incl, diff, 0.0)), 0.0)
+                gam = np.exp(G)
+                be = beta[b, t0:t1, h]
+                At = np.tril((Kh @ Kh.T) * Gam, k=-1)          # A / beta_i
+                A = be[:, None] * At
+                Tm = solve_triangular(np.eye(n) + A, np.eye(n), lower=True, unit_diagonal=True)
+                W = Tm @ ((be * gam)[:, None] * Kh)
+                Ut = Tm @ (be[:, None] * v[b, t0:t1, h])
+                QK = (Qh @ Kh.T) * Gam                          # P / scale
+                dec = np.exp(G[-1] - G)                         # gamma_n / gamma
+                chunks.append(dict(t0=t0, t1=t1, Qh=Qh, Kh=Kh, rq=rq, rk=rk, qr=qr, kr=kr, V=v[b, t0:t1, h],
+                                   be=be, gam=gam, gn=gam[-1], dec=dec, Gam=Gam, At=At, A=A, Tm=Tm, W=W,
+                                   Ut=Ut, QK=QK, dY=dy[b, t0:t1, h]))
+            S = np.zeros((dk, dv)) if s0 is None else np.array(s0[b, h], dtype=np.float64)
+            for c in chunks:                                   # forward chain
+                c["S"] = S
+                c["U"] = c["Ut"] - c["W"] @ S
+                S = c["gn"] * S + c["Kh"].T @ (c["dec"][:, None] * c["U"])
+            dS = dsf[b, h].copy()
+            for c in reversed(chunks):                         # reverse chain
+                c["dSp"] = dS
+                c["dU"] = c["dec"][:, None] * (c["Kh"] @ dS) + scale * c["QK"].T @ c["dY"]
+                dS = c["gn"] * dS + scale * c["Qh"].T @ (c["gam"][:, None] * c["dY"]) - c["W"].T @ c["dU"]
+            out["ds0"][b, h] = dS
+            for c in chunks:                                   # chunk-local gradients
+                S, dSp, U, dU, dY = c["S"], c["dSp"], c["U"], c["dU"], c["dY"]
+                Tm, Kh, Qh, be, gam, Gam = c["Tm"], c["Kh"], c["Qh"], c["be"], c["gam"], c["Gam"]
+                n = len(be)
+                Z1 = Tm.T @ dU
+                dV = be[:, None] * Z1
+                dbe = np.sum(c["V"] * Z1, axis=1)
+                dW = -dU @ S.T
+                Z2 = Tm.T @ dW
+                dKh = (be * gam)[:, None] * Z2
+                dbg = np.sum(Kh * Z2, axis=1)                   # d (beta gamma)
+                dbe += dbg * gam
+                dgam = dbg * be
+                dT = dU @ (be[:, None] * c["V"]).T + dW @ ((be * gam)[:, None] * Kh).T
+                dA = np.tril(-(Tm.T @ dT @ Tm.T), k=-1)
+                G1 = dY @ S.T
+                dQh = scale * gam[:, None] * G1
+                dgam += scale * np.sum(Qh * G1, axis=1)
+                G2 = U @ dSp.T
+                dKh += c["dec"][:, None] * G2
+                ddec = np.sum(Kh * G2, axis=1)                  # d (gamma_n / gamma_i)
+                dgn = np.sum(S * dSp) + np.sum(ddec / gam)
+                dgam -= ddec * c["gn"] / gam ** 2
+                dP = np.tril(scale * (dY @ U.T))
+                E = dA * be[:, None] * Gam
+                F = dP * Gam
+                dKh += E @ Kh + E.T @ Kh + F.T @ Qh
+                dQh += F @ Kh
+                dbe += np.sum(dA * c["At"], axis=1)
+                M = dA * c["A"] + dP * c["QK"]
+                dG = dgam * gam + M.sum(axis=1) - M.sum(axis=0)
+                dG[-1] += dgn * c["gn"]
+                dlna = np.cumsum(dG[::-1])[::-1]
+                t0, t1 = c["t0"], c["t1"]
+                if l2norm:
+                    dq = c["rq"][:, None] * (dQh - Qh * np.sum(Qh * dQh, axis=1, keepdims=True))
+                    dkk = c["rk"][:, None] * (dKh - Kh * np.sum(Kh * dKh, axis=1, keepdims=True))
+                else:
+                    dq, dkk = dQh, dKh
+                out["dq"][b, t0:t1, h] = dq
+                out["dk"][b, t0:t1, h] = dkk
+                out["dv"][b, t0:t1, h] = dV
+                out["dalpha"][b, t0:t1, h] = dlna / alpha[b, t0:t1, h]
+                out["dbeta"][b, t0:t1, h] = dbe
+    return out

@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 
 import oracle
-from oracle.chunked import forward_chunked
+from oracle.chunked import backward_chunked, forward_chunked
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -244,6 +244,25 @@ def test_chunked_form_small_alpha_no_overflow():
     yc, sc = forward_chunked(q, k, v, alpha, beta, S0, C=64)
     assert np.all(np.isfinite(yc)) and np.all(np.isfinite(sc))
     np.testing.assert_allclose(yc, y, rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("C", [16, 64])
+@pytest.mark.parametrize("l2norm", [True, False])
+def test_chunked_backward_matches_reverse_recurrence(C, l2norm):
+    """The chunked backward (the forward chain transposed plus chunk-local gradients, the form the
+    CUDA backward runs) agrees with the token-by-token reverse recurrence: dk != dv, T not a
+    multiple of C, a nonzero dS_final and a scale."""
+    rng = np.random.default_rng(16)
+    q, k, v, alpha, beta, S0 = _rand(rng, 2, 150, 2, 16, 24)
+    if not l2norm:
+        q, k = _l2n(q), _l2n(k)
+    dy = rng.standard_normal((2, 150, 2, 24))
+    dsf = rng.standard_normal((2, 2, 16, 24))
+    ref = oracle.backward(q, k, v, alpha, beta, s0=S0, dy=dy, ds_final=dsf, scale=0.7, l2norm=l2norm)
+    got = backward_chunked(q, k, v, alpha, beta, s0=S0, dy=dy, ds_final=dsf, C=C, scale=0.7,
+                           l2norm=l2norm)
+    for name in ("dq", "dk", "dv", "dalpha", "dbeta", "ds0"):
+        np.testing.assert_allclose(got[name], ref[name], rtol=1e-9, atol=1e-11, err_msg=name)
 
 
 # ------------------------------------------------------------------ backward pins
