@@ -86,17 +86,15 @@ __device__ __forceinline__ void mm_nn(float* acc, const float* a, int as, const 
     }
 }
 
-// acc[n] += sum_k a[k] * b[n * bs + k], k contiguous in both (16-byte aligned), K % 4 == 0.
-// GLOBAL: b is read-only global memory (read through the non-coherent cache).
-template <int NC, bool GLOBAL>
+// acc[n] += sum_k a[k] * b[n * bs + k], k contiguous in both (16-byte aligned), K % 4 == 0
+template <int NC>
 __device__ __forceinline__ void mm_nt(float* acc, const float* a, const float* b, int bs, int K) {
 #pragma unroll 2
     for (int k = 0; k < K; k += 4) {
         const float4 x = *reinterpret_cast<const float4*>(a + k);
 #pragma unroll
         for (int n = 0; n < NC; ++n) {
-            const float4* p = reinterpret_cast<const float4*>(b + (size_t)n * bs + k);
-            const float4 y = GLOBAL ? __ldg(p) : *p;
+            const float4 y = *reinterpret_cast<const float4*>(b + (size_t)n * bs + k);
             acc[n] = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc[n]))));
         }
     }
@@ -247,8 +245,8 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
         float kk[16], qk[16];
 #pragma unroll
         for (int n = 0; n < 16; ++n) kk[n] = qk[n] = 0.f;
-        mm_nt<16, false>(kk, kh + i * LD, kh + g * LD, 4 * LD, D);
-        mm_nt<16, false>(qk, qh + i * LD, kh + g * LD, 4 * LD, D);
+        mm_nt<16>(kk, kh + i * LD, kh + g * LD, 4 * LD, D);
+        mm_nt<16>(qk, qh + i * LD, kh + g * LD, 4 * LD, D);
         float* Atg = ws + w.At + r * kCB * kCB + i * kCB;
         float* Pg = ws + w.P + r * kCB * kCB + i * kCB;
 #pragma unroll
@@ -348,11 +346,10 @@ struct ChainB {
 // memory: the copy for the next chunk is issued before the current chunk's arithmetic.
 template <int D>
 struct ChunkRegs {
-    static constexpr int PW = kCB * D / 4 / 256;    // float4 of W
-    static constexpr int PP = kCB * kCB / 4 / 256;  // float4 of P
-    static constexpr int PR = kCB * D / 8 / 256;    // 8-element groups of a token tile
-    float4 w[PW], pm[PP];
-    float k[PR][8], q[PR][8], y[8];
+    static constexpr int PW = kCB * D / 4 / 256;  // float4 of W
+    static constexpr int PR = kCB * D / 8 / 256;  // 8-element groups of a token tile
+    float4 w[PW];
+    float k[PR][8], y[8];
 };
 
 // Forward: S^c and U of every chunk, 32 state columns per CTA.
