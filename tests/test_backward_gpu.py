@@ -58,6 +58,17 @@ def test_backward_with_state_gradient_scale_and_no_norm():
     _check(out, ref)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_long_with_states(d):
+    """13 chunks (ragged last) through both chunk chains, with a nonzero S0, dS_final and scale."""
+    B, T, H = 1, 777, 2
+    inp = make_inputs(B, T, H, d, d, seed=31 + d, with_s0=True, with_dy=True)
+    rng = np.random.default_rng(d)
+    dsf = torch.from_numpy(rng.standard_normal((B, H, d, d)).astype(np.float32))
+    out, ref = _run(inp, ds_final=dsf, scale=0.9)
+    _check(out, ref)
+
+
 def test_backward_training_config_sampled():
     """Training shape B=8, T=4096, H=32, dk=dv=128, bf16, dy ~ N(0,1), S0 = 0, dS_final = 0.
     The oracle recomputes 3 sampled (sequence, head) chains in full."""
