@@ -53,6 +53,7 @@ PIN_TESTS = [
     lambda: pins.test_hand_worked_examples("scalar_three_tokens.txt"),
     lambda: pins.test_hand_worked_examples("two_by_three.txt"),
     lambda: pins.test_hand_worked_examples("l2norm_one_token.txt"),
+    pins.test_hand_worked_backward,
     pins.test_alpha1_beta0_is_identity,
     pins.test_one_token_outer_product,
     pins.test_beta1_unit_key_writes_exactly,

@@ -49,6 +49,26 @@ def test_hand_worked_examples(name):
     np.testing.assert_allclose(sf, g["s_final"], rtol=0, atol=1e-14)
 
 
+
+def test_hand_worked_backward():
+    """Hand-computed gradients of eqs. (1)-(4) for dk = dv = 1 (scalar chain rule; the
+    derivation is in the fixture), compared with the oracle's reverse recurrence."""
+    g = _load_golden("scalar_three_tokens_backward.txt")
+    T = int(g["T"][0])
+    sh = (1, T, 1, 1)
+    args = (g["q"].reshape(sh), g["k"].reshape(sh), g["v"].reshape(sh),
+            g["alpha"].reshape(1, T, 1), g["beta"].reshape(1, T, 1))
+    s0 = g["s0"].reshape(1, 1, 1, 1)
+    y, sf = oracle.forward(*args, s0, l2norm=False)
+    np.testing.assert_allclose(y.reshape(-1), g["y"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(sf.reshape(-1), g["s_final"], rtol=0, atol=1e-14)
+    out = oracle.backward(*args, s0, dy=g["dy"].reshape(sh),
+                          ds_final=g["ds_final"].reshape(1, 1, 1, 1), l2norm=False)
+    for name, key in (("dq", "dq"), ("dk", "dk_grad"), ("dv", "dv_grad"),
+                      ("dalpha", "dalpha"), ("dbeta", "dbeta"), ("ds0", "ds0")):
+        np.testing.assert_allclose(out[name].reshape(-1), g[key], rtol=0, atol=1e-14,
+                                   err_msg=name)
+
 def _rand(rng, B, T, H, dk, dv, s0=True):
     q = rng.standard_normal((B, T, H, dk))
     k = rng.standard_normal((B, T, H, dk))
