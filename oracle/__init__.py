@@ -11,9 +11,12 @@ Two independent fp64 forms of the same recurrence live here:
   gated delta rule (Qwen3.8-Flash-Next summary, picx.dev, "Theoretical
   foundations", eqs. (1)-(4)) with L2-normalised q and k ("Methodology",
   "1. GDN Hybrid Token Mixing") and its reverse-mode derivative.
-* ``chunked.forward_chunked``: numpy form of the same recurrence in chunks
-  (the WY/UT representation), used only to check that derivation against
-  the token loop.
+* ``chunked.forward_chunked`` / ``chunked.backward_chunked``: numpy form of
+  the same recurrence in chunks (the WY/UT representation), used only to
+  check that derivation against the token loop.
+* ``gates``: numpy fp64 form of the gates of eqs. (9)-(10) and the gated
+  RMSNorm of eq. (11) ("Methodology", "1. GDN Hybrid Token Mixing"), with
+  their reverse modes, chained around the token loop by ``layer_core``.
 
 Every array crosses the boundary as a C-contiguous float64 numpy array; the
 caller upcasts bf16/fp32 inputs (exactly) before calling.

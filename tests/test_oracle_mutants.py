@@ -1,16 +1,20 @@
 """Mutation check of the oracle's pins.
 
-Each case below plants one plausible mistake in a copy of the oracle's C source
-(on the CPU, in a temporary directory), builds it, and runs the pin tests of
-``test_oracle_pins`` against that build.  The pins must reject every mutant;
-a mutant that survives means a mistake of that kind would go unnoticed.
+Each case below plants one plausible mistake in a copy of the oracle's source (on
+the CPU, in a temporary directory) and runs the pin tests against that copy: the C
+token loop against ``test_oracle_pins``, the gates and gated output of
+``oracle/gates.py`` against ``test_oracle_gates``.  The pins must reject every
+mutant; a mutant that survives means a mistake of that kind would go unnoticed.
 """
+import importlib.util
 import os
 import subprocess
 
+import numpy as np
 import pytest
 
 import oracle
+import tests.test_oracle_gates as gate_pins
 import tests.test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")
@@ -82,4 +86,52 @@ def test_pins_reject_mutant(tmp_path, name, old, new):
                 t()
             except AssertionError:
                 caught.append(t)
+    assert caught, f"no pin rejects the planted mistake {name!r}"
+
+
+GATES_SRC = os.path.join(os.path.dirname(oracle.__file__), "gates.py")
+
+GATE_MUTANTS = [
+    ("decay_rate_not_exponentiated", "g = -np.exp(A_log) * softplus(a + b_alpha)",
+     "g = -A_log * softplus(a + b_alpha)"),
+    ("decay_bias_outside_softplus", "g = -np.exp(A_log) * softplus(a + b_alpha)",
+     "g = -np.exp(A_log) * (softplus(a) + b_alpha)"),
+    ("softplus_as_log1p", "return np.logaddexp(0.0, _f64(x))", "return np.log1p(_f64(x))"),
+    ("sigmoid_sign", "return 1.0 / (1.0 + np.exp(-x))", "return 1.0 / (1.0 + np.exp(x))"),
+    ("norm_not_zero_centred", "return (1.0 + w) * y * r", "return w * y * r"),
+    ("norm_sum_not_mean",
+     "r = 1.0 / np.sqrt(np.mean(y * y, axis=-1, keepdims=True) + eps)\n    return",
+     "r = 1.0 / np.sqrt(np.sum(y * y, axis=-1, keepdims=True) + eps)\n    return"),
+    ("bwd_alpha_chain_dropped", "dg_tot += _f64(dalpha) * alpha", "dg_tot += _f64(dalpha)"),
+    ("bwd_dA_missing_g", "dA_log = np.sum(dg_tot * g, axis=(0, 1))",
+     "dA_log = np.sum(dg_tot, axis=(0, 1))"),
+    ("bwd_db_alpha_sign", "db_alpha = np.sum(da, axis=(0, 1))",
+     "db_alpha = -np.sum(da, axis=(0, 1))"),
+    ("bwd_beta_derivative", "* beta * (1.0 - beta)", "* beta"),
+    ("bwd_gate_derivative", "dz = do * (1.0 + w) * n * s * (1.0 - s)",
+     "dz = do * (1.0 + w) * n * s"),
+    ("bwd_norm_projection_dropped",
+     "dy = r * (dn - n * np.mean(dn * n, axis=-1, keepdims=True))", "dy = r * dn"),
+    ("layer_gate_swapped", "return gated_output(y, z, w, eps), y, sf",
+     "return gated_output(z, y, w, eps), y, sf"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", GATE_MUTANTS, ids=[m[0] for m in GATE_MUTANTS])
+def test_gate_pins_reject_mutant(tmp_path, name, old, new):
+    src = open(GATES_SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    path = tmp_path / f"gates_{name}.py"
+    path.write_text(src.replace(old, new))
+    # a submodule of the oracle package, so that its relative imports resolve
+    spec = importlib.util.spec_from_file_location(f"oracle._mutant_{name}", str(path))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    caught = []
+    for check in gate_pins.CHECKS:
+        try:
+            with np.errstate(all="ignore"):
+                check(mod)
+        except AssertionError:
+            caught.append(check)
     assert caught, f"no pin rejects the planted mistake {name!r}"
