@@ -54,6 +54,7 @@ SIGNATURES = {
     "gdn_backward_noalloc": (_I, [_P] * 14 + [_I] * 6 + [_F, _I, _P]),
     "gdn_backward_noalloc_max_workspace": (_S, []),
     "gdn_read_device_status": (_I, [_I, ctypes.POINTER(_I)]),
+    "gdn_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
 }
 
 _lock = threading.Lock()

@@ -76,6 +76,10 @@ size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv);
 size_t backward_chunked_workspace_bytes(int B, int T, int H, int dk, int dv);
 cudaError_t launch_backward_chunked(const BackwardArgs& a, cudaStream_t st);
 
+// A kernel whose bounded wait runs out (nothing arrives on its barrier): it records
+// GDN_ERR_TIMEOUT in `status` after about limit_ns and returns.
+cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns, cudaStream_t st);
+
 // Size of the fixed device scratch array behind gdn_backward_noalloc.
 constexpr size_t kBackwardFixedScratchBytes = size_t(32) << 20;
 // Device address of that array on the current device (looked up on first use per device).

@@ -173,6 +173,12 @@ def test_backward_needs_its_workspace(lib):
     assert f(*bad, A, 1 << 30, None) == _abi.GDN_ERR_INVALID_ARG
 
 
+def test_selftest_rejects_limits_out_of_range(lib):
+    assert lib.gdn_selftest_wait_timeout(0, None) == _abi.GDN_ERR_INVALID_ARG
+    assert lib.gdn_selftest_wait_timeout(999, None) == _abi.GDN_ERR_INVALID_ARG
+    assert lib.gdn_selftest_wait_timeout(2_000_000_000, None) == _abi.GDN_ERR_INVALID_ARG
+
+
 def test_device_status_rejects_null(lib):
     assert lib.gdn_read_device_status(0, None) == _abi.GDN_ERR_INVALID_ARG
 
