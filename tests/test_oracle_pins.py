@@ -256,6 +256,22 @@ def test_chunked_form_matches_token_loop(C, l2norm, chunked=None):
     np.testing.assert_allclose(sc, sf, rtol=1e-10, atol=1e-12)
 
 
+@pytest.mark.parametrize("unroll", [False, True])
+def test_coupled_chunk_form_matches_token_loop(unroll, chunked=None):
+    """The coupled form the CUDA prefill's sequential kernel runs (U_c from U_{c-1} and a state
+    one chunk back through X_c = -W_c K_{c-1}^T), and its two-chunk unrolling, agree with the
+    token-by-token form (T not a multiple of C, nonzero S0, a scale)."""
+    fc = (chunked or oracle_chunked).forward_chunked_coupled
+    rng = np.random.default_rng(17)
+    q, k, v, alpha, beta, S0 = _rand(rng, 2, 330, 2, 16, 12)
+    slow = rng.uniform(0.9, 0.999, alpha.shape)  # chunk decays near 1: every coupling term counts
+    for a in (alpha, slow):
+        y, sf = oracle.forward(q, k, v, a, beta, S0, scale=0.8)
+        yc, sc = fc(q, k, v, a, beta, S0, C=32, scale=0.8, unroll=unroll)
+        np.testing.assert_allclose(yc, y, rtol=1e-9, atol=1e-11)
+        np.testing.assert_allclose(sc, sf, rtol=1e-9, atol=1e-11)
+
+
 def test_chunked_form_small_alpha_no_overflow(chunked=None):
     """Cumulative log-decay far below -88 within a chunk (exp(-G) alone would overflow
     fp64 only much later, but the relative form must stay finite and exact)."""
