@@ -68,6 +68,34 @@ def forward_chunked(q, k, v, alpha, beta, s0=None, C=64, scale=1.0, l2norm=True,
     return y, sf
 
 
+def blocked_unit_lower_inverse(A, bs=16):
+    """T = (I + A)^-1 for strictly lower-triangular A (n x n), in the blocked order the CUDA
+    kernels use: the diagonal bs x bs blocks by forward substitution, then the off-diagonal
+    blocks by increasing block distance, T_ij = -T_ii sum_{j <= m < i} A_im T_mj (blocks)."""
+    A = np.asarray(A, dtype=np.float64)
+    n = A.shape[0]
+    nb = (n + bs - 1) // bs
+    T = np.zeros((n, n))
+    blk = lambda i: slice(i * bs, min(n, (i + 1) * bs))
+    for b in range(nb):                       # diagonal blocks: (I + A_bb) T_bb = I
+        s = blk(b)
+        m = s.stop - s.start
+        Ab = A[s, s]
+        Tb = np.zeros((m, m))
+        for col in range(m):
+            x = np.zeros(m)
+            for r in range(m):
+                x[r] = (1.0 if r == col else 0.0) - Ab[r, :r] @ x[:r]
+            Tb[:, col] = x
+        T[s, s] = Tb
+    for dist in range(1, nb):                  # off-diagonal blocks, nearest first
+        for bj in range(nb - dist):
+            bi = bj + dist
+            acc = sum(A[blk(bi), blk(mb)] @ T[blk(mb), blk(bj)] for mb in range(bj, bi))
+            T[blk(bi), blk(bj)] = -T[blk(bi), blk(bi)] @ acc
+    return T
+
+
 def forward_chunked_coupled(q, k, v, alpha, beta, s0=None, C=64, scale=1.0, l2norm=True,
                             eps=EPS, unroll=False):
     """The chunked forward in the coupled form the CUDA prefill's sequential kernel runs, same

@@ -179,6 +179,8 @@ CHUNKED_CHECKS = [
     lambda m: pins.test_chunked_backward_matches_reverse_recurrence(64, False, m),
     lambda m: pins.test_coupled_chunk_form_matches_token_loop(False, m),
     lambda m: pins.test_coupled_chunk_form_matches_token_loop(True, m),
+    lambda m: pins.test_blocked_inverse_matches_dense_inverse(64, m),
+    lambda m: pins.test_blocked_inverse_matches_dense_inverse(50, m),
 ]
 
 CHUNKED_MUTANTS = [
@@ -201,6 +203,11 @@ CHUNKED_MUTANTS = [
      'U.append(d["Ut"] + (-d["W"] @ S[c - 1]) + d["X"] @ (m["D"] * U[c - 1]))'),
     ("unrolled_A2_second_term_dropped",
      'A2 = d["X"] @ (m["D"] * m["X"]) - m["g"] * d["W"] @ mm["K"].T', 'A2 = d["X"] @ (m["D"] * m["X"])'),
+    ("inverse_offdiag_sign", "T[blk(bi), blk(bj)] = -T[blk(bi), blk(bi)] @ acc",
+     "T[blk(bi), blk(bj)] = T[blk(bi), blk(bi)] @ acc"),
+    ("inverse_offdiag_missing_far_terms",
+     "acc = sum(A[blk(bi), blk(mb)] @ T[blk(mb), blk(bj)] for mb in range(bj, bi))",
+     "acc = A[blk(bi), blk(bj)] @ T[blk(bj), blk(bj)]"),
     ("bwd_dU_without_decay", 'c["dU"] = c["dec"][:, None] * (c["Kh"] @ dS) + scale * c["QK"].T @ c["dY"]',
      'c["dU"] = (c["Kh"] @ dS) + scale * c["QK"].T @ c["dY"]'),
 ]
