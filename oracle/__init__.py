@@ -13,7 +13,9 @@ Two independent fp64 forms of the same recurrence live here:
   "1. GDN Hybrid Token Mixing") and its reverse-mode derivative.
 * ``chunked.forward_chunked`` / ``chunked.backward_chunked``: numpy form of
   the same recurrence in chunks (the WY/UT representation), used only to
-  check that derivation against the token loop.
+  check that derivation against the token loop; with it the coupled form the
+  sequential prefill kernel runs (and its two-chunk unrolling) and the
+  blocked inversion of I + A the kernels use.
 * ``gates``: numpy fp64 form of the gates of eqs. (9)-(10) and the gated
   RMSNorm of eq. (11) ("Methodology", "1. GDN Hybrid Token Mixing"), with
   their reverse modes, chained around the token loop by ``layer_core``.
