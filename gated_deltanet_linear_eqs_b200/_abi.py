@@ -53,6 +53,13 @@ SIGNATURES = {
     "gdn_backward": (_I, [_P] * 14 + [_I] * 6 + [_F, _I, _P, _S, _P]),
     "gdn_backward_noalloc": (_I, [_P] * 14 + [_I] * 6 + [_F, _I, _P]),
     "gdn_backward_noalloc_max_workspace": (_S, []),
+    "gdn_prefill_gated": (_I, [_P] * 10 + [_I] * 6 + [_F, _I, _P, _S, _P]),
+    "gdn_prefill_varlen_gated": (_I, [_P] * 8 + [_I] + [_P] * 3 + [_I] * 5 + [_F, _I, _P, _S,
+                                                                            _P]),
+    "gdn_decode_step_gated": (_I, [_P] * 9 + [_I] * 5 + [_F, _I, _P]),
+    "gdn_backward_gated": (_I, [_P] * 18 + [_I] * 6 + [_F, _I, _P, _S, _P]),
+    "gdn_gated_rmsnorm": (_I, [_P] * 4 + [ctypes.c_int64, _I, _I, _F, _P]),
+    "gdn_gated_rmsnorm_backward": (_I, [_P] * 7 + [ctypes.c_int64, _I, _I, _F, _P]),
     "gdn_read_device_status": (_I, [_I, ctypes.POINTER(_I)]),
 }
 

@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
                                                  const Tin* __restrict__ v, const float* __restrict__ alpha,
                                                  const float* __restrict__ beta, float* __restrict__ ws,
                                                  const BwdChunkWs w, int T, int H, int nch, float scale,
-                                                 int l2norm) {
+                                                 int l2norm, const float* __restrict__ A_log,
+                                                 const float* __restrict__ b_alpha) {
     constexpr int LD = PrepB<D>::LD;
     extern __shared__ float smf[];
     float* qh = smf;
@@ -212,8 +213,14 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
     load_rows<D, LD, 256>(kh, k, b, t0, nv, h, T, H, nullptr, tid);
     if (tid < kCB) {
         const size_t o = tok_off(b, t0 + tid, h, T, H);
-        be[tid] = tid < nv ? beta[o] : 0.f;
-        Lg[tid] = tid < nv ? logf(alpha[o]) : 0.f;
+        float bt = 0.f, lg = 0.f;  // rows past the end: beta = 0, alpha = 1
+        if (tid < nv) {
+            // gated form: alpha, beta hold the logits of eqs. (9)-(10)
+            bt = A_log ? gate_sigmoid(beta[o]) : beta[o];
+            lg = A_log ? gate_log_decay(alpha[o], A_log[h], b_alpha[h]) : logf(alpha[o]);
+        }
+        be[tid] = bt;
+        Lg[tid] = lg;
     }
     __syncthreads();
     for (int rr = 0; rr < 16; ++rr) {  // warp w: rows 16 w .. 16 w + 15 of [q; k]
@@ -628,7 +635,11 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
                                                      Tin* __restrict__ dk, Tin* __restrict__ dv,
                                                      float* __restrict__ dalpha, float* __restrict__ dbeta,
                                                      const float* __restrict__ ws, const BwdChunkWs w, int T,
-                                                     int H, int nch, float scale, int l2norm) {
+                                                     int H, int nch, float scale, int l2norm,
+                                                     const float* __restrict__ A_log,
+                                                     const float* __restrict__ b_alpha,
+                                                     float* __restrict__ dA_log,
+                                                     float* __restrict__ db_alpha) {
     constexpr int LD = LocalB<D>::LD;
     constexpr int CT = D / 32;  // 8-column tiles per warp in 64 x D results
     extern __shared__ float smf[];
@@ -910,11 +921,32 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
         }
     }
     __syncthreads();
+    float pA = 0.f, pba = 0.f;  // this token's share of dA_log[h], db_alpha[h] (gated form)
     if (tid < nv) {
         const int i = tid;
         const size_t o = tok_off(b, t0 + i, h, T, H);
-        dalpha[o] = dLg[i] / alpha[o];
-        dbeta[o] = r_dbe[i] + r_dbg[i] * gam[i];
+        const float dbe = r_dbe[i] + r_dbg[i] * gam[i];
+        if (A_log) {
+            // ln alpha = -e^A softplus(x), x = a + b_alpha: d a = -e^A sigmoid(x) d ln alpha,
+            // d A = ln alpha d ln alpha, d b_alpha = d a; beta = sigmoid(b): d b = beta (1-beta) d beta
+            const float xa = alpha[o] + b_alpha[h], ea = expf(A_log[h]);
+            const float da = -ea * gate_sigmoid(xa) * dLg[i];
+            dalpha[o] = da;
+            dbeta[o] = dbe * be[i] * (1.f - be[i]);
+            pA = -ea * gate_softplus(xa) * dLg[i];
+            pba = da;
+        } else {
+            dalpha[o] = dLg[i] / alpha[o];
+            dbeta[o] = dbe;
+        }
+    }
+    if (A_log && tid < kCB) {  // warps 0 and 1, whole warps
+        pA = warp_sum(pA);
+        pba = warp_sum(pba);
+        if (lane == 0) {
+            atomicAdd(&dA_log[h], pA);
+            atomicAdd(&db_alpha[h], pba);
+        }
     }
     // 11b. dx = r (dx^ - x^ (x^ . dx^))
 #pragma unroll
@@ -955,16 +987,22 @@ cudaError_t launch_chunked(const BackwardArgs& a, cudaStream_t st) {
                                   LocalB<D>::BYTES)) != cudaSuccess)
         return e;
     bwdc_prep<D, Tin><<<R, 256, PrepB<D>::BYTES, st>>>(q, k, v, a.alpha, a.beta, ws, w, a.T, a.H, nch,
-                                                        a.scale, a.l2norm);
+                                                        a.scale, a.l2norm, a.A_log, a.b_alpha);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwdc_fwd<D, Tin><<<chains, 256, ChainB<D>::FWD_BYTES, st>>>(k, a.s0, ws, w, a.T, a.H, nch);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwdc_rev<D, Tin><<<chains, 256, ChainB<D>::REV_BYTES, st>>>(q, k, dy, a.ds_final, a.ds0, ws, w, a.T,
                                                                  a.H, nch, a.scale);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.A_log) {
+        if ((e = cudaMemsetAsync(a.dA_log, 0, sizeof(float) * a.H, st)) != cudaSuccess ||
+            (e = cudaMemsetAsync(a.db_alpha, 0, sizeof(float) * a.H, st)) != cudaSuccess)
+            return e;
+    }
     bwdc_local<D, Tin><<<R, 512, LocalB<D>::BYTES, st>>>(
         q, k, v, dy, a.alpha, static_cast<Tin*>(a.dq), static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv),
-        a.dalpha, a.dbeta, ws, w, a.T, a.H, nch, a.scale, a.l2norm);
+        a.dalpha, a.dbeta, ws, w, a.T, a.H, nch, a.scale, a.l2norm, a.A_log, a.b_alpha, a.dA_log,
+        a.db_alpha);
     return cudaGetLastError();
 }
 
