@@ -61,6 +61,7 @@ SIGNATURES = {
     "gdn_gated_rmsnorm": (_I, [_P] * 4 + [ctypes.c_int64, _I, _I, _F, _P]),
     "gdn_gated_rmsnorm_backward": (_I, [_P] * 7 + [ctypes.c_int64, _I, _I, _F, _P]),
     "gdn_read_device_status": (_I, [_I, ctypes.POINTER(_I)]),
+    "gdn_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
 }
 
 _lock = threading.Lock()

@@ -439,3 +439,10 @@ def gdn_read_device_status(reset=True):
     _check(_lib().gdn_read_device_status(int(bool(reset)), ctypes.byref(st)),
            "gdn_read_device_status")
     return int(st.value)
+
+
+def gdn_selftest_wait_timeout(limit_ns=1_000_000, stream=None):
+    """Launch the kernel whose bounded wait runs out (see include/gdn.h); afterwards
+    gdn_read_device_status() reports GDN_ERR_TIMEOUT."""
+    _check(_lib().gdn_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+           "gdn_selftest_wait_timeout")

@@ -368,6 +368,14 @@ int gdn_backward_noalloc(const void* q, const void* k, const void* v, const floa
 
 size_t gdn_backward_noalloc_max_workspace(void) { return gdn::kBackwardFixedScratchBytes; }
 
+int gdn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+    if (limit_ns < 1000 || limit_ns > 1000000000ull) return GDN_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    return map_cuda(gdn::launch_wait_timeout_selftest(dev.status, limit_ns,
+                                                      static_cast<cudaStream_t>(stream)));
+}
+
 int gdn_read_device_status(int reset, int* device_status) {
     if (!device_status) return GDN_ERR_INVALID_ARG;
     DeviceInfo dev;

@@ -104,6 +104,10 @@ struct GatedNormArgs {
 cudaError_t launch_gated_norm(const GatedNormArgs& a, cudaStream_t st);
 cudaError_t launch_gated_norm_backward(const GatedNormArgs& a, cudaStream_t st);
 
+// A kernel whose bounded wait runs out (nothing arrives on its barrier): it records
+// GDN_ERR_TIMEOUT in `status` after about limit_ns and returns.
+cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns, cudaStream_t st);
+
 // Size of the fixed device scratch array behind gdn_backward_noalloc.
 constexpr size_t kBackwardFixedScratchBytes = size_t(32) << 20;
 // Device address of that array on the current device (looked up on first use per device).

@@ -279,6 +279,17 @@ int gdn_gated_rmsnorm_backward(const void* y, const void* z, const float* w, con
  */
 int gdn_read_device_status(int reset, int* device_status);
 
+/*
+ * gdn_selftest_wait_timeout -- exercises the failure path of the library's bounded waits.
+ * Every wait inside the kernels gives up after a limit, records GDN_ERR_TIMEOUT in the device
+ * status word and returns, so that a lost arrival is reported rather than left to hang the GPU.
+ * This call launches one small kernel whose wait, on a barrier that nothing arrives on, runs
+ * out after about limit_ns nanoseconds (1e3 <= limit_ns <= 1e9, else GDN_ERR_INVALID_ARG).
+ * Afterwards gdn_read_device_status() reports GDN_ERR_TIMEOUT (clear it with reset != 0) and
+ * the device stays usable.  It touches no caller memory.
+ */
+int gdn_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

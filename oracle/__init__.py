@@ -17,6 +17,9 @@ Two independent fp64 forms of the same recurrence live here:
 * ``gates``: numpy fp64 form of the gates of eqs. (9)-(10) and the gated
   RMSNorm of eq. (11) ("Methodology", "1. GDN Hybrid Token Mixing"), with
   their reverse modes, chained around the token loop by ``layer_core``.
+* ``segments``: the recurrence as affine maps of runs of tokens (S -> M S + N),
+  their composition and scan, and a segment-parallel forward built on them
+  (the exchange that splitting one sequence across processors needs).
 
 Every array crosses the boundary as a C-contiguous float64 numpy array; the
 caller upcasts bf16/fp32 inputs (exactly) before calling.

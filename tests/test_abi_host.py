@@ -221,6 +221,10 @@ def test_gated_rmsnorm_rejects_bad_arguments(lib):
     assert bwd(dw=0) == _abi.GDN_ERR_INVALID_ARG
     assert bwd(do=0) == _abi.GDN_ERR_INVALID_ARG
     assert bwd(dv=32) == _abi.GDN_ERR_UNSUPPORTED_SHAPE
+def test_selftest_rejects_limits_out_of_range(lib):
+    assert lib.gdn_selftest_wait_timeout(0, None) == _abi.GDN_ERR_INVALID_ARG
+    assert lib.gdn_selftest_wait_timeout(999, None) == _abi.GDN_ERR_INVALID_ARG
+    assert lib.gdn_selftest_wait_timeout(2_000_000_000, None) == _abi.GDN_ERR_INVALID_ARG
 
 
 def test_device_status_rejects_null(lib):

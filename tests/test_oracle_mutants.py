@@ -16,6 +16,7 @@ import pytest
 import oracle
 import tests.test_oracle_gates as gate_pins
 import tests.test_oracle_pins as pins
+import tests.test_oracle_segments as seg_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")
 
@@ -117,21 +118,52 @@ GATE_MUTANTS = [
 ]
 
 
-@pytest.mark.parametrize("name,old,new", GATE_MUTANTS, ids=[m[0] for m in GATE_MUTANTS])
-def test_gate_pins_reject_mutant(tmp_path, name, old, new):
-    src = open(GATES_SRC).read()
+def _python_mutant_caught(tmp_path, src_path, checks, name, old, new):
+    src = open(src_path).read()
     assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
-    path = tmp_path / f"gates_{name}.py"
+    path = tmp_path / f"mutant_{name}.py"
     path.write_text(src.replace(old, new))
     # a submodule of the oracle package, so that its relative imports resolve
     spec = importlib.util.spec_from_file_location(f"oracle._mutant_{name}", str(path))
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
     caught = []
-    for check in gate_pins.CHECKS:
+    for check in checks:
         try:
             with np.errstate(all="ignore"):
                 check(mod)
         except AssertionError:
             caught.append(check)
+    return caught
+
+
+@pytest.mark.parametrize("name,old,new", GATE_MUTANTS, ids=[m[0] for m in GATE_MUTANTS])
+def test_gate_pins_reject_mutant(tmp_path, name, old, new):
+    caught = _python_mutant_caught(tmp_path, GATES_SRC, gate_pins.CHECKS, name, old, new)
+    assert caught, f"no pin rejects the planted mistake {name!r}"
+
+
+SEGMENTS_SRC = os.path.join(os.path.dirname(oracle.__file__), "segments.py")
+
+SEGMENT_MUTANTS = [
+    ("token_map_without_decay", "M = alpha_t * (np.eye(kh.shape[0]) - beta_t * np.outer(kh, kh))",
+     "M = np.eye(kh.shape[0]) - beta_t * np.outer(kh, kh)"),
+    ("token_map_sign", "M = alpha_t * (np.eye(kh.shape[0]) - beta_t * np.outer(kh, kh))",
+     "M = alpha_t * (np.eye(kh.shape[0]) + beta_t * np.outer(kh, kh))"),
+    ("token_write_without_beta", "N = beta_t * np.outer(kh, v_t)", "N = np.outer(kh, v_t)"),
+    ("compose_order", "return M2 @ M1, M2 @ N1 + N2", "return M1 @ M2, M2 @ N1 + N2"),
+    ("compose_offset_not_carried", "return M2 @ M1, M2 @ N1 + N2", "return M2 @ M1, N1 + N2"),
+    ("scan_inclusive", "        starts.append(S)\n        S = apply(m, S)",
+     "        S = apply(m, S)\n        starts.append(S)"),
+    ("chunk_map_decay_dropped", "mc = (gam[-1] * np.eye(dk) - Kd.T @ W, Kd.T @ Ut)",
+     "mc = (np.eye(dk) - Kd.T @ W, Kd.T @ Ut)"),
+    ("chunk_map_unscaled_keys", "Kd = Gam[-1][:, None] * K", "Kd = K"),
+    ("segments_restart_from_s0", "                                beta[b:b + 1, t0:t1, h:h + 1], Ss[None, None], scale=scale,",
+     "                                beta[b:b + 1, t0:t1, h:h + 1], S0[None, None], scale=scale,"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", SEGMENT_MUTANTS, ids=[m[0] for m in SEGMENT_MUTANTS])
+def test_segment_pins_reject_mutant(tmp_path, name, old, new):
+    caught = _python_mutant_caught(tmp_path, SEGMENTS_SRC, seg_pins.CHECKS, name, old, new)
     assert caught, f"no pin rejects the planted mistake {name!r}"
