@@ -231,6 +231,23 @@ def test_device_status_rejects_null(lib):
     assert lib.gdn_read_device_status(0, None) == _abi.GDN_ERR_INVALID_ARG
 
 
+def test_binding_refuses_host_tensors():
+    """The Python binding computes nothing itself: tensors that are not on a CUDA device are
+    rejected before any call, so no host path can stand in for the kernels."""
+    import torch
+
+    from gated_deltanet_linear_eqs_b200 import api
+    q = torch.zeros((1, 64, 1, 64), dtype=torch.bfloat16)
+    a = torch.full((1, 64, 1), 0.5)
+    with pytest.raises(ValueError, match="CUDA"):
+        api.gdn_prefill(q, q, q, a, a)
+    with pytest.raises(ValueError, match="CUDA"):
+        api.gdn_decode_step(q[:, 0], q[:, 0], q[:, 0], a[:, 0], a[:, 0],
+                            torch.zeros((1, 1, 64, 64)))
+    with pytest.raises(ValueError, match="CUDA"):
+        api.gdn_backward(q, q, q, a, a, q)
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     saved = _abi._lib
     try:
