@@ -86,20 +86,6 @@ __device__ __forceinline__ void mm_nn(float* acc, const float* a, int as, const 
     }
 }
 
-// acc[n] += sum_k a[k] * b[n * bs + k], k contiguous in both (16-byte aligned), K % 4 == 0
-template <int NC>
-__device__ __forceinline__ void mm_nt(float* acc, const float* a, const float* b, int bs, int K) {
-#pragma unroll 2
-    for (int k = 0; k < K; k += 4) {
-        const float4 x = *reinterpret_cast<const float4*>(a + k);
-#pragma unroll
-        for (int n = 0; n < NC; ++n) {
-            const float4 y = *reinterpret_cast<const float4*>(b + (size_t)n * bs + k);
-            acc[n] = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc[n]))));
-        }
-    }
-}
-
 __device__ __forceinline__ size_t tok_off(int b, int t, int h, int T, int H) {
     return ((size_t)b * T + t) * H + h;
 }
@@ -175,6 +161,33 @@ __device__ __forceinline__ void mma_tf32(float* c, uint32_t a0, uint32_t a1, uin
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// acc[t] (16 x 8 tile t at rows r0.., columns c0 + 8 t ..) += A B over k < K, tf32
+template <int CT, typename FA, typename FB>
+__device__ __forceinline__ void wmma_acc(float (&acc)[CT][4], int K, int r0, int c0, FA a, FB b, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = to_tf32(a(r0 + gid, k0 + tig)), a1 = to_tf32(a(r0 + gid + 8, k0 + tig));
+        const uint32_t a2 = to_tf32(a(r0 + gid, k0 + tig + 4)), a3 = to_tf32(a(r0 + gid + 8, k0 + tig + 4));
+#pragma unroll
+        for (int t = 0; t < CT; ++t) {
+            const int n = c0 + 8 * t + gid;
+            mma_tf32(acc[t], a0, a1, a2, a3, to_tf32(b(k0 + tig, n)), to_tf32(b(k0 + tig + 4, n)));
+        }
+    }
+}
+template <int CT>
+__device__ __forceinline__ void zero_acc(float (&acc)[CT][4]) {
+#pragma unroll
+    for (int t = 0; t < CT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+}
+// sum over the 4 lanes of a quad (the lanes that share a tile row)
+__device__ __forceinline__ float quad_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    return x;
+}
+
 // ============================================================================ bwdc_prep
 template <int D>
 struct PrepB {
@@ -183,7 +196,7 @@ struct PrepB {
 };
 
 template <int D, typename Tin>
-__global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, const Tin* __restrict__ k,
+__global__ void __launch_bounds__(256, 2) bwdc_prep(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                  const Tin* __restrict__ v, const float* __restrict__ alpha,
                                                  const float* __restrict__ beta, float* __restrict__ ws,
                                                  const BwdChunkWs w, int T, int H, int nch, float scale,
@@ -239,25 +252,38 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
         kh[i * LD + m] *= rk[i];
     }
     __syncthreads();
-    // A / beta and P
-    {  // thread: row i, columns j = g + 4 n (rows g + 4 n of K^ sit in distinct banks)
-        const int i = tid >> 2, g = tid & 3;
-        float kk[16], qk[16];
+    // A / beta and P: K^ K^T and Q^ K^T as 16 x 8 tensor-core tiles (tf32 operands, fp32
+    // accumulation); warp w owns rows 16 (w & 3) .. +15 and columns 32 (w >> 2) .. +31, and lane
+    // (gid, tig) of tile t holds rows gid, gid + 8 and columns 8 t + 2 tig, 8 t + 2 tig + 1
+    {
+        const int gid = lane >> 2, tig = lane & 3;
+        const int r0 = (warp & 3) * 16, c0 = (warp >> 2) * 32;
+        const float* khp = kh;
+        const float* qhp = qh;
+        float kk[4][4], qk[4][4];
+        zero_acc(kk);
+        zero_acc(qk);
+        auto bKt = [khp](int k2, int n) { return khp[n * LD + k2]; };
+        wmma_acc(kk, D, r0, c0, [khp](int i, int k2) { return khp[i * LD + k2]; }, bKt, lane);
+        wmma_acc(qk, D, r0, c0, [qhp](int i, int k2) { return qhp[i * LD + k2]; }, bKt, lane);
+        float* Atg = ws + w.At + r * kCB * kCB;
+        float* Pg = ws + w.P + r * kCB * kCB;
 #pragma unroll
-        for (int n = 0; n < 16; ++n) kk[n] = qk[n] = 0.f;
-        mm_nt<16>(kk, kh + i * LD, kh + g * LD, 4 * LD, D);
-        mm_nt<16>(qk, qh + i * LD, kh + g * LD, 4 * LD, D);
-        float* Atg = ws + w.At + r * kCB * kCB + i * kCB;
-        float* Pg = ws + w.P + r * kCB * kCB + i * kCB;
+        for (int t = 0; t < 4; ++t)
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            const int j = g + 4 * n;
-            const float gm = expf(fminf(Lg[i] - Lg[j], 0.f));
-            const float at = j < i ? kk[n] * gm : 0.f;
-            Atg[j] = at;
-            Am[i * kL64 + j] = be[i] * at;
-            Pg[j] = j <= i ? scale * qk[n] * gm : 0.f;
-        }
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = r0 + gid + 8 * hh, j = c0 + 8 * t + 2 * tig;
+                float at[2], pp[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const float gm = expf(fminf(Lg[i] - Lg[j + u], 0.f));
+                    at[u] = j + u < i ? kk[t][2 * hh + u] * gm : 0.f;
+                    pp[u] = j + u <= i ? scale * qk[t][2 * hh + u] * gm : 0.f;
+                    Am[i * kL64 + j + u] = be[i] * at[u];
+                }
+                *reinterpret_cast<float2*>(Atg + i * kCB + j) = make_float2(at[0], at[1]);
+                *reinterpret_cast<float2*>(Pg + i * kCB + j) = make_float2(pp[0], pp[1]);
+            }
     }
     __syncthreads();
     load_rows<D, LD, 256>(vs, v, b, t0, nv, h, T, H, nullptr, tid);  // Q is no longer read
@@ -297,35 +323,36 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
         __syncthreads();
     }
     for (int e = tid; e < kCB * kCB; e += 256) ws[w.Tm + r * kCB * kCB + e] = Tm[(e / kCB) * kL64 + e % kCB];
-    // W = T diag(beta gam) K^, Ut = T diag(beta) V
-    {  // thread: row i, column chunks 4 g + 16 u
-        constexpr int NC = D / 4;
-        const int i = tid >> 2, g = tid & 3;
-        float wa[NC], ua[NC];
+    // W = T diag(beta gam) K^, Ut = T diag(beta) V: 64 x D tensor-core tiles (tf32, fp32
+    // accumulation), the diagonal scales folded into the B operand; warp w owns rows
+    // 16 (w & 3) .. +15 and columns (D / 2)(w >> 2) .. +D/2-1
+    {
+        constexpr int CT = D / 16;
+        const int gid = lane >> 2, tig = lane & 3;
+        const int r0 = (warp & 3) * 16, c0 = (warp >> 2) * (D / 2);
+        const float* Tp = Tm;
+        const float* khp = kh;
+        const float* vp = vs;
+        const float* bep = be;
+        const float* gp = gam;
+        float wa[CT][4], ua[CT][4];
+        zero_acc(wa);
+        zero_acc(ua);
+        auto aT = [Tp](int i, int j) { return Tp[i * kL64 + j]; };
+        wmma_acc(wa, kCB, r0, c0, aT,
+                 [bep, gp, khp](int j, int n) { return bep[j] * gp[j] * khp[j * LD + n]; }, lane);
+        wmma_acc(ua, kCB, r0, c0, aT, [bep, vp](int j, int n) { return bep[j] * vp[j * LD + n]; },
+                 lane);
+        float* Wg = ws + w.W + r * kCB * D;
+        float* Ug = ws + w.Ut + r * kCB * D;
 #pragma unroll
-        for (int n = 0; n < NC; ++n) wa[n] = ua[n] = 0.f;
-        for (int j = 0; j < kCB; ++j) {
-            const float tij = Tm[i * kL64 + j];
-            const float fw = tij * be[j] * gam[j], fu = tij * be[j];
-            const float* kr = kh + j * LD + 4 * g;
-            const float* vr = vs + j * LD + 4 * g;
+        for (int t = 0; t < CT; ++t)
 #pragma unroll
-            for (int n = 0; n < NC / 4; ++n) {
-                const float4 y = *reinterpret_cast<const float4*>(kr + 16 * n);
-                const float4 z = *reinterpret_cast<const float4*>(vr + 16 * n);
-                wa[4 * n] = fmaf(fw, y.x, wa[4 * n]); wa[4 * n + 1] = fmaf(fw, y.y, wa[4 * n + 1]);
-                wa[4 * n + 2] = fmaf(fw, y.z, wa[4 * n + 2]); wa[4 * n + 3] = fmaf(fw, y.w, wa[4 * n + 3]);
-                ua[4 * n] = fmaf(fu, z.x, ua[4 * n]); ua[4 * n + 1] = fmaf(fu, z.y, ua[4 * n + 1]);
-                ua[4 * n + 2] = fmaf(fu, z.z, ua[4 * n + 2]); ua[4 * n + 3] = fmaf(fu, z.w, ua[4 * n + 3]);
+            for (int hh = 0; hh < 2; ++hh) {
+                const size_t o = (size_t)(r0 + gid + 8 * hh) * D + c0 + 8 * t + 2 * tig;
+                *reinterpret_cast<float2*>(Wg + o) = make_float2(wa[t][2 * hh], wa[t][2 * hh + 1]);
+                *reinterpret_cast<float2*>(Ug + o) = make_float2(ua[t][2 * hh], ua[t][2 * hh + 1]);
             }
-        }
-        float* Wg = ws + w.W + r * kCB * D + (size_t)i * D + 4 * g;
-        float* Ug = ws + w.Ut + r * kCB * D + (size_t)i * D + 4 * g;
-#pragma unroll
-        for (int n = 0; n < NC / 4; ++n) {
-            *reinterpret_cast<float4*>(Wg + 16 * n) = make_float4(wa[4 * n], wa[4 * n + 1], wa[4 * n + 2], wa[4 * n + 3]);
-            *reinterpret_cast<float4*>(Ug + 16 * n) = make_float4(ua[4 * n], ua[4 * n + 1], ua[4 * n + 2], ua[4 * n + 3]);
-        }
     }
     if (tid < kCB) {
         float* sc = ws + w.SC + r * 256;
@@ -575,33 +602,6 @@ struct LocalB {
     static constexpr int NROW = 10;  // row accumulators
     static constexpr int BYTES = (5 * kCB * LD + 3 * kCB * kL64 + (5 + NROW + 1) * kCB + 32) * 4;
 };
-
-// acc[t] (16 x 8 tile t at rows r0.., columns c0 + 8 t ..) += A B over k < K, tf32
-template <int CT, typename FA, typename FB>
-__device__ __forceinline__ void wmma_acc(float (&acc)[CT][4], int K, int r0, int c0, FA a, FB b, int lane) {
-    const int gid = lane >> 2, tig = lane & 3;
-#pragma unroll 2
-    for (int k0 = 0; k0 < K; k0 += 8) {
-        const uint32_t a0 = to_tf32(a(r0 + gid, k0 + tig)), a1 = to_tf32(a(r0 + gid + 8, k0 + tig));
-        const uint32_t a2 = to_tf32(a(r0 + gid, k0 + tig + 4)), a3 = to_tf32(a(r0 + gid + 8, k0 + tig + 4));
-#pragma unroll
-        for (int t = 0; t < CT; ++t) {
-            const int n = c0 + 8 * t + gid;
-            mma_tf32(acc[t], a0, a1, a2, a3, to_tf32(b(k0 + tig, n)), to_tf32(b(k0 + tig + 4, n)));
-        }
-    }
-}
-template <int CT>
-__device__ __forceinline__ void zero_acc(float (&acc)[CT][4]) {
-#pragma unroll
-    for (int t = 0; t < CT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-}
-// sum over the 4 lanes of a quad (the lanes that share a tile row)
-__device__ __forceinline__ float quad_sum(float x) {
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
-    return x;
-}
 
 // acc += A G^T for the warp's tiles, G [D][D] fp32 in global memory, staged in `buf` (row stride
 // LD) 64 rows at a time: the warps whose output columns fall in the staged rows compute.  Every
