@@ -188,6 +188,35 @@ __device__ __forceinline__ float quad_sum(float x) {
     return x;
 }
 
+// acc[t] += A B like wmma_acc, with every operand split into its tf32 value and a tf32
+// remainder: A_lo B_hi + A_hi B_lo + A_hi B_hi.  That keeps the products' relative error near
+// 2^-22 instead of tf32's 2^-11, for the products whose rounding accumulates along a chain.
+template <int CT, typename FA, typename FB>
+__device__ __forceinline__ void wmma_acc3(float (&acc)[CT][4], int K, int r0, int c0, FA a, FB b, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const float af[4] = {a(r0 + gid, k0 + tig), a(r0 + gid + 8, k0 + tig), a(r0 + gid, k0 + tig + 4),
+                             a(r0 + gid + 8, k0 + tig + 4)};
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            ah[e] = to_tf32(af[e]);
+            al[e] = to_tf32(af[e] - __uint_as_float(ah[e]));
+        }
+#pragma unroll
+        for (int t = 0; t < CT; ++t) {
+            const int n = c0 + 8 * t + gid;
+            const float b0 = b(k0 + tig, n), b1 = b(k0 + tig + 4, n);
+            const uint32_t bh0 = to_tf32(b0), bh1 = to_tf32(b1);
+            const uint32_t bl0 = to_tf32(b0 - __uint_as_float(bh0)), bl1 = to_tf32(b1 - __uint_as_float(bh1));
+            mma_tf32(acc[t], al[0], al[1], al[2], al[3], bh0, bh1);
+            mma_tf32(acc[t], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+            mma_tf32(acc[t], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+        }
+    }
+}
+
 // ============================================================================ bwdc_prep
 template <int D>
 struct PrepB {
@@ -363,7 +392,7 @@ __global__ void __launch_bounds__(256, 2) bwdc_prep(const Tin* __restrict__ q, c
 // ============================================================================ chains
 template <int D>
 struct ChainB {
-    static constexpr int LDS = kNVB + 4;
+    static constexpr int LDS = kNVB + 8;  // rows k and k + 1..3 of a B operand: distinct banks
     static constexpr int LD = D + 4;
     static constexpr int FWD_BYTES = (D * LDS + 2 * kCB * LD + kCB * LDS + 2 * kCB) * 4;
     static constexpr int REV_BYTES = (D * LDS + 2 * kCB * LD + 2 * kCB * LDS + 3 * kCB) * 4;
@@ -376,7 +405,8 @@ struct ChunkRegs {
     static constexpr int PW = kCB * D / 4 / 256;  // float4 of W
     static constexpr int PR = kCB * D / 8 / 256;  // 8-element groups of a token tile
     float4 w[PW];
-    float k[PR][8], y[8];
+    float k[PR][8];
+    float2 y[4];  // Ut at this lane's positions of the U tiles (tile t, row half hh: y[2 t + hh])
 };
 
 // Forward: S^c and U of every chunk, 32 state columns per CTA.
@@ -396,8 +426,10 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
     float* rks = dec + kCB;
     constexpr int nsl = D / kNVB;
     const int jsl = blockIdx.x % nsl, h = (blockIdx.x / nsl) % H, b = blockIdx.x / (nsl * H);
-    const int col0 = jsl * kNVB, tid = threadIdx.x;
-    const int iu = tid >> 2, nu = (tid & 3) * 8;  // U element block of this thread
+    const int col0 = jsl * kNVB, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    // U (64 x 32) tiles: warp w owns rows 16 (w & 3) .. +15 and columns 16 (w >> 2) .. +15
+    const int ur0 = (warp & 3) * 16, uc0 = (warp >> 2) * 16;
     R rg;
     auto fetch = [&](int c) {
         const size_t r = ((size_t)b * nch + c) * H + h;
@@ -414,7 +446,13 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
                 for (int j = 0; j < 8; ++j) rg.k[u][j] = 0.f;
             }
         }
-        ld8(ws + w.Ut + r * kCB * D + (size_t)iu * D + col0 + nu, rg.y);  // Ut of this thread's U block
+        const float* Utg = ws + w.Ut + r * kCB * D + col0;  // Ut at this lane's U tile positions
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                rg.y[2 * t + hh] = *reinterpret_cast<const float2*>(
+                    Utg + (size_t)(ur0 + gid + 8 * hh) * D + uc0 + 8 * t + 2 * tig);
     };
     for (int e = tid; e < D * kNVB; e += 256) {
         const int m = e / kNVB, n = e % kNVB;
@@ -439,9 +477,9 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
             const int e = (tid + u * 256) * 8;
             st8(Kt + (e / D) * LD + e % D, rg.k[u], 1.f);
         }
-        float ut[8];
+        float2 ut[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) ut[j] = rg.y[j];
+        for (int j = 0; j < 4; ++j) ut[j] = rg.y[j];
         const float* SCg = ws + w.SC + r * 256;
         if (tid < kCB) {
             dec[tid] = expf(SCg[128 + kCB - 1] - SCg[128 + tid]);
@@ -450,38 +488,48 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
         const float gC = expf(SCg[128 + kCB - 1]);
         __syncthreads();
         if (c + 1 < nch) fetch(c + 1);
-        {  // U = Ut - W S: row iu, 8 columns
-            float acc[8];
+        {  // U = Ut - W S as 16 x 8 tensor-core tiles (tf32 operands, fp32 accumulation)
+            float acc[2][4];
+            zero_acc(acc);
+            const float* Wp = Wt;
+            const float* Sp = Ss;
+            wmma_acc(acc, D, ur0, uc0, [Wp](int i, int k2) { return Wp[i * LD + k2]; },
+                     [Sp](int k2, int n) { return Sp[k2 * LDS + n]; }, lane);
+            float* Ug = ws + w.U + r * kCB * D + col0;
 #pragma unroll
-            for (int n = 0; n < 8; ++n) acc[n] = 0.f;
-            mm_nn<8>(acc, Wt + iu * LD, 1, Ss + nu, LDS, D);
-            float* Ug = ws + w.U + r * kCB * D + (size_t)iu * D + col0 + nu;
+            for (int t = 0; t < 2; ++t)
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const float u = ut[n] - acc[n];
-                Us[iu * LDS + nu + n] = u;
-                Ug[n] = u;
-            }
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int i = ur0 + gid + 8 * hh, n = uc0 + 8 * t + 2 * tig;
+                    const float2 u = make_float2(ut[2 * t + hh].x - acc[t][2 * hh],
+                                                 ut[2 * t + hh].y - acc[t][2 * hh + 1]);
+                    *reinterpret_cast<float2*>(Us + i * LDS + n) = u;
+                    *reinterpret_cast<float2*>(Ug + (size_t)i * D + n) = u;
+                }
         }
         __syncthreads();
-        {  // S = gC S + K^T diag(rk gC / gam) U
-            constexpr int TPR = 256 / D, NC = kNVB / TPR;
-            const int m = tid / TPR, n0 = (tid % TPR) * NC;
-            float acc[NC];
+        {  // S = gC S + K^T diag(rk gC / gam) U as tensor-core tiles (tf32, fp32 accumulation);
+           // the D x 32 slice is D / 16 row blocks by 8 / (D / 16) column groups, one per warp
+            constexpr int RB = D / 16, CG = 8 / RB, CT = 4 / CG;
+            const int sr0 = 16 * (warp % RB), sc0 = (32 / CG) * (warp / RB);
+            float acc[CT][4];
+            zero_acc(acc);
+            const float* Kp = Kt;
+            const float* Up = Us;
+            const float* dp = dec;
+            const float* rp = rks;
+            wmma_acc(acc, kCB, sr0, sc0,
+                     [Kp, dp, rp](int m, int i) { return Kp[i * LD + m] * (dp[i] * rp[i]); },
+                     [Up](int i, int n) { return Up[i * LDS + n]; }, lane);
 #pragma unroll
-            for (int n = 0; n < NC; ++n) acc[n] = 0.f;
-            for (int i = 0; i < kCB; ++i) {
-                const float x = Kt[i * LD + m] * (dec[i] * rks[i]);
-                const float4* ur = reinterpret_cast<const float4*>(Us + i * LDS + n0);
+            for (int t = 0; t < CT; ++t)
 #pragma unroll
-                for (int n = 0; n < NC / 4; ++n) {
-                    const float4 y = ur[n];
-                    acc[4 * n] = fmaf(x, y.x, acc[4 * n]); acc[4 * n + 1] = fmaf(x, y.y, acc[4 * n + 1]);
-                    acc[4 * n + 2] = fmaf(x, y.z, acc[4 * n + 2]); acc[4 * n + 3] = fmaf(x, y.w, acc[4 * n + 3]);
+                for (int hh = 0; hh < 2; ++hh) {
+                    float* sp = Ss + (sr0 + gid + 8 * hh) * LDS + sc0 + 8 * t + 2 * tig;
+                    const float2 o = *reinterpret_cast<const float2*>(sp);
+                    *reinterpret_cast<float2*>(sp) =
+                        make_float2(fmaf(gC, o.x, acc[t][2 * hh]), fmaf(gC, o.y, acc[t][2 * hh + 1]));
                 }
-            }
-#pragma unroll
-            for (int n = 0; n < NC; ++n) Ss[m * LDS + n0 + n] = fmaf(gC, Ss[m * LDS + n0 + n], acc[n]);
         }
     }
 }
@@ -506,7 +554,13 @@ __global__ void __launch_bounds__(256, 2) bwdc_rev(const Tin* __restrict__ q, co
     float* rks = ysc + kCB;
     constexpr int nsl = D / kNVB;
     const int jsl = blockIdx.x % nsl, h = (blockIdx.x / nsl) % H, b = blockIdx.x / (nsl * H);
-    const int col0 = jsl * kNVB, tid = threadIdx.x;
+    const int col0 = jsl * kNVB, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    // dU (64 x 32) tiles: warp w owns rows 16 (w & 3) .. +15 and columns 16 (w >> 2) .. +15;
+    // dS (D x 32): D / 16 row blocks by 8 / (D / 16) column groups, one per warp
+    const int ur0 = (warp & 3) * 16, uc0 = (warp >> 2) * 16;
+    constexpr int RB = D / 16, CG = 8 / RB, SCT = 4 / CG;
+    const int sr0 = 16 * (warp % RB), sc0 = (32 / CG) * (warp / RB);
     for (int e = tid; e < D * kNVB; e += 256) {
         const int m = e / kNVB, n = e % kNVB;
         Ss[m * LDS + n] = ds_final ? ds_final[(((size_t)b * H + h) * D + m) * D + col0 + n] : 0.f;
@@ -541,46 +595,57 @@ __global__ void __launch_bounds__(256, 2) bwdc_rev(const Tin* __restrict__ q, co
         const int nvc = min(kCB, T - c * kCB);
         load_rows<D, LD, 256>(X1, k, b, c * kCB, nvc, h, T, H, rks, tid);
         __syncthreads();
-        {  // dU = diag(gC / gam) K^ dS + P^T dY
-            const int i = tid >> 2, n0 = (tid & 3) * 8;
-            float a1[8], a2[8];
+        {  // dU = diag(gC / gam) K^ dS + P^T dY as tensor-core tiles (tf32, fp32 accumulation)
+            float a1[2][4], a2[2][4];
+            zero_acc(a1);
+            zero_acc(a2);
+            const float* Kp = X1;
+            const float* Pp = X2;
+            const float* Sp = Ss;
+            const float* Yp = dYs;
+            wmma_acc(a1, D, ur0, uc0, [Kp](int i, int m) { return Kp[i * LD + m]; },
+                     [Sp](int m, int n) { return Sp[m * LDS + n]; }, lane);
+            wmma_acc(a2, kCB, ur0, uc0, [Pp](int i, int j) { return Pp[j * kL64 + i]; },
+                     [Yp](int j, int n) { return Yp[j * LDS + n]; }, lane);
+            float* dUg = ws + w.dU + r * kCB * D + col0;
 #pragma unroll
-            for (int n = 0; n < 8; ++n) a1[n] = a2[n] = 0.f;
-            mm_nn<8>(a1, X1 + i * LD, 1, Ss + n0, LDS, D);
-            mm_nn<8>(a2, X2 + i, kL64, dYs + n0, LDS, kCB);
-            float* dUg = ws + w.dU + r * kCB * D + (size_t)i * D + col0 + n0;
+            for (int t = 0; t < 2; ++t)
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const float du = fmaf(dec[i], a1[n], a2[n]);
-                dUs[i * LDS + n0 + n] = du;
-                dUg[n] = du;
-            }
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int i = ur0 + gid + 8 * hh, n = uc0 + 8 * t + 2 * tig;
+                    const float2 du = make_float2(fmaf(dec[i], a1[t][2 * hh], a2[t][2 * hh]),
+                                                  fmaf(dec[i], a1[t][2 * hh + 1], a2[t][2 * hh + 1]));
+                    *reinterpret_cast<float2*>(dUs + i * LDS + n) = du;
+                    *reinterpret_cast<float2*>(dUg + (size_t)i * D + n) = du;
+                }
         }
         __syncthreads();
         load_rows<D, LD, 256>(X1, q, b, c * kCB, nvc, h, T, H, ysc, tid);
         load_rec<D, LD, 256>(X2, ws + w.W + r * kCB * D, tid);
         __syncthreads();
-        {  // dS = gC dS + (scale gam Q^)^T dY - W^T dU
-            constexpr int TPR = 256 / D, NC = kNVB / TPR;
-            const int m = tid / TPR, n0 = (tid % TPR) * NC;
-            float acc[NC];
+        {  // dS = gC dS + (scale gam Q^)^T dY - W^T dU as tensor-core tiles with split (3 x tf32)
+           // operands: these products feed the state gradient along the whole chain
+            float a1[SCT][4], a2[SCT][4];
+            zero_acc(a1);
+            zero_acc(a2);
+            const float* Qp = X1;
+            const float* Wp = X2;
+            const float* Yp = dYs;
+            const float* Up = dUs;
+            wmma_acc3(a1, kCB, sr0, sc0, [Qp](int m, int i) { return Qp[i * LD + m]; },
+                      [Yp](int i, int n) { return Yp[i * LDS + n]; }, lane);
+            wmma_acc3(a2, kCB, sr0, sc0, [Wp](int m, int i) { return Wp[i * LD + m]; },
+                      [Up](int i, int n) { return Up[i * LDS + n]; }, lane);
 #pragma unroll
-            for (int n = 0; n < NC; ++n) acc[n] = 0.f;
-            for (int i = 0; i < kCB; ++i) {
-                const float xq = X1[i * LD + m], xw = X2[i * LD + m];
-                const float4* yr = reinterpret_cast<const float4*>(dYs + i * LDS + n0);
-                const float4* ur = reinterpret_cast<const float4*>(dUs + i * LDS + n0);
+            for (int t = 0; t < SCT; ++t)
 #pragma unroll
-                for (int n = 0; n < NC / 4; ++n) {
-                    const float4 y = yr[n], u = ur[n];
-                    acc[4 * n] = fmaf(xq, y.x, fmaf(-xw, u.x, acc[4 * n]));
-                    acc[4 * n + 1] = fmaf(xq, y.y, fmaf(-xw, u.y, acc[4 * n + 1]));
-                    acc[4 * n + 2] = fmaf(xq, y.z, fmaf(-xw, u.z, acc[4 * n + 2]));
-                    acc[4 * n + 3] = fmaf(xq, y.w, fmaf(-xw, u.w, acc[4 * n + 3]));
+                for (int hh = 0; hh < 2; ++hh) {
+                    float* sp = Ss + (sr0 + gid + 8 * hh) * LDS + sc0 + 8 * t + 2 * tig;
+                    const float2 o = *reinterpret_cast<const float2*>(sp);
+                    *reinterpret_cast<float2*>(sp) =
+                        make_float2(fmaf(gC, o.x, a1[t][2 * hh] - a2[t][2 * hh]),
+                                    fmaf(gC, o.y, a1[t][2 * hh + 1] - a2[t][2 * hh + 1]));
                 }
-            }
-#pragma unroll
-            for (int n = 0; n < NC; ++n) Ss[m * LDS + n0 + n] = fmaf(gC, Ss[m * LDS + n0 + n], acc[n]);
         }
     }
     __syncthreads();
