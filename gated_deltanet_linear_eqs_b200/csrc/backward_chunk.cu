@@ -1,6 +1,8 @@
 // backward_chunk.cu -- the backward pass of eqs. (1)-(4) (Qwen3.8-Flash-Next summary, picx.dev,
 // "Theoretical foundations"; the reverse recurrence of its Appendix B) in the chunked WY form of
-// the forward, on 64-token chunks, in fp32.
+// the forward, on 64-token chunks, in fp32 with the products on tensor cores (warp-level
+// m16n8k8 tf32 tiles, fp32 accumulation; the reverse chain's dS products with split 3 x tf32
+// operands, since their rounding accumulates into dS0 along the whole chain).
 //
 // Per chunk, with q^ = rq q, k^ = rk k the normalised rows, Lg the inclusive cumsum of ln(alpha),
 // gam = e^Lg, gC = gam of the chunk's last token, Gam_ij = e^(Lg_i - Lg_j), S = S^c the state at
