@@ -200,17 +200,18 @@ __device__ __forceinline__ void wmma_acc3(float (&acc)[CT][4], int K, int r0, in
     for (int k0 = 0; k0 < K; k0 += 8) {
         const float af[4] = {a(r0 + gid, k0 + tig), a(r0 + gid + 8, k0 + tig), a(r0 + gid, k0 + tig + 4),
                              a(r0 + gid + 8, k0 + tig + 4)};
+        // the high part's low 13 bits are cleared so that it reads back as the exact tf32 value
         uint32_t ah[4], al[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            ah[e] = to_tf32(af[e]);
+            ah[e] = to_tf32(af[e]) & 0xffffe000u;
             al[e] = to_tf32(af[e] - __uint_as_float(ah[e]));
         }
 #pragma unroll
         for (int t = 0; t < CT; ++t) {
             const int n = c0 + 8 * t + gid;
             const float b0 = b(k0 + tig, n), b1 = b(k0 + tig + 4, n);
-            const uint32_t bh0 = to_tf32(b0), bh1 = to_tf32(b1);
+            const uint32_t bh0 = to_tf32(b0) & 0xffffe000u, bh1 = to_tf32(b1) & 0xffffe000u;
             const uint32_t bl0 = to_tf32(b0 - __uint_as_float(bh0)), bl1 = to_tf32(b1 - __uint_as_float(bh1));
             mma_tf32(acc[t], al[0], al[1], al[2], al[3], bh0, bh1);
             mma_tf32(acc[t], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
