@@ -291,7 +291,56 @@ def run_ours(args, rank, world, local_rank):
     if args.only in ("all", "gated"):
         out["gated_norm"] = run_gated_norm(args, dev, uuid, peaks, peak_src, max_over_ranks,
                                            barrier)
+    if args.only in ("all", "segmented"):
+        out["segmented"] = run_segmented(args, dev, max_over_ranks, barrier, rank, world)
     return out
+
+
+SEG_B, SEG_T, SEG_H = 1, 131072, 4  # few, long chains: 4 heads x 4 column slices of 2048 chunks
+
+
+def run_segmented(args, dev, max_over_ranks, barrier, rank, world=1):
+    """One long sequence with few heads, where the plain prefill runs only B H dv/32 = 16 chains:
+    the plain call against gdn_prefill_segmented at several segment counts."""
+    import torch
+    from gated_deltanet_linear_eqs_b200 import api
+    from gated_deltanet_linear_eqs_b200._abi import GDN_OP_PREFILL, GDN_OP_PREFILL_SEGMENTED
+    from gated_deltanet_linear_eqs_b200.inputs import make_inputs
+    inp = make_inputs(SEG_B, SEG_T, SEG_H, D, D, seed=rank, with_s0=True)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    y = torch.empty((SEG_B, SEG_T, SEG_H, D), dtype=torch.bfloat16, device=dev)
+    sf = torch.empty((SEG_B, SEG_H, D, D), dtype=torch.float32, device=dev)
+    res = {"config": {"workload": f"one sequence: B={SEG_B}, T={SEG_T}, H={SEG_H}, dk=dv={D}, "
+                                  "bf16, S0 ~ N(0, 0.02^2)"}}
+    for P in (1, 8, 16):
+        op = GDN_OP_PREFILL if P == 1 else GDN_OP_PREFILL_SEGMENTED
+        ws = torch.empty(api.gdn_workspace_bytes(op, SEG_B, SEG_T, SEG_H, D, D, P),
+                         dtype=torch.uint8, device=dev)
+
+        def run():
+            if P == 1:
+                api.gdn_prefill(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["s0"], y=y,
+                                s_final=sf, ws=ws)
+            else:
+                api.gdn_prefill_segmented(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                          g["s0"], num_segments=P, y=y, s_final=sf, ws=ws)
+        for _ in range(max(3, args.warmup)):
+            run()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        n = max(3, min(args.steps, 10))
+        e0.record()
+        for _ in range(n):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1) / n)
+        res[f"segments_{P}"] = {"ms_per_step": ms,
+                                "tokens_per_s": world * SEG_B * SEG_T / (ms / 1e3)}
+        del ws
+    return res
 
 
 NORM_ROWS = T_TOTAL * H  # one gated RMSNorm row per (token, head) of the prefill workload
@@ -555,7 +604,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "train", "gated"],
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "train", "gated", "segmented"],
                     default="all")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--train-steps", type=int, default=3)
@@ -608,6 +657,8 @@ def main():
                     clocks=p["clocks"], e2e=res["e2e"], gpu_launches=3 * args.steps)
     if "train" in res:
         line["train"] = res["train"]
+    if "segmented" in res:
+        line["segmented"] = res["segmented"]
     if "gated_norm" in res:
         line["gated_norm"] = res["gated_norm"]
         if "prefill" not in res and "decode" not in res:

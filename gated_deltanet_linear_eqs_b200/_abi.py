@@ -30,6 +30,7 @@ GDN_OP_PREFILL = 0
 GDN_OP_PREFILL_VARLEN = 1
 GDN_OP_DECODE = 2
 GDN_OP_BACKWARD = 3
+GDN_OP_PREFILL_SEGMENTED = 4
 
 _P = ctypes.c_void_p
 _F = ctypes.c_float
@@ -62,6 +63,7 @@ SIGNATURES = {
     "gdn_gated_rmsnorm_backward": (_I, [_P] * 7 + [ctypes.c_int64, _I, _I, _F, _P]),
     "gdn_read_device_status": (_I, [_I, ctypes.POINTER(_I)]),
     "gdn_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
+    "gdn_prefill_segmented": (_I, [_P] * 8 + [_I] * 6 + [_F, _I, _I, _P, _S, _P]),
 }
 
 _lock = threading.Lock()

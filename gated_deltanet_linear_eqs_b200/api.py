@@ -95,6 +95,39 @@ def gdn_prefill(q, k, v, alpha, beta, s0=None, scale=1.0, l2norm_qk=True, y=None
     return y, s_final
 
 
+def gdn_prefill_segmented(q, k, v, alpha, beta, s0=None, num_segments=1, scale=1.0,
+                          l2norm_qk=True, y=None, s_final=None, want_final=True, ws=None,
+                          stream=None):
+    """gdn_prefill with every sequence cut into ``num_segments`` segments that run side by side
+    (affine state maps, a scan, and a pass from every segment's start state).  Same tensors as
+    gdn_prefill.  Returns (y, s_final)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _need(q, "q", dt)
+    _need(k, "k", dt, q.shape)
+    _need(v, "v", dt, (B, T, H, dv))
+    _need(alpha, "alpha", torch.float32, (B, T, H))
+    _need(beta, "beta", torch.float32, (B, T, H))
+    _need(s0, "s0", torch.float32, (B, H, dk, dv), optional=True)
+    if y is None:
+        y = torch.empty((B, T, H, dv), dtype=dt, device=q.device)
+    _need(y, "y", dt, (B, T, H, dv))
+    if s_final is None and want_final:
+        s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(s_final, "s_final", torch.float32, (B, H, dk, dv), optional=True)
+    ws, wsb = _workspace(_abi.GDN_OP_PREFILL_SEGMENTED, q.device, B, T, H, dk, dv,
+                         int(num_segments), ws=ws)
+    rc = _lib().gdn_prefill_segmented(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(s0), _p(y),
+                                      _p(s_final), B, T, H, dk, dv, _DT[dt], float(scale),
+                                      int(bool(l2norm_qk)), int(num_segments), _p(ws), wsb,
+                                      _stream(stream))
+    _check(rc, "gdn_prefill_segmented")
+    return y, s_final
+
+
 def gdn_prefill_varlen(q, k, v, alpha, beta, cu_seqlens, s0=None, scale=1.0, l2norm_qk=True,
                        y=None, s_final=None, ws=None, stream=None):
     """Packed documents: q,k [1,T,H,dk] (or [T,H,dk]), v likewise, alpha,beta [1,T,H],

@@ -104,6 +104,13 @@ int gdn_workspace_bytes(int op, int B, int T, int H, int dk, int dv, int num_seq
             if (B < 1) return GDN_ERR_INVALID_ARG;
             *bytes = gdn::backward_chunked_workspace_bytes(B, T, H, dk, dv);
             return GDN_OK;
+        case GDN_OP_PREFILL_SEGMENTED: {  // num_seqs carries the number of segments
+            if (B < 1 || num_seqs < 1) return GDN_ERR_INVALID_ARG;
+            const size_t a = gdn::segmented_layout(B, T, H, dk, num_seqs, GDN_BF16).total;
+            const size_t f = gdn::segmented_layout(B, T, H, dk, num_seqs, GDN_FP32).total;
+            *bytes = a > f ? a : f;
+            return GDN_OK;
+        }
         default:
             return GDN_ERR_INVALID_ARG;
     }
@@ -374,6 +381,25 @@ int gdn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
     if (int rc = current_device_info(&dev)) return rc;
     return map_cuda(gdn::launch_wait_timeout_selftest(dev.status, limit_ns,
                                                       static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_prefill_segmented(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* beta, const float* s0, void* y, float* s_final, int B,
+                          int T, int H, int dk, int dv, int dtype, float scale, int l2norm_qk,
+                          int num_segments, void* ws, size_t ws_bytes, void* stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
+        !ok_ptr(y) || !ok_opt_ptr(s0) || !ok_opt_ptr(s_final))
+        return GDN_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || H < 1 || num_segments < 1) return GDN_ERR_INVALID_ARG;
+    if (int rc = check_dims(dk, dv, dtype)) return rc;
+    const size_t need = gdn::segmented_layout(B, T, H, dk, num_segments, dtype).total;
+    if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return GDN_ERR_WORKSPACE;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::PrefillArgs a{q, k, v, alpha, beta, s0, y, s_final, nullptr, B, T, H, dk, dv,
+                       dtype, scale, l2norm_qk ? 1 : 0, dev.status, ws, ws_bytes};
+    return map_cuda(gdn::launch_prefill_segmented(a, num_segments,
+                                                  static_cast<cudaStream_t>(stream)));
 }
 
 int gdn_read_device_status(int reset, int* device_status) {

@@ -108,6 +108,16 @@ cudaError_t launch_gated_norm_backward(const GatedNormArgs& a, cudaStream_t st);
 // GDN_ERR_TIMEOUT in `status` after about limit_ns and returns.
 cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns, cudaStream_t st);
 
+// Segment-parallel prefill of a dense batch (segmented.cu): every sequence cut into P segments
+// of L tokens (whole chunks), the segments' affine state maps formed by two prefill passes, a
+// scan of the maps from s0, and a third pass from the segments' start states.
+struct SegmentedLayout {
+    int L, P;  // segment length in tokens; number of non-empty segments
+    size_t off_inner, inner_bytes, off_cu, off_vzero, off_eye, off_m, off_n, off_start, total;
+};
+SegmentedLayout segmented_layout(int B, int T, int H, int D, int P, int dtype);
+cudaError_t launch_prefill_segmented(const PrefillArgs& a, int P, cudaStream_t st);
+
 // Size of the fixed device scratch array behind gdn_backward_noalloc.
 constexpr size_t kBackwardFixedScratchBytes = size_t(32) << 20;
 // Device address of that array on the current device (looked up on first use per device).

@@ -60,7 +60,8 @@ typedef enum {
     GDN_OP_PREFILL = 0,
     GDN_OP_PREFILL_VARLEN = 1,
     GDN_OP_DECODE = 2,
-    GDN_OP_BACKWARD = 3
+    GDN_OP_BACKWARD = 3,
+    GDN_OP_PREFILL_SEGMENTED = 4  /* num_seqs carries the number of segments */
 } gdn_op;
 
 /* Static description of a status code.  Never NULL. */
@@ -278,6 +279,28 @@ int gdn_gated_rmsnorm_backward(const void* y, const void* z, const float* w, con
  * Synchronises the current device.  If reset != 0 the word is cleared.
  */
 int gdn_read_device_status(int reset, int* device_status);
+
+/*
+ * gdn_prefill_segmented -- gdn_prefill of a dense batch with every sequence cut along time into
+ * num_segments segments that run side by side.  By eqs. (1)-(3) one token maps the state
+ * affinely (S -> alpha (I - beta k k^T) S + beta k v^T), so each segment acts on its start state
+ * as S -> M S + N, computable from its own tokens.  The call runs the B * P segments as packed
+ * documents: once with v = 0 from S0 = I (giving every M), once from S0 = 0 (every N), scans
+ * the maps from s0 for every segment's start state (fp32), and once more from the start states
+ * (giving y).  This pays three prefill passes for B * P independent chains instead of B: it is
+ * for batches of few, long sequences, where the plain call leaves most SMs idle.
+ *   - Arguments and layouts as gdn_prefill; num_segments >= 1.  Segments are whole 64-token
+ *     chunks of ceil(ceil(T / 64) / num_segments) chunks each, so fewer may result; with one
+ *     segment the call is gdn_prefill.  dk == dv.
+ *   - s_final (if non-NULL) is the scan's state after the last segment.
+ *   - ws/ws_bytes: gdn_workspace_bytes(GDN_OP_PREFILL_SEGMENTED, B, T, H, dk, dv, num_segments).
+ *     It holds the inner packed prefill's workspace (bf16), a zero copy of v, and four fp32
+ *     states per (segment, head).
+ */
+int gdn_prefill_segmented(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* beta, const float* s0, void* y, float* s_final, int B,
+                          int T, int H, int dk, int dv, int dtype, float scale, int l2norm_qk,
+                          int num_segments, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * gdn_selftest_wait_timeout -- exercises the failure path of the library's bounded waits.

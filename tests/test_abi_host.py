@@ -227,6 +227,30 @@ def test_selftest_rejects_limits_out_of_range(lib):
     assert lib.gdn_selftest_wait_timeout(2_000_000_000, None) == _abi.GDN_ERR_INVALID_ARG
 
 
+def test_segmented_workspace_and_validation(lib):
+    n = ctypes.c_size_t(0)
+    plain = ctypes.c_size_t(0)
+    # one segment is the plain prefill, with its workspace
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL_SEGMENTED, 1, 4096, 16, 128, 128, 1,
+                                   ctypes.byref(n)) == 0
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL, 1, 4096, 16, 128, 128, 0,
+                                   ctypes.byref(plain)) == 0
+    assert n.value == plain.value
+    # four segments of 1024 tokens: the packed prefill's workspace for 4 documents, the zero
+    # copy of v (bf16 here, fp32 for fp32 inputs: the larger is reported) and 4 state arrays
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL_SEGMENTED, 1, 4096, 16, 128, 128, 4,
+                                   ctypes.byref(n)) == 0
+    states = 4 * 4 * 16 * 128 * 128 * 4
+    assert n.value >= 4096 * 16 * 128 * 4 + states
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL_SEGMENTED, 1, 4096, 16, 128, 128, 0,
+                                   ctypes.byref(n)) == _abi.GDN_ERR_INVALID_ARG
+    f = lib.gdn_prefill_segmented
+    args = [A] * 5 + [0, A, 0, 1, 4096, 2, 128, 128, 0, 1.0, 1]
+    assert f(*args, 0, A, 1 << 40, None) == _abi.GDN_ERR_INVALID_ARG    # no segments
+    assert f(*args, 4, None, 0, None) == _abi.GDN_ERR_WORKSPACE
+    assert f(*args, 4, A, 16, None) == _abi.GDN_ERR_WORKSPACE
+
+
 def test_device_status_rejects_null(lib):
     assert lib.gdn_read_device_status(0, None) == _abi.GDN_ERR_INVALID_ARG
 
