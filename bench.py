@@ -284,9 +284,10 @@ def run_ours(args, rank, world, local_rank):
                       "ms_per_step": e2e_ms}
 
     if args.only in ("all", "decode") and args.decode_steps > 0:
-        out["decode"] = run_decode(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier)
+        out["decode"] = run_decode(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier,
+                                    world)
     if args.only in ("all", "train") and args.train_steps > 0:
-        out["train"] = run_train(args, dev, uuid, max_over_ranks, barrier, rank)
+        out["train"] = run_train(args, dev, uuid, max_over_ranks, barrier, rank, world)
     if args.only in ("all", "gated"):
         out["gated_norm"] = run_gated_norm(args, dev, uuid, peaks, peak_src, max_over_ranks,
                                            barrier)
@@ -350,7 +351,7 @@ def train_inputs(dev, seed=0):
     return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
 
 
-def run_train(args, dev, uuid, max_over_ranks, barrier, rank):
+def run_train(args, dev, uuid, max_over_ranks, barrier, rank, world=1):
     """Training shape: forward (gdn_prefill: prep and chain kernels) + backward (gdn_backward:
     chunk-matrix, forward-chain, reverse-chain and local-gradient kernels) per step."""
     import torch
@@ -385,9 +386,9 @@ def run_train(args, dev, uuid, max_over_ranks, barrier, rank):
         torch.cuda.synchronize()
     f_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
     b_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
-    tokens = TRAIN_B * TRAIN_T
+    tokens = TRAIN_B * TRAIN_T  # per rank; the value is the whole job's
     return {"metric": "GDN fwd+bwd tokens/s (training shape)", "unit": "tokens/s",
-            "value": tokens / ((f_ms + b_ms) / 1e3), "ms_per_step": f_ms + b_ms,
+            "value": world * tokens / ((f_ms + b_ms) / 1e3), "ms_per_step": f_ms + b_ms,
             "fwd_ms": f_ms, "bwd_ms": b_ms, "steps": steps, "gpu_launches": 6 * steps,
             "config": {"workload": f"train: B={TRAIN_B}, T={TRAIN_T}, H={TRAIN_H}, dk=dv={D}, "
                                    "bf16, dy ~ N(0,1), S0 = 0"},
@@ -436,7 +437,7 @@ def run_profile(args):
     return 0
 
 
-def run_decode(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier):
+def run_decode(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier, world=1):
     import torch
     from gated_deltanet_linear_eqs_b200 import api
     from gated_deltanet_linear_eqs_b200.inputs import make_decode_state, make_decode_step_inputs
@@ -469,8 +470,8 @@ def run_decode(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier):
         torch.cuda.synchronize()
     step_ms = max_over_ranks(e0.elapsed_time(e1) / nsteps)
     bytes_step = DEC_N * H * (2 * D * D * 4 + BYTES_PER_TOKEN_HEAD)
-    gbs = bytes_step / (step_ms / 1e3) / 1e9
-    return {"metric": "decode-step state GB/s", "value": gbs, "unit": "GB/s",
+    gbs = bytes_step / (step_ms / 1e3) / 1e9  # per GPU (the roofline's); the value is the job's
+    return {"metric": "decode-step state GB/s", "value": world * gbs, "unit": "GB/s",
             "ms_per_step": step_ms, "steps": nsteps, "gpu_launches": nsteps,
             "config": {"workload": f"decode: {DEC_N} sequences x {H} heads, dk=dv={D}, fp32 "
                                    f"state updated in place, bf16 tokens, {nsteps} steps",

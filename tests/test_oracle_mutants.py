@@ -167,3 +167,35 @@ SEGMENT_MUTANTS = [
 def test_segment_pins_reject_mutant(tmp_path, name, old, new):
     caught = _python_mutant_caught(tmp_path, SEGMENTS_SRC, seg_pins.CHECKS, name, old, new)
     assert caught, f"no pin rejects the planted mistake {name!r}"
+
+
+CHUNKED_SRC = os.path.join(os.path.dirname(oracle.__file__), "chunked.py")
+
+CHUNKED_CHECKS = [
+    lambda m: pins.test_chunked_form_matches_token_loop(16, True, m),
+    lambda m: pins.test_chunked_form_matches_token_loop(64, False, m),
+    lambda m: pins.test_chunked_form_small_alpha_no_overflow(m),
+    lambda m: pins.test_chunked_backward_matches_reverse_recurrence(16, True, m),
+    lambda m: pins.test_chunked_backward_matches_reverse_recurrence(64, False, m),
+]
+
+CHUNKED_MUTANTS = [
+    ("A_sign", "A = np.tril(be[:, None] * (K @ K.T) * Gam, k=-1)",
+     "A = -np.tril(be[:, None] * (K @ K.T) * Gam, k=-1)"),
+    ("output_without_decay_mask", "((Q @ K.T) * Gam) @ U", "(Q @ K.T) @ U"),
+    ("state_not_decayed", "S = gam[-1] * S + (Gam[-1][:, None] * K).T @ U", "S = S + (Gam[-1][:, None] * K).T @ U"),
+    ("W_without_gamma", "W = solve_triangular(IA, (be * gam)[:, None] * K",
+     "W = solve_triangular(IA, be[:, None] * K"),
+    ("bwd_dV_without_beta", "dV = be[:, None] * Z1", "dV = Z1"),
+    ("bwd_dA_sign", "dA = np.tril(-(Tm.T @ dT @ Tm.T), k=-1)", "dA = np.tril(Tm.T @ dT @ Tm.T, k=-1)"),
+    ("bwd_forward_cumsum", "dlna = np.cumsum(dG[::-1])[::-1]", "dlna = np.cumsum(dG)"),
+    ("bwd_E_transpose_dropped", "dKh += E @ Kh + E.T @ Kh + F.T @ Qh", "dKh += E @ Kh + F.T @ Qh"),
+    ("bwd_dU_without_decay", 'c["dU"] = c["dec"][:, None] * (c["Kh"] @ dS) + scale * c["QK"].T @ c["dY"]',
+     'c["dU"] = (c["Kh"] @ dS) + scale * c["QK"].T @ c["dY"]'),
+]
+
+
+@pytest.mark.parametrize("name,old,new", CHUNKED_MUTANTS, ids=[m[0] for m in CHUNKED_MUTANTS])
+def test_chunked_pins_reject_mutant(tmp_path, name, old, new):
+    caught = _python_mutant_caught(tmp_path, CHUNKED_SRC, CHUNKED_CHECKS, name, old, new)
+    assert caught, f"no pin rejects the planted mistake {name!r}"
