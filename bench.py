@@ -386,7 +386,38 @@ def run_gated_norm(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier):
     res["config"] = {"workload": f"gated RMSNorm (eq. (11) bracket): {NORM_ROWS} rows "
                                  f"(T={T_TOTAL} x H={H}) of dv={D}, bf16 y/z/o, fp32 w",
                      "l2": "each launch streams >= 403 MB, beyond the 126 MB L2; no flush"}
-    res["gpu_launches"] = 2 * args.steps
+    # the gated recurrence on the headline workload: logits of eqs. (9)-(10) in place of alpha,
+    # beta; the same bytes per token as the plain call, the gates evaluated where alpha is loaded
+    from gated_deltanet_linear_eqs_b200._abi import GDN_OP_PREFILL_VARLEN
+    from gated_deltanet_linear_eqs_b200.inputs import make_gate_inputs
+    _, inp = varlen_workload(seed=0)
+    gv = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    gi = {k: v.to(dev) for k, v in make_gate_inputs((1, T_TOTAL, H), H, seed=0).items()}
+    ws = torch.empty(api.gdn_workspace_bytes(GDN_OP_PREFILL_VARLEN, 1, T_TOTAL, H, D, D, NDOCS),
+                     dtype=torch.uint8, device=dev)
+    y = torch.empty((1, T_TOTAL, H, D), dtype=torch.bfloat16, device=dev)
+    sf = torch.empty((NDOCS, H, D, D), dtype=torch.float32, device=dev)
+
+    def gated_step():
+        api.gdn_prefill_varlen_gated(gv["q"], gv["k"], gv["v"], gi["a"], gi["b"], gi["A_log"],
+                                     gi["b_alpha"], gv["cu_seqlens"], gv["s0"], y=y, s_final=sf,
+                                     ws=ws)
+    for _ in range(max(3, args.warmup)):
+        gated_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        gated_step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    res["gated_prefill"] = {"ms_per_step": ms, "tokens_per_s": T_TOTAL / (ms / 1e3),
+                            "workload": "the headline varlen workload with gate logits a, b ~ N(0, 1), "
+                                        "A_log ~ U(-1, 1), b_alpha ~ N(0, 0.5^2) per head"}
+    res["gpu_launches"] = 2 * args.steps + 3 * args.steps
     return res
 
 
