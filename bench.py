@@ -586,6 +586,18 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline(target_s=12.0):
     cores = cpu_cores()
     threads = min(cores, H)
@@ -594,7 +606,8 @@ def cpu_baseline(target_s=12.0):
     dt, _ = oracle_sample(n, threads)
     return {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"fp64 token-loop oracle on the first {n} tokens of the 16749-token "
-                      f"document, all {H} heads (threads over heads), {dt:.1f} s"}
+                      f"document, all {H} heads (threads over heads), {dt:.1f} s",
+            "host_cpus": cores, "cpu_model": cpu_model()}
 
 
 def run_reference(args):
@@ -617,7 +630,8 @@ def run_reference(args):
         "config": {"workload": WORKLOAD_NAME, "sample_tokens_per_step": n_tok},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": f"each step: fp64 oracle on {n_tok} tokens x {H} heads of "
-                                   "the longest document"},
+                                   "the longest document",
+                         "host_cpus": cores, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,

@@ -54,4 +54,5 @@ def test_reference_arm_prints_one_json_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["host_cpus"] >= d["cpu_baseline"]["cores"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["gpu_launches"] == 0
