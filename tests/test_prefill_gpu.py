@@ -214,3 +214,21 @@ def test_prefill_slow_decay_state_accuracy():
     yr, sr = oracle.forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["s0"])
     assert max_rel(y, yr) <= Y_TOL
     assert frob_rel(sf, sr) <= S_TOL
+
+
+def test_prefill_varlen_many_documents_beyond_the_shared_map():
+    """More documents than the chunk-base scan keeps in shared memory (8192): the record map is
+    searched in global memory.  Lengths 0..4 tokens, so most documents are a single ragged chunk."""
+    import numpy as np
+    rng = np.random.default_rng(12)
+    lengths = [int(x) for x in rng.integers(0, 5, 9000)]
+    H, d = 1, 64
+    inp = make_varlen_inputs(lengths, H, d, d, seed=13)
+    g = _cuda(inp)
+    y, sf = api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                   g["cu_seqlens"], g["s0"])
+    torch.cuda.synchronize()
+    yr, sr = oracle.forward_varlen(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                                   inp["cu_seqlens"].numpy(), inp["s0"])
+    assert max_rel(y, yr) <= Y_TOL
+    assert frob_rel(sf, sr) <= S_TOL
