@@ -232,3 +232,18 @@ def test_prefill_varlen_many_documents_beyond_the_shared_map():
                                    inp["cu_seqlens"].numpy(), inp["s0"])
     assert max_rel(y, yr) <= Y_TOL
     assert frob_rel(sf, sr) <= S_TOL
+
+
+@pytest.mark.parametrize("lengths", [[1, 63, 64, 65, 130], [0, 300, 7]])
+def test_prefill_varlen_d64(lengths):
+    """The packed bf16 path at dk = dv = 64 (two 32-column chain slices per head)."""
+    H, d = 3, 64
+    inp = make_varlen_inputs(lengths, H, d, d, seed=7 + sum(lengths))
+    g = _cuda(inp)
+    y, sf = api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                   g["cu_seqlens"], g["s0"], scale=0.6)
+    torch.cuda.synchronize()
+    yr, sr = oracle.forward_varlen(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                                   inp["cu_seqlens"].numpy(), inp["s0"], scale=0.6)
+    assert max_rel(y, yr) <= Y_TOL
+    assert frob_rel(sf, sr) <= S_TOL
