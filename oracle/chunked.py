@@ -68,6 +68,103 @@ def forward_chunked(q, k, v, alpha, beta, s0=None, C=64, scale=1.0, l2norm=True,
     return y, sf
 
 
+def blocked_unit_lower_inverse(A, bs=16):
+    """T = (I + A)^-1 for strictly lower-triangular A (n x n), in the blocked order the CUDA
+    kernels use: the diagonal bs x bs blocks by forward substitution, then the off-diagonal
+    blocks by increasing block distance, T_ij = -T_ii sum_{j <= m < i} A_im T_mj (blocks)."""
+    A = np.asarray(A, dtype=np.float64)
+    n = A.shape[0]
+    nb = (n + bs - 1) // bs
+    T = np.zeros((n, n))
+    blk = lambda i: slice(i * bs, min(n, (i + 1) * bs))
+    for b in range(nb):                       # diagonal blocks: (I + A_bb) T_bb = I
+        s = blk(b)
+        m = s.stop - s.start
+        Ab = A[s, s]
+        Tb = np.zeros((m, m))
+        for col in range(m):
+            x = np.zeros(m)
+            for r in range(m):
+                x[r] = (1.0 if r == col else 0.0) - Ab[r, :r] @ x[:r]
+            Tb[:, col] = x
+        T[s, s] = Tb
+    for dist in range(1, nb):                  # off-diagonal blocks, nearest first
+        for bj in range(nb - dist):
+            bi = bj + dist
+            acc = sum(A[blk(bi), blk(mb)] @ T[blk(mb), blk(bj)] for mb in range(bj, bi))
+            T[blk(bi), blk(bj)] = -T[blk(bi), blk(bi)] @ acc
+    return T
+
+
+def forward_chunked_coupled(q, k, v, alpha, beta, s0=None, C=64, scale=1.0, l2norm=True,
+                            eps=EPS, unroll=False):
+    """The chunked forward in the coupled form the CUDA prefill's sequential kernel runs, same
+    contract as ``forward_chunked``.  With S^c the state at the start of chunk c, gamma_c the
+    chunk's total decay, D_c = diag(Gam_{n,.}) (so that S^{c+1} = gamma_c S^c + K_c^T D_c U_c) and
+    X_c = -W_c K_{c-1}^T:
+
+        U_c = Ut_c + gamma_{c-1} (-W_c S^{c-1}) + X_c D_{c-1} U_{c-1}      (c >= 1)
+
+    so the only chunk-to-chunk dependence is through U and a state one chunk back.  With
+    ``unroll`` the recurrence is also stepped two chunks at a time:
+
+        U_{c+1} = Ut_{c+1} + X_{c+1} D_c Ut_c + A1 S^{c-1} + A2 D_{c-1} U_{c-1},
+        A1 = -gamma_c gamma_{c-1} W_{c+1} - gamma_{c-1} X_{c+1} D_c W_c,
+        A2 = X_{c+1} D_c X_c - gamma_c W_{c+1} K_{c-1}^T,
+
+    which depends on chunk c only through chunk-local quantities."""
+    q, k, v, alpha, beta = (np.asarray(x, dtype=np.float64) for x in (q, k, v, alpha, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    y = np.zeros((B, T, H, dv))
+    sf = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            ch = []
+            for t0 in range(0, T, C):
+                t1 = min(T, t0 + C)
+                n = t1 - t0
+                K = _l2n(k[b, t0:t1, h], eps, l2norm)
+                Q = _l2n(q[b, t0:t1, h], eps, l2norm)
+                be = beta[b, t0:t1, h]
+                G = np.cumsum(np.log(alpha[b, t0:t1, h]))
+                lower = np.tril(np.ones((n, n), dtype=bool))
+                Gam = np.where(lower, np.exp(np.where(lower, G[:, None] - G[None, :], 0.0)), 0.0)
+                gam = np.exp(G)
+                IA = np.eye(n) + np.tril(be[:, None] * (K @ K.T) * Gam, k=-1)
+                W = solve_triangular(IA, (be * gam)[:, None] * K, lower=True, unit_diagonal=True)
+                Ut = solve_triangular(IA, be[:, None] * v[b, t0:t1, h], lower=True,
+                                      unit_diagonal=True)
+                ch.append(dict(t0=t0, t1=t1, K=K, Q=Q, W=W, Ut=Ut, gam=gam, g=gam[-1],
+                               D=Gam[-1][:, None], P=(Q @ K.T) * Gam))
+            for c in range(1, len(ch)):
+                ch[c]["X"] = -ch[c]["W"] @ ch[c - 1]["K"].T
+            S = [np.zeros((dk, dv)) if s0 is None else np.array(s0[b, h], dtype=np.float64)]
+            U = []
+            c = 0
+            while c < len(ch):
+                d = ch[c]
+                if c == 0:
+                    U.append(d["Ut"] - d["W"] @ S[0])
+                elif unroll and c >= 2 and c % 2 == 0:
+                    # U_c from (S^{c-2}, U_{c-2}) through the unrolled pair coefficients
+                    m, mm = ch[c - 1], ch[c - 2]
+                    A1 = -m["g"] * mm["g"] * d["W"] - mm["g"] * d["X"] @ (m["D"] * m["W"])
+                    A2 = d["X"] @ (m["D"] * m["X"]) - m["g"] * d["W"] @ mm["K"].T
+                    U.append(d["Ut"] + d["X"] @ (m["D"] * m["Ut"]) + A1 @ S[c - 2]
+                             + A2 @ (mm["D"] * U[c - 2]))
+                else:
+                    m = ch[c - 1]
+                    U.append(d["Ut"] + m["g"] * (-d["W"] @ S[c - 1]) + d["X"] @ (m["D"] * U[c - 1]))
+                S.append(d["g"] * S[c] + d["K"].T @ (d["D"] * U[c]))
+                c += 1
+            for c, d in enumerate(ch):
+                y[b, d["t0"]:d["t1"], h] = scale * (d["gam"][:, None] * (d["Q"] @ S[c])
+                                                    + d["P"] @ U[c])
+            sf[b, h] = S[-1]
+    return y, sf
+
+
 def backward_chunked(q, k, v, alpha, beta, s0=None, dy=None, ds_final=None, C=64, scale=1.0,
                      l2norm=True, eps=EPS):
     """Gradients of L = <dy, y> + <ds_final, S_T> in the chunked form; same contract as

@@ -177,6 +177,10 @@ CHUNKED_CHECKS = [
     lambda m: pins.test_chunked_form_small_alpha_no_overflow(m),
     lambda m: pins.test_chunked_backward_matches_reverse_recurrence(16, True, m),
     lambda m: pins.test_chunked_backward_matches_reverse_recurrence(64, False, m),
+    lambda m: pins.test_coupled_chunk_form_matches_token_loop(False, m),
+    lambda m: pins.test_coupled_chunk_form_matches_token_loop(True, m),
+    lambda m: pins.test_blocked_inverse_matches_dense_inverse(64, m),
+    lambda m: pins.test_blocked_inverse_matches_dense_inverse(50, m),
 ]
 
 CHUNKED_MUTANTS = [
@@ -184,12 +188,26 @@ CHUNKED_MUTANTS = [
      "A = -np.tril(be[:, None] * (K @ K.T) * Gam, k=-1)"),
     ("output_without_decay_mask", "((Q @ K.T) * Gam) @ U", "(Q @ K.T) @ U"),
     ("state_not_decayed", "S = gam[-1] * S + (Gam[-1][:, None] * K).T @ U", "S = S + (Gam[-1][:, None] * K).T @ U"),
-    ("W_without_gamma", "W = solve_triangular(IA, (be * gam)[:, None] * K",
-     "W = solve_triangular(IA, be[:, None] * K"),
+    ("W_without_gamma", "W = solve_triangular(IA, (be * gam)[:, None] * K, lower=True, unit_diagonal=True)\n"
+     "                Ut = solve_triangular(IA, be[:, None] * V,",
+     "W = solve_triangular(IA, be[:, None] * K, lower=True, unit_diagonal=True)\n"
+     "                Ut = solve_triangular(IA, be[:, None] * V,"),
     ("bwd_dV_without_beta", "dV = be[:, None] * Z1", "dV = Z1"),
     ("bwd_dA_sign", "dA = np.tril(-(Tm.T @ dT @ Tm.T), k=-1)", "dA = np.tril(Tm.T @ dT @ Tm.T, k=-1)"),
     ("bwd_forward_cumsum", "dlna = np.cumsum(dG[::-1])[::-1]", "dlna = np.cumsum(dG)"),
     ("bwd_E_transpose_dropped", "dKh += E @ Kh + E.T @ Kh + F.T @ Qh", "dKh += E @ Kh + F.T @ Qh"),
+    ("coupled_X_sign", 'ch[c]["X"] = -ch[c]["W"] @ ch[c - 1]["K"].T',
+     'ch[c]["X"] = ch[c]["W"] @ ch[c - 1]["K"].T'),
+    ("coupled_state_one_back_undecayed",
+     'U.append(d["Ut"] + m["g"] * (-d["W"] @ S[c - 1]) + d["X"] @ (m["D"] * U[c - 1]))',
+     'U.append(d["Ut"] + (-d["W"] @ S[c - 1]) + d["X"] @ (m["D"] * U[c - 1]))'),
+    ("unrolled_A2_second_term_dropped",
+     'A2 = d["X"] @ (m["D"] * m["X"]) - m["g"] * d["W"] @ mm["K"].T', 'A2 = d["X"] @ (m["D"] * m["X"])'),
+    ("inverse_offdiag_sign", "T[blk(bi), blk(bj)] = -T[blk(bi), blk(bi)] @ acc",
+     "T[blk(bi), blk(bj)] = T[blk(bi), blk(bi)] @ acc"),
+    ("inverse_offdiag_missing_far_terms",
+     "acc = sum(A[blk(bi), blk(mb)] @ T[blk(mb), blk(bj)] for mb in range(bj, bi))",
+     "acc = A[blk(bi), blk(bj)] @ T[blk(bj), blk(bj)]"),
     ("bwd_dU_without_decay", 'c["dU"] = c["dec"][:, None] * (c["Kh"] @ dS) + scale * c["QK"].T @ c["dY"]',
      'c["dU"] = (c["Kh"] @ dS) + scale * c["QK"].T @ c["dY"]'),
 ]

@@ -256,6 +256,38 @@ def test_chunked_form_matches_token_loop(C, l2norm, chunked=None):
     np.testing.assert_allclose(sc, sf, rtol=1e-10, atol=1e-12)
 
 
+@pytest.mark.parametrize("n", [64, 50, 16, 1])
+def test_blocked_inverse_matches_dense_inverse(n, chunked=None):
+    """The 16 x 16 blocked inversion of the unit lower-triangular I + A that the kernels use
+    (diagonal blocks by substitution, off-diagonal blocks by distance) equals the dense inverse,
+    for A of the method's form strictLower(diag(beta) (K K^T * Gam))."""
+    inv = (chunked or oracle_chunked).blocked_unit_lower_inverse
+    rng = np.random.default_rng(19 + n)
+    K = _l2n(rng.standard_normal((n, 8)))
+    beta = rng.uniform(0.05, 0.95, n)
+    G = np.cumsum(np.log(rng.uniform(0.5, 0.999, n)))
+    Gam = np.exp(np.minimum(G[:, None] - G[None, :], 0.0))
+    A = np.tril(beta[:, None] * (K @ K.T) * Gam, k=-1)
+    ref = np.linalg.inv(np.eye(n) + A)
+    np.testing.assert_allclose(inv(A), ref, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("unroll", [False, True])
+def test_coupled_chunk_form_matches_token_loop(unroll, chunked=None):
+    """The coupled form the CUDA prefill's sequential kernel runs (U_c from U_{c-1} and a state
+    one chunk back through X_c = -W_c K_{c-1}^T), and its two-chunk unrolling, agree with the
+    token-by-token form (T not a multiple of C, nonzero S0, a scale)."""
+    fc = (chunked or oracle_chunked).forward_chunked_coupled
+    rng = np.random.default_rng(17)
+    q, k, v, alpha, beta, S0 = _rand(rng, 2, 330, 2, 16, 12)
+    slow = rng.uniform(0.9, 0.999, alpha.shape)  # chunk decays near 1: every coupling term counts
+    for a in (alpha, slow):
+        y, sf = oracle.forward(q, k, v, a, beta, S0, scale=0.8)
+        yc, sc = fc(q, k, v, a, beta, S0, C=32, scale=0.8, unroll=unroll)
+        np.testing.assert_allclose(yc, y, rtol=1e-9, atol=1e-11)
+        np.testing.assert_allclose(sc, sf, rtol=1e-9, atol=1e-11)
+
+
 def test_chunked_form_small_alpha_no_overflow(chunked=None):
     """Cumulative log-decay far below -88 within a chunk (exp(-G) alone would overflow
     fp64 only much later, but the relative form must stay finite and exact)."""
