@@ -6,7 +6,8 @@ Headline workload: one packed T = 32768 token stream of 4 seeded documents
 per-document initial state S0 ~ N(0, 0.02^2): one step = one gdn_prefill_varlen over the
 stream (norms, decay, intra-chunk WY, state passes, outputs, final states).  Also measured:
 the decode step (256 sequences x 16 heads, fp32 128x128 states, 1000 consecutive steps with
-fresh tokens) as a secondary object.
+fresh tokens), the training step (forward + backward) and the gated RMSNorm of eq. (11) over the
+workload's y (forward and backward) as secondary objects.
 
 Prints ONE JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own stream (weak
 scaling, no data-path collective); time is the max over ranks.
@@ -287,7 +288,137 @@ def run_ours(args, rank, world, local_rank):
                                     world)
     if args.only in ("all", "train") and args.train_steps > 0:
         out["train"] = run_train(args, dev, uuid, max_over_ranks, barrier, rank, world)
+    if args.only in ("all", "gated"):
+        out["gated_norm"] = run_gated_norm(args, dev, uuid, peaks, peak_src, max_over_ranks,
+                                           barrier)
+    if args.only in ("all", "segmented"):
+        out["segmented"] = run_segmented(args, dev, max_over_ranks, barrier, rank, world)
     return out
+
+
+SEG_B, SEG_T, SEG_H = 1, 131072, 4  # few, long chains: 4 heads x 4 column slices of 2048 chunks
+
+
+def run_segmented(args, dev, max_over_ranks, barrier, rank, world=1):
+    """One long sequence with few heads, where the plain prefill runs only B H dv/32 = 16 chains:
+    the plain call against gdn_prefill_segmented at several segment counts."""
+    import torch
+    from gated_deltanet_linear_eqs_b200 import api
+    from gated_deltanet_linear_eqs_b200._abi import GDN_OP_PREFILL, GDN_OP_PREFILL_SEGMENTED
+    from gated_deltanet_linear_eqs_b200.inputs import make_inputs
+    inp = make_inputs(SEG_B, SEG_T, SEG_H, D, D, seed=rank, with_s0=True)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    y = torch.empty((SEG_B, SEG_T, SEG_H, D), dtype=torch.bfloat16, device=dev)
+    sf = torch.empty((SEG_B, SEG_H, D, D), dtype=torch.float32, device=dev)
+    res = {"config": {"workload": f"one sequence: B={SEG_B}, T={SEG_T}, H={SEG_H}, dk=dv={D}, "
+                                  "bf16, S0 ~ N(0, 0.02^2)"}}
+    for P in (1, 8, 16):
+        op = GDN_OP_PREFILL if P == 1 else GDN_OP_PREFILL_SEGMENTED
+        ws = torch.empty(api.gdn_workspace_bytes(op, SEG_B, SEG_T, SEG_H, D, D, P),
+                         dtype=torch.uint8, device=dev)
+
+        def run():
+            if P == 1:
+                api.gdn_prefill(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["s0"], y=y,
+                                s_final=sf, ws=ws)
+            else:
+                api.gdn_prefill_segmented(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                          g["s0"], num_segments=P, y=y, s_final=sf, ws=ws)
+        for _ in range(max(3, args.warmup)):
+            run()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        n = max(3, min(args.steps, 10))
+        e0.record()
+        for _ in range(n):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1) / n)
+        res[f"segments_{P}"] = {"ms_per_step": ms,
+                                "tokens_per_s": world * SEG_B * SEG_T / (ms / 1e3)}
+        del ws
+    return res
+
+
+NORM_ROWS = T_TOTAL * H  # one gated RMSNorm row per (token, head) of the prefill workload
+
+
+def run_gated_norm(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier):
+    """The bracket of eq. (11) over the prefill workload's y (T*H rows of dv = 128, bf16):
+    forward and backward, each timed alone with CUDA events; both are HBM-bound streams."""
+    import torch
+    from gated_deltanet_linear_eqs_b200 import api
+    from gated_deltanet_linear_eqs_b200.inputs import make_norm_inputs
+    g = {k: v.to(dev) for k, v in make_norm_inputs(NORM_ROWS, D, seed=0, with_do=True).items()}
+    o = torch.empty_like(g["y"])
+    res = {}
+    for name, n_io, fn in (
+            ("forward", 3, lambda: api.gdn_gated_rmsnorm(g["y"], g["z"], g["w"], o=o)),
+            ("backward", 5, lambda: api.gdn_gated_rmsnorm_backward(g["y"], g["z"], g["w"],
+                                                                   g["d_o"]))):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with ClockSampler(uuid) as clk:
+            e0.record()
+            for _ in range(args.steps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        nbytes = NORM_ROWS * D * 2 * n_io + D * 4 * (1 if name == "forward" else 2)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        res[name] = {"ms_per_launch": ms, "bytes_per_launch": nbytes, "GB/s": gbs,
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                                  "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                                  "traffic": profile_traffic(
+                                      "gated_norm_rows524288.md",
+                                      "gated_deltanet_linear_eqs_b200/csrc/gated_norm.cu",
+                                      key=f"{name}_dram_bytes_per_launch"),
+                                  "peak_source": peak_src},
+                     "clocks": clk.summary()}
+    res["config"] = {"workload": f"gated RMSNorm (eq. (11) bracket): {NORM_ROWS} rows "
+                                 f"(T={T_TOTAL} x H={H}) of dv={D}, bf16 y/z/o, fp32 w",
+                     "l2": "each launch streams >= 403 MB, beyond the 126 MB L2; no flush"}
+    # the gated recurrence on the headline workload: logits of eqs. (9)-(10) in place of alpha,
+    # beta; the same bytes per token as the plain call, the gates evaluated where alpha is loaded
+    from gated_deltanet_linear_eqs_b200._abi import GDN_OP_PREFILL_VARLEN
+    from gated_deltanet_linear_eqs_b200.inputs import make_gate_inputs
+    _, inp = varlen_workload(seed=0)
+    gv = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    gi = {k: v.to(dev) for k, v in make_gate_inputs((1, T_TOTAL, H), H, seed=0).items()}
+    ws = torch.empty(api.gdn_workspace_bytes(GDN_OP_PREFILL_VARLEN, 1, T_TOTAL, H, D, D, NDOCS),
+                     dtype=torch.uint8, device=dev)
+    y = torch.empty((1, T_TOTAL, H, D), dtype=torch.bfloat16, device=dev)
+    sf = torch.empty((NDOCS, H, D, D), dtype=torch.float32, device=dev)
+
+    def gated_step():
+        api.gdn_prefill_varlen_gated(gv["q"], gv["k"], gv["v"], gi["a"], gi["b"], gi["A_log"],
+                                     gi["b_alpha"], gv["cu_seqlens"], gv["s0"], y=y, s_final=sf,
+                                     ws=ws)
+    for _ in range(max(3, args.warmup)):
+        gated_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        gated_step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    res["gated_prefill"] = {"ms_per_step": ms, "tokens_per_s": T_TOTAL / (ms / 1e3),
+                            "workload": "the headline varlen workload with gate logits a, b ~ N(0, 1), "
+                                        "A_log ~ U(-1, 1), b_alpha ~ N(0, 0.5^2) per head"}
+    res["gpu_launches"] = 2 * args.steps + 3 * args.steps
+    return res
 
 
 TRAIN_B, TRAIN_T, TRAIN_H = 8, 4096, 32
@@ -367,6 +498,12 @@ def run_profile(args):
              if isinstance(v, torch.Tensor)}
         for _ in range(n + 1):
             api.gdn_decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S)
+    elif args.profile == "gated":
+        from gated_deltanet_linear_eqs_b200.inputs import make_norm_inputs
+        g = {k: v.to(dev) for k, v in make_norm_inputs(NORM_ROWS, D, seed=0, with_do=True).items()}
+        for _ in range(n + 1):
+            api.gdn_gated_rmsnorm(g["y"], g["z"], g["w"])
+            api.gdn_gated_rmsnorm_backward(g["y"], g["z"], g["w"], g["d_o"])
     else:
         from gated_deltanet_linear_eqs_b200._abi import GDN_OP_BACKWARD
         g = train_inputs(dev)
@@ -512,10 +649,11 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "train"], default="all")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "train", "gated", "segmented"],
+                    default="all")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--train-steps", type=int, default=3)
-    ap.add_argument("--profile", choices=["prefill", "decode", "backward"], default=None,
+    ap.add_argument("--profile", choices=["prefill", "decode", "backward", "gated"], default=None,
                     help="launch-only mode for ncu (no timing, no JSON)")
     ap.add_argument("--launches", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -564,6 +702,16 @@ def main():
                     clocks=p["clocks"], e2e=res["e2e"], gpu_launches=3 * args.steps)
     if "train" in res:
         line["train"] = res["train"]
+    if "segmented" in res:
+        line["segmented"] = res["segmented"]
+    if "gated_norm" in res:
+        line["gated_norm"] = res["gated_norm"]
+        if "prefill" not in res and "decode" not in res:
+            gn = res["gated_norm"]
+            line.update(value=gn["forward"]["GB/s"], unit="GB/s",
+                        ms_per_step=gn["forward"]["ms_per_launch"], config=gn["config"],
+                        roofline=gn["forward"]["roofline"], clocks=gn["forward"]["clocks"],
+                        gpu_launches=gn["gpu_launches"])
     if "decode" in res:
         line["decode"] = res["decode"]
         if "prefill" not in res:

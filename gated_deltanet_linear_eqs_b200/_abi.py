@@ -30,6 +30,7 @@ GDN_OP_PREFILL = 0
 GDN_OP_PREFILL_VARLEN = 1
 GDN_OP_DECODE = 2
 GDN_OP_BACKWARD = 3
+GDN_OP_PREFILL_SEGMENTED = 4
 
 _P = ctypes.c_void_p
 _F = ctypes.c_float
@@ -53,8 +54,16 @@ SIGNATURES = {
     "gdn_backward": (_I, [_P] * 14 + [_I] * 6 + [_F, _I, _P, _S, _P]),
     "gdn_backward_noalloc": (_I, [_P] * 14 + [_I] * 6 + [_F, _I, _P]),
     "gdn_backward_noalloc_max_workspace": (_S, []),
+    "gdn_prefill_gated": (_I, [_P] * 10 + [_I] * 6 + [_F, _I, _P, _S, _P]),
+    "gdn_prefill_varlen_gated": (_I, [_P] * 8 + [_I] + [_P] * 3 + [_I] * 5 + [_F, _I, _P, _S,
+                                                                            _P]),
+    "gdn_decode_step_gated": (_I, [_P] * 9 + [_I] * 5 + [_F, _I, _P]),
+    "gdn_backward_gated": (_I, [_P] * 18 + [_I] * 6 + [_F, _I, _P, _S, _P]),
+    "gdn_gated_rmsnorm": (_I, [_P] * 4 + [ctypes.c_int64, _I, _I, _F, _P]),
+    "gdn_gated_rmsnorm_backward": (_I, [_P] * 7 + [ctypes.c_int64, _I, _I, _F, _P]),
     "gdn_read_device_status": (_I, [_I, ctypes.POINTER(_I)]),
     "gdn_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
+    "gdn_prefill_segmented": (_I, [_P] * 8 + [_I] * 6 + [_F, _I, _I, _P, _S, _P]),
 }
 
 _lock = threading.Lock()

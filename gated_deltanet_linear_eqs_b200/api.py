@@ -95,6 +95,39 @@ def gdn_prefill(q, k, v, alpha, beta, s0=None, scale=1.0, l2norm_qk=True, y=None
     return y, s_final
 
 
+def gdn_prefill_segmented(q, k, v, alpha, beta, s0=None, num_segments=1, scale=1.0,
+                          l2norm_qk=True, y=None, s_final=None, want_final=True, ws=None,
+                          stream=None):
+    """gdn_prefill with every sequence cut into ``num_segments`` segments that run side by side
+    (affine state maps, a scan, and a pass from every segment's start state).  Same tensors as
+    gdn_prefill.  Returns (y, s_final)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _need(q, "q", dt)
+    _need(k, "k", dt, q.shape)
+    _need(v, "v", dt, (B, T, H, dv))
+    _need(alpha, "alpha", torch.float32, (B, T, H))
+    _need(beta, "beta", torch.float32, (B, T, H))
+    _need(s0, "s0", torch.float32, (B, H, dk, dv), optional=True)
+    if y is None:
+        y = torch.empty((B, T, H, dv), dtype=dt, device=q.device)
+    _need(y, "y", dt, (B, T, H, dv))
+    if s_final is None and want_final:
+        s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(s_final, "s_final", torch.float32, (B, H, dk, dv), optional=True)
+    ws, wsb = _workspace(_abi.GDN_OP_PREFILL_SEGMENTED, q.device, B, T, H, dk, dv,
+                         int(num_segments), ws=ws)
+    rc = _lib().gdn_prefill_segmented(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(s0), _p(y),
+                                      _p(s_final), B, T, H, dk, dv, _DT[dt], float(scale),
+                                      int(bool(l2norm_qk)), int(num_segments), _p(ws), wsb,
+                                      _stream(stream))
+    _check(rc, "gdn_prefill_segmented")
+    return y, s_final
+
+
 def gdn_prefill_varlen(q, k, v, alpha, beta, cu_seqlens, s0=None, scale=1.0, l2norm_qk=True,
                        y=None, s_final=None, ws=None, stream=None):
     """Packed documents: q,k [1,T,H,dk] (or [T,H,dk]), v likewise, alpha,beta [1,T,H],
@@ -268,6 +301,170 @@ def gdn_backward_noalloc(q, k, v, alpha, beta, dy, s0=None, ds_final=None, scale
 
 def gdn_backward_noalloc_max_workspace():
     return int(_lib().gdn_backward_noalloc_max_workspace())
+
+
+def _need_gate(a, b, A_log, b_alpha, shape, H):
+    _need(a, "a", torch.float32, shape)
+    _need(b, "b", torch.float32, shape)
+    _need(A_log, "A_log", torch.float32, (H,))
+    _need(b_alpha, "b_alpha", torch.float32, (H,))
+
+
+def gdn_prefill_gated(q, k, v, a, b, A_log, b_alpha, s0=None, scale=1.0, l2norm_qk=True,
+                      y=None, s_final=None, want_final=True, ws=None, stream=None):
+    """gdn_prefill with alpha and beta given by eqs. (9)-(10): a = W_alpha x, b = W_beta x
+    [B,T,H] fp32, A_log and b_alpha [H] fp32.  Returns (y, s_final)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _need(q, "q", dt)
+    _need(k, "k", dt, q.shape)
+    _need(v, "v", dt, (B, T, H, dv))
+    _need_gate(a, b, A_log, b_alpha, (B, T, H), H)
+    _need(s0, "s0", torch.float32, (B, H, dk, dv), optional=True)
+    if y is None:
+        y = torch.empty((B, T, H, dv), dtype=dt, device=q.device)
+    _need(y, "y", dt, (B, T, H, dv))
+    if s_final is None and want_final:
+        s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(s_final, "s_final", torch.float32, (B, H, dk, dv), optional=True)
+    ws, wsb = _workspace(_abi.GDN_OP_PREFILL, q.device, B, T, H, dk, dv, ws=ws)
+    rc = _lib().gdn_prefill_gated(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(b_alpha),
+                                  _p(s0), _p(y), _p(s_final), B, T, H, dk, dv, _DT[dt],
+                                  float(scale), int(bool(l2norm_qk)), _p(ws), wsb,
+                                  _stream(stream))
+    _check(rc, "gdn_prefill_gated")
+    return y, s_final
+
+
+def gdn_prefill_varlen_gated(q, k, v, a, b, A_log, b_alpha, cu_seqlens, s0=None, scale=1.0,
+                             l2norm_qk=True, y=None, s_final=None, ws=None, stream=None):
+    """gdn_prefill_varlen with alpha and beta given by eqs. (9)-(10) (a, b [1,T,H] or [T,H]
+    fp32; A_log, b_alpha [H]).  Returns (y, s_final)."""
+    if q.dim() == 3:
+        q, k, v, a, b = (x.unsqueeze(0) for x in (q, k, v, a, b))
+    _, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError("q/k/v must be bf16 or fp32")
+    N = cu_seqlens.numel() - 1
+    _need(q, "q", dt)
+    _need(k, "k", dt, q.shape)
+    _need(v, "v", dt, (1, T, H, dv))
+    _need_gate(a, b, A_log, b_alpha, (1, T, H), H)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,))
+    _need(s0, "s0", torch.float32, (N, H, dk, dv), optional=True)
+    if y is None:
+        y = torch.empty((1, T, H, dv), dtype=dt, device=q.device)
+    _need(y, "y", dt, (1, T, H, dv))
+    if s_final is None:
+        s_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(s_final, "s_final", torch.float32, (N, H, dk, dv))
+    ws, wsb = _workspace(_abi.GDN_OP_PREFILL_VARLEN, q.device, 1, T, H, dk, dv, N, ws=ws)
+    rc = _lib().gdn_prefill_varlen_gated(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log),
+                                         _p(b_alpha), _p(cu_seqlens), N, _p(s0), _p(y),
+                                         _p(s_final), T, H, dk, dv, _DT[dt], float(scale),
+                                         int(bool(l2norm_qk)), _p(ws), wsb, _stream(stream))
+    _check(rc, "gdn_prefill_varlen_gated")
+    return y, s_final
+
+
+def gdn_decode_step_gated(q, k, v, a, b, A_log, b_alpha, state, scale=1.0, l2norm_qk=True,
+                          y=None, stream=None):
+    """gdn_decode_step with alpha and beta given by eqs. (9)-(10) (a, b [N,H] fp32; A_log,
+    b_alpha [H]).  The state is updated in place.  Returns y [N,H,dv]."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _need(q, "q", dt)
+    _need(k, "k", dt, q.shape)
+    _need(v, "v", dt, (N, H, dv))
+    _need_gate(a, b, A_log, b_alpha, (N, H), H)
+    _need(state, "state", torch.float32, (N, H, dk, dv))
+    if y is None:
+        y = torch.empty((N, H, dv), dtype=dt, device=q.device)
+    _need(y, "y", dt, (N, H, dv))
+    rc = _lib().gdn_decode_step_gated(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(b_alpha),
+                                      _p(state), _p(y), N, H, dk, dv, _DT[dt], float(scale),
+                                      int(bool(l2norm_qk)), _stream(stream))
+    _check(rc, "gdn_decode_step_gated")
+    return y
+
+
+def gdn_backward_gated(q, k, v, a, b, A_log, b_alpha, dy, s0=None, ds_final=None, scale=1.0,
+                       l2norm_qk=True, want_ds0=True, ws=None, stream=None):
+    """Gradients of (y, s_final) for the gated form.  Returns dict dq, dk, dv, da, db,
+    dA_log, db_alpha, ds0."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _need(q, "q", dt)
+    _need(k, "k", dt, q.shape)
+    _need(v, "v", dt, (B, T, H, dv))
+    _need_gate(a, b, A_log, b_alpha, (B, T, H), H)
+    _need(dy, "dy", dt, (B, T, H, dv))
+    _need(s0, "s0", torch.float32, (B, H, dk, dv), optional=True)
+    _need(ds_final, "ds_final", torch.float32, (B, H, dk, dv), optional=True)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               da=torch.empty_like(a), db=torch.empty_like(b), dA_log=torch.empty_like(A_log),
+               db_alpha=torch.empty_like(b_alpha),
+               ds0=torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+               if want_ds0 else None)
+    ws, wsb = _workspace(_abi.GDN_OP_BACKWARD, q.device, B, T, H, dk, dv, ws=ws)
+    rc = _lib().gdn_backward_gated(_p(q), _p(k), _p(v), _p(a), _p(b), _p(A_log), _p(b_alpha),
+                                   _p(s0), _p(dy), _p(ds_final), _p(out["dq"]), _p(out["dk"]),
+                                   _p(out["dv"]), _p(out["da"]), _p(out["db"]),
+                                   _p(out["dA_log"]), _p(out["db_alpha"]), _p(out["ds0"]), B, T,
+                                   H, dk, dv, _DT[dt], float(scale), int(bool(l2norm_qk)), _p(ws),
+                                   wsb, _stream(stream))
+    _check(rc, "gdn_backward_gated")
+    return out
+
+
+def gdn_gated_rmsnorm(y, z, w, eps=1e-6, o=None, stream=None):
+    """The bracket of eq. (11): sigmoid(z) * (1 + w) * y / sqrt(mean(y^2) + eps) over the last
+    axis.  y, z [..., dv] (bf16 or fp32, same dtype), w [dv] fp32.  Returns o like y."""
+    dt = y.dtype
+    if dt not in _DT:
+        raise ValueError("y/z must be bf16 or fp32")
+    dv = y.shape[-1]
+    _need(y, "y", dt)
+    _need(z, "z", dt, y.shape)
+    _need(w, "w", torch.float32, (dv,))
+    if o is None:
+        o = torch.empty_like(y)
+    _need(o, "o", dt, y.shape)
+    rows = y.numel() // dv if dv else 0
+    rc = _lib().gdn_gated_rmsnorm(_p(y), _p(z), _p(w), _p(o), rows, dv, _DT[dt], float(eps),
+                                  _stream(stream))
+    _check(rc, "gdn_gated_rmsnorm")
+    return o
+
+
+def gdn_gated_rmsnorm_backward(y, z, w, d_o, eps=1e-6, stream=None):
+    """Gradients of gdn_gated_rmsnorm given d_o.  Returns dict dy, dz (like y) and dw [dv]."""
+    dt = y.dtype
+    if dt not in _DT:
+        raise ValueError("y/z must be bf16 or fp32")
+    dv = y.shape[-1]
+    _need(y, "y", dt)
+    _need(z, "z", dt, y.shape)
+    _need(w, "w", torch.float32, (dv,))
+    _need(d_o, "d_o", dt, y.shape)
+    out = dict(dy=torch.empty_like(y), dz=torch.empty_like(z), dw=torch.empty_like(w))
+    rows = y.numel() // dv if dv else 0
+    rc = _lib().gdn_gated_rmsnorm_backward(_p(y), _p(z), _p(w), _p(d_o), _p(out["dy"]),
+                                           _p(out["dz"]), _p(out["dw"]), rows, dv, _DT[dt],
+                                           float(eps), _stream(stream))
+    _check(rc, "gdn_gated_rmsnorm_backward")
+    return out
 
 
 def gdn_read_device_status(reset=True):

@@ -1,6 +1,8 @@
 // backward_chunk.cu -- the backward pass of eqs. (1)-(4) (Qwen3.8-Flash-Next summary, picx.dev,
 // "Theoretical foundations"; the reverse recurrence of its Appendix B) in the chunked WY form of
-// the forward, on 64-token chunks, in fp32.
+// the forward, on 64-token chunks, in fp32 with the products on tensor cores (warp-level
+// m16n8k8 tf32 tiles, fp32 accumulation; the reverse chain's dS products with split 3 x tf32
+// operands, since their rounding accumulates into dS0 along the whole chain).
 //
 // Per chunk, with q^ = rq q, k^ = rk k the normalised rows, Lg the inclusive cumsum of ln(alpha),
 // gam = e^Lg, gC = gam of the chunk's last token, Gam_ij = e^(Lg_i - Lg_j), S = S^c the state at
@@ -86,20 +88,6 @@ __device__ __forceinline__ void mm_nn(float* acc, const float* a, int as, const 
     }
 }
 
-// acc[n] += sum_k a[k] * b[n * bs + k], k contiguous in both (16-byte aligned), K % 4 == 0
-template <int NC>
-__device__ __forceinline__ void mm_nt(float* acc, const float* a, const float* b, int bs, int K) {
-#pragma unroll 2
-    for (int k = 0; k < K; k += 4) {
-        const float4 x = *reinterpret_cast<const float4*>(a + k);
-#pragma unroll
-        for (int n = 0; n < NC; ++n) {
-            const float4 y = *reinterpret_cast<const float4*>(b + (size_t)n * bs + k);
-            acc[n] = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc[n]))));
-        }
-    }
-}
-
 __device__ __forceinline__ size_t tok_off(int b, int t, int h, int T, int H) {
     return ((size_t)b * T + t) * H + h;
 }
@@ -175,6 +163,63 @@ __device__ __forceinline__ void mma_tf32(float* c, uint32_t a0, uint32_t a1, uin
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// acc[t] (16 x 8 tile t at rows r0.., columns c0 + 8 t ..) += A B over k < K, tf32
+template <int CT, typename FA, typename FB>
+__device__ __forceinline__ void wmma_acc(float (&acc)[CT][4], int K, int r0, int c0, FA a, FB b, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = to_tf32(a(r0 + gid, k0 + tig)), a1 = to_tf32(a(r0 + gid + 8, k0 + tig));
+        const uint32_t a2 = to_tf32(a(r0 + gid, k0 + tig + 4)), a3 = to_tf32(a(r0 + gid + 8, k0 + tig + 4));
+#pragma unroll
+        for (int t = 0; t < CT; ++t) {
+            const int n = c0 + 8 * t + gid;
+            mma_tf32(acc[t], a0, a1, a2, a3, to_tf32(b(k0 + tig, n)), to_tf32(b(k0 + tig + 4, n)));
+        }
+    }
+}
+template <int CT>
+__device__ __forceinline__ void zero_acc(float (&acc)[CT][4]) {
+#pragma unroll
+    for (int t = 0; t < CT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+}
+// sum over the 4 lanes of a quad (the lanes that share a tile row)
+__device__ __forceinline__ float quad_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    return x;
+}
+
+// acc[t] += A B like wmma_acc, with every operand split into its tf32 value and a tf32
+// remainder: A_lo B_hi + A_hi B_lo + A_hi B_hi.  That keeps the products' relative error near
+// 2^-22 instead of tf32's 2^-11, for the products whose rounding accumulates along a chain.
+template <int CT, typename FA, typename FB>
+__device__ __forceinline__ void wmma_acc3(float (&acc)[CT][4], int K, int r0, int c0, FA a, FB b, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const float af[4] = {a(r0 + gid, k0 + tig), a(r0 + gid + 8, k0 + tig), a(r0 + gid, k0 + tig + 4),
+                             a(r0 + gid + 8, k0 + tig + 4)};
+        // the high part's low 13 bits are cleared so that it reads back as the exact tf32 value
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            ah[e] = to_tf32(af[e]) & 0xffffe000u;
+            al[e] = to_tf32(af[e] - __uint_as_float(ah[e]));
+        }
+#pragma unroll
+        for (int t = 0; t < CT; ++t) {
+            const int n = c0 + 8 * t + gid;
+            const float b0 = b(k0 + tig, n), b1 = b(k0 + tig + 4, n);
+            const uint32_t bh0 = to_tf32(b0) & 0xffffe000u, bh1 = to_tf32(b1) & 0xffffe000u;
+            const uint32_t bl0 = to_tf32(b0 - __uint_as_float(bh0)), bl1 = to_tf32(b1 - __uint_as_float(bh1));
+            mma_tf32(acc[t], al[0], al[1], al[2], al[3], bh0, bh1);
+            mma_tf32(acc[t], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+            mma_tf32(acc[t], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+        }
+    }
+}
+
 // ============================================================================ bwdc_prep
 template <int D>
 struct PrepB {
@@ -183,11 +228,12 @@ struct PrepB {
 };
 
 template <int D, typename Tin>
-__global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, const Tin* __restrict__ k,
+__global__ void __launch_bounds__(256, 2) bwdc_prep(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                  const Tin* __restrict__ v, const float* __restrict__ alpha,
                                                  const float* __restrict__ beta, float* __restrict__ ws,
                                                  const BwdChunkWs w, int T, int H, int nch, float scale,
-                                                 int l2norm) {
+                                                 int l2norm, const float* __restrict__ A_log,
+                                                 const float* __restrict__ b_alpha) {
     constexpr int LD = PrepB<D>::LD;
     extern __shared__ float smf[];
     float* qh = smf;
@@ -212,8 +258,14 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
     load_rows<D, LD, 256>(kh, k, b, t0, nv, h, T, H, nullptr, tid);
     if (tid < kCB) {
         const size_t o = tok_off(b, t0 + tid, h, T, H);
-        be[tid] = tid < nv ? beta[o] : 0.f;
-        Lg[tid] = tid < nv ? logf(alpha[o]) : 0.f;
+        float bt = 0.f, lg = 0.f;  // rows past the end: beta = 0, alpha = 1
+        if (tid < nv) {
+            // gated form: alpha, beta hold the logits of eqs. (9)-(10)
+            bt = A_log ? gate_sigmoid(beta[o]) : beta[o];
+            lg = A_log ? gate_log_decay(alpha[o], A_log[h], b_alpha[h]) : logf(alpha[o]);
+        }
+        be[tid] = bt;
+        Lg[tid] = lg;
     }
     __syncthreads();
     for (int rr = 0; rr < 16; ++rr) {  // warp w: rows 16 w .. 16 w + 15 of [q; k]
@@ -239,25 +291,38 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
         kh[i * LD + m] *= rk[i];
     }
     __syncthreads();
-    // A / beta and P
-    {  // thread: row i, columns j = g + 4 n (rows g + 4 n of K^ sit in distinct banks)
-        const int i = tid >> 2, g = tid & 3;
-        float kk[16], qk[16];
+    // A / beta and P: K^ K^T and Q^ K^T as 16 x 8 tensor-core tiles (tf32 operands, fp32
+    // accumulation); warp w owns rows 16 (w & 3) .. +15 and columns 32 (w >> 2) .. +31, and lane
+    // (gid, tig) of tile t holds rows gid, gid + 8 and columns 8 t + 2 tig, 8 t + 2 tig + 1
+    {
+        const int gid = lane >> 2, tig = lane & 3;
+        const int r0 = (warp & 3) * 16, c0 = (warp >> 2) * 32;
+        const float* khp = kh;
+        const float* qhp = qh;
+        float kk[4][4], qk[4][4];
+        zero_acc(kk);
+        zero_acc(qk);
+        auto bKt = [khp](int k2, int n) { return khp[n * LD + k2]; };
+        wmma_acc(kk, D, r0, c0, [khp](int i, int k2) { return khp[i * LD + k2]; }, bKt, lane);
+        wmma_acc(qk, D, r0, c0, [qhp](int i, int k2) { return qhp[i * LD + k2]; }, bKt, lane);
+        float* Atg = ws + w.At + r * kCB * kCB;
+        float* Pg = ws + w.P + r * kCB * kCB;
 #pragma unroll
-        for (int n = 0; n < 16; ++n) kk[n] = qk[n] = 0.f;
-        mm_nt<16>(kk, kh + i * LD, kh + g * LD, 4 * LD, D);
-        mm_nt<16>(qk, qh + i * LD, kh + g * LD, 4 * LD, D);
-        float* Atg = ws + w.At + r * kCB * kCB + i * kCB;
-        float* Pg = ws + w.P + r * kCB * kCB + i * kCB;
+        for (int t = 0; t < 4; ++t)
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            const int j = g + 4 * n;
-            const float gm = expf(fminf(Lg[i] - Lg[j], 0.f));
-            const float at = j < i ? kk[n] * gm : 0.f;
-            Atg[j] = at;
-            Am[i * kL64 + j] = be[i] * at;
-            Pg[j] = j <= i ? scale * qk[n] * gm : 0.f;
-        }
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = r0 + gid + 8 * hh, j = c0 + 8 * t + 2 * tig;
+                float at[2], pp[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const float gm = expf(fminf(Lg[i] - Lg[j + u], 0.f));
+                    at[u] = j + u < i ? kk[t][2 * hh + u] * gm : 0.f;
+                    pp[u] = j + u <= i ? scale * qk[t][2 * hh + u] * gm : 0.f;
+                    Am[i * kL64 + j + u] = be[i] * at[u];
+                }
+                *reinterpret_cast<float2*>(Atg + i * kCB + j) = make_float2(at[0], at[1]);
+                *reinterpret_cast<float2*>(Pg + i * kCB + j) = make_float2(pp[0], pp[1]);
+            }
     }
     __syncthreads();
     load_rows<D, LD, 256>(vs, v, b, t0, nv, h, T, H, nullptr, tid);  // Q is no longer read
@@ -297,35 +362,36 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
         __syncthreads();
     }
     for (int e = tid; e < kCB * kCB; e += 256) ws[w.Tm + r * kCB * kCB + e] = Tm[(e / kCB) * kL64 + e % kCB];
-    // W = T diag(beta gam) K^, Ut = T diag(beta) V
-    {  // thread: row i, column chunks 4 g + 16 u
-        constexpr int NC = D / 4;
-        const int i = tid >> 2, g = tid & 3;
-        float wa[NC], ua[NC];
+    // W = T diag(beta gam) K^, Ut = T diag(beta) V: 64 x D tensor-core tiles (tf32, fp32
+    // accumulation), the diagonal scales folded into the B operand; warp w owns rows
+    // 16 (w & 3) .. +15 and columns (D / 2)(w >> 2) .. +D/2-1
+    {
+        constexpr int CT = D / 16;
+        const int gid = lane >> 2, tig = lane & 3;
+        const int r0 = (warp & 3) * 16, c0 = (warp >> 2) * (D / 2);
+        const float* Tp = Tm;
+        const float* khp = kh;
+        const float* vp = vs;
+        const float* bep = be;
+        const float* gp = gam;
+        float wa[CT][4], ua[CT][4];
+        zero_acc(wa);
+        zero_acc(ua);
+        auto aT = [Tp](int i, int j) { return Tp[i * kL64 + j]; };
+        wmma_acc(wa, kCB, r0, c0, aT,
+                 [bep, gp, khp](int j, int n) { return bep[j] * gp[j] * khp[j * LD + n]; }, lane);
+        wmma_acc(ua, kCB, r0, c0, aT, [bep, vp](int j, int n) { return bep[j] * vp[j * LD + n]; },
+                 lane);
+        float* Wg = ws + w.W + r * kCB * D;
+        float* Ug = ws + w.Ut + r * kCB * D;
 #pragma unroll
-        for (int n = 0; n < NC; ++n) wa[n] = ua[n] = 0.f;
-        for (int j = 0; j < kCB; ++j) {
-            const float tij = Tm[i * kL64 + j];
-            const float fw = tij * be[j] * gam[j], fu = tij * be[j];
-            const float* kr = kh + j * LD + 4 * g;
-            const float* vr = vs + j * LD + 4 * g;
+        for (int t = 0; t < CT; ++t)
 #pragma unroll
-            for (int n = 0; n < NC / 4; ++n) {
-                const float4 y = *reinterpret_cast<const float4*>(kr + 16 * n);
-                const float4 z = *reinterpret_cast<const float4*>(vr + 16 * n);
-                wa[4 * n] = fmaf(fw, y.x, wa[4 * n]); wa[4 * n + 1] = fmaf(fw, y.y, wa[4 * n + 1]);
-                wa[4 * n + 2] = fmaf(fw, y.z, wa[4 * n + 2]); wa[4 * n + 3] = fmaf(fw, y.w, wa[4 * n + 3]);
-                ua[4 * n] = fmaf(fu, z.x, ua[4 * n]); ua[4 * n + 1] = fmaf(fu, z.y, ua[4 * n + 1]);
-                ua[4 * n + 2] = fmaf(fu, z.z, ua[4 * n + 2]); ua[4 * n + 3] = fmaf(fu, z.w, ua[4 * n + 3]);
+            for (int hh = 0; hh < 2; ++hh) {
+                const size_t o = (size_t)(r0 + gid + 8 * hh) * D + c0 + 8 * t + 2 * tig;
+                *reinterpret_cast<float2*>(Wg + o) = make_float2(wa[t][2 * hh], wa[t][2 * hh + 1]);
+                *reinterpret_cast<float2*>(Ug + o) = make_float2(ua[t][2 * hh], ua[t][2 * hh + 1]);
             }
-        }
-        float* Wg = ws + w.W + r * kCB * D + (size_t)i * D + 4 * g;
-        float* Ug = ws + w.Ut + r * kCB * D + (size_t)i * D + 4 * g;
-#pragma unroll
-        for (int n = 0; n < NC / 4; ++n) {
-            *reinterpret_cast<float4*>(Wg + 16 * n) = make_float4(wa[4 * n], wa[4 * n + 1], wa[4 * n + 2], wa[4 * n + 3]);
-            *reinterpret_cast<float4*>(Ug + 16 * n) = make_float4(ua[4 * n], ua[4 * n + 1], ua[4 * n + 2], ua[4 * n + 3]);
-        }
     }
     if (tid < kCB) {
         float* sc = ws + w.SC + r * 256;
@@ -336,7 +402,7 @@ __global__ void __launch_bounds__(256) bwdc_prep(const Tin* __restrict__ q, cons
 // ============================================================================ chains
 template <int D>
 struct ChainB {
-    static constexpr int LDS = kNVB + 4;
+    static constexpr int LDS = kNVB + 8;  // rows k and k + 1..3 of a B operand: distinct banks
     static constexpr int LD = D + 4;
     static constexpr int FWD_BYTES = (D * LDS + 2 * kCB * LD + kCB * LDS + 2 * kCB) * 4;
     static constexpr int REV_BYTES = (D * LDS + 2 * kCB * LD + 2 * kCB * LDS + 3 * kCB) * 4;
@@ -349,7 +415,8 @@ struct ChunkRegs {
     static constexpr int PW = kCB * D / 4 / 256;  // float4 of W
     static constexpr int PR = kCB * D / 8 / 256;  // 8-element groups of a token tile
     float4 w[PW];
-    float k[PR][8], y[8];
+    float k[PR][8];
+    float2 y[4];  // Ut at this lane's positions of the U tiles (tile t, row half hh: y[2 t + hh])
 };
 
 // Forward: S^c and U of every chunk, 32 state columns per CTA.
@@ -369,8 +436,10 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
     float* rks = dec + kCB;
     constexpr int nsl = D / kNVB;
     const int jsl = blockIdx.x % nsl, h = (blockIdx.x / nsl) % H, b = blockIdx.x / (nsl * H);
-    const int col0 = jsl * kNVB, tid = threadIdx.x;
-    const int iu = tid >> 2, nu = (tid & 3) * 8;  // U element block of this thread
+    const int col0 = jsl * kNVB, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    // U (64 x 32) tiles: warp w owns rows 16 (w & 3) .. +15 and columns 16 (w >> 2) .. +15
+    const int ur0 = (warp & 3) * 16, uc0 = (warp >> 2) * 16;
     R rg;
     auto fetch = [&](int c) {
         const size_t r = ((size_t)b * nch + c) * H + h;
@@ -387,7 +456,13 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
                 for (int j = 0; j < 8; ++j) rg.k[u][j] = 0.f;
             }
         }
-        ld8(ws + w.Ut + r * kCB * D + (size_t)iu * D + col0 + nu, rg.y);  // Ut of this thread's U block
+        const float* Utg = ws + w.Ut + r * kCB * D + col0;  // Ut at this lane's U tile positions
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                rg.y[2 * t + hh] = *reinterpret_cast<const float2*>(
+                    Utg + (size_t)(ur0 + gid + 8 * hh) * D + uc0 + 8 * t + 2 * tig);
     };
     for (int e = tid; e < D * kNVB; e += 256) {
         const int m = e / kNVB, n = e % kNVB;
@@ -412,9 +487,9 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
             const int e = (tid + u * 256) * 8;
             st8(Kt + (e / D) * LD + e % D, rg.k[u], 1.f);
         }
-        float ut[8];
+        float2 ut[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) ut[j] = rg.y[j];
+        for (int j = 0; j < 4; ++j) ut[j] = rg.y[j];
         const float* SCg = ws + w.SC + r * 256;
         if (tid < kCB) {
             dec[tid] = expf(SCg[128 + kCB - 1] - SCg[128 + tid]);
@@ -423,38 +498,48 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
         const float gC = expf(SCg[128 + kCB - 1]);
         __syncthreads();
         if (c + 1 < nch) fetch(c + 1);
-        {  // U = Ut - W S: row iu, 8 columns
-            float acc[8];
+        {  // U = Ut - W S as 16 x 8 tensor-core tiles (tf32 operands, fp32 accumulation)
+            float acc[2][4];
+            zero_acc(acc);
+            const float* Wp = Wt;
+            const float* Sp = Ss;
+            wmma_acc(acc, D, ur0, uc0, [Wp](int i, int k2) { return Wp[i * LD + k2]; },
+                     [Sp](int k2, int n) { return Sp[k2 * LDS + n]; }, lane);
+            float* Ug = ws + w.U + r * kCB * D + col0;
 #pragma unroll
-            for (int n = 0; n < 8; ++n) acc[n] = 0.f;
-            mm_nn<8>(acc, Wt + iu * LD, 1, Ss + nu, LDS, D);
-            float* Ug = ws + w.U + r * kCB * D + (size_t)iu * D + col0 + nu;
+            for (int t = 0; t < 2; ++t)
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const float u = ut[n] - acc[n];
-                Us[iu * LDS + nu + n] = u;
-                Ug[n] = u;
-            }
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int i = ur0 + gid + 8 * hh, n = uc0 + 8 * t + 2 * tig;
+                    const float2 u = make_float2(ut[2 * t + hh].x - acc[t][2 * hh],
+                                                 ut[2 * t + hh].y - acc[t][2 * hh + 1]);
+                    *reinterpret_cast<float2*>(Us + i * LDS + n) = u;
+                    *reinterpret_cast<float2*>(Ug + (size_t)i * D + n) = u;
+                }
         }
         __syncthreads();
-        {  // S = gC S + K^T diag(rk gC / gam) U
-            constexpr int TPR = 256 / D, NC = kNVB / TPR;
-            const int m = tid / TPR, n0 = (tid % TPR) * NC;
-            float acc[NC];
+        {  // S = gC S + K^T diag(rk gC / gam) U as tensor-core tiles (tf32, fp32 accumulation);
+           // the D x 32 slice is D / 16 row blocks by 8 / (D / 16) column groups, one per warp
+            constexpr int RB = D / 16, CG = 8 / RB, CT = 4 / CG;
+            const int sr0 = 16 * (warp % RB), sc0 = (32 / CG) * (warp / RB);
+            float acc[CT][4];
+            zero_acc(acc);
+            const float* Kp = Kt;
+            const float* Up = Us;
+            const float* dp = dec;
+            const float* rp = rks;
+            wmma_acc(acc, kCB, sr0, sc0,
+                     [Kp, dp, rp](int m, int i) { return Kp[i * LD + m] * (dp[i] * rp[i]); },
+                     [Up](int i, int n) { return Up[i * LDS + n]; }, lane);
 #pragma unroll
-            for (int n = 0; n < NC; ++n) acc[n] = 0.f;
-            for (int i = 0; i < kCB; ++i) {
-                const float x = Kt[i * LD + m] * (dec[i] * rks[i]);
-                const float4* ur = reinterpret_cast<const float4*>(Us + i * LDS + n0);
+            for (int t = 0; t < CT; ++t)
 #pragma unroll
-                for (int n = 0; n < NC / 4; ++n) {
-                    const float4 y = ur[n];
-                    acc[4 * n] = fmaf(x, y.x, acc[4 * n]); acc[4 * n + 1] = fmaf(x, y.y, acc[4 * n + 1]);
-                    acc[4 * n + 2] = fmaf(x, y.z, acc[4 * n + 2]); acc[4 * n + 3] = fmaf(x, y.w, acc[4 * n + 3]);
+                for (int hh = 0; hh < 2; ++hh) {
+                    float* sp = Ss + (sr0 + gid + 8 * hh) * LDS + sc0 + 8 * t + 2 * tig;
+                    const float2 o = *reinterpret_cast<const float2*>(sp);
+                    *reinterpret_cast<float2*>(sp) =
+                        make_float2(fmaf(gC, o.x, acc[t][2 * hh]), fmaf(gC, o.y, acc[t][2 * hh + 1]));
                 }
-            }
-#pragma unroll
-            for (int n = 0; n < NC; ++n) Ss[m * LDS + n0 + n] = fmaf(gC, Ss[m * LDS + n0 + n], acc[n]);
         }
     }
 }
@@ -479,7 +564,13 @@ __global__ void __launch_bounds__(256, 2) bwdc_rev(const Tin* __restrict__ q, co
     float* rks = ysc + kCB;
     constexpr int nsl = D / kNVB;
     const int jsl = blockIdx.x % nsl, h = (blockIdx.x / nsl) % H, b = blockIdx.x / (nsl * H);
-    const int col0 = jsl * kNVB, tid = threadIdx.x;
+    const int col0 = jsl * kNVB, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    // dU (64 x 32) tiles: warp w owns rows 16 (w & 3) .. +15 and columns 16 (w >> 2) .. +15;
+    // dS (D x 32): D / 16 row blocks by 8 / (D / 16) column groups, one per warp
+    const int ur0 = (warp & 3) * 16, uc0 = (warp >> 2) * 16;
+    constexpr int RB = D / 16, CG = 8 / RB, SCT = 4 / CG;
+    const int sr0 = 16 * (warp % RB), sc0 = (32 / CG) * (warp / RB);
     for (int e = tid; e < D * kNVB; e += 256) {
         const int m = e / kNVB, n = e % kNVB;
         Ss[m * LDS + n] = ds_final ? ds_final[(((size_t)b * H + h) * D + m) * D + col0 + n] : 0.f;
@@ -514,46 +605,57 @@ __global__ void __launch_bounds__(256, 2) bwdc_rev(const Tin* __restrict__ q, co
         const int nvc = min(kCB, T - c * kCB);
         load_rows<D, LD, 256>(X1, k, b, c * kCB, nvc, h, T, H, rks, tid);
         __syncthreads();
-        {  // dU = diag(gC / gam) K^ dS + P^T dY
-            const int i = tid >> 2, n0 = (tid & 3) * 8;
-            float a1[8], a2[8];
+        {  // dU = diag(gC / gam) K^ dS + P^T dY as tensor-core tiles (tf32, fp32 accumulation)
+            float a1[2][4], a2[2][4];
+            zero_acc(a1);
+            zero_acc(a2);
+            const float* Kp = X1;
+            const float* Pp = X2;
+            const float* Sp = Ss;
+            const float* Yp = dYs;
+            wmma_acc(a1, D, ur0, uc0, [Kp](int i, int m) { return Kp[i * LD + m]; },
+                     [Sp](int m, int n) { return Sp[m * LDS + n]; }, lane);
+            wmma_acc(a2, kCB, ur0, uc0, [Pp](int i, int j) { return Pp[j * kL64 + i]; },
+                     [Yp](int j, int n) { return Yp[j * LDS + n]; }, lane);
+            float* dUg = ws + w.dU + r * kCB * D + col0;
 #pragma unroll
-            for (int n = 0; n < 8; ++n) a1[n] = a2[n] = 0.f;
-            mm_nn<8>(a1, X1 + i * LD, 1, Ss + n0, LDS, D);
-            mm_nn<8>(a2, X2 + i, kL64, dYs + n0, LDS, kCB);
-            float* dUg = ws + w.dU + r * kCB * D + (size_t)i * D + col0 + n0;
+            for (int t = 0; t < 2; ++t)
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const float du = fmaf(dec[i], a1[n], a2[n]);
-                dUs[i * LDS + n0 + n] = du;
-                dUg[n] = du;
-            }
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int i = ur0 + gid + 8 * hh, n = uc0 + 8 * t + 2 * tig;
+                    const float2 du = make_float2(fmaf(dec[i], a1[t][2 * hh], a2[t][2 * hh]),
+                                                  fmaf(dec[i], a1[t][2 * hh + 1], a2[t][2 * hh + 1]));
+                    *reinterpret_cast<float2*>(dUs + i * LDS + n) = du;
+                    *reinterpret_cast<float2*>(dUg + (size_t)i * D + n) = du;
+                }
         }
         __syncthreads();
         load_rows<D, LD, 256>(X1, q, b, c * kCB, nvc, h, T, H, ysc, tid);
         load_rec<D, LD, 256>(X2, ws + w.W + r * kCB * D, tid);
         __syncthreads();
-        {  // dS = gC dS + (scale gam Q^)^T dY - W^T dU
-            constexpr int TPR = 256 / D, NC = kNVB / TPR;
-            const int m = tid / TPR, n0 = (tid % TPR) * NC;
-            float acc[NC];
+        {  // dS = gC dS + (scale gam Q^)^T dY - W^T dU as tensor-core tiles with split (3 x tf32)
+           // operands: these products feed the state gradient along the whole chain
+            float a1[SCT][4], a2[SCT][4];
+            zero_acc(a1);
+            zero_acc(a2);
+            const float* Qp = X1;
+            const float* Wp = X2;
+            const float* Yp = dYs;
+            const float* Up = dUs;
+            wmma_acc3(a1, kCB, sr0, sc0, [Qp](int m, int i) { return Qp[i * LD + m]; },
+                      [Yp](int i, int n) { return Yp[i * LDS + n]; }, lane);
+            wmma_acc3(a2, kCB, sr0, sc0, [Wp](int m, int i) { return Wp[i * LD + m]; },
+                      [Up](int i, int n) { return Up[i * LDS + n]; }, lane);
 #pragma unroll
-            for (int n = 0; n < NC; ++n) acc[n] = 0.f;
-            for (int i = 0; i < kCB; ++i) {
-                const float xq = X1[i * LD + m], xw = X2[i * LD + m];
-                const float4* yr = reinterpret_cast<const float4*>(dYs + i * LDS + n0);
-                const float4* ur = reinterpret_cast<const float4*>(dUs + i * LDS + n0);
+            for (int t = 0; t < SCT; ++t)
 #pragma unroll
-                for (int n = 0; n < NC / 4; ++n) {
-                    const float4 y = yr[n], u = ur[n];
-                    acc[4 * n] = fmaf(xq, y.x, fmaf(-xw, u.x, acc[4 * n]));
-                    acc[4 * n + 1] = fmaf(xq, y.y, fmaf(-xw, u.y, acc[4 * n + 1]));
-                    acc[4 * n + 2] = fmaf(xq, y.z, fmaf(-xw, u.z, acc[4 * n + 2]));
-                    acc[4 * n + 3] = fmaf(xq, y.w, fmaf(-xw, u.w, acc[4 * n + 3]));
+                for (int hh = 0; hh < 2; ++hh) {
+                    float* sp = Ss + (sr0 + gid + 8 * hh) * LDS + sc0 + 8 * t + 2 * tig;
+                    const float2 o = *reinterpret_cast<const float2*>(sp);
+                    *reinterpret_cast<float2*>(sp) =
+                        make_float2(fmaf(gC, o.x, a1[t][2 * hh] - a2[t][2 * hh]),
+                                    fmaf(gC, o.y, a1[t][2 * hh + 1] - a2[t][2 * hh + 1]));
                 }
-            }
-#pragma unroll
-            for (int n = 0; n < NC; ++n) Ss[m * LDS + n0 + n] = fmaf(gC, Ss[m * LDS + n0 + n], acc[n]);
         }
     }
     __syncthreads();
@@ -575,33 +677,6 @@ struct LocalB {
     static constexpr int NROW = 10;  // row accumulators
     static constexpr int BYTES = (5 * kCB * LD + 3 * kCB * kL64 + (5 + NROW + 1) * kCB + 32) * 4;
 };
-
-// acc[t] (16 x 8 tile t at rows r0.., columns c0 + 8 t ..) += A B over k < K, tf32
-template <int CT, typename FA, typename FB>
-__device__ __forceinline__ void wmma_acc(float (&acc)[CT][4], int K, int r0, int c0, FA a, FB b, int lane) {
-    const int gid = lane >> 2, tig = lane & 3;
-#pragma unroll 2
-    for (int k0 = 0; k0 < K; k0 += 8) {
-        const uint32_t a0 = to_tf32(a(r0 + gid, k0 + tig)), a1 = to_tf32(a(r0 + gid + 8, k0 + tig));
-        const uint32_t a2 = to_tf32(a(r0 + gid, k0 + tig + 4)), a3 = to_tf32(a(r0 + gid + 8, k0 + tig + 4));
-#pragma unroll
-        for (int t = 0; t < CT; ++t) {
-            const int n = c0 + 8 * t + gid;
-            mma_tf32(acc[t], a0, a1, a2, a3, to_tf32(b(k0 + tig, n)), to_tf32(b(k0 + tig + 4, n)));
-        }
-    }
-}
-template <int CT>
-__device__ __forceinline__ void zero_acc(float (&acc)[CT][4]) {
-#pragma unroll
-    for (int t = 0; t < CT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-}
-// sum over the 4 lanes of a quad (the lanes that share a tile row)
-__device__ __forceinline__ float quad_sum(float x) {
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
-    return x;
-}
 
 // acc += A G^T for the warp's tiles, G [D][D] fp32 in global memory, staged in `buf` (row stride
 // LD) 64 rows at a time: the warps whose output columns fall in the staged rows compute.  Every
@@ -628,7 +703,11 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
                                                      Tin* __restrict__ dk, Tin* __restrict__ dv,
                                                      float* __restrict__ dalpha, float* __restrict__ dbeta,
                                                      const float* __restrict__ ws, const BwdChunkWs w, int T,
-                                                     int H, int nch, float scale, int l2norm) {
+                                                     int H, int nch, float scale, int l2norm,
+                                                     const float* __restrict__ A_log,
+                                                     const float* __restrict__ b_alpha,
+                                                     float* __restrict__ dA_log,
+                                                     float* __restrict__ db_alpha) {
     constexpr int LD = LocalB<D>::LD;
     constexpr int CT = D / 32;  // 8-column tiles per warp in 64 x D results
     extern __shared__ float smf[];
@@ -910,11 +989,32 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
         }
     }
     __syncthreads();
+    float pA = 0.f, pba = 0.f;  // this token's share of dA_log[h], db_alpha[h] (gated form)
     if (tid < nv) {
         const int i = tid;
         const size_t o = tok_off(b, t0 + i, h, T, H);
-        dalpha[o] = dLg[i] / alpha[o];
-        dbeta[o] = r_dbe[i] + r_dbg[i] * gam[i];
+        const float dbe = r_dbe[i] + r_dbg[i] * gam[i];
+        if (A_log) {
+            // ln alpha = -e^A softplus(x), x = a + b_alpha: d a = -e^A sigmoid(x) d ln alpha,
+            // d A = ln alpha d ln alpha, d b_alpha = d a; beta = sigmoid(b): d b = beta (1-beta) d beta
+            const float xa = alpha[o] + b_alpha[h], ea = expf(A_log[h]);
+            const float da = -ea * gate_sigmoid(xa) * dLg[i];
+            dalpha[o] = da;
+            dbeta[o] = dbe * be[i] * (1.f - be[i]);
+            pA = -ea * gate_softplus(xa) * dLg[i];
+            pba = da;
+        } else {
+            dalpha[o] = dLg[i] / alpha[o];
+            dbeta[o] = dbe;
+        }
+    }
+    if (A_log && tid < kCB) {  // warps 0 and 1, whole warps
+        pA = warp_sum(pA);
+        pba = warp_sum(pba);
+        if (lane == 0) {
+            atomicAdd(&dA_log[h], pA);
+            atomicAdd(&db_alpha[h], pba);
+        }
     }
     // 11b. dx = r (dx^ - x^ (x^ . dx^))
 #pragma unroll
@@ -955,16 +1055,22 @@ cudaError_t launch_chunked(const BackwardArgs& a, cudaStream_t st) {
                                   LocalB<D>::BYTES)) != cudaSuccess)
         return e;
     bwdc_prep<D, Tin><<<R, 256, PrepB<D>::BYTES, st>>>(q, k, v, a.alpha, a.beta, ws, w, a.T, a.H, nch,
-                                                        a.scale, a.l2norm);
+                                                        a.scale, a.l2norm, a.A_log, a.b_alpha);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwdc_fwd<D, Tin><<<chains, 256, ChainB<D>::FWD_BYTES, st>>>(k, a.s0, ws, w, a.T, a.H, nch);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwdc_rev<D, Tin><<<chains, 256, ChainB<D>::REV_BYTES, st>>>(q, k, dy, a.ds_final, a.ds0, ws, w, a.T,
                                                                  a.H, nch, a.scale);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.A_log) {
+        if ((e = cudaMemsetAsync(a.dA_log, 0, sizeof(float) * a.H, st)) != cudaSuccess ||
+            (e = cudaMemsetAsync(a.db_alpha, 0, sizeof(float) * a.H, st)) != cudaSuccess)
+            return e;
+    }
     bwdc_local<D, Tin><<<R, 512, LocalB<D>::BYTES, st>>>(
         q, k, v, dy, a.alpha, static_cast<Tin*>(a.dq), static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv),
-        a.dalpha, a.dbeta, ws, w, a.T, a.H, nch, a.scale, a.l2norm);
+        a.dalpha, a.dbeta, ws, w, a.T, a.H, nch, a.scale, a.l2norm, a.A_log, a.b_alpha, a.dA_log,
+        a.db_alpha);
     return cudaGetLastError();
 }
 

@@ -10,6 +10,7 @@
 namespace gdn {
 
 constexpr float kNormEps = 1e-6f;  // x / sqrt(|x|^2 + eps): the library's reading of "L2 norm"
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e): ln x * kLog2e = log2 x
 
 // ---- element conversion -----------------------------------------------------------------
 __device__ __forceinline__ float to_f32(float x) { return x; }
@@ -48,6 +49,21 @@ __device__ __forceinline__ float warp_sum(float x) {
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
     return x;
 }
+
+// ---- gates, eqs. (9)-(10) of the Qwen3.8-Flash-Next summary (picx.dev, "Methodology",
+// "1. GDN Hybrid Token Mixing") -------------------------------------------------------------
+//   beta_t = sigmoid(b_t),  ln alpha_t = -exp(A) softplus(a_t + b_alpha)
+// with a_t = W_alpha x_t and b_t = W_beta x_t given per (token, head) and A (as A_log) and
+// b_alpha per head.  The decay stays in log space: the chunked kernels consume ln alpha, and
+// exp of it would underflow to 0 for strong decays.
+// softplus(x) = ln(1 + e^x) = max(x, 0) + ln(1 + e^-|x|): the second term never overflows.
+__device__ __forceinline__ float gate_softplus(float x) {
+    return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));
+}
+__device__ __forceinline__ float gate_log_decay(float a, float A_log, float b_alpha) {
+    return -expf(A_log) * gate_softplus(a + b_alpha);
+}
+__device__ __forceinline__ float gate_sigmoid(float x) { return 1.f / (1.f + expf(-x)); }
 
 // Record the first device-side error in the library's status word (never traps).
 __device__ __forceinline__ void record_status(int* status, int code) {

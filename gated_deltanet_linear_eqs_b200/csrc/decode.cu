@@ -27,7 +27,8 @@ template <int DK, typename T>
 __global__ void __launch_bounds__(kDecodeThreads)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
               const float* __restrict__ alpha, const float* __restrict__ beta,
-              float* __restrict__ state, T* __restrict__ y, int DV, float scale, int l2norm) {
+              float* __restrict__ state, T* __restrict__ y, int DV, float scale, int l2norm,
+              int H, const float* __restrict__ A_log, const float* __restrict__ b_alpha) {
     constexpr int LPR = kDecodeCols / 4;          // lanes per row (16)
     constexpr int RPW = 32 / LPR;                 // rows per warp instruction (2)
     constexpr int NW = kDecodeThreads / 32;       // warps (4)
@@ -111,7 +112,11 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         r.x += b.x; r.y += b.y; r.z += b.z; r.w += b.w;
     }
 
-    const float a = alpha[nh], b = beta[nh], kq = s_kq;
+    // gated form: alpha, beta hold the logits of eqs. (9)-(10)
+    const int h = nh % H;
+    const float a = A_log ? expf(gate_log_decay(alpha[nh], A_log[h], b_alpha[h])) : alpha[nh];
+    const float b = A_log ? gate_sigmoid(beta[nh]) : beta[nh];
+    const float kq = s_kq;
     const float4 vv = load4(v + (size_t)nh * DV + col);
     float4 e;
     e.x = vv.x - a * p.x; e.y = vv.y - a * p.y; e.z = vv.z - a * p.z; e.w = vv.w - a * p.w;
@@ -138,7 +143,8 @@ cudaError_t launch(const DecodeArgs& a, cudaStream_t st) {
     dim3 grid((unsigned)(a.N * a.H), (unsigned)(a.dv / kDecodeCols));
     decode_kernel<DK, T><<<grid, kDecodeThreads, 0, st>>>(
         static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
-        a.alpha, a.beta, a.state, static_cast<T*>(a.y), a.dv, a.scale, a.l2norm);
+        a.alpha, a.beta, a.state, static_cast<T*>(a.y), a.dv, a.scale, a.l2norm, a.H, a.A_log,
+        a.b_alpha);
     return cudaGetLastError();
 }
 

@@ -104,15 +104,27 @@ int gdn_workspace_bytes(int op, int B, int T, int H, int dk, int dv, int num_seq
             if (B < 1) return GDN_ERR_INVALID_ARG;
             *bytes = gdn::backward_chunked_workspace_bytes(B, T, H, dk, dv);
             return GDN_OK;
+        case GDN_OP_PREFILL_SEGMENTED: {  // num_seqs carries the number of segments
+            if (B < 1 || num_seqs < 1) return GDN_ERR_INVALID_ARG;
+            const size_t a = gdn::segmented_layout(B, T, H, dk, num_seqs, GDN_BF16).total;
+            const size_t f = gdn::segmented_layout(B, T, H, dk, num_seqs, GDN_FP32).total;
+            *bytes = a > f ? a : f;
+            return GDN_OK;
+        }
         default:
             return GDN_ERR_INVALID_ARG;
     }
 }
 
-int gdn_prefill(const void* q, const void* k, const void* v, const float* alpha,
-                const float* beta, const float* s0, void* y, float* s_final, int B, int T, int H,
-                int dk, int dv, int dtype, float scale, int l2norm_qk, void* ws, size_t ws_bytes,
-                void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The plain and the gated entry points share these bodies; A_log == nullptr is the plain form.
+int prefill_dense(const void* q, const void* k, const void* v, const float* alpha,
+                  const float* beta, const float* A_log, const float* b_alpha, const float* s0,
+                  void* y, float* s_final, int B, int T, int H, int dk, int dv, int dtype,
+                  float scale, int l2norm_qk, void* ws, size_t ws_bytes, void* stream) {
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
         !ok_ptr(y) || !ok_opt_ptr(s0) || !ok_opt_ptr(s_final))
         return GDN_ERR_INVALID_ARG;
@@ -125,15 +137,15 @@ int gdn_prefill(const void* q, const void* k, const void* v, const float* alpha,
     DeviceInfo dev;
     if (int rc = current_device_info(&dev)) return rc;
     gdn::PrefillArgs a{q, k, v, alpha, beta, s0, y, s_final, nullptr, B, T, H, dk, dv,
-                       dtype, scale, l2norm_qk ? 1 : 0, dev.status, ws, ws_bytes};
+                       dtype, scale, l2norm_qk ? 1 : 0, dev.status, ws, ws_bytes, A_log, b_alpha};
     return map_cuda(gdn::launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 
-int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float* alpha,
-                       const float* beta, const int32_t* cu_seqlens, int num_seqs,
-                       const float* s0, void* y, float* s_final, int T, int H, int dk, int dv,
-                       int dtype, float scale, int l2norm_qk, void* ws, size_t ws_bytes,
-                       void* stream) {
+int prefill_varlen(const void* q, const void* k, const void* v, const float* alpha,
+                   const float* beta, const float* A_log, const float* b_alpha,
+                   const int32_t* cu_seqlens, int num_seqs, const float* s0, void* y,
+                   float* s_final, int T, int H, int dk, int dv, int dtype, float scale,
+                   int l2norm_qk, void* ws, size_t ws_bytes, void* stream) {
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
         !ok_ptr(y) || cu_seqlens == nullptr || !ok_opt_ptr(s0) || !ok_opt_ptr(s_final))
         return GDN_ERR_INVALID_ARG;
@@ -146,8 +158,88 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
     DeviceInfo dev;
     if (int rc = current_device_info(&dev)) return rc;
     gdn::PrefillArgs a{q, k, v, alpha, beta, s0, y, s_final, cu_seqlens, num_seqs, T, H, dk, dv,
-                       dtype, scale, l2norm_qk ? 1 : 0, dev.status, ws, ws_bytes};
+                       dtype, scale, l2norm_qk ? 1 : 0, dev.status, ws, ws_bytes, A_log, b_alpha};
     return map_cuda(gdn::launch_prefill(a, static_cast<cudaStream_t>(stream)));
+}
+
+int decode_step(const void* q, const void* k, const void* v, const float* alpha,
+                const float* beta, const float* A_log, const float* b_alpha, float* state,
+                void* y, int N, int H, int dk, int dv, int dtype, float scale, int l2norm_qk,
+                void* stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
+        !ok_ptr(state) || !ok_ptr(y))
+        return GDN_ERR_INVALID_ARG;
+    if (N < 1 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (int rc = check_dims(dk, dv, dtype)) return rc;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::DecodeArgs a{q, k, v, alpha, beta, state, y, N, H, dk, dv, dtype, scale,
+                      l2norm_qk ? 1 : 0, A_log, b_alpha};
+    return map_cuda(gdn::launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+int backward_chunked(const void* q, const void* k, const void* v, const float* alpha,
+                     const float* beta, const float* A_log, const float* b_alpha,
+                     const float* s0, const void* dy, const float* ds_final, void* dq,
+                     void* dk_out, void* dv_out, float* dalpha, float* dbeta, float* dA_log,
+                     float* db_alpha, float* ds0, int B, int T, int H, int dk, int dv, int dtype,
+                     float scale, int l2norm_qk, void* ws, size_t ws_bytes, void* stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
+        !ok_ptr(dy) || !ok_ptr(dq) || !ok_ptr(dk_out) || !ok_ptr(dv_out) || !ok_ptr(dalpha) ||
+        !ok_ptr(dbeta) || !ok_opt_ptr(s0) || !ok_opt_ptr(ds_final) || !ok_opt_ptr(ds0))
+        return GDN_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (int rc = check_dims(dk, dv, dtype)) return rc;
+    const size_t need = gdn::backward_chunked_workspace_bytes(B, T, H, dk, dv);
+    if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return GDN_ERR_WORKSPACE;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::BackwardArgs a{q, k, v, alpha, beta, s0, dy, ds_final, dq, dk_out, dv_out, dalpha,
+                        dbeta, ds0, B, T, H, dk, dv, dtype, scale, l2norm_qk ? 1 : 0, ws,
+                        ws_bytes, dev.status, A_log, b_alpha, dA_log, db_alpha};
+    return map_cuda(gdn::launch_backward_chunked(a, static_cast<cudaStream_t>(stream)));
+}
+
+bool ok_gate(const float* A_log, const float* b_alpha) { return ok_ptr(A_log) && ok_ptr(b_alpha); }
+
+}  // namespace
+
+extern "C" {
+
+int gdn_prefill(const void* q, const void* k, const void* v, const float* alpha,
+                const float* beta, const float* s0, void* y, float* s_final, int B, int T, int H,
+                int dk, int dv, int dtype, float scale, int l2norm_qk, void* ws, size_t ws_bytes,
+                void* stream) {
+    return prefill_dense(q, k, v, alpha, beta, nullptr, nullptr, s0, y, s_final, B, T, H, dk, dv,
+                         dtype, scale, l2norm_qk, ws, ws_bytes, stream);
+}
+
+int gdn_prefill_gated(const void* q, const void* k, const void* v, const float* a,
+                      const float* b, const float* A_log, const float* b_alpha, const float* s0,
+                      void* y, float* s_final, int B, int T, int H, int dk, int dv, int dtype,
+                      float scale, int l2norm_qk, void* ws, size_t ws_bytes, void* stream) {
+    if (!ok_gate(A_log, b_alpha)) return GDN_ERR_INVALID_ARG;
+    return prefill_dense(q, k, v, a, b, A_log, b_alpha, s0, y, s_final, B, T, H, dk, dv, dtype,
+                         scale, l2norm_qk, ws, ws_bytes, stream);
+}
+
+int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float* alpha,
+                       const float* beta, const int32_t* cu_seqlens, int num_seqs,
+                       const float* s0, void* y, float* s_final, int T, int H, int dk, int dv,
+                       int dtype, float scale, int l2norm_qk, void* ws, size_t ws_bytes,
+                       void* stream) {
+    return prefill_varlen(q, k, v, alpha, beta, nullptr, nullptr, cu_seqlens, num_seqs, s0, y,
+                          s_final, T, H, dk, dv, dtype, scale, l2norm_qk, ws, ws_bytes, stream);
+}
+
+int gdn_prefill_varlen_gated(const void* q, const void* k, const void* v, const float* a,
+                             const float* b, const float* A_log, const float* b_alpha,
+                             const int32_t* cu_seqlens, int num_seqs, const float* s0, void* y,
+                             float* s_final, int T, int H, int dk, int dv, int dtype, float scale,
+                             int l2norm_qk, void* ws, size_t ws_bytes, void* stream) {
+    if (!ok_gate(A_log, b_alpha)) return GDN_ERR_INVALID_ARG;
+    return prefill_varlen(q, k, v, a, b, A_log, b_alpha, cu_seqlens, num_seqs, s0, y, s_final, T,
+                          H, dk, dv, dtype, scale, l2norm_qk, ws, ws_bytes, stream);
 }
 
 int gdn_prefill_varlen_prepare(const void* q, const void* k, const void* v, const float* alpha,
@@ -191,16 +283,17 @@ int gdn_prefill_varlen_finish(const void* q, const void* k, const int32_t* cu_se
 int gdn_decode_step(const void* q, const void* k, const void* v, const float* alpha,
                     const float* beta, float* state, void* y, int N, int H, int dk, int dv,
                     int dtype, float scale, int l2norm_qk, void* stream) {
-    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
-        !ok_ptr(state) || !ok_ptr(y))
-        return GDN_ERR_INVALID_ARG;
-    if (N < 1 || H < 1) return GDN_ERR_INVALID_ARG;
-    if (int rc = check_dims(dk, dv, dtype)) return rc;
-    DeviceInfo dev;
-    if (int rc = current_device_info(&dev)) return rc;
-    gdn::DecodeArgs a{q, k, v, alpha, beta, state, y, N, H, dk, dv, dtype, scale,
-                      l2norm_qk ? 1 : 0};
-    return map_cuda(gdn::launch_decode(a, static_cast<cudaStream_t>(stream)));
+    return decode_step(q, k, v, alpha, beta, nullptr, nullptr, state, y, N, H, dk, dv, dtype,
+                       scale, l2norm_qk, stream);
+}
+
+int gdn_decode_step_gated(const void* q, const void* k, const void* v, const float* a,
+                          const float* b, const float* A_log, const float* b_alpha, float* state,
+                          void* y, int N, int H, int dk, int dv, int dtype, float scale,
+                          int l2norm_qk, void* stream) {
+    if (!ok_gate(A_log, b_alpha)) return GDN_ERR_INVALID_ARG;
+    return decode_step(q, k, v, a, b, A_log, b_alpha, state, y, N, H, dk, dv, dtype, scale,
+                       l2norm_qk, stream);
 }
 
 int gdn_backward(const void* q, const void* k, const void* v, const float* alpha,
@@ -208,20 +301,53 @@ int gdn_backward(const void* q, const void* k, const void* v, const float* alpha
                  void* dq, void* dk_out, void* dv_out, float* dalpha, float* dbeta, float* ds0,
                  int B, int T, int H, int dk, int dv, int dtype, float scale, int l2norm_qk,
                  void* ws, size_t ws_bytes, void* stream) {
-    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
-        !ok_ptr(dy) || !ok_ptr(dq) || !ok_ptr(dk_out) || !ok_ptr(dv_out) || !ok_ptr(dalpha) ||
-        !ok_ptr(dbeta) || !ok_opt_ptr(s0) || !ok_opt_ptr(ds_final) || !ok_opt_ptr(ds0))
+    return backward_chunked(q, k, v, alpha, beta, nullptr, nullptr, s0, dy, ds_final, dq, dk_out,
+                            dv_out, dalpha, dbeta, nullptr, nullptr, ds0, B, T, H, dk, dv, dtype,
+                            scale, l2norm_qk, ws, ws_bytes, stream);
+}
+
+int gdn_backward_gated(const void* q, const void* k, const void* v, const float* a,
+                       const float* b, const float* A_log, const float* b_alpha, const float* s0,
+                       const void* dy, const float* ds_final, void* dq, void* dk_out,
+                       void* dv_out, float* da, float* db, float* dA_log, float* db_alpha,
+                       float* ds0, int B, int T, int H, int dk, int dv, int dtype, float scale,
+                       int l2norm_qk, void* ws, size_t ws_bytes, void* stream) {
+    if (!ok_gate(A_log, b_alpha) || !ok_ptr(dA_log) || !ok_ptr(db_alpha))
         return GDN_ERR_INVALID_ARG;
-    if (B < 1 || T < 1 || H < 1) return GDN_ERR_INVALID_ARG;
-    if (int rc = check_dims(dk, dv, dtype)) return rc;
-    const size_t need = gdn::backward_chunked_workspace_bytes(B, T, H, dk, dv);
-    if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return GDN_ERR_WORKSPACE;
+    return backward_chunked(q, k, v, a, b, A_log, b_alpha, s0, dy, ds_final, dq, dk_out, dv_out,
+                            da, db, dA_log, db_alpha, ds0, B, T, H, dk, dv, dtype, scale,
+                            l2norm_qk, ws, ws_bytes, stream);
+}
+
+int gdn_gated_rmsnorm(const void* y, const void* z, const float* w, void* o, int64_t rows,
+                      int dv, int dtype, float eps, void* stream) {
+    if (rows < 0 || !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    // no rows: nothing is read or written, and the (empty) tensors may be NULL
+    const auto ok = [rows](const void* p) { return rows == 0 ? aligned16(p) : ok_ptr(p); };
+    if (!ok(y) || !ok(z) || !ok(w) || !ok(o)) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 && dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (dv != 64 && dv != 128) return GDN_ERR_UNSUPPORTED_SHAPE;
     DeviceInfo dev;
     if (int rc = current_device_info(&dev)) return rc;
-    gdn::BackwardArgs a{q, k, v, alpha, beta, s0, dy, ds_final, dq, dk_out, dv_out, dalpha,
-                        dbeta, ds0, B, T, H, dk, dv, dtype, scale, l2norm_qk ? 1 : 0, ws,
-                        ws_bytes, dev.status};
-    return map_cuda(gdn::launch_backward_chunked(a, static_cast<cudaStream_t>(stream)));
+    gdn::GatedNormArgs a{y, z, w, nullptr, o, nullptr, nullptr, nullptr, (long long)rows, dv,
+                         dtype, eps};
+    return map_cuda(gdn::launch_gated_norm(a, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_gated_rmsnorm_backward(const void* y, const void* z, const float* w, const void* d_o,
+                               void* dy, void* dz, float* dw, int64_t rows, int dv, int dtype,
+                               float eps, void* stream) {
+    if (rows < 0 || !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    // no rows: only dw is written (zeros); the empty row tensors may be NULL
+    const auto ok = [rows](const void* p) { return rows == 0 ? aligned16(p) : ok_ptr(p); };
+    if (!ok(y) || !ok(z) || !ok(w) || !ok(d_o) || !ok(dy) || !ok(dz) || !ok_ptr(dw))
+        return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 && dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (dv != 64 && dv != 128) return GDN_ERR_UNSUPPORTED_SHAPE;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::GatedNormArgs a{y, z, w, d_o, nullptr, dy, dz, dw, (long long)rows, dv, dtype, eps};
+    return map_cuda(gdn::launch_gated_norm_backward(a, static_cast<cudaStream_t>(stream)));
 }
 
 int gdn_backward_noalloc(const void* q, const void* k, const void* v, const float* alpha,
@@ -255,6 +381,25 @@ int gdn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
     if (int rc = current_device_info(&dev)) return rc;
     return map_cuda(gdn::launch_wait_timeout_selftest(dev.status, limit_ns,
                                                       static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_prefill_segmented(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* beta, const float* s0, void* y, float* s_final, int B,
+                          int T, int H, int dk, int dv, int dtype, float scale, int l2norm_qk,
+                          int num_segments, void* ws, size_t ws_bytes, void* stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(alpha) || !ok_ptr(beta) ||
+        !ok_ptr(y) || !ok_opt_ptr(s0) || !ok_opt_ptr(s_final))
+        return GDN_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || H < 1 || num_segments < 1) return GDN_ERR_INVALID_ARG;
+    if (int rc = check_dims(dk, dv, dtype)) return rc;
+    const size_t need = gdn::segmented_layout(B, T, H, dk, num_segments, dtype).total;
+    if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return GDN_ERR_WORKSPACE;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::PrefillArgs a{q, k, v, alpha, beta, s0, y, s_final, nullptr, B, T, H, dk, dv,
+                       dtype, scale, l2norm_qk ? 1 : 0, dev.status, ws, ws_bytes};
+    return map_cuda(gdn::launch_prefill_segmented(a, num_segments,
+                                                  static_cast<cudaStream_t>(stream)));
 }
 
 int gdn_read_device_status(int reset, int* device_status) {

@@ -15,6 +15,10 @@ struct DecodeArgs {
     int N, H, dk, dv, dtype;
     float scale;
     int l2norm;
+    // Gated form (eqs. (9)-(10)): when A_log != nullptr, alpha and beta hold the logits
+    // a = W_alpha x and b = W_beta x, and A_log, b_alpha [H] the per-head parameters.
+    const float* A_log;
+    const float* b_alpha;
 };
 
 // Dense prefill is the varlen case with B documents of T tokens each (cu_seqlens == nullptr).
@@ -33,6 +37,8 @@ struct PrefillArgs {
     int* status;                // device status word
     void* ws;                   // workspace (bf16 path), see prefill_workspace
     size_t ws_bytes;
+    const float* A_log;         // gated form, as in DecodeArgs
+    const float* b_alpha;
 };
 
 // Workspace of the bf16 prefill: per (chunk record, head) the operand tiles that the prep kernel
@@ -56,6 +62,12 @@ struct BackwardArgs {
     void* ws;
     size_t ws_bytes;
     int* status;
+    // Gated form, as in DecodeArgs; dalpha and dbeta then receive d a and d b, and the
+    // per-head gradients are summed into dA_log, db_alpha [H] (cleared by the launcher).
+    const float* A_log;
+    const float* b_alpha;
+    float* dA_log;
+    float* db_alpha;
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
@@ -76,9 +88,35 @@ size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv);
 size_t backward_chunked_workspace_bytes(int B, int T, int H, int dk, int dv);
 cudaError_t launch_backward_chunked(const BackwardArgs& a, cudaStream_t st);
 
+// The bracket of eq. (11), sigma(z) * RMSNorm(y) with the zero-centred gain (1 + w), over rows
+// of dv values, and its reverse mode (dw summed over all rows; cleared by the launcher).
+struct GatedNormArgs {
+    const void *y, *z;
+    const float* w;
+    const void* d_o;       // backward only
+    void* o;               // forward: o; backward: unused
+    void *dy, *dz;         // backward only
+    float* dw;             // backward only
+    long long rows;
+    int dv, dtype;
+    float eps;
+};
+cudaError_t launch_gated_norm(const GatedNormArgs& a, cudaStream_t st);
+cudaError_t launch_gated_norm_backward(const GatedNormArgs& a, cudaStream_t st);
+
 // A kernel whose bounded wait runs out (nothing arrives on its barrier): it records
 // GDN_ERR_TIMEOUT in `status` after about limit_ns and returns.
 cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns, cudaStream_t st);
+
+// Segment-parallel prefill of a dense batch (segmented.cu): every sequence cut into P segments
+// of L tokens (whole chunks), the segments' affine state maps formed by two prefill passes, a
+// scan of the maps from s0, and a third pass from the segments' start states.
+struct SegmentedLayout {
+    int L, P;  // segment length in tokens; number of non-empty segments
+    size_t off_inner, inner_bytes, off_cu, off_vzero, off_eye, off_m, off_n, off_start, total;
+};
+SegmentedLayout segmented_layout(int B, int T, int H, int D, int P, int dtype);
+cudaError_t launch_prefill_segmented(const PrefillArgs& a, int P, cudaStream_t st);
 
 // Size of the fixed device scratch array behind gdn_backward_noalloc.
 constexpr size_t kBackwardFixedScratchBytes = size_t(32) << 20;

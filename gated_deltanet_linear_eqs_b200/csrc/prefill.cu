@@ -238,6 +238,8 @@ struct PrepParams {
     uint8_t* ws_x;
     int* status;
     long long ab_elems;
+    const float* A_log;         // gated form: alpha, beta hold the logits of eqs. (9)-(10)
+    const float* b_alpha;
 };
 
 constexpr int kPrepThreads = 320;  // warp 0 loads, warp 1 TMEM + tensor cores, 2..9 compute
@@ -302,8 +304,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     if (warp == 0) {
         // ---------------------------------------------------------------- loads
-        // the tile copies first (lane 0's arrival carries the byte count), then alpha and beta;
-        // the other 31 arrivals follow the alpha / beta stores of all lanes
+        // the tile copies first (lane 0's arrival carries the byte count), then log2(alpha) and
+        // beta; the other 31 arrivals follow the stores of all lanes
         if (lane == 0) {
             mbar_arrive_expect_tx(&bars[PB_FULL], L::TX + (has_prev ? KB * 8192 : 0));
             const int z = (int)base;
@@ -322,8 +324,19 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int i = lane + 32 * u;
             const long t = base + i;
             const bool ok = i < nvalid && GUARD(t * p.H + h < p.ab_elems, DBG_GLOBAL_OOB, 1);
-            ab[i] = ok ? p.alpha[t * p.H + h] : 1.f;
-            ab[64 + i] = ok ? p.beta[t * p.H + h] : 0.f;
+            float lg = 0.f, bt = 0.f;  // rows past the end: alpha = 1, beta = 0
+            if (ok) {
+                const float av = p.alpha[t * p.H + h], bv = p.beta[t * p.H + h];
+                if (p.A_log) {
+                    lg = gate_log_decay(av, p.A_log[h], p.b_alpha[h]) * kLog2e;
+                    bt = gate_sigmoid(bv);
+                } else {
+                    lg = lg2(av);
+                    bt = bv;
+                }
+            }
+            ab[i] = lg;
+            ab[64 + i] = bt;
         }
         __syncwarp();
         if (lane != 0) mbar_arrive(&bars[PB_FULL]);
@@ -439,7 +452,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         bool ok = wwait(PB_FULL, 0);
         if (ok && hf == 0) {
             if (t < 64) {
-                float gl = lg2(ab[t]);
+                float gl = ab[t];  // log2(alpha)
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const float x = __shfl_up_sync(0xffffffffu, gl, o);
@@ -1273,7 +1286,7 @@ cudaError_t launch_prep(const PrefillArgs& a, cudaStream_t st) {
     PrepParams pp{a.alpha, a.beta, varlen ? map : nullptr, a.num_seqs, a.T, a.H,
                   nchunk_dense, ntask, 2 * nsm, a.scale, a.l2norm, ws + w.off_w, ws + w.off_p,
                   ws + w.off_u, reinterpret_cast<float*>(ws + w.off_s), ws + w.off_x, a.status,
-                  (long long)tokens * a.H};
+                  (long long)tokens * a.H, a.A_log, a.b_alpha};
     const int smem1 = PrepLayout<D>::BYTES + 1024;
     if ((e = cudaFuncSetAttribute(prep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   smem1)) != cudaSuccess)

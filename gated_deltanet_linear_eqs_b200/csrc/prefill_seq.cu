@@ -22,7 +22,8 @@ seq_prefill_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
                    const float* __restrict__ alpha, const float* __restrict__ beta,
                    const float* __restrict__ s0, T* __restrict__ y, float* __restrict__ s_final,
                    const int32_t* __restrict__ cu_seqlens, int T_len, int H, float scale,
-                   int l2norm) {
+                   int l2norm, const float* __restrict__ A_log,
+                   const float* __restrict__ b_alpha) {
     constexpr int NW = D / 8, CPL = D / 32, PL = D / 32;
     __shared__ float s_kh[2][D];
     __shared__ float s_qh[2][D];
@@ -93,7 +94,10 @@ seq_prefill_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
             s_red[buf][warp][1][c0 + j] = pq[j];
         }
         __syncthreads();
-        const float a = alpha[th], b = beta[th], kq = s_kq[buf];
+        // gated form: alpha, beta hold the logits of eqs. (9)-(10)
+        const float a = A_log ? expf(gate_log_decay(alpha[th], A_log[h], b_alpha[h])) : alpha[th];
+        const float b = A_log ? gate_sigmoid(beta[th]) : beta[th];
+        const float kq = s_kq[buf];
         float e[CPL];
 #pragma unroll
         for (int j = 0; j < CPL; ++j) {
@@ -124,7 +128,7 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st) {
     seq_prefill_kernel<D, T><<<a.num_seqs * a.H, D * 4, 0, st>>>(
         static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
         a.alpha, a.beta, a.s0, static_cast<T*>(a.y), a.s_final, a.cu_seqlens, a.T, a.H, a.scale,
-        a.l2norm);
+        a.l2norm, a.A_log, a.b_alpha);
     return cudaGetLastError();
 }
 

@@ -11,6 +11,10 @@ Recipe (per call, ``numpy.random.default_rng(seed)``, drawn in this order):
                                  stored as float32 (alpha, beta in (0, 1))
   S0       ~ N(0, 0.02^2)       float32, only if requested
   dy       ~ N(0, 1)            float32 draws rounded like q, only if requested
+
+Gated form (``make_gate_inputs``, its own generator): the logits a, b ~ N(0, 1) per
+(token, head), A_log ~ U(-1, 1) and b_alpha ~ N(0, 0.5^2) per head, all float32.
+Gated output (``make_norm_inputs``): y, z ~ N(0, 1) rounded like q, w ~ N(0, 0.1^2) float32.
 """
 from __future__ import annotations
 
@@ -93,3 +97,27 @@ def make_decode_state(N, H, dk, dv, seed=0, std=S0_STD):
     """Initial decode state S ~ N(0, 0.02^2), fp32 [N,H,dk,dv]."""
     rng = np.random.default_rng(seed)
     return torch.from_numpy((rng.standard_normal((N, H, dk, dv)) * std).astype(np.float32))
+
+
+def make_gate_inputs(shape, H, seed=0):
+    """Logits of the gated form: a, b fp32 of ``shape`` (last axis H) and the per-head
+    parameters A_log, b_alpha [H] fp32."""
+    rng = np.random.default_rng(seed)
+    a = rng.standard_normal(shape, dtype=np.float32)
+    b = rng.standard_normal(shape, dtype=np.float32)
+    A_log = rng.uniform(-1.0, 1.0, H).astype(np.float32)
+    b_alpha = (rng.standard_normal(H) * 0.5).astype(np.float32)
+    return dict(a=torch.from_numpy(a), b=torch.from_numpy(b), A_log=torch.from_numpy(A_log),
+                b_alpha=torch.from_numpy(b_alpha))
+
+
+def make_norm_inputs(rows, dv, dtype="bf16", seed=0, with_do=False):
+    """Inputs of the gated RMSNorm: y, z [rows, dv] in ``dtype``, w [dv] fp32, and the
+    upstream gradient d_o [rows, dv] when ``with_do``."""
+    rng = np.random.default_rng(seed)
+    out = dict(y=_round(rng.standard_normal((rows, dv), dtype=np.float32), dtype),
+               z=_round(rng.standard_normal((rows, dv), dtype=np.float32), dtype),
+               w=torch.from_numpy((rng.standard_normal(dv) * 0.1).astype(np.float32)), d_o=None)
+    if with_do:
+        out["d_o"] = _round(rng.standard_normal((rows, dv), dtype=np.float32), dtype)
+    return out

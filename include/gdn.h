@@ -60,7 +60,8 @@ typedef enum {
     GDN_OP_PREFILL = 0,
     GDN_OP_PREFILL_VARLEN = 1,
     GDN_OP_DECODE = 2,
-    GDN_OP_BACKWARD = 3
+    GDN_OP_BACKWARD = 3,
+    GDN_OP_PREFILL_SEGMENTED = 4  /* num_seqs carries the number of segments */
 } gdn_op;
 
 /* Static description of a status code.  Never NULL. */
@@ -202,11 +203,104 @@ int gdn_backward_noalloc(const void* q, const void* k, const void* v, const floa
 size_t gdn_backward_noalloc_max_workspace(void);
 
 /*
+ * Gated form: the same calls with alpha and beta given by their parameterisation (same page,
+ * "Methodology", "1. GDN Hybrid Token Mixing", eqs. (9)-(10)):
+ *
+ *     beta_t  = sigmoid(b_t)
+ *     alpha_t = exp[-exp(A) softplus(a_t + b_alpha)]
+ *
+ *   a [.., H] fp32: a_t = W_alpha x_t per (token, head), before the bias (in place of alpha);
+ *   b [.., H] fp32: b_t = W_beta x_t per (token, head) (in place of beta);
+ *   A_log [H], b_alpha [H] fp32: the per-head parameters A and b_alpha (this library's reading:
+ *   one each per head, like alpha_t itself).
+ * The projections W_alpha x, W_beta x are the caller's (dense products with learned weights).
+ * The decay is evaluated in log space, ln alpha = -exp(A) softplus(a + b_alpha), which is what
+ * the chunked kernels use, so strong decays never pass through an alpha that underflows.  Every
+ * other argument, layout, workspace and error is that of the plain call; A_log and b_alpha must
+ * be non-NULL and 16-byte aligned (else GDN_ERR_INVALID_ARG).  a and b may take any finite
+ * value; the domain precondition on alpha and beta holds by construction.
+ */
+int gdn_prefill_gated(const void* q, const void* k, const void* v, const float* a,
+                      const float* b, const float* A_log, const float* b_alpha, const float* s0,
+                      void* y, float* s_final, int B, int T, int H, int dk, int dv, int dtype,
+                      float scale, int l2norm_qk, void* ws, size_t ws_bytes, void* stream);
+int gdn_prefill_varlen_gated(const void* q, const void* k, const void* v, const float* a,
+                             const float* b, const float* A_log, const float* b_alpha,
+                             const int32_t* cu_seqlens, int num_seqs, const float* s0, void* y,
+                             float* s_final, int T, int H, int dk, int dv, int dtype, float scale,
+                             int l2norm_qk, void* ws, size_t ws_bytes, void* stream);
+int gdn_decode_step_gated(const void* q, const void* k, const void* v, const float* a,
+                          const float* b, const float* A_log, const float* b_alpha, float* state,
+                          void* y, int N, int H, int dk, int dv, int dtype, float scale,
+                          int l2norm_qk, void* stream);
+/*
+ * gdn_backward_gated -- gdn_backward for the gated form: writes da, db [B,T,H] fp32 (gradients
+ * with respect to a and b) in place of dalpha, dbeta, and dA_log, db_alpha [H] fp32 (sums over
+ * every token of the batch; the call overwrites them).  Workspace: GDN_OP_BACKWARD.  The
+ * per-head sums are accumulated with atomic adds, so their last bits may differ between runs.
+ */
+int gdn_backward_gated(const void* q, const void* k, const void* v, const float* a,
+                       const float* b, const float* A_log, const float* b_alpha, const float* s0,
+                       const void* dy, const float* ds_final, void* dq, void* dk_out,
+                       void* dv_out, float* da, float* db, float* dA_log, float* db_alpha,
+                       float* ds0, int B, int T, int H, int dk, int dv, int dtype, float scale,
+                       int l2norm_qk, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * gdn_gated_rmsnorm -- the bracket of eq. (11) of the same section,
+ *
+ *     o = sigmoid(z) * RMSNorm(y),   RMSNorm(y) = (1 + w) * y / sqrt(mean(y^2) + eps),
+ *
+ * over `rows` independent rows of dv values: one row is one head of one token (y as the
+ * recurrence writes it, [B,T,H,dv] being B*T*H rows).  "Zero-centered RMSNorm" is read as the
+ * gain (1 + w), so that w = 0 is the identity; no mean is subtracted.  W_z x (= z) and the W_o
+ * product after it are the caller's.
+ *   y, z, o [rows, dv] in dtype (bf16 or fp32); w [dv] fp32; dv in {64, 128}; eps >= 0
+ *   (1e-6 is this library's choice elsewhere); rows >= 0 (0 launches nothing, and y, z, w, o
+ *   may then be NULL).
+ * Errors: GDN_ERR_INVALID_ARG (null or misaligned pointer, rows < 0, eps < 0 or NaN, bad dtype),
+ * GDN_ERR_UNSUPPORTED_SHAPE (dv), GDN_ERR_CUDA.  No workspace.
+ */
+int gdn_gated_rmsnorm(const void* y, const void* z, const float* w, void* o, int64_t rows,
+                      int dv, int dtype, float eps, void* stream);
+/*
+ * gdn_gated_rmsnorm_backward -- gradients of the above given d_o [rows, dv]: dy, dz [rows, dv]
+ * in dtype and dw [dv] fp32 (summed over all rows; the call overwrites it, accumulating with
+ * atomic adds, so its last bits may differ between runs).  Same sizes and errors; with rows = 0
+ * only dw (zeros) is written and dw alone must be non-NULL.
+ */
+int gdn_gated_rmsnorm_backward(const void* y, const void* z, const float* w, const void* d_o,
+                               void* dy, void* dz, float* dw, int64_t rows, int dv, int dtype,
+                               float eps, void* stream);
+
+/*
  * Device status word of the current device: 0 when no kernel has recorded an
  * error, otherwise the first gdn_status a kernel recorded (GDN_ERR_TIMEOUT).
  * Synchronises the current device.  If reset != 0 the word is cleared.
  */
 int gdn_read_device_status(int reset, int* device_status);
+
+/*
+ * gdn_prefill_segmented -- gdn_prefill of a dense batch with every sequence cut along time into
+ * num_segments segments that run side by side.  By eqs. (1)-(3) one token maps the state
+ * affinely (S -> alpha (I - beta k k^T) S + beta k v^T), so each segment acts on its start state
+ * as S -> M S + N, computable from its own tokens.  The call runs the B * P segments as packed
+ * documents: once with v = 0 from S0 = I (giving every M), once from S0 = 0 (every N), scans
+ * the maps from s0 for every segment's start state (fp32), and once more from the start states
+ * (giving y).  This pays three prefill passes for B * P independent chains instead of B: it is
+ * for batches of few, long sequences, where the plain call leaves most SMs idle.
+ *   - Arguments and layouts as gdn_prefill; num_segments >= 1.  Segments are whole 64-token
+ *     chunks of ceil(ceil(T / 64) / num_segments) chunks each, so fewer may result; with one
+ *     segment the call is gdn_prefill.  dk == dv.
+ *   - s_final (if non-NULL) is the scan's state after the last segment.
+ *   - ws/ws_bytes: gdn_workspace_bytes(GDN_OP_PREFILL_SEGMENTED, B, T, H, dk, dv, num_segments).
+ *     It holds the inner packed prefill's workspace (bf16), a zero copy of v, and four fp32
+ *     states per (segment, head).
+ */
+int gdn_prefill_segmented(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* beta, const float* s0, void* y, float* s_final, int B,
+                          int T, int H, int dk, int dv, int dtype, float scale, int l2norm_qk,
+                          int num_segments, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * gdn_selftest_wait_timeout -- exercises the failure path of the library's bounded waits.

@@ -173,10 +173,82 @@ def test_backward_needs_its_workspace(lib):
     assert f(*bad, A, 1 << 30, None) == _abi.GDN_ERR_INVALID_ARG
 
 
+def test_gated_calls_reject_bad_arguments(lib):
+    """The gated entry points validate like the plain ones and also need A_log and b_alpha."""
+    pre = lambda **kw: lib.gdn_prefill_gated(
+        *[kw.get(n, A) for n in ("q", "k", "v", "a", "b", "Al", "ba")], 0, kw.get("y", A), 0, 1,
+        64, 1, kw.get("dk", 64), 64, 0, 1.0, 1, kw.get("ws", A), 1 << 30, None)
+    assert pre(Al=0) == _abi.GDN_ERR_INVALID_ARG
+    assert pre(ba=A + 4) == _abi.GDN_ERR_INVALID_ARG
+    assert pre(q=0) == _abi.GDN_ERR_INVALID_ARG
+    assert pre(dk=96) == _abi.GDN_ERR_UNSUPPORTED_SHAPE
+    assert pre(ws=0) == _abi.GDN_ERR_WORKSPACE
+    var = lambda **kw: lib.gdn_prefill_varlen_gated(
+        *[kw.get(n, A) for n in ("q", "k", "v", "a", "b", "Al", "ba", "cu")], 2, 0, A, A, 100, 2,
+        64, 64, 0, 1.0, 1, A, 1 << 30, None)
+    assert var(ba=0) == _abi.GDN_ERR_INVALID_ARG
+    assert var(cu=0) == _abi.GDN_ERR_INVALID_ARG
+    dec = lambda **kw: lib.gdn_decode_step_gated(
+        *[kw.get(n, A) for n in ("q", "k", "v", "a", "b", "Al", "ba", "st", "y")], 4, 2, 128, 128,
+        0, 1.0, 1, None)
+    assert dec(Al=0) == _abi.GDN_ERR_INVALID_ARG
+    assert dec(st=0) == _abi.GDN_ERR_INVALID_ARG
+    bwd = lambda **kw: lib.gdn_backward_gated(
+        *[kw.get(n, A) for n in ("q", "k", "v", "a", "b", "Al", "ba")], 0, A, 0,
+        *[kw.get(n, A) for n in ("dq", "dk", "dv", "da", "db", "dA", "dba")], 0, 1, 64, 1, 64, 64,
+        0, 1.0, 1, kw.get("ws", A), kw.get("wsb", 1 << 30), None)
+    assert bwd(dA=0) == _abi.GDN_ERR_INVALID_ARG
+    assert bwd(dba=A + 8) == _abi.GDN_ERR_INVALID_ARG
+    assert bwd(Al=0) == _abi.GDN_ERR_INVALID_ARG
+    assert bwd(ws=0) == _abi.GDN_ERR_WORKSPACE
+    assert bwd(wsb=16) == _abi.GDN_ERR_WORKSPACE
+
+
+def test_gated_rmsnorm_rejects_bad_arguments(lib):
+    fwd = lambda **kw: lib.gdn_gated_rmsnorm(
+        *[kw.get(n, A) for n in ("y", "z", "w", "o")], kw.get("rows", 10), kw.get("dv", 128),
+        kw.get("dt", 0), kw.get("eps", 1e-6), None)
+    assert fwd(y=0) == _abi.GDN_ERR_INVALID_ARG
+    assert fwd(w=A + 4) == _abi.GDN_ERR_INVALID_ARG
+    assert fwd(rows=-1) == _abi.GDN_ERR_INVALID_ARG
+    assert fwd(eps=-1.0) == _abi.GDN_ERR_INVALID_ARG
+    assert fwd(eps=float("nan")) == _abi.GDN_ERR_INVALID_ARG
+    assert fwd(dt=7) == _abi.GDN_ERR_INVALID_ARG
+    assert fwd(dv=96) == _abi.GDN_ERR_UNSUPPORTED_SHAPE
+    bwd = lambda **kw: lib.gdn_gated_rmsnorm_backward(
+        *[kw.get(n, A) for n in ("y", "z", "w", "do", "dy", "dz", "dw")], kw.get("rows", 10),
+        kw.get("dv", 64), 0, 1e-6, None)
+    assert bwd(dw=0) == _abi.GDN_ERR_INVALID_ARG
+    assert bwd(do=0) == _abi.GDN_ERR_INVALID_ARG
+    assert bwd(dv=32) == _abi.GDN_ERR_UNSUPPORTED_SHAPE
 def test_selftest_rejects_limits_out_of_range(lib):
     assert lib.gdn_selftest_wait_timeout(0, None) == _abi.GDN_ERR_INVALID_ARG
     assert lib.gdn_selftest_wait_timeout(999, None) == _abi.GDN_ERR_INVALID_ARG
     assert lib.gdn_selftest_wait_timeout(2_000_000_000, None) == _abi.GDN_ERR_INVALID_ARG
+
+
+def test_segmented_workspace_and_validation(lib):
+    n = ctypes.c_size_t(0)
+    plain = ctypes.c_size_t(0)
+    # one segment is the plain prefill, with its workspace
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL_SEGMENTED, 1, 4096, 16, 128, 128, 1,
+                                   ctypes.byref(n)) == 0
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL, 1, 4096, 16, 128, 128, 0,
+                                   ctypes.byref(plain)) == 0
+    assert n.value == plain.value
+    # four segments of 1024 tokens: the packed prefill's workspace for 4 documents, the zero
+    # copy of v (bf16 here, fp32 for fp32 inputs: the larger is reported) and 4 state arrays
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL_SEGMENTED, 1, 4096, 16, 128, 128, 4,
+                                   ctypes.byref(n)) == 0
+    states = 4 * 4 * 16 * 128 * 128 * 4
+    assert n.value >= 4096 * 16 * 128 * 4 + states
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_PREFILL_SEGMENTED, 1, 4096, 16, 128, 128, 0,
+                                   ctypes.byref(n)) == _abi.GDN_ERR_INVALID_ARG
+    f = lib.gdn_prefill_segmented
+    args = [A] * 5 + [0, A, 0, 1, 4096, 2, 128, 128, 0, 1.0, 1]
+    assert f(*args, 0, A, 1 << 40, None) == _abi.GDN_ERR_INVALID_ARG    # no segments
+    assert f(*args, 4, None, 0, None) == _abi.GDN_ERR_WORKSPACE
+    assert f(*args, 4, A, 16, None) == _abi.GDN_ERR_WORKSPACE
 
 
 def test_device_status_rejects_null(lib):

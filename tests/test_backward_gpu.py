@@ -102,3 +102,14 @@ def test_backward_workspace_is_caller_owned():
     ref = oracle.backward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], dy=inp["dy"])
     for k in ("dq", "dk", "dv", "dalpha", "dbeta"):
         assert max_rel(out[k], ref[k]) <= G_TOL, k
+
+
+def test_backward_slow_decay():
+    """Slow decays (alpha uniform in [0.97, 0.9995]) carry state and its gradient across many
+    chunks; every gradient and dS0 stay within their bars."""
+    B, T, H, d = 1, 1000, 2, 128
+    inp = make_inputs(B, T, H, d, d, seed=17, with_s0=True, with_dy=True)
+    rng = np.random.default_rng(18)
+    inp["alpha"] = torch.from_numpy(rng.uniform(0.97, 0.9995, (B, T, H)).astype(np.float32))
+    out, ref = _run(inp)
+    _check(out, ref)

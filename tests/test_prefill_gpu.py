@@ -199,3 +199,51 @@ def test_prefill_split_phases():
                                      None, scale=0.7)
     assert max_rel(y3, yr0) <= Y_TOL and frob_rel(s3, sr0) <= S_TOL
     assert api.gdn_read_device_status(reset=True) == 0
+
+
+def test_prefill_slow_decay_state_accuracy():
+    """Slow decays (alpha uniform in [0.97, 0.9995]) keep old state in play for many chunks, the
+    hard case for the state's bf16 operand in -W S.  An emulation of the kernel's rounding points
+    puts the state error near 6e-4 here; the bar is 1e-3."""
+    import numpy as np
+    B, T, H, d = 1, 4096, 2, 128
+    inp = make_inputs(B, T, H, d, d, seed=5, with_s0=True)
+    rng = np.random.default_rng(1)
+    inp["alpha"] = torch.from_numpy(rng.uniform(0.97, 0.9995, (B, T, H)).astype(np.float32))
+    y, sf = _run_dense(inp)
+    yr, sr = oracle.forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["s0"])
+    assert max_rel(y, yr) <= Y_TOL
+    assert frob_rel(sf, sr) <= S_TOL
+
+
+def test_prefill_varlen_many_documents_beyond_the_shared_map():
+    """More documents than the chunk-base scan keeps in shared memory (8192): the record map is
+    searched in global memory.  Lengths 0..4 tokens, so most documents are a single ragged chunk."""
+    import numpy as np
+    rng = np.random.default_rng(12)
+    lengths = [int(x) for x in rng.integers(0, 5, 9000)]
+    H, d = 1, 64
+    inp = make_varlen_inputs(lengths, H, d, d, seed=13)
+    g = _cuda(inp)
+    y, sf = api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                   g["cu_seqlens"], g["s0"])
+    torch.cuda.synchronize()
+    yr, sr = oracle.forward_varlen(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                                   inp["cu_seqlens"].numpy(), inp["s0"])
+    assert max_rel(y, yr) <= Y_TOL
+    assert frob_rel(sf, sr) <= S_TOL
+
+
+@pytest.mark.parametrize("lengths", [[1, 63, 64, 65, 130], [0, 300, 7]])
+def test_prefill_varlen_d64(lengths):
+    """The packed bf16 path at dk = dv = 64 (two 32-column chain slices per head)."""
+    H, d = 3, 64
+    inp = make_varlen_inputs(lengths, H, d, d, seed=7 + sum(lengths))
+    g = _cuda(inp)
+    y, sf = api.gdn_prefill_varlen(g["q"], g["k"], g["v"], g["alpha"], g["beta"],
+                                   g["cu_seqlens"], g["s0"], scale=0.6)
+    torch.cuda.synchronize()
+    yr, sr = oracle.forward_varlen(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                                   inp["cu_seqlens"].numpy(), inp["s0"], scale=0.6)
+    assert max_rel(y, yr) <= Y_TOL
+    assert frob_rel(sf, sr) <= S_TOL
