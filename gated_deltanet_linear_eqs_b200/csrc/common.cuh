@@ -72,10 +72,11 @@ __device__ __forceinline__ void record_status(int* status, int code) {
 
 }  // namespace gdn
 
-// ---- debug-build self checks ---------------------------------------------------------------
-// Compiled in only with -DGDN_DEBUG (libgdn_debug.so).  A failed check records
+// ---- self checks ---------------------------------------------------------------------------
+// Compiled in where GDN_DEBUG is defined: always in prefill.cu, which defines it itself, and in
+// every other source only with -DGDN_DEBUG (libgdn_debug.so).  A failed check records
 // (code, detail, block) in the device status words and the guarded access is skipped, so a
-// bad index is reported instead of faulting.  In the normal build every guard is `true`.
+// bad index is reported instead of faulting.  Where GDN_DEBUG is undefined every guard is `true`.
 namespace gdn {
 enum DebugCode {
     DBG_GLOBAL_OOB = 100,   // global index out of the tensor's extent

@@ -766,8 +766,11 @@ struct ChainLayout {
 // ring barriers (full / empty per slot), then per-step arrivals and tensor-core completions
 enum {
     CB_QWF = 0, CB_QWE = 2, CB_PXF = 4, CB_PXE = 6, CB_KF = 8, CB_KE = 10, CB_UF = 12, CB_UE = 14,
-    CB_AD = 16, CB_BD = 18, CB_YD = 20, CB_M4A = 22, CB_M4B = 24, CB_M5 = 26, CB_COUNT = 28
+    CB_AD = 16, CB_BD = 18, CB_YD = 20, CB_M4A = 22, CB_M4B = 24, CB_M5 = 26,
+    CB_FIN = 28,  // one per issuer: the commit that covers every product it issued
+    CB_COUNT = 30
 };
+static_assert(CB_COUNT <= 32, "the barrier area holds 32 barriers");
 
 struct ChainParams {
     const float* s0;
@@ -1000,6 +1003,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 mma_commit(&bars[CB_M4A + (j & 1)]);
                 mma_commit(&bars[CB_QWE + (j & 1)]);
             }
+            // no product of this thread may still be writing TMEM or arriving on a barrier when
+            // the CTA ends, also when a wait above gave up
+            mma_commit(&bars[CB_FIN]);
+            mbar_wait(&bars[CB_FIN], 0, never, 100000000ull);
         }
         __syncwarp();
     } else if (warp == 13) {
@@ -1029,6 +1036,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 mma_commit(&bars[CB_M5 + s]);
                 mma_commit(&bars[CB_KE + s]);
             }
+            mma_commit(&bars[CB_FIN + 1]);  // as for the other issuer
+            mbar_wait(&bars[CB_FIN + 1], 0, never, 100000000ull);
         }
         __syncwarp();
     } else {
@@ -1209,11 +1218,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #undef GUARD
     __syncwarp();
     __syncthreads();
+    // every product has completed (the issuers' final commits) and every copy has landed (the
+    // loaders' final waits), whether or not a wait gave up: TMEM can be released
     if (warp == 1) {
-        if (*abort_flag) {  // a wait gave up: let products already issued drain first
-            const long long t = clock64();
-            while (clock64() - t < 400000) {}
-        }
         tc_fence_after();
         tmem_dealloc(tmem, L::T_COLS);
     }

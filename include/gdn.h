@@ -32,7 +32,10 @@
  *    found inside a kernel (a bounded wait that ran out) are recorded in a
  *    device status word read with gdn_read_device_status().  Nothing throws.
  *  - The calls are thread safe: no global mutable host state is touched after
- *    the first call on a device (which caches its properties).
+ *    the first call on a device (which caches its properties and the device
+ *    addresses of the library's own device arrays).  Those cached addresses do
+ *    not survive cudaDeviceReset: do not call the library on a device after a
+ *    reset of it in the same process.
  */
 #ifndef GDN_H
 #define GDN_H
@@ -187,7 +190,10 @@ int gdn_backward(const void* q, const void* k, const void* v, const float* alpha
  *     gdn_backward's to rounding (both are fp32).
  *   - The first call on each device looks up the scratch array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call before any
- *     stream capture.
+ *     stream capture.  The address is kept for the life of the process, so the library must
+ *     not be used on a device after cudaDeviceReset (or any teardown of its primary context)
+ *     has run on it; the device status word behind gdn_read_device_status is kept the same
+ *     way.
  *   - All calls share the one array and it keeps the last call's contents; every byte a call
  *     reads from it is written earlier by the same call, so nothing needs clearing.  Calls
  *     whose kernels overlap on the GPU (other streams, other host threads) race on the array:

@@ -69,24 +69,25 @@ def test_backward_long_with_states(d):
     _check(out, ref)
 
 
-def test_backward_training_config_sampled():
+def test_backward_training_config_full():
     """Training shape B=8, T=4096, H=32, dk=dv=128, bf16, dy ~ N(0,1), S0 = 0, dS_final = 0.
-    The oracle recomputes 3 sampled (sequence, head) chains in full."""
+    Every (sequence, head) chain against the oracle's reverse recurrence, one sequence at a
+    time to bound host memory; the bars hold per sequence and for dS0 per chain."""
     B, T, H, d = 8, 4096, 32, 128
     inp = make_inputs(B, T, H, d, d, seed=0, with_dy=True)
     g = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
     out = api.gdn_backward(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["dy"])
     torch.cuda.synchronize()
-    for n in NAMES:
-        assert torch.isfinite(out[n]).all(), n
-    for b, h in [(0, 0), (3, 17), (7, 31)]:
-        sub = {n: inp[n][b:b + 1, :, h:h + 1].contiguous() for n in
-               ("q", "k", "v", "alpha", "beta", "dy")}
+    out = {n: out[n].cpu() for n in NAMES}
+    del g
+    for b in range(B):
+        sub = {n: inp[n][b:b + 1].contiguous() for n in ("q", "k", "v", "alpha", "beta", "dy")}
         ref = oracle.backward(sub["q"], sub["k"], sub["v"], sub["alpha"], sub["beta"],
                               dy=sub["dy"])
         for n in ("dq", "dk", "dv", "dalpha", "dbeta"):
-            assert max_rel(out[n][b:b + 1, :, h:h + 1], ref[n]) <= G_TOL, (n, b, h)
-        assert frob_rel(out["ds0"][b:b + 1, h:h + 1], ref["ds0"]) <= S_TOL
+            assert max_rel(out[n][b:b + 1], ref[n]) <= G_TOL, (n, b)
+        for h in range(H):
+            assert frob_rel(out["ds0"][b, h], ref["ds0"][0, h]) <= S_TOL, (b, h)
 
 
 def test_backward_workspace_is_caller_owned():

@@ -53,28 +53,26 @@ def test_decode_many_steps_small():
     assert frob_rel(Sg, Sr) <= 1e-5
 
 
-def test_decode_full_size_1000_steps_sampled():
+def test_decode_full_size_1000_steps_full():
     """Full decode workload (256 sequences x 16 heads x 128 x 128 fp32 state, 1000 steps with
-    fresh seeded tokens); the oracle follows 6 sampled (sequence, head) pairs all the way."""
+    fresh seeded tokens); the oracle follows every (sequence, head) pair all the way: y of
+    every step within the y bar, and the final state within the state bar per pair."""
     N, H, d, steps = 256, 16, 128, 1000
     S = make_decode_state(N, H, d, d, seed=0)
     Sg = S.cuda()
-    pairs = [(0, 0), (17, 3), (128, 15), (200, 7), (255, 0), (99, 9)]
-    Sr = np.stack([S[n, h].double().numpy() for n, h in pairs])[:, None]  # [P,1,d,d]
+    Sr = S.double().numpy()
     worst_y = 0.0
     for t in range(steps):
         inp = make_decode_step_inputs(N, H, d, d, step=t)
         g = _dev(inp)
         y = api.gdn_decode_step(g["q"], g["k"], g["v"], g["alpha"], g["beta"], Sg)
-        sel = {n: torch.stack([inp[n][a, b] for a, b in pairs])[:, None] for n in
-               ("q", "k", "v", "alpha", "beta")}
-        yr, Sr = oracle.decode_step(sel["q"], sel["k"], sel["v"], sel["alpha"], sel["beta"], Sr)
-        yg = torch.stack([y[a, b] for a, b in pairs])[:, None]
-        worst_y = max(worst_y, max_rel(yg, yr))
-    Sg_sel = torch.stack([Sg[a, b] for a, b in pairs])[:, None]
+        yr, Sr = oracle.decode_step(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], Sr)
+        worst_y = max(worst_y, max_rel(y, yr))
     assert worst_y <= Y_TOL
-    assert frob_rel(Sg_sel, Sr) <= S_TOL
-    assert torch.isfinite(Sg).all()
+    Sg = Sg.cpu()
+    assert frob_rel(Sg, Sr) <= S_TOL
+    for n in range(N):
+        assert frob_rel(Sg[n], Sr[n]) <= S_TOL, n
 
 
 def test_decode_equals_oracle_prefill_of_same_tokens():
