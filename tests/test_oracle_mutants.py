@@ -217,3 +217,26 @@ CHUNKED_MUTANTS = [
 def test_chunked_pins_reject_mutant(tmp_path, name, old, new):
     caught = _python_mutant_caught(tmp_path, CHUNKED_SRC, CHUNKED_CHECKS, name, old, new)
     assert caught, f"no pin rejects the planted mistake {name!r}"
+
+
+CONV_SRC = os.path.join(os.path.dirname(oracle.__file__), "short_conv.py")
+
+CONV_MUTANTS = [
+    ("taps_reversed", "acc += w[:, i] * ext[t + i]", "acc += w[:, W - 1 - i] * ext[t + i]"),
+    ("window_off_by_one", "acc += w[:, i] * ext[t + i]",
+     "acc += w[:, i] * ext[min(t + i + 1, ext.shape[0] - 1)]"),
+    ("state_ignored", "ext = np.concatenate([st[n], x[a:b]], axis=0)",
+     "ext = np.concatenate([0.0 * st[n], x[a:b]], axis=0)"),
+    ("final_state_from_first_rows", "final[n] = ext[ext.shape[0] - (W - 1):] if W > 1 else final[n]",
+     "final[n] = ext[:W - 1] if W > 1 else final[n]"),
+    ("silu_as_sigmoid", "return x / (1.0 + np.exp(-x))", "return 1.0 / (1.0 + np.exp(-x))"),
+    ("documents_not_reset", "ext = np.concatenate([st[n], x[a:b]], axis=0)",
+     "ext = np.concatenate([x[max(a - (W - 1), 0):a] if a >= W - 1 else st[n], x[a:b]], axis=0)"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", CONV_MUTANTS, ids=[m[0] for m in CONV_MUTANTS])
+def test_short_conv_pins_reject_mutant(tmp_path, name, old, new):
+    import tests.test_oracle_short_conv as conv_pins
+    caught = _python_mutant_caught(tmp_path, CONV_SRC, conv_pins.CHECKS, name, old, new)
+    assert caught, f"no pin rejects the planted mistake {name!r}"
