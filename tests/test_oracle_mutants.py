@@ -240,3 +240,27 @@ def test_short_conv_pins_reject_mutant(tmp_path, name, old, new):
     import tests.test_oracle_short_conv as conv_pins
     caught = _python_mutant_caught(tmp_path, CONV_SRC, conv_pins.CHECKS, name, old, new)
     assert caught, f"no pin rejects the planted mistake {name!r}"
+
+
+QSA_SRC = os.path.join(os.path.dirname(oracle.__file__), "qsa_indexer.py")
+
+QSA_MUTANTS = [
+    ("relu_dropped", "out.append(np.maximum(sim, 0.0).sum(axis=0))", "out.append(sim.sum(axis=0))"),
+    ("max_over_heads", "out.append(np.maximum(sim, 0.0).sum(axis=0))",
+     "out.append(np.maximum(sim, 0.0).max(axis=0))"),
+    ("mask_misses_completed_block", "nvis = (i + 1) // r", "nvis = i // r"),
+    ("mask_admits_partial_block", "nvis = (i + 1) // r", "nvis = (i + r) // r"),
+    ("ties_to_higher_index", "key=lambda b: (-s[b], b)", "key=lambda b: (-s[b], -b)"),
+    ("norm_without_gain", "return _f64(g) * x / np.sqrt(", "return x / np.sqrt("),
+    ("partial_block_pooled", "nb = (b - a) // r", "nb = -(-(b - a) // r)"),
+    ("selection_in_score_order", "sel = sorted(order)", "sel = list(order)"),
+    ("blocks_from_stream_start", "rows.append(np.mean(k[a + r * j:a + r * (j + 1)], axis=0))",
+     "rows.append(np.mean(k[r * j:r * (j + 1)], axis=0))"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", QSA_MUTANTS, ids=[m[0] for m in QSA_MUTANTS])
+def test_qsa_pins_reject_mutant(tmp_path, name, old, new):
+    import tests.test_oracle_qsa as qsa_pins
+    caught = _python_mutant_caught(tmp_path, QSA_SRC, qsa_pins.CHECKS, name, old, new)
+    assert caught, f"no pin rejects the planted mistake {name!r}"
