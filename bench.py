@@ -293,7 +293,148 @@ def run_ours(args, rank, world, local_rank):
                                            barrier)
     if args.only in ("all", "segmented"):
         out["segmented"] = run_segmented(args, dev, max_over_ranks, barrier, rank, world)
+    if args.only in ("all", "qsa"):
+        out["qsa_indexer"] = run_qsa(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier)
+    if args.only in ("all", "conv"):
+        out["short_conv"] = run_short_conv(args, dev, uuid, peaks, peak_src, max_over_ranks,
+                                           barrier)
     return out
+
+
+QSA_BUDGET = 512
+
+
+def run_qsa(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier):
+    """The QSA block indexer over the prefill workload's stream (T = 32768, 4 documents) with
+    4 indexer query heads and one key head of dim 128 and the budget of 512 blocks: the scores
+    call (pooling + tcgen05 products) and the selection call, each timed alone."""
+    import torch
+    from gated_deltanet_linear_eqs_b200 import api
+    from gated_deltanet_linear_eqs_b200.inputs import make_qsa_inputs, varlen_lengths
+    lengths = varlen_lengths(T_TOTAL, NDOCS, seed=0)
+    g = {k: v.to(dev) for k, v in make_qsa_inputs(lengths, seed=0).items()}
+    maxlen = max(lengths)
+    res = {}
+    k_hat, base, scores = api.gdn_qsa_block_scores(g["q"], g["k"], g["g"], g["cu_seqlens"], maxlen)
+    sel = api.gdn_qsa_select_blocks(scores, g["cu_seqlens"], QSA_BUDGET)
+    # visible (token, block) pairs: sum over documents of sum_i floor((i + 1) / 4)
+    pairs = sum(sum((i + 1) // 4 for i in range(n)) for n in lengths)
+    flops = 2 * 4 * 128 * pairs                      # the causal products, 4 heads
+    sel_bytes = pairs * 4 + T_TOTAL * QSA_BUDGET * 4   # scores read once, selection written
+
+    def scores_call():
+        api.gdn_qsa_block_scores(g["q"], g["k"], g["g"], g["cu_seqlens"], maxlen)
+
+    def select_call():
+        api.gdn_qsa_select_blocks(scores, g["cu_seqlens"], QSA_BUDGET, sel=sel)
+    for name, fn in (("scores", scores_call), ("select", select_call)):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with ClockSampler(uuid) as clk:
+            e0.record()
+            for _ in range(args.steps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        if name == "scores":
+            tf = flops / (ms / 1e3) / 1e12
+            roof = {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"], "flops_per_launch": flops,
+                    "traffic": None, "peak_source": peak_src}
+        else:
+            gbs = sel_bytes / (ms / 1e3) / 1e9
+            roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": sel_bytes,
+                    "traffic": None, "peak_source": peak_src}
+        res[name] = {"ms_per_launch": ms, "roofline": roof, "clocks": clk.summary()}
+    res["config"] = {"workload": f"QSA indexer: {T_TOTAL} tokens in {NDOCS} seeded documents, "
+                                 f"4 query heads + 1 key head of dim 128, blocks of 4 tokens, "
+                                 f"budget {QSA_BUDGET}; {pairs} visible (token, block) pairs",
+                     "l2": "the scores (185 MB) exceed the 126 MB L2; no flush"}
+    res["gpu_launches"] = 3 * args.steps + args.steps
+    return res
+
+
+CONV_W = 4
+
+
+def run_short_conv(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier):
+    """The short causal convolution over the prefill workload's q, k, v as one fused
+    [T, 3 H d] bf16 tensor (W = 4 taps, SiLU, a conv state per document), and its decode-step
+    form over the decode workload's tokens (256 sequences); both HBM-bound streams."""
+    import torch
+    from gated_deltanet_linear_eqs_b200 import api
+    from gated_deltanet_linear_eqs_b200.inputs import make_conv_inputs, varlen_lengths
+    C = 3 * H * D
+    lengths = varlen_lengths(T_TOTAL, NDOCS, seed=0)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v)
+         for k, v in make_conv_inputs(lengths, C, CONV_W, seed=0).items()}
+    y = torch.empty_like(g["x"])
+    sf = torch.empty_like(g["conv_state"])
+    stn = make_conv_inputs([1] * DEC_N, C, CONV_W, seed=1)
+    xs, ws_, st = stn["x"].to(dev), stn["w"].to(dev), stn["conv_state"].to(dev)
+    ys = torch.empty_like(xs)
+    res = {}
+
+    def varlen():
+        api.gdn_short_conv_varlen(g["x"], g["w"], g["cu_seqlens"], g["conv_state"],
+                                  activation="silu", y=y)
+
+    # the step form is a few microseconds of work: its launches are replayed from a CUDA graph
+    # so that the host's per-call cost stays out of the timed region
+    n_graph = 100
+    api.gdn_short_conv_step(xs, ws_, st, activation="silu", y=ys)  # loads the library
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(n_graph):
+            api.gdn_short_conv_step(xs, ws_, st, activation="silu", y=ys)
+
+    def step():
+        graph.replay()
+    states = NDOCS * (CONV_W - 1) * C * 2
+    for name, fn, nbytes, reps in (
+            ("varlen", varlen, 2 * T_TOTAL * C * 2 + 2 * states + C * CONV_W * 4, args.steps),
+            ("step", step, n_graph * (2 * DEC_N * C * 2 + 2 * DEC_N * (CONV_W - 1) * C * 2
+                                      + C * CONV_W * 4), max(3, args.steps // 4))):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with ClockSampler(uuid) as clk:
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1) / reps)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        if name == "step":  # per launch, from a replay of n_graph launches
+            ms, nbytes = ms / n_graph, nbytes // n_graph
+        res[name] = {"ms_per_launch": ms, "bytes_per_launch": nbytes, "GB/s": gbs,
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                                  "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                                  "traffic": profile_traffic(
+                                      "short_conv_T32768_C6144.md",
+                                      "gated_deltanet_linear_eqs_b200/csrc/short_conv.cu",
+                                      key=f"{name}_dram_bytes_per_launch"),
+                                  "peak_source": peak_src},
+                     "clocks": clk.summary()}
+    res["config"] = {"workload": f"short causal conv: fused q/k/v [{T_TOTAL}, {C}] bf16 of the "
+                                 f"varlen workload ({NDOCS} documents), W={CONV_W}, SiLU, conv "
+                                 f"state per document; step form: {DEC_N} sequences x {C} channels",
+                     "l2": "the varlen launch streams 805 MB, beyond the 126 MB L2; the step "
+                           "form's 25 MB stays in L2 (no flush), so its GB/s is an L2 figure"}
+    res["gpu_launches"] = args.steps + n_graph * max(3, args.steps // 4)
+    del graph
+    return res
 
 
 SEG_B, SEG_T, SEG_H = 1, 131072, 4  # few, long chains: 4 heads x 4 column slices of 2048 chunks
@@ -504,6 +645,21 @@ def run_profile(args):
         for _ in range(n + 1):
             api.gdn_gated_rmsnorm(g["y"], g["z"], g["w"])
             api.gdn_gated_rmsnorm_backward(g["y"], g["z"], g["w"], g["d_o"])
+    elif args.profile == "qsa":
+        from gated_deltanet_linear_eqs_b200.inputs import make_qsa_inputs, varlen_lengths
+        lengths = varlen_lengths(T_TOTAL, NDOCS, seed=0)
+        g = {k: v.to(dev) for k, v in make_qsa_inputs(lengths, seed=0).items()}
+        for _ in range(n + 1):
+            api.gdn_qsa_indexer(g["q"], g["k"], g["g"], g["cu_seqlens"], max(lengths),
+                                budget=QSA_BUDGET)
+    elif args.profile == "conv":
+        from gated_deltanet_linear_eqs_b200.inputs import make_conv_inputs, varlen_lengths
+        g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v)
+             for k, v in make_conv_inputs(varlen_lengths(T_TOTAL, NDOCS, seed=0), 3 * H * D,
+                                          CONV_W, seed=0).items()}
+        for _ in range(n + 1):
+            api.gdn_short_conv_varlen(g["x"], g["w"], g["cu_seqlens"], g["conv_state"],
+                                      activation="silu")
     else:
         from gated_deltanet_linear_eqs_b200._abi import GDN_OP_BACKWARD
         g = train_inputs(dev)
@@ -649,11 +805,13 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "train", "gated", "segmented"],
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "train", "gated", "segmented",
+                                       "conv", "qsa"],
                     default="all")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--train-steps", type=int, default=3)
-    ap.add_argument("--profile", choices=["prefill", "decode", "backward", "gated"], default=None,
+    ap.add_argument("--profile", choices=["prefill", "decode", "backward", "gated", "conv", "qsa"],
+                    default=None,
                     help="launch-only mode for ncu (no timing, no JSON)")
     ap.add_argument("--launches", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -704,6 +862,10 @@ def main():
         line["train"] = res["train"]
     if "segmented" in res:
         line["segmented"] = res["segmented"]
+    if "short_conv" in res:
+        line["short_conv"] = res["short_conv"]
+    if "qsa_indexer" in res:
+        line["qsa_indexer"] = res["qsa_indexer"]
     if "gated_norm" in res:
         line["gated_norm"] = res["gated_norm"]
         if "prefill" not in res and "decode" not in res:

@@ -31,6 +31,7 @@ GDN_OP_PREFILL_VARLEN = 1
 GDN_OP_DECODE = 2
 GDN_OP_BACKWARD = 3
 GDN_OP_PREFILL_SEGMENTED = 4
+GDN_OP_QSA_SCORES = 5
 
 _P = ctypes.c_void_p
 _F = ctypes.c_float
@@ -62,6 +63,11 @@ SIGNATURES = {
     "gdn_gated_rmsnorm": (_I, [_P] * 4 + [ctypes.c_int64, _I, _I, _F, _P]),
     "gdn_gated_rmsnorm_backward": (_I, [_P] * 7 + [ctypes.c_int64, _I, _I, _F, _P]),
     "gdn_read_device_status": (_I, [_I, ctypes.POINTER(_I)]),
+    "gdn_short_conv_varlen": (_I, [_P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "gdn_short_conv_step": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "gdn_qsa_block_scores": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _I, _P, _S, _P]),
+    "gdn_qsa_select_blocks": (_I, [_P, _I, _P, _I, _I, _I, _P, _P]),
+    "gdn_qsa_indexer": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _S, _P]),
     "gdn_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
     "gdn_prefill_segmented": (_I, [_P] * 8 + [_I] * 6 + [_F, _I, _I, _P, _S, _P]),
 }

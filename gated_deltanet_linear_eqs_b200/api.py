@@ -479,3 +479,102 @@ def gdn_selftest_wait_timeout(limit_ns=1_000_000, stream=None):
     gdn_read_device_status() reports GDN_ERR_TIMEOUT."""
     _check(_lib().gdn_selftest_wait_timeout(int(limit_ns), _stream(stream)),
            "gdn_selftest_wait_timeout")
+
+
+_ACT = {"none": 0, "silu": 1}
+
+
+def gdn_short_conv_varlen(x, w, cu_seqlens, conv_state=None, activation="none",
+                          return_state=True, y=None, stream=None):
+    """Short causal convolution of packed documents: x [T, C] (bf16 or fp32, C % 8 == 0),
+    w [C, W] fp32, cu_seqlens [N+1] int32 (CUDA), conv_state [N, W-1, C] like x or None (zero).
+    Returns (y [T, C], final conv state [N, W-1, C] or None)."""
+    dt = x.dtype
+    if dt not in _DT:
+        raise ValueError("x must be bf16 or fp32")
+    if x.dim() != 2 or w.dim() != 2:
+        raise ValueError("x must be [T, C] and w [C, W]")
+    T, C = x.shape
+    W = w.shape[1]
+    _need(x, "x", dt)
+    _need(w, "w", torch.float32, (C, W))
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    N = cu_seqlens.numel() - 1
+    _need(conv_state, "conv_state", dt, (N, W - 1, C), optional=True)
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", dt, (T, C))
+    sf = torch.empty((N, W - 1, C), dtype=dt, device=x.device) if return_state else None
+    rc = _lib().gdn_short_conv_varlen(_p(x), _p(w), _p(cu_seqlens), N, _p(conv_state), _p(sf),
+                                      _p(y), T, C, W, _DT[dt], _ACT[activation], _stream(stream))
+    _check(rc, "gdn_short_conv_varlen")
+    return y, sf
+
+
+def gdn_short_conv_step(x, w, conv_state, activation="none", y=None, stream=None):
+    """One decode token per sequence: x [N, C], w [C, W] fp32, conv_state [N, W-1, C] like x,
+    updated in place.  Returns y [N, C]."""
+    dt = x.dtype
+    if dt not in _DT:
+        raise ValueError("x must be bf16 or fp32")
+    N, C = x.shape
+    W = w.shape[1]
+    _need(x, "x", dt)
+    _need(w, "w", torch.float32, (C, W))
+    _need(conv_state, "conv_state", dt, (N, W - 1, C))
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", dt, (N, C))
+    rc = _lib().gdn_short_conv_step(_p(x), _p(w), _p(conv_state), _p(y), N, C, W, _DT[dt],
+                                    _ACT[activation], _stream(stream))
+    _check(rc, "gdn_short_conv_step")
+    return y
+
+
+def _qsa_ld(max_doc_len):
+    return ((max_doc_len // 4) + 3) // 4 * 4
+
+
+def gdn_qsa_block_scores(q, k, g, cu_seqlens, max_doc_len, stream=None):
+    """QSA indexer, pooled keys and block scores: q [T, 4, 128] bf16, k [T, 128] bf16, g [128]
+    fp32, cu_seqlens [N+1] int32 (CUDA), every document at most max_doc_len tokens.  Returns
+    (k_hat [T//4, 128] bf16, block_base [N+1] int32, scores [T, ld] fp32); row t of scores holds
+    its visible blocks' scores (document-local block order), the rest is not written."""
+    T = q.shape[0]
+    _need(q, "q", torch.bfloat16, (T, 4, 128))
+    _need(k, "k", torch.bfloat16, (T, 128))
+    _need(g, "g", torch.float32, (128,))
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    N = cu_seqlens.numel() - 1
+    ld = _qsa_ld(max_doc_len)
+    dev = q.device
+    k_hat = torch.empty((T // 4, 128), dtype=torch.bfloat16, device=dev)
+    base = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn_workspace_bytes(_abi.GDN_OP_QSA_SCORES, 1, max(T, 1), 1, 128, 128, N),
+                     dtype=torch.uint8, device=dev)
+    rc = _lib().gdn_qsa_block_scores(_p(q), _p(k), _p(g), _p(cu_seqlens), N, T, int(max_doc_len),
+                                     _p(k_hat), _p(base), _p(scores), ld, _p(ws), ws.numel(),
+                                     _stream(stream))
+    _check(rc, "gdn_qsa_block_scores")
+    return k_hat, base, scores
+
+
+def gdn_qsa_select_blocks(scores, cu_seqlens, budget=512, sel=None, stream=None):
+    """Top-budget block selection from gdn_qsa_block_scores' scores: sel [T, budget] int32."""
+    _need(scores, "scores", torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    T, ld = scores.shape
+    if sel is None:
+        sel = torch.empty((T, budget), dtype=torch.int32, device=scores.device)
+    _need(sel, "sel", torch.int32, (T, budget))
+    rc = _lib().gdn_qsa_select_blocks(_p(scores), ld, _p(cu_seqlens), cu_seqlens.numel() - 1, T,
+                                      int(budget), _p(sel), _stream(stream))
+    _check(rc, "gdn_qsa_select_blocks")
+    return sel
+
+
+def gdn_qsa_indexer(q, k, g, cu_seqlens, max_doc_len, budget=512, stream=None):
+    """Both steps: returns (sel [T, budget] int32, k_hat, block_base, scores)."""
+    k_hat, base, scores = gdn_qsa_block_scores(q, k, g, cu_seqlens, max_doc_len, stream)
+    return gdn_qsa_select_blocks(scores, cu_seqlens, budget, stream=stream), k_hat, base, scores

@@ -111,6 +111,10 @@ int gdn_workspace_bytes(int op, int B, int T, int H, int dk, int dv, int num_seq
             *bytes = a > f ? a : f;
             return GDN_OK;
         }
+        case GDN_OP_QSA_SCORES:
+            if (num_seqs < 1) return GDN_ERR_INVALID_ARG;
+            *bytes = gdn::qsa_workspace_bytes(num_seqs);
+            return GDN_OK;
         default:
             return GDN_ERR_INVALID_ARG;
     }
@@ -374,6 +378,83 @@ int gdn_backward_noalloc(const void* q, const void* k, const void* v, const floa
 }
 
 size_t gdn_backward_noalloc_max_workspace(void) { return gdn::kBackwardFixedScratchBytes; }
+
+static int check_conv(const float* w, int C, int width, int dtype, int activation) {
+    if (!ok_ptr(w) || C < 8 || C % 8 != 0 || width < 1 || width > 8) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 && dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (activation != 0 && activation != 1) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+int gdn_short_conv_varlen(const void* x, const float* w, const int32_t* cu_seqlens,
+                          int num_seqs, const void* conv_state_in, void* conv_state_out, void* y,
+                          int T, int C, int width, int dtype, int activation, void* stream) {
+    if (int rc = check_conv(w, C, width, dtype, activation)) return rc;
+    if (T < 0 || num_seqs < 1 || !ok_ptr(cu_seqlens)) return GDN_ERR_INVALID_ARG;
+    const auto ok_tok = [T](const void* p) { return T == 0 ? aligned16(p) : ok_ptr(p); };
+    if (!ok_tok(x) || !ok_tok(y) || !ok_opt_ptr(conv_state_in) || !ok_opt_ptr(conv_state_out))
+        return GDN_ERR_INVALID_ARG;
+    if (conv_state_in != nullptr && conv_state_in == conv_state_out) return GDN_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::ShortConvArgs a{x, w, cu_seqlens, num_seqs, conv_state_in, conv_state_out, y, T, C,
+                         width, dtype, activation == 1};
+    return map_cuda(gdn::launch_short_conv(a, false, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_short_conv_step(const void* x, const float* w, void* conv_state, void* y, int N, int C,
+                        int width, int dtype, int activation, void* stream) {
+    if (int rc = check_conv(w, C, width, dtype, activation)) return rc;
+    if (N < 1 || !ok_ptr(x) || !ok_ptr(y)) return GDN_ERR_INVALID_ARG;
+    if (width > 1 ? !ok_ptr(conv_state) : !ok_opt_ptr(conv_state)) return GDN_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::ShortConvArgs a{x, w, nullptr, N, conv_state, conv_state, y, 1, C, width, dtype,
+                         activation == 1};
+    return map_cuda(gdn::launch_short_conv(a, true, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_qsa_block_scores(const void* q, const void* k, const float* g, const int32_t* cu_seqlens,
+                         int num_seqs, int T, int max_doc_len, void* k_hat, int32_t* block_base,
+                         float* scores, int ld, void* ws, size_t ws_bytes, void* stream) {
+    if (T < 0 || num_seqs < 1 || max_doc_len < 0 || max_doc_len > T) return GDN_ERR_INVALID_ARG;
+    if (ld < max_doc_len / 4 || ld % 4 != 0) return GDN_ERR_INVALID_ARG;
+    const auto ok_tok = [T](const void* p) { return T == 0 ? aligned16(p) : ok_ptr(p); };
+    if (!ok_tok(q) || !ok_tok(k) || !ok_ptr(g) || !ok_ptr(cu_seqlens) || !ok_ptr(block_base) ||
+        !ok_tok(scores))
+        return GDN_ERR_INVALID_ARG;
+    if (T / 4 > 0 ? !ok_ptr(k_hat) : !aligned16(k_hat)) return GDN_ERR_INVALID_ARG;
+    if (ws == nullptr || !aligned16(ws) || ws_bytes < gdn::qsa_workspace_bytes(num_seqs))
+        return GDN_ERR_WORKSPACE;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::QsaArgs a{q, k, g, cu_seqlens, num_seqs, T, max_doc_len, k_hat, block_base, scores, ld,
+                   0, nullptr, dev.status, ws, ws_bytes};
+    return map_cuda(gdn::launch_qsa_scores(a, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_qsa_select_blocks(const float* scores, int ld, const int32_t* cu_seqlens, int num_seqs,
+                          int T, int budget, int32_t* sel, void* stream) {
+    if (T < 0 || num_seqs < 1 || budget < 1 || ld < 0 || ld % 4 != 0) return GDN_ERR_INVALID_ARG;
+    const auto ok_tok = [T](const void* p) { return T == 0 ? aligned16(p) : ok_ptr(p); };
+    if (!ok_tok(scores) || !ok_tok(sel) || !ok_ptr(cu_seqlens)) return GDN_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if (int rc = current_device_info(&dev)) return rc;
+    gdn::QsaArgs a{nullptr, nullptr, nullptr, cu_seqlens, num_seqs, T, 0, nullptr, nullptr,
+                   const_cast<float*>(scores), ld, budget, sel, dev.status, nullptr, 0};
+    return map_cuda(gdn::launch_qsa_select(a, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_qsa_indexer(const void* q, const void* k, const float* g, const int32_t* cu_seqlens,
+                    int num_seqs, int T, int max_doc_len, int budget, void* k_hat,
+                    int32_t* block_base, float* scores, int ld, int32_t* sel, void* ws,
+                    size_t ws_bytes, void* stream) {
+    if (budget < 1 || (T > 0 && !ok_ptr(sel))) return GDN_ERR_INVALID_ARG;
+    if (int rc = gdn_qsa_block_scores(q, k, g, cu_seqlens, num_seqs, T, max_doc_len, k_hat,
+                                      block_base, scores, ld, ws, ws_bytes, stream))
+        return rc;
+    return gdn_qsa_select_blocks(scores, ld, cu_seqlens, num_seqs, T, budget, sel, stream);
+}
 
 int gdn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
     if (limit_ns < 1000 || limit_ns > 1000000000ull) return GDN_ERR_INVALID_ARG;

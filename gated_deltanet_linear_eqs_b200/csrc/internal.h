@@ -118,6 +118,44 @@ struct SegmentedLayout {
 SegmentedLayout segmented_layout(int B, int T, int H, int D, int P, int dtype);
 cudaError_t launch_prefill_segmented(const PrefillArgs& a, int P, cudaStream_t st);
 
+// The short causal convolution (short_conv.cu): depthwise, W taps per channel, over [T, C]
+// tensors with per-document conv states of W - 1 rows.  The varlen form reads state_in (nullable)
+// and writes state_out (nullable); the step form (one token per sequence, num_seqs sequences)
+// updates state_out in place.
+struct ShortConvArgs {
+    const void* x;
+    const float* w;              // [C, W] fp32
+    const int32_t* cu_seqlens;   // varlen form: device, [num_seqs + 1]
+    int num_seqs;
+    const void* state_in;        // [num_seqs, W - 1, C], dtype of x
+    void* state_out;
+    void* y;
+    int T, C, width, dtype;
+    bool silu;
+};
+cudaError_t launch_short_conv(const ShortConvArgs& a, bool step, cudaStream_t st);
+
+// The QSA block indexer (qsa_indexer.cu): pooled key blocks, block scores, top-budget selection.
+struct QsaArgs {
+    const void* q;               // [T, 4, 128] bf16 indexer queries
+    const void* k;               // [T, 128] bf16 indexer keys (one shared head)
+    const float* g;              // [128] RMSNorm gain
+    const int32_t* cu_seqlens;   // device, [num_seqs + 1]
+    int num_seqs, T, max_doc_len;
+    void* k_hat;                 // [T / 4, 128] bf16: pooled keys, packed by document
+    int32_t* block_base;         // [num_seqs + 1]: first pooled key of every document
+    float* scores;               // [T, ld] fp32: row t holds its visible blocks' scores
+    int ld;
+    int budget;
+    int32_t* sel;                // [T, budget]
+    int* status;
+    void* ws;
+    size_t ws_bytes;
+};
+size_t qsa_workspace_bytes(int num_seqs);
+cudaError_t launch_qsa_scores(const QsaArgs& a, cudaStream_t st);
+cudaError_t launch_qsa_select(const QsaArgs& a, cudaStream_t st);
+
 // Size of the fixed device scratch array behind gdn_backward_noalloc.
 constexpr size_t kBackwardFixedScratchBytes = size_t(32) << 20;
 // Device address of that array on the current device (looked up on first use per device).

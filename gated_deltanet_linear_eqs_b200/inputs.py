@@ -15,6 +15,10 @@ Recipe (per call, ``numpy.random.default_rng(seed)``, drawn in this order):
 Gated form (``make_gate_inputs``, its own generator): the logits a, b ~ N(0, 1) per
 (token, head), A_log ~ U(-1, 1) and b_alpha ~ N(0, 0.5^2) per head, all float32.
 Gated output (``make_norm_inputs``): y, z ~ N(0, 1) rounded like q, w ~ N(0, 0.1^2) float32.
+QSA indexer (``make_qsa_inputs``): q ~ N(0, 1) [T, 4, 128] and k ~ N(0, 1) [T, 128] rounded to
+bf16, gain g ~ 1 + N(0, 0.1^2) [128] float32.
+Short convolution (``make_conv_inputs``): x ~ N(0, 1) [T, C] rounded like q, taps
+w ~ N(0, 1/W) [C, W] float32, conv states ~ N(0, 1) [N, W-1, C] rounded like x.
 """
 from __future__ import annotations
 
@@ -121,3 +125,28 @@ def make_norm_inputs(rows, dv, dtype="bf16", seed=0, with_do=False):
     if with_do:
         out["d_o"] = _round(rng.standard_normal((rows, dv), dtype=np.float32), dtype)
     return out
+
+
+def make_conv_inputs(lengths, C, W, dtype="bf16", seed=0, with_state=True):
+    """Inputs of the short causal convolution over packed documents of the given lengths:
+    x [T, C], w [C, W] fp32, conv_state [N, W-1, C] (or None) and cu_seqlens [N+1] int32."""
+    rng = np.random.default_rng(seed)
+    T = int(sum(lengths))
+    out = dict(x=_round(rng.standard_normal((T, C), dtype=np.float32), dtype),
+               w=torch.from_numpy((rng.standard_normal((C, W)) / np.sqrt(W)).astype(np.float32)),
+               conv_state=None, cu_seqlens=cu_seqlens_from(lengths))
+    if with_state:
+        out["conv_state"] = _round(
+            rng.standard_normal((len(lengths), W - 1, C), dtype=np.float32), dtype)
+    return out
+
+
+def make_qsa_inputs(lengths, seed=0, hq=4, d=128):
+    """Inputs of the QSA block indexer over packed documents: q [T, hq, d], k [T, d] bf16,
+    g [d] fp32 and cu_seqlens [N+1] int32."""
+    rng = np.random.default_rng(seed)
+    T = int(sum(lengths))
+    return dict(q=_round(rng.standard_normal((T, hq, d), dtype=np.float32), "bf16"),
+                k=_round(rng.standard_normal((T, d), dtype=np.float32), "bf16"),
+                g=torch.from_numpy((1.0 + 0.1 * rng.standard_normal(d)).astype(np.float32)),
+                cu_seqlens=cu_seqlens_from(lengths))

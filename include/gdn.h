@@ -64,7 +64,8 @@ typedef enum {
     GDN_OP_PREFILL_VARLEN = 1,
     GDN_OP_DECODE = 2,
     GDN_OP_BACKWARD = 3,
-    GDN_OP_PREFILL_SEGMENTED = 4  /* num_seqs carries the number of segments */
+    GDN_OP_PREFILL_SEGMENTED = 4, /* num_seqs carries the number of segments */
+    GDN_OP_QSA_SCORES = 5         /* gdn_qsa_block_scores: only num_seqs matters */
 } gdn_op;
 
 /* Static description of a status code.  Never NULL. */
@@ -307,6 +308,79 @@ int gdn_prefill_segmented(const void* q, const void* k, const void* v, const flo
                           const float* beta, const float* s0, void* y, float* s_final, int B,
                           int T, int H, int dk, int dv, int dtype, float scale, int l2norm_qk,
                           int num_segments, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Short causal convolution ahead of the recurrence (same page, "Methodology", "1. GDN Hybrid
+ * Token Mixing": "short causal convolutions").  The page fixes neither the width nor the form;
+ * this library's reading is a depthwise causal convolution of each [T, C] input (q, k or v with
+ * C = H * d, or a fused [T, 2 H dk + H dv] tensor), W taps per channel and no bias:
+ *
+ *     y[t, c] = act( sum_{i=0}^{W-1} w[c, i] * x[t - (W - 1) + i, c] ),
+ *
+ * tap W - 1 weighing the current token; act = identity (activation 0) or SiLU, x sigmoid(x)
+ * (activation 1).  Its outputs are the q, k, v the recurrence calls take; the L2 norm of q and
+ * k stays fused inside those calls.
+ *
+ * gdn_short_conv_varlen -- packed documents.
+ *   x, y [T, C] in dtype (bf16 or fp32), C a multiple of 8; w [C, W] fp32, 1 <= W <= 8.
+ *   cu_seqlens [num_seqs + 1] int32 on the device (monotone, cu[0] = 0, cu[num_seqs] = T;
+ *   not checked on the host).  T >= 0, num_seqs >= 1.
+ *   conv_state_in [num_seqs, W - 1, C] in dtype (NULL: zero): row j holds the input at
+ *   position start - (W - 1) + j of each document, i.e. its W - 1 inputs before its start.
+ *   conv_state_out [num_seqs, W - 1, C] (NULL: not written): the last W - 1 inputs of each
+ *   document (rows of the initial state where a document is shorter; empty documents keep
+ *   theirs).  It must not overlap conv_state_in (equal pointers give GDN_ERR_INVALID_ARG).
+ *   Every pointer 16-byte aligned.  One launch; HBM-bound (x read once, y written once).
+ * gdn_short_conv_step -- one token per sequence (decode): x, y [N, C]; conv_state
+ *   [N, W - 1, C] in dtype, read and then updated in place (shifted by the new token).
+ * Errors: GDN_ERR_INVALID_ARG for a null or misaligned pointer, C % 8 != 0, W outside 1..8,
+ * an unknown activation or dtype; nothing is launched then.
+ */
+int gdn_short_conv_varlen(const void* x, const float* w, const int32_t* cu_seqlens,
+                          int num_seqs, const void* conv_state_in, void* conv_state_out, void* y,
+                          int T, int C, int width, int dtype, int activation, void* stream);
+int gdn_short_conv_step(const void* x, const float* w, void* conv_state, void* y, int N, int C,
+                        int width, int dtype, int activation, void* stream);
+
+/*
+ * QSA block indexer (same page, "Methodology", "2. Qwen Sparse Attention (QSA)", eq. (13); the
+ * bud-325 wiki entry, "Key claims": an MQA indexer with 4 query heads and 1 shared key head of
+ * dimension 128, a budget of 512 blocks).  Per document (packed by cu_seqlens), keys are cut
+ * into blocks of 4 tokens from the document's first token and compressed,
+ *     k^_b = g * m / sqrt(mean(m^2) + 1e-6),   m = the mean of the block's 4 key rows;
+ * a trailing partial block is never scored.  Query token t at position i of its document scores
+ * the blocks complete at or before it (b < floor((i + 1) / 4)) by
+ *     I[t, b] = sum_{h<4} ReLU(q[t, h] . k^_b)
+ * and selects the budget highest (ties to the lower block index).
+ *
+ * gdn_qsa_block_scores -- pooled keys and scores.
+ *   q [T, 4, 128] bf16, k [T, 128] bf16, g [128] fp32; cu_seqlens [num_seqs + 1] int32 on the
+ *   device (monotone, cu[0] = 0, cu[num_seqs] = T), every document at most max_doc_len tokens
+ *   (a longer one is recorded as GDN_ERR_INVALID_ARG in the device status word and its scores
+ *   are not written).
+ *   k_hat [T / 4, 128] bf16 (out): the pooled keys of every document, packed (document n's at
+ *   rows block_base[n] .. block_base[n + 1] - 1); block_base [num_seqs + 1] int32 (out).
+ *   scores [T, ld] fp32 (out), ld >= floor(max_doc_len / 4) and a multiple of 4: row t holds
+ *   I[t, b] for its visible blocks b (document-local indices); the rest of the row is not
+ *   written.  ws/ws_bytes: gdn_workspace_bytes(GDN_OP_QSA_SCORES, 1, T, 1, 128, 128, num_seqs).
+ *   Launches: a scan of the documents, the pooling, and one tcgen05 product per 32-token query
+ *   tile against 128-block key tiles (TMA-fed), ReLU and the head sum in its epilogue.
+ * gdn_qsa_select_blocks -- the selection from those scores: sel [T, budget] int32 (out), the
+ *   min(budget, visible) selected document-local block indices in increasing order, then -1.
+ *   1 <= budget.  One CTA per query token (radix selection over the scores' bit patterns).
+ * gdn_qsa_indexer -- both calls, in stream order.
+ * Errors: GDN_ERR_INVALID_ARG for a null or misaligned pointer or a bad size; nothing is
+ * launched then.
+ */
+int gdn_qsa_block_scores(const void* q, const void* k, const float* g, const int32_t* cu_seqlens,
+                         int num_seqs, int T, int max_doc_len, void* k_hat, int32_t* block_base,
+                         float* scores, int ld, void* ws, size_t ws_bytes, void* stream);
+int gdn_qsa_select_blocks(const float* scores, int ld, const int32_t* cu_seqlens, int num_seqs,
+                          int T, int budget, int32_t* sel, void* stream);
+int gdn_qsa_indexer(const void* q, const void* k, const float* g, const int32_t* cu_seqlens,
+                    int num_seqs, int T, int max_doc_len, int budget, void* k_hat,
+                    int32_t* block_base, float* scores, int ld, int32_t* sel, void* ws,
+                    size_t ws_bytes, void* stream);
 
 /*
  * gdn_selftest_wait_timeout -- exercises the failure path of the library's bounded waits.

@@ -251,6 +251,58 @@ def test_segmented_workspace_and_validation(lib):
     assert f(*args, 4, A, 16, None) == _abi.GDN_ERR_WORKSPACE
 
 
+def test_short_conv_rejects_bad_arguments(lib):
+    var = lambda **kw: lib.gdn_short_conv_varlen(
+        kw.get("x", A), kw.get("w", A), kw.get("cu", A), kw.get("n", 2), kw.get("si", 0),
+        kw.get("so", A), kw.get("y", A), kw.get("T", 100), kw.get("C", 2048), kw.get("W", 4),
+        kw.get("dt", 0), kw.get("act", 0), None)
+    assert var(x=0) == _abi.GDN_ERR_INVALID_ARG
+    assert var(w=A + 4) == _abi.GDN_ERR_INVALID_ARG
+    assert var(cu=0) == _abi.GDN_ERR_INVALID_ARG
+    assert var(n=0) == _abi.GDN_ERR_INVALID_ARG
+    assert var(T=-1) == _abi.GDN_ERR_INVALID_ARG
+    assert var(C=2044) == _abi.GDN_ERR_INVALID_ARG      # not a multiple of 8
+    assert var(W=0) == _abi.GDN_ERR_INVALID_ARG
+    assert var(W=9) == _abi.GDN_ERR_INVALID_ARG
+    assert var(dt=5) == _abi.GDN_ERR_INVALID_ARG
+    assert var(act=2) == _abi.GDN_ERR_INVALID_ARG
+    assert var(si=A, so=A) == _abi.GDN_ERR_INVALID_ARG  # the state may not be updated in place
+    assert var(so=A + 8) == _abi.GDN_ERR_INVALID_ARG
+    step = lambda **kw: lib.gdn_short_conv_step(
+        kw.get("x", A), kw.get("w", A), kw.get("s", A), kw.get("y", A), kw.get("N", 4),
+        kw.get("C", 64), kw.get("W", 4), 0, kw.get("act", 1), None)
+    assert step(s=0) == _abi.GDN_ERR_INVALID_ARG       # W > 1 needs a state
+    assert step(N=0) == _abi.GDN_ERR_INVALID_ARG
+    assert step(C=12) == _abi.GDN_ERR_INVALID_ARG
+    assert step(y=A + 2) == _abi.GDN_ERR_INVALID_ARG
+
+
+def test_qsa_rejects_bad_arguments(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.gdn_workspace_bytes(_abi.GDN_OP_QSA_SCORES, 1, 100, 1, 128, 128, 3,
+                                   ctypes.byref(n)) == 0
+    assert n.value >= 16 and n.value % 256 == 0
+    sc = lambda **kw: lib.gdn_qsa_block_scores(
+        kw.get("q", A), kw.get("k", A), kw.get("g", A), kw.get("cu", A), kw.get("n", 2),
+        kw.get("T", 100), kw.get("ml", 60), kw.get("kh", A), kw.get("bb", A), kw.get("s", A),
+        kw.get("ld", 16), kw.get("ws", A), kw.get("wsb", 256), None)
+    assert sc(q=0) == _abi.GDN_ERR_INVALID_ARG
+    assert sc(g=A + 4) == _abi.GDN_ERR_INVALID_ARG
+    assert sc(n=0) == _abi.GDN_ERR_INVALID_ARG
+    assert sc(ml=101) == _abi.GDN_ERR_INVALID_ARG     # longer than the stream
+    assert sc(ld=12) == _abi.GDN_ERR_INVALID_ARG      # below floor(60 / 4)
+    assert sc(ld=18) == _abi.GDN_ERR_INVALID_ARG      # not a multiple of 4
+    assert sc(kh=0) == _abi.GDN_ERR_INVALID_ARG
+    assert sc(ws=0) == _abi.GDN_ERR_WORKSPACE
+    assert sc(wsb=8) == _abi.GDN_ERR_WORKSPACE
+    sl = lambda **kw: lib.gdn_qsa_select_blocks(
+        kw.get("s", A), kw.get("ld", 16), kw.get("cu", A), kw.get("n", 2), kw.get("T", 100),
+        kw.get("b", 512), kw.get("sel", A), None)
+    assert sl(b=0) == _abi.GDN_ERR_INVALID_ARG
+    assert sl(sel=0) == _abi.GDN_ERR_INVALID_ARG
+    assert sl(ld=6) == _abi.GDN_ERR_INVALID_ARG
+
+
 def test_device_status_rejects_null(lib):
     assert lib.gdn_read_device_status(0, None) == _abi.GDN_ERR_INVALID_ARG
 
