@@ -97,7 +97,7 @@ def blocked_unit_lower_inverse(A, bs=16):
 
 
 def forward_chunked_coupled(q, k, v, alpha, beta, s0=None, C=64, scale=1.0, l2norm=True,
-                            eps=EPS, unroll=False):
+                            eps=EPS, unroll=False, lag2=False):
     """The chunked forward in the coupled form the CUDA prefill's sequential kernel runs, same
     contract as ``forward_chunked``.  With S^c the state at the start of chunk c, gamma_c the
     chunk's total decay, D_c = diag(Gam_{n,.}) (so that S^{c+1} = gamma_c S^c + K_c^T D_c U_c) and
@@ -112,7 +112,13 @@ def forward_chunked_coupled(q, k, v, alpha, beta, s0=None, C=64, scale=1.0, l2no
         A1 = -gamma_c gamma_{c-1} W_{c+1} - gamma_{c-1} X_{c+1} D_c W_c,
         A2 = X_{c+1} D_c X_c - gamma_c W_{c+1} K_{c-1}^T,
 
-    which depends on chunk c only through chunk-local quantities."""
+    which depends on chunk c only through chunk-local quantities.  With ``lag2`` the state is
+    taken two chunks back instead (substituting S^{c-1} = gamma_{c-2} S^{c-2} + K_{c-2}^T D U_{c-2}),
+
+        U_c = Ut_c + gamma_{c-1} gamma_{c-2} (-W_c S^{c-2}) + gamma_{c-1} X2_c D_{c-2} U_{c-2}
+              + X_c D_{c-1} U_{c-1},   X2_c = -W_c K_{c-2}^T      (c >= 2),
+
+    so that the product with the state may lag the pseudo-value recursion by two chunks."""
     q, k, v, alpha, beta = (np.asarray(x, dtype=np.float64) for x in (q, k, v, alpha, beta))
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -146,6 +152,11 @@ def forward_chunked_coupled(q, k, v, alpha, beta, s0=None, C=64, scale=1.0, l2no
                 d = ch[c]
                 if c == 0:
                     U.append(d["Ut"] - d["W"] @ S[0])
+                elif lag2 and c >= 2:
+                    m, mm = ch[c - 1], ch[c - 2]
+                    X2 = -d["W"] @ mm["K"].T
+                    U.append(d["Ut"] + m["g"] * mm["g"] * (-d["W"] @ S[c - 2])
+                             + m["g"] * (X2 @ (mm["D"] * U[c - 2])) + d["X"] @ (m["D"] * U[c - 1]))
                 elif unroll and c >= 2 and c % 2 == 0:
                     # U_c from (S^{c-2}, U_{c-2}) through the unrolled pair coefficients
                     m, mm = ch[c - 1], ch[c - 2]

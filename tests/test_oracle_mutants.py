@@ -179,6 +179,7 @@ CHUNKED_CHECKS = [
     lambda m: pins.test_chunked_backward_matches_reverse_recurrence(64, False, m),
     lambda m: pins.test_coupled_chunk_form_matches_token_loop(False, m),
     lambda m: pins.test_coupled_chunk_form_matches_token_loop(True, m),
+    lambda m: pins.test_lag2_coupled_chunk_form_matches_token_loop(m),
     lambda m: pins.test_blocked_inverse_matches_dense_inverse(64, m),
     lambda m: pins.test_blocked_inverse_matches_dense_inverse(50, m),
 ]
@@ -201,6 +202,11 @@ CHUNKED_MUTANTS = [
     ("coupled_state_one_back_undecayed",
      'U.append(d["Ut"] + m["g"] * (-d["W"] @ S[c - 1]) + d["X"] @ (m["D"] * U[c - 1]))',
      'U.append(d["Ut"] + (-d["W"] @ S[c - 1]) + d["X"] @ (m["D"] * U[c - 1]))'),
+    ("lag2_X2_term_dropped",
+     '                             + m["g"] * (X2 @ (mm["D"] * U[c - 2])) + d["X"] @ (m["D"] * U[c - 1]))',
+     '                             + d["X"] @ (m["D"] * U[c - 1]))'),
+    ("lag2_state_decay_single", 'U.append(d["Ut"] + m["g"] * mm["g"] * (-d["W"] @ S[c - 2])',
+     'U.append(d["Ut"] + m["g"] * (-d["W"] @ S[c - 2])'),
     ("unrolled_A2_second_term_dropped",
      'A2 = d["X"] @ (m["D"] * m["X"]) - m["g"] * d["W"] @ mm["K"].T', 'A2 = d["X"] @ (m["D"] * m["X"])'),
     ("inverse_offdiag_sign", "T[blk(bi), blk(bj)] = -T[blk(bi), blk(bi)] @ acc",

@@ -288,6 +288,21 @@ def test_coupled_chunk_form_matches_token_loop(unroll, chunked=None):
         np.testing.assert_allclose(sc, sf, rtol=1e-9, atol=1e-11)
 
 
+def test_lag2_coupled_chunk_form_matches_token_loop(chunked=None):
+    """The coupled form with the state product two chunks behind (the extra coupling X2_c =
+    -W_c K_{c-2}^T) agrees with the token-by-token form, at the benchmark's decays and at decays
+    near 1 where every coupling term counts."""
+    fc = (chunked or oracle_chunked).forward_chunked_coupled
+    rng = np.random.default_rng(19)
+    q, k, v, alpha, beta, S0 = _rand(rng, 2, 330, 2, 16, 12)
+    slow = rng.uniform(0.9, 0.999, alpha.shape)
+    for a in (alpha, slow):
+        y, sf = oracle.forward(q, k, v, a, beta, S0, scale=0.8)
+        yc, sc = fc(q, k, v, a, beta, S0, C=32, scale=0.8, lag2=True)
+        np.testing.assert_allclose(yc, y, rtol=1e-9, atol=1e-11)
+        np.testing.assert_allclose(sc, sf, rtol=1e-9, atol=1e-11)
+
+
 def test_chunked_form_small_alpha_no_overflow(chunked=None):
     """Cumulative log-decay far below -88 within a chunk (exp(-G) alone would overflow
     fp64 only much later, but the relative form must stay finite and exact)."""
