@@ -69,6 +69,29 @@ def _kernel_prefill(q, k, v, alpha, beta, s0, scale, l2norm_qk):
     return api.gdn_prefill(q, k, v, alpha, beta, s0, scale=scale, l2norm_qk=l2norm_qk)
 
 
+def segment_map(q, k, v, alpha, beta, scale=1.0, l2norm_qk=True,
+                prefill: Optional[Callable] = None):
+    """The affine map S -> M S + N of a run of tokens (q, k [B,T,H,d], v [B,T,H,d], alpha,
+    beta [B,T,H], T >= 1), from two kernel runs: v = 0 from S0 = I gives M, S0 = 0 gives N.
+    Returns (M [B,H,d,d], N [B,H,d,d]) fp32."""
+    run = prefill or _kernel_prefill
+    B, T, H, dk = q.shape
+    eye = torch.eye(dk, dtype=torch.float32, device=q.device).expand(B, H, dk, dk).contiguous()
+    _, M = run(q, k, torch.zeros_like(k), alpha, beta, eye, scale, l2norm_qk)
+    _, N = run(q, k, v, alpha, beta, None, scale, l2norm_qk)
+    return M.contiguous(), N.contiguous()
+
+
+def start_states(Ms, Ns, S0):
+    """The state before every segment, given the segments' maps in order: S^(0) = S0,
+    S^(p+1) = M_p S^(p) + N_p.  Returns the list [S^(0), .., S^(P)] (the last one is the state
+    after the last segment)."""
+    out = [S0]
+    for M, N in zip(Ms, Ns):
+        out.append(torch.matmul(M, out[-1]) + N)
+    return out
+
+
 def context_parallel_prefill(q, k, v, alpha, beta, s0=None, scale=1.0, l2norm_qk=True,
                              group=None, prefill: Optional[Callable] = None):
     """Prefill of ONE batch of sequences split along time across the ranks of ``group``, in rank
@@ -98,10 +121,7 @@ def context_parallel_prefill(q, k, v, alpha, beta, s0=None, scale=1.0, l2norm_qk
     rank = dist.get_rank(group)
     # 1. this rank's map S -> M S + N, from its own tokens
     if T > 0:
-        eye = torch.eye(dk, **f32).expand(B, H, dk, dk).contiguous()
-        _, M = run(q, k, torch.zeros_like(k), alpha, beta, eye, scale, l2norm_qk)
-        _, N = run(q, k, v, alpha, beta, None, scale, l2norm_qk)
-        M, N = M.contiguous(), N.contiguous()
+        M, N = segment_map(q, k, v, alpha, beta, scale, l2norm_qk, run)
     else:
         M = torch.eye(dk, **f32).expand(B, H, dk, dk).contiguous()
         N = torch.zeros((B, H, dk, dv), **f32)
@@ -111,9 +131,7 @@ def context_parallel_prefill(q, k, v, alpha, beta, s0=None, scale=1.0, l2norm_qk
     dist.all_gather(Ms, M, group=group)
     dist.all_gather(Ns, N, group=group)
     # 3. start state: the maps of ranks 0 .. rank-1 applied to S0 in order
-    S = S0
-    for p in range(rank):
-        S = torch.matmul(Ms[p], S) + Ns[p]
+    S = start_states(Ms[:rank], Ns[:rank], S0)[-1]
     # 4. this rank's tokens from their start state
     if T == 0:
         return v.new_zeros((B, 0, H, dv)), S

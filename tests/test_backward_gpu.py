@@ -113,4 +113,6 @@ def test_backward_slow_decay():
     rng = np.random.default_rng(18)
     inp["alpha"] = torch.from_numpy(rng.uniform(0.97, 0.9995, (B, T, H)).astype(np.float32))
     out, ref = _run(inp)
+    print("slow decays: " + ", ".join(f"{n} {max_rel(out[n], ref[n]):.2e}" for n in NAMES)
+          + f", dS0 frob {frob_rel(out['ds0'], ref['ds0']):.2e}")
     _check(out, ref)

@@ -3,8 +3,9 @@
 Such callers (a plugin whose device memory belongs to its host framework's pool, a server
 that reserves all memory at start-up) cannot hand the backward pass a workspace from
 cudaMalloc.  This entry point runs the token-loop form of the backward on a fixed scratch
-array built into the library (gdn_backward runs the chunked form).  The GPU test calls it through the C ABI twice in a row, on different inputs,
-and compares each result with gdn_backward's on the same inputs.  The second call checks
+array built into the library (gdn_backward runs the chunked form).  The GPU test calls it
+through the C ABI twice in a row, on different inputs, and compares each result with the fp64
+oracle's reverse recurrence and with gdn_backward's on the same inputs.  The second call checks
 that the contents the first call leaves in the shared array cannot leak into the next result.
 This file is collected last; it passes alone in a fresh process and after the other tests.
 """
@@ -12,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from gated_deltanet_linear_eqs_b200 import _abi, api
 from gated_deltanet_linear_eqs_b200.build import build
 from gated_deltanet_linear_eqs_b200.inputs import make_inputs
@@ -31,9 +33,12 @@ def test_noalloc_matches_backward_on_two_calls(B, T, H, d, dtype):
     assert need <= api.gdn_backward_noalloc_max_workspace()
     rng = np.random.default_rng(7)
     for call in range(2):
-        g = _cuda(make_inputs(B, T, H, d, d, dtype=dtype, seed=100 + call, with_s0=True,
-                              with_dy=True))
-        dsf = torch.from_numpy(rng.standard_normal((B, H, d, d)).astype(np.float32)).cuda()
+        inp = make_inputs(B, T, H, d, d, dtype=dtype, seed=100 + call, with_s0=True, with_dy=True)
+        g = _cuda(inp)
+        dsf_h = torch.from_numpy(rng.standard_normal((B, H, d, d)).astype(np.float32))
+        dsf = dsf_h.cuda()
+        exact = oracle.backward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                                s0=inp["s0"], dy=inp["dy"], ds_final=dsf_h, scale=0.8)
         ref = api.gdn_backward(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["dy"],
                                s0=g["s0"], ds_final=dsf, scale=0.8)
         out = api.gdn_backward_noalloc(g["q"], g["k"], g["v"], g["alpha"], g["beta"], g["dy"],
@@ -41,7 +46,9 @@ def test_noalloc_matches_backward_on_two_calls(B, T, H, d, dtype):
         torch.cuda.synchronize()
         for n in NAMES:
             assert torch.isfinite(out[n]).all(), (call, n)
+            assert max_rel(out[n], exact[n]) <= G_TOL, (call, n)
             assert max_rel(out[n], ref[n]) <= G_TOL, (call, n)
+        assert frob_rel(out["ds0"], exact["ds0"]) <= S_TOL, call
         assert frob_rel(out["ds0"], ref["ds0"]) <= S_TOL, call
 
 
