@@ -342,22 +342,37 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (lane != 0) mbar_arrive(&bars[PB_FULL]);
         // Warm L2 with the tiles of the CTA that will most likely run next on this SM (CTAs are
         // dispatched in index order as slots free up), so that its loads do not wait on DRAM.
+        // The same CTA's alpha and beta go in too (one line per token and head), or its loader
+        // would wait on DRAM for them.
         const int nt = bid + p.ahead;
-        if (lane == 0 && nt < p.ntask) {
+        if (nt < p.ntask) {
             const int g2 = nt / p.H, h2 = nt % p.H;
-            int z2 = -1;
+            int z2 = -1, nv2 = 0;
             if (p.map) {
                 const int2 m = p.map[g2];
-                if (m.y > 0) z2 = m.x;
+                if ((m.y & 0xffff) > 0) { z2 = m.x; nv2 = m.y & 0xffff; }
             } else {
-                z2 = (g2 / p.nchunk_dense) * p.T + (g2 % p.nchunk_dense) * kChunk;
+                const int c2 = g2 % p.nchunk_dense;
+                z2 = (g2 / p.nchunk_dense) * p.T + c2 * kChunk;
+                nv2 = min(kChunk, p.T - c2 * kChunk);
             }
             if (z2 >= 0) {
+                if (lane == 0) {
 #pragma unroll
-                for (int b = 0; b < KB; ++b) {
-                    tma_prefetch_3d(&tm_k, 64 * b, h2, z2);
-                    tma_prefetch_3d(&tm_q, 64 * b, h2, z2);
-                    tma_prefetch_3d(&tm_v, 64 * b, h2, z2);
+                    for (int b = 0; b < KB; ++b) {
+                        tma_prefetch_3d(&tm_k, 64 * b, h2, z2);
+                        tma_prefetch_3d(&tm_q, 64 * b, h2, z2);
+                        tma_prefetch_3d(&tm_v, 64 * b, h2, z2);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int i = lane + 32 * u;
+                    const long long e = ((long long)z2 + i) * p.H + h2;
+                    if (i < nv2 && e < p.ab_elems) {
+                        prefetch_l2(p.alpha + e);
+                        prefetch_l2(p.beta + e);
+                    }
                 }
             }
         }
@@ -750,8 +765,7 @@ struct ChainLayout {
     static constexpr int QWR = 0;                   // slot j: per dk block [Q_{j-1} | -W_j], 16 KB
     static constexpr int PXR = QWR + 2 * KB * 16384; // slot u: [P_u | X_{u+1}], 16 KB
     static constexpr int KR = PXR + 32768;          // slot: K_c, KB x 8 KB
-    static constexpr int USR = KR + 2 * KB * 8192;  // slot: Ut slice 8 KB, then the scalars 1 KB
-    static constexpr int SB = USR + 2 * 9216;       // 2 buffers: S^c in bf16, D rows x 64 cols
+    static constexpr int SB = KR + 2 * KB * 8192;   // 2 buffers: S^c in bf16, D rows x 64 cols
     static constexpr int UU = SB + 2 * D * 128;     // 2 buffers: [U'_hi | U'_lo] then [U_bf16 | 0]
     static constexpr int BAR = UU + 2 * 16384;
     static constexpr int MISC = BAR + 32 * 8;       // tmem base, abort flag, zero word
@@ -765,7 +779,7 @@ struct ChainLayout {
 };
 // ring barriers (full / empty per slot), then per-step arrivals and tensor-core completions
 enum {
-    CB_QWF = 0, CB_QWE = 2, CB_PXF = 4, CB_PXE = 6, CB_KF = 8, CB_KE = 10, CB_UF = 12, CB_UE = 14,
+    CB_QWF = 0, CB_QWE = 2, CB_PXF = 4, CB_PXE = 6, CB_KF = 8, CB_KE = 10,  // 12-15 unused
     CB_AD = 16, CB_BD = 18, CB_YD = 20, CB_M4A = 22, CB_M4B = 24, CB_M5 = 26,
     CB_FIN = 28,  // one per issuer: the commit that covers every product it issued
     CB_COUNT = 30
@@ -792,7 +806,8 @@ struct ChainParams {
 constexpr int kChainThreads = 512;
 
 // Warp roles: 0 loads the [Q; -W] and [P; X] rings, 1 owns the TMEM allocation and loads the
-// Ut / scalar and K rings; 2, 3, 4, 5, 8, 9, 14, 15 hold the state (16 columns each: rows
+// K ring (the Ut slices and scalars go straight from global memory into the registers of the
+// warps that use them, one chunk ahead); 2, 3, 4, 5, 8, 9, 14, 15 hold the state (16 columns each: rows
 // 32 (w % 4) .. +31, columns 0-15 for w < 8, 16-31 otherwise) for the readout (A), warps 4, 5,
 // 8, 9 also write Y; 6, 7, 10, 11 run the pseudo-value epilogue (B) on rows 64-127 (16 columns
 // each); 12 issues M4a, 13 issues M4b and M5.  Warp w reads TMEM lanes 32 (w % 4) .. +31.
@@ -848,7 +863,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     if (tid == 0) {
         for (int b = 0; b < CB_COUNT; ++b) {
             int cnt = 1;
-            if (b == CB_UE || b == CB_UE + 1) cnt = 12;  // 8 readout warps + 4 pseudo-value warps
             if (b == CB_AD || b == CB_AD + 1) cnt = 8;
             if (b == CB_BD || b == CB_BD + 1 || b == CB_YD || b == CB_YD + 1) cnt = 4;
             mbar_init(&bars[b], cnt);
@@ -894,7 +908,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     constexpr uint32_t kRecW = D * 128, kRecU = D * 256;
     auto recof = [&](int c) { return (size_t)(cbase + c) * p.H + h; };
     auto zof = [&](int c) { return (int)(t0 + (long)c * kChunk); };
-    auto usc_of = [&](int s) { return reinterpret_cast<const float*>(sm + L::USR + s * 9216 + 8192); };
     constexpr uint32_t ID_KN = idesc_bf16(128, 64, false, true);
     constexpr uint32_t ID_KN128 = idesc_bf16(128, 128, false, true);
     constexpr uint32_t ID_M5 = idesc_bf16(128, 64, true, true);
@@ -947,18 +960,14 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- loads: Ut / scalars, K
+        // ---------------------------------------------------------------- loads: K; L2 warming
+        // (the Ut slice and the scalars are read from global memory by the warps that use them,
+        // one chunk ahead; here they are only prefetched into L2 two chunks ahead)
         if (lane == 0) {
             prefetch_tmap(&tm_k);
             int nl = 0;
             for (int c = 0; c < nch; ++c) {
-                const size_t rec = recof(c);
                 const int s = c & 1;
-                if (!slot_wait(CB_UE, c, true)) break;
-                uint64_t* uf = &bars[CB_UF + s];
-                mbar_arrive_expect_tx(uf, 8192 + kRecS);
-                bulk_load(sm + L::USR + s * 9216, p.ws_u + rec * kRecU + (size_t)jsl * 8192, 8192, uf);
-                bulk_load(sm + L::USR + s * 9216 + 8192, p.ws_s + rec * (kRecS / 4), kRecS, uf);
                 if (!slot_wait(CB_KE, c, true)) break;
                 uint64_t* kf = &bars[CB_KF + s];
                 mbar_arrive_expect_tx(kf, KB * 8192);
@@ -975,7 +984,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 }
             }
             for (int u = nl - 2 < 0 ? 0 : nl - 2; u < nl; ++u) {
-                mbar_wait(&bars[CB_UF + (u & 1)], (u >> 1) & 1, never, 100000000ull);
                 mbar_wait(&bars[CB_KF + (u & 1)], (u >> 1) & 1, never, 100000000ull);
                 mbar_wait(&bars[CB_KE + (u & 1)], (u >> 1) & 1, abort_flag);
             }
@@ -1072,18 +1080,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     S[4 * q] = v.x; S[4 * q + 1] = v.y; S[4 * q + 2] = v.z; S[4 * q + 3] = v.w;
                 }
             }
-            // gamma of the previous chunk; the output scale of the previous chunk's rows, read
-            // while its slot is held
+            // gamma of the previous chunk; the output scale of the previous chunk's rows.  Chunk
+            // a's values are loaded at the top of step a and first used at step a + 1.
             float gprev = 1.f, ysprev = 0.f;
             for (int a = 0; a <= nch; ++a) {
                 float g_a = 1.f, ys_a = 0.f;
                 if (a < nch) {
-                    ok = wwait(CB_UF + (a & 1), (a >> 1) & 1, a) && ok;
-                    const float* sc = usc_of(a & 1);
-                    g_a = sc[128];
-                    if (ywarp) ys_a = sc[64 + srow];
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars[CB_UE + (a & 1)]);
+                    const float* sc = p.ws_s + recof(a) * (kRecS / 4);
+                    g_a = __ldg(sc + 128);
+                    if (ywarp) ys_a = __ldg(sc + 64 + srow);
                 }
                 if (a >= 1) {
                     ok = wwait(CB_M5 + ((a - 1) & 1), ((a - 1) >> 1) & 1, a) && ok;
@@ -1151,17 +1156,26 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const int col0 = 16 * hf;
             const int i = srow - 64;
             float gprev = 1.f;
-            for (int c = 0; c < nch; ++c) {
-                const int s = c & 1;
-                // this chunk's Ut row and scalars first: their loads overlap the product waits
-                ok = wwait(CB_UF + s, (c >> 1) & 1, c) && ok;
-                const float* sc = usc_of(s);
-                const float us = sc[i], gnext = sc[128];
-                const uint8_t* urow = sm + L::USR + s * 9216 + i * 128;
-                float4 utq[4];
+            // this row's Ut values (16-byte chunk q of row i at position q ^ (i % 8)) and
+            // scalars, loaded from the workspace record one chunk before they are used
+            auto load_u = [&](int c, float4* u4, float& usv, float& gn) {
+                const size_t rec = recof(c);
+                const float* scg = p.ws_s + rec * (kRecS / 4);
+                usv = __ldg(scg + i);
+                gn = __ldg(scg + 128);
+                const uint8_t* urow = p.ws_u + rec * kRecU + (size_t)jsl * 8192 + (size_t)i * 128;
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    utq[q] = *reinterpret_cast<const float4*>(urow + (((4 * hf + q) ^ (i & 7)) << 4));
+                    u4[q] = __ldg(reinterpret_cast<const float4*>(urow + (((4 * hf + q) ^ (i & 7)) << 4)));
+            };
+            float4 utq[4];
+            float us = 0.f, gnext = 1.f;
+            load_u(0, utq, us, gnext);
+            for (int c = 0; c < nch; ++c) {
+                const int s = c & 1;
+                float4 nutq[4] = {};
+                float nus = 0.f, ngn = 1.f;
+                if (c + 1 < nch) load_u(c + 1, nutq, nus, ngn);
                 ok = wwait(CB_M4A + s, (c >> 1) & 1, c) && ok;
                 if (c >= 1) ok = wwait(CB_M4B + ((c - 1) & 1), ((c - 1) >> 1) & 1, c) && ok;
                 tc_fence_after();
@@ -1208,8 +1222,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     }
                 }
                 gprev = gnext;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[CB_UE + s]);
+                us = nus;
+                gnext = ngn;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) utq[q] = nutq[q];
                 signal(CB_BD + s);
             }
         }
