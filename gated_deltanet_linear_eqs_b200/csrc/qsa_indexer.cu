@@ -16,7 +16,8 @@
 //                     TMEM lanes, so a reduce-scatter over lane pairs) and stores the visible scores
 //   qsa_select_kernel one CTA per query token: radix selection of the budget-th largest score over
 //                     the token's visible blocks (4 passes of 8 bits on the scores' bit patterns,
-//                     which order like the non-negative scores), then an ordered compaction
+//                     which order like the non-negative scores; the row staged once in shared
+//                     memory), then an ordered compaction
 #include <mutex>
 
 #include "common.cuh"
@@ -146,7 +147,9 @@ struct ScoreLayout {
     static constexpr uint32_t T_COLS = 256;      // two 128-column accumulators
 };
 enum { QB_A = 0, QB_BF = 1, QB_BE = 3, QB_AF = 5, QB_AE = 7, QB_FIN = 9, QB_COUNT = 10 };
-constexpr int kScoreThreads = 192;  // warp 0 loads, warp 1 TMEM + tensor cores, 2..5 epilogue
+// warp 0 loads, warp 1 TMEM + tensor cores, 2..9 epilogue (two per TMEM lane quadrant, each
+// taking half of a tile's columns)
+constexpr int kScoreThreads = 320;
 
 struct ScoreParams {
     const int32_t* cu;
@@ -182,7 +185,7 @@ qsa_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
     volatile int* never = reinterpret_cast<volatile int*>(sm + L::MISC + 8);
     if (tid == 0) {
-        for (int b = 0; b < QB_COUNT; ++b) mbar_init(&bars[b], (b == QB_AE || b == QB_AE + 1) ? 4 : 1);
+        for (int b = 0; b < QB_COUNT; ++b) mbar_init(&bars[b], (b == QB_AE || b == QB_AE + 1) ? 8 : 1);
         *abort_flag = 0;
         *never = 0;
         fence_mbar_init();
@@ -255,8 +258,9 @@ qsa_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- epilogue
-        // row = 32 q + lane of the accumulator: token 8 q + lane / 4, head lane % 4
-        const int q = warp & 3, h = lane & 3;
+        // row = 32 q + lane of the accumulator: token 8 q + lane / 4, head lane % 4; this warp
+        // takes the 32-column chunks 2 hc and 2 hc + 1 of every tile
+        const int q = warp & 3, h = lane & 3, hc = (warp - 2) >> 2;
         const int tl = 8 * q + (lane >> 2);
         const bool row_ok = tl < ntok;
         const int i = i0 + tl;
@@ -271,7 +275,7 @@ qsa_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * hc; c < 2 * hc + 2; ++c) {
                 float v[32];
                 tmem_ld32(tmem + s * kNB + 32 * c + lane_base, v);
 #pragma unroll
@@ -313,9 +317,11 @@ qsa_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 }
 
 // ============================================================================ selection
-constexpr int kSelThreads = 128;
+constexpr int kSelThreads = 256;
+constexpr int kSelSmemKeys = 12288;  // rows of up to this many blocks are staged in shared memory
 
-__device__ __forceinline__ int block_excl_sum(int x, int* sh, int& total) {
+// exclusive prefix sum of x over the block; *total receives the sum
+__device__ __forceinline__ int block_excl_sum(int x, int* sh, int* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int v = x;
 #pragma unroll
@@ -332,16 +338,22 @@ __device__ __forceinline__ int block_excl_sum(int x, int* sh, int& total) {
         tot += sh[w];
     }
     __syncthreads();
-    total = tot;
+    *total = tot;
     return pre + v - x;
 }
 
 // scores' bit patterns order like the scores (all >= 0); the sign bit of a -0 is dropped
 __device__ __forceinline__ uint32_t score_key(float s) { return __float_as_uint(s) & 0x7fffffffu; }
 
+// One CTA per query token.  The row's keys are read once into shared memory (when they fit);
+// each of the 4 radix passes builds a 256-bin histogram of one byte of the keys that match the
+// bytes chosen so far, and a suffix sum over the bins (one bin per thread) picks the byte of
+// the budget-th largest key.
+template <bool kStage>
 __global__ void __launch_bounds__(kSelThreads) qsa_select_kernel(const float* __restrict__ scores,
                                                                  int ld, const int32_t* __restrict__ cu,
                                                                  int n, int budget, int32_t* __restrict__ sel) {
+    extern __shared__ uint32_t skeys[];
     __shared__ int hist[256];
     __shared__ int sh[kSelThreads / 32];
     __shared__ uint32_t s_prefix;
@@ -357,23 +369,28 @@ __global__ void __launch_bounds__(kSelThreads) qsa_select_kernel(const float* __
         return;
     }
     const float* row = scores + t * ld;
+    auto key_at = [&](int b) -> uint32_t {
+        return kStage ? skeys[b] : score_key(__ldg(row + b));
+    };
+    if (kStage) {
+        for (int b = tid; b < nvis; b += kSelThreads) skeys[b] = score_key(__ldg(row + b));
+    }
     uint32_t prefix = 0, mask = 0;
     int need = budget;
 #pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int j = tid; j < 256; j += kSelThreads) hist[j] = 0;
+        hist[tid] = 0;  // kSelThreads == 256 bins
         __syncthreads();
         for (int b = tid; b < nvis; b += kSelThreads) {
-            const uint32_t key = score_key(__ldg(row + b));
+            const uint32_t key = key_at(b);
             if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
         }
         __syncthreads();
-        if (tid == 0) {
-            int above = 0, d = 255;
-            for (; d > 0; --d) {
-                if (above + hist[d] >= need) break;
-                above += hist[d];
-            }
+        // suffix sum: above = number of matching keys whose byte is larger than bin 255 - tid
+        const int d = 255 - tid, hd = hist[d];
+        int total;
+        const int above = block_excl_sum(hd, sh, &total);
+        if (above < need && above + hd >= need) {
             s_prefix = prefix | ((uint32_t)d << shift);
             s_need = need - above;
         }
@@ -388,16 +405,16 @@ __global__ void __launch_bounds__(kSelThreads) qsa_select_kernel(const float* __
     const int b0 = min(nvis, tid * per), b1 = min(nvis, b0 + per);
     int gt = 0, eq = 0;
     for (int b = b0; b < b1; ++b) {
-        const uint32_t key = score_key(__ldg(row + b));
+        const uint32_t key = key_at(b);
         gt += key > prefix;
         eq += key == prefix;
     }
     int tot_gt, tot_eq;
-    const int gt_before = block_excl_sum(gt, sh, tot_gt);
-    const int eq_before = block_excl_sum(eq, sh, tot_eq);
+    const int gt_before = block_excl_sum(gt, sh, &tot_gt);
+    const int eq_before = block_excl_sum(eq, sh, &tot_eq);
     int pos = gt_before + min(eq_before, need), eq_rank = eq_before;
     for (int b = b0; b < b1; ++b) {
-        const uint32_t key = score_key(__ldg(row + b));
+        const uint32_t key = key_at(b);
         bool take = key > prefix;
         if (key == prefix) take = eq_rank++ < need;
         if (take && pos < budget) out[pos++] = b;
@@ -470,8 +487,19 @@ cudaError_t launch_qsa_scores(const QsaArgs& a, cudaStream_t st) {
 
 cudaError_t launch_qsa_select(const QsaArgs& a, cudaStream_t st) {
     if (a.T == 0) return cudaSuccess;
-    qsa_select_kernel<<<(unsigned)a.T, kSelThreads, 0, st>>>(a.scores, a.ld, a.cu_seqlens, a.num_seqs,
-                                                            a.budget, a.sel);
+    if (a.ld <= kSelSmemKeys) {
+        const int smem = a.ld * 4;
+        cudaError_t e;
+        if (smem > 48 * 1024 &&
+            (e = cudaFuncSetAttribute(qsa_select_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+            return e;
+        qsa_select_kernel<true><<<(unsigned)a.T, kSelThreads, smem, st>>>(
+            a.scores, a.ld, a.cu_seqlens, a.num_seqs, a.budget, a.sel);
+    } else {
+        qsa_select_kernel<false><<<(unsigned)a.T, kSelThreads, 0, st>>>(
+            a.scores, a.ld, a.cu_seqlens, a.num_seqs, a.budget, a.sel);
+    }
     return cudaGetLastError();
 }
 
