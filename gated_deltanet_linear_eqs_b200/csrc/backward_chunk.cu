@@ -40,6 +40,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace gdn {
 namespace {
@@ -154,6 +155,8 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
     return r;
 }
+// x rounded to tf32 (nearest, ties away) as an fp32 value with the low 13 bits clear
+__device__ __forceinline__ float rtf(float x) { return __uint_as_float(to_tf32(x) & 0xffffe000u); }
 __device__ __forceinline__ void mma_tf32(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -361,7 +364,7 @@ __global__ void __launch_bounds__(256, 2) bwdc_prep(const Tin* __restrict__ q, c
         }
         __syncthreads();
     }
-    for (int e = tid; e < kCB * kCB; e += 256) ws[w.Tm + r * kCB * kCB + e] = Tm[(e / kCB) * kL64 + e % kCB];
+    for (int e = tid; e < kCB * kCB; e += 256) ws[w.Tm + r * kCB * kCB + e] = rtf(Tm[(e / kCB) * kL64 + e % kCB]);
     // W = T diag(beta gam) K^, Ut = T diag(beta) V: 64 x D tensor-core tiles (tf32, fp32
     // accumulation), the diagonal scales folded into the B operand; warp w owns rows
     // 16 (w & 3) .. +15 and columns (D / 2)(w >> 2) .. +D/2-1
@@ -475,7 +478,7 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
         float* Sg = ws + w.S + r * D * D;
         for (int e = tid; e < D * kNVB; e += 256) {
             const int m = e / kNVB, n = e % kNVB;
-            Sg[(size_t)m * D + col0 + n] = Ss[m * LDS + n];
+            Sg[(size_t)m * D + col0 + n] = rtf(Ss[m * LDS + n]);
         }
 #pragma unroll
         for (int u = 0; u < R::PW; ++u) {
@@ -514,7 +517,7 @@ __global__ void __launch_bounds__(256) bwdc_fwd(const Tin* __restrict__ k, const
                     const float2 u = make_float2(ut[2 * t + hh].x - acc[t][2 * hh],
                                                  ut[2 * t + hh].y - acc[t][2 * hh + 1]);
                     *reinterpret_cast<float2*>(Us + i * LDS + n) = u;
-                    *reinterpret_cast<float2*>(Ug + (size_t)i * D + n) = u;
+                    *reinterpret_cast<float2*>(Ug + (size_t)i * D + n) = make_float2(rtf(u.x), rtf(u.y));
                 }
         }
         __syncthreads();
@@ -581,7 +584,7 @@ __global__ void __launch_bounds__(256, 2) bwdc_rev(const Tin* __restrict__ q, co
         float* dSg = ws + w.dSp + r * D * D;
         for (int e = tid; e < D * kNVB; e += 256) {
             const int m = e / kNVB, n = e % kNVB;
-            dSg[(size_t)m * D + col0 + n] = Ss[m * LDS + n];
+            dSg[(size_t)m * D + col0 + n] = rtf(Ss[m * LDS + n]);
         }
         const float* SCg = ws + w.SC + r * 256;
         if (tid < kCB) {
@@ -626,7 +629,7 @@ __global__ void __launch_bounds__(256, 2) bwdc_rev(const Tin* __restrict__ q, co
                     const float2 du = make_float2(fmaf(dec[i], a1[t][2 * hh], a2[t][2 * hh]),
                                                   fmaf(dec[i], a1[t][2 * hh + 1], a2[t][2 * hh + 1]));
                     *reinterpret_cast<float2*>(dUs + i * LDS + n) = du;
-                    *reinterpret_cast<float2*>(dUg + (size_t)i * D + n) = du;
+                    *reinterpret_cast<float2*>(dUg + (size_t)i * D + n) = make_float2(rtf(du.x), rtf(du.y));
                 }
         }
         __syncthreads();
@@ -667,34 +670,120 @@ __global__ void __launch_bounds__(256, 2) bwdc_rev(const Tin* __restrict__ q, co
 }
 
 // ============================================================================ bwdc_local
-// Every product runs as warp-level tf32 MMA tiles (m16n8k8, fp32 accumulation).  Warp w owns rows
-// 16 (w % 4) .. +15 and, in 64 x D results, columns (w / 4) D/4 .. +D/4 - 1 (in 64 x 64 results
-// columns 16 (w / 4) .. +15); lane (gid, tig) holds rows gid, gid + 8 and columns 2 tig, 2 tig + 1
-// of each 16 x 8 tile.  dq^ and dk^ stay in registers in that layout across the products.
-template <int D>
-struct LocalB {
-    static constexpr int LD = D + 4;
-    static constexpr int NROW = 10;  // row accumulators
-    static constexpr int BYTES = (5 * kCB * LD + 3 * kCB * kL64 + (5 + NROW + 1) * kCB + 32) * 4;
-};
+// Every product runs on tcgen05 tensor cores as M = 64 tiles with tf32 operands and fp32
+// accumulators in TMEM; one thread issues the products and the tensor copies, all 16 warps stage
+// the token tiles and run the epilogues.  Operands sit in shared memory as 128-byte-swizzled
+// panels (below), K-major on both sides; a product that contracts over the token index takes a
+// transposed copy, written when the operand is staged or produced.  The fp32 records of the
+// workspace (dU, U, S, dS', T; rounded to tf32 by the kernels that write them) arrive by TMA
+// straight into panels.  Each warp owns the same part of every 64-row result as the fragment
+// layout of a warp-level m16n8 MMA: rows 16 (w % 4) .. +15 and, in 64 x D results, columns
+// (w / 4) D/4 .. +D/4 - 1 (in 64 x 64 results columns 16 (w / 4) .. +15); lane (gid, tig) holds
+// rows gid, gid + 8 and columns 2 tig, 2 tig + 1 of each 16 x 8 tile, read out of TMEM with the
+// 16x256b load shape from the warp's own quarter of the lanes.  dq^ and dk^ stay in registers in
+// that layout across the products that feed them.
+//
+// Shared-memory panels: a matrix of R rows (a multiple of 8) and C columns (a multiple of 32) is
+// stored as C / 32 panels of R rows x 128 bytes, 1024-byte aligned; the 16-byte chunk c of row r
+// of a panel sits at chunk position c ^ (r % 8) (the layout a 32 x R fp32 TMA box with the
+// 128-byte swizzle writes).  Values are tf32 (rounded to nearest), so that the MMA's truncation
+// to tf32 is exact.
+__device__ __forceinline__ uint32_t pan(int R, int r, int c) {
+    return (uint32_t)((((c >> 5) * R + r) << 7) + (((((c & 31) >> 2) ^ (r & 7))) << 4) + ((c & 3) << 2));
+}
 
-// acc += A G^T for the warp's tiles, G [D][D] fp32 in global memory, staged in `buf` (row stride
-// LD) 64 rows at a time: the warps whose output columns fall in the staged rows compute.  Every
-// thread of the CTA calls it.
-template <int D, int LD, int CT, typename FA>
-__device__ __forceinline__ void gemm_staged(float (&acc)[CT][4], FA a, const float* G, float* buf, int r0,
-                                            int cD, int tid, int lane) {
-    for (int hh = 0; hh < D / 64; ++hh) {
-        __syncthreads();
-        load_rec<D, LD, 512>(buf, G + (size_t)hh * 64 * D, tid);
-        __syncthreads();
-        if (cD / 64 == hh) {
-            const float* bb = buf;
-            const int off = hh * 64;
-            wmma_acc(acc, D, r0, cD, a, [bb, off](int kk, int n) { return bb[(n - off) * LD + kk]; }, lane);
+// Stage rows 0..63 x C columns (C = 64 or 128) into panels: row-major into `dst` (64 rows) and/or
+// transposed into `dstT` (C rows x 64 columns).  `src(r, c, x)` yields the 8 values of row r,
+// columns c .. c + 7.  Lane l of warp w takes row 32 (w % 2) + l and the 8-column groups
+// w / 2 + 8 u: a warp's transposed stores then fill one 128-byte row (distinct banks), its
+// row-major 16-byte stores spread over the 8 swizzled chunk positions.  All loads are issued
+// before any store.
+template <int C, typename Src>
+__device__ __forceinline__ void stage(uint8_t* dst, uint8_t* dstT, Src src, int tid) {
+    constexpr int PER = C / 64;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int r = 32 * (warp & 1) + lane;
+    float x[PER][8];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) src(r, 8 * ((warp >> 1) + 8 * u), x[u]);
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int c = 8 * ((warp >> 1) + 8 * u);
+        float y[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) y[j] = rtf(x[u][j]);
+        if (dst) {
+            *reinterpret_cast<float4*>(dst + pan(kCB, r, c)) = make_float4(y[0], y[1], y[2], y[3]);
+            *reinterpret_cast<float4*>(dst + pan(kCB, r, c + 4)) = make_float4(y[4], y[5], y[6], y[7]);
+        }
+        if (dstT) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) *reinterpret_cast<float*>(dstT + pan(C, c + j, r)) = y[j];
         }
     }
 }
+// 8 values of row r, columns c .. c + 7, of a 64-row panel tile in shared memory
+__device__ __forceinline__ void pan_ld8(const uint8_t* t, int r, int c, float* x) {
+    const float4 a = *reinterpret_cast<const float4*>(t + pan(kCB, r, c));
+    const float4 b = *reinterpret_cast<const float4*>(t + pan(kCB, r, c + 4));
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+// D[0..63][0..N) (+)= A B^T over K (a multiple of 8): A = 64-row panels at shared address a,
+// B = b_rows-row panels at b (its first N rows are used), both K-major.  One thread issues.
+__device__ __forceinline__ void tc_gemm(uint32_t d, uint32_t a, uint32_t b, int b_rows, int K, uint32_t idesc,
+                                        bool accumulate) {
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t kc = (uint32_t)(k0 & 31) * 4;
+        const uint64_t da = sm100::sdesc(a + (uint32_t)(k0 >> 5) * kCB * 128 + kc, 16, 1024);
+        const uint64_t db = sm100::sdesc(b + (uint32_t)(k0 >> 5) * b_rows * 128 + kc, 16, 1024);
+        sm100::mma_tf32_tc(d, da, db, idesc, (accumulate || k0 > 0) ? 1u : 0u);
+    }
+}
+// TMA copy of a 64 x C fp32 record (rows y0 .. y0 + 63 of a C-wide tensor map) into 64-row panels
+__device__ __forceinline__ void tma_rec(uint8_t* dst, const CUtensorMap* map, int C, long y0, uint64_t* bar) {
+    for (int p = 0; p < C / 32; ++p) sm100::tma_load_2d(dst + p * kCB * 128, map, 32 * p, (int)y0, bar);
+}
+
+__device__ __forceinline__ float2 ld2(const __nv_bfloat16* p) {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+__device__ __forceinline__ float2 ld2(const float* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ void st2(__nv_bfloat16* p, float a, float b) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+}
+__device__ __forceinline__ void st2(float* p, float a, float b) {
+    *reinterpret_cast<float2*>(p) = make_float2(a, b);
+}
+
+// Shared-memory layout (bytes from a 1024-byte aligned base) and TMEM columns of bwdc_local.
+// Five 64 x D tiles (B0..B4) and three 64 x 64 tiles (S0..S2) are reused as the products go:
+//   B0: dU, dW, dS' rows 0..63, F      B1: dY, k^T            B2: S rows 0..63 (then 64..127), k
+//   B3: dU^T, dW^T, dS' rows 64..127, F^T diag(rq)           B4: V, U, q^T
+//   S0: T^T, M2 = T^T dT               S1: T, E^T diag(rk)    S2: dT^T, E diag(rk)
+// (k and q unnormalised: the row scales rk, rq are applied in the epilogues and folded into the
+// other operand of the products that contract over the token index.)
+// TMEM: Z (T^T dU, T^T dW, then dk^'s last products), W (dU S^T, U dS'^T, then F K^), G (dY S^T,
+// then dP), X (dU V^T, then M2), Y (dW k^T, then M2 T^T).
+template <int D>
+struct LocalB {
+    static constexpr int BIG = kCB * D * 4, SMALL = kCB * kCB * 4;
+    static constexpr int B0 = 0, B1 = B0 + BIG, B2 = B1 + BIG, B3 = B2 + BIG, B4 = B3 + BIG;
+    static constexpr int S0 = B4 + BIG, S1 = S0 + SMALL, S2 = S1 + SMALL;
+    static constexpr int NROW = 10;                       // row accumulators of 64
+    static constexpr int SCAL = S2 + SMALL;               // rq, rk, Lg, beta, gam
+    static constexpr int RACC = SCAL + 5 * kCB * 4;
+    static constexpr int BAR = RACC + (NROW * kCB + 32) * 4;
+    static constexpr int NBAR = 16;
+    static constexpr int MISC = BAR + NBAR * 8;           // TMEM base, abort flag, zero word
+    static constexpr int BYTES = MISC + 16 + 1024;        // + alignment slack
+    static constexpr uint32_t TZ = 0, TW = D, TG = 2 * D, TX = 3 * D, TY = 3 * D + 64, TCOLS = 512;
+    static_assert(TY + 64 <= TCOLS, "TMEM columns");
+    static_assert(BAR % 8 == 0, "mbarrier alignment");
+};
+// mbarriers: products (one commit each) and tensor copies
+enum LocalBar { LB_P0 = 0, LB_P1, LB_P2, LB_P3, LB_P4, LB_P5, LB_DRAIN, LB_C0, LB_C1, LB_C2, LB_C3 };
 
 template <int D, typename Tin>
 __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, const Tin* __restrict__ k,
@@ -707,24 +796,19 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
                                                      const float* __restrict__ A_log,
                                                      const float* __restrict__ b_alpha,
                                                      float* __restrict__ dA_log,
-                                                     float* __restrict__ db_alpha) {
-    constexpr int LD = LocalB<D>::LD;
+                                                     float* __restrict__ db_alpha, int* __restrict__ status,
+                                                     const __grid_constant__ CUtensorMap map_d,
+                                                     const __grid_constant__ CUtensorMap map_64) {
+    using L = LocalB<D>;
     constexpr int CT = D / 32;  // 8-column tiles per warp in 64 x D results
-    extern __shared__ float smf[];
-    float* KH = smf;
-    float* QH = KH + kCB * LD;
-    float* B1 = QH + kCB * LD;   // dU, later dY
-    float* B2 = B1 + kCB * LD;   // V, later U
-    float* B3 = B2 + kCB * LD;   // dW
-    float* Tm = B3 + kCB * LD;
-    float* M1 = Tm + kCB * kL64;  // dT, then dA, then E
-    float* M2 = M1 + kCB * kL64;  // T^T dT, then F
-    float* rq = M2 + kCB * kL64;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* rq = reinterpret_cast<float*>(sm + L::SCAL);
     float* rk = rq + kCB;
     float* Lg = rk + kCB;
     float* be = Lg + kCB;
     float* gam = be + kCB;
-    float* racc = gam + kCB;      // NROW row accumulators of 64
+    float* racc = reinterpret_cast<float*>(sm + L::RACC);  // NROW row accumulators of 64
     float* r_dbe = racc;          // v . T^T dU  + sum_j dA_ij At_ij
     float* r_dbg = racc + 64;     // k^ . T^T dW  (d (beta gam))
     float* r_g1 = racc + 128;     // q^ . dY S^T
@@ -735,6 +819,10 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
     float* r_pk = racc + 448;     // k^ . dk^
     float* dLg = racc + 512;
     float* red = racc + 640;      // [0]: gC d gC
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
+    volatile int* never = reinterpret_cast<volatile int*>(sm + L::MISC + 8);
     const size_t r = blockIdx.x;
     const int h = (int)(r % H);
     const int gr = (int)(r / H);
@@ -745,26 +833,95 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
     const int r0 = (warp & 3) * 16;             // tile rows of this warp
     const int cD = (warp >> 2) * (D / 4);       // first column in 64 x D results
     const int c64 = (warp >> 2) * 16;           // first column in 64 x 64 results
+    const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;  // this warp's TMEM lane quarter
     const float* Sg = ws + w.S + r * D * D;
-    const float* dSg = ws + w.dSp + r * D * D;
+    const float* Atg = ws + w.At + r * kCB * kCB;
+    const float* Pg = ws + w.P + r * kCB * kCB;
+    // rows of the workspace's records in the D-wide and 64-wide tensor maps
+    const long y_dU = (long)(w.dU / D) + (long)r * kCB, y_U = (long)(w.U / D) + (long)r * kCB;
+    const long y_S = (long)(w.S / D) + (long)r * D, y_dS = (long)(w.dSp / D) + (long)r * D;
+    const long y_T = (long)(w.Tm / kCB) + (long)r * kCB;
+    const uint32_t sa = sm100::smem_u32(sm);
 
-    const float* SCg = ws + w.SC + r * 256;
-    if (tid < kCB) {
-        rq[tid] = SCg[tid]; rk[tid] = SCg[64 + tid]; Lg[tid] = SCg[128 + tid]; be[tid] = SCg[192 + tid];
-        gam[tid] = expf(SCg[128 + tid]);
+    if (tid == 0) {
+        for (int i = 0; i < L::NBAR; ++i) sm100::mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        *never = 0;
+        sm100::fence_mbar_init();
+        sm100::prefetch_tmap(&map_d);
+        sm100::prefetch_tmap(&map_64);
     }
-    for (int e = tid; e < LocalB<D>::NROW * kCB + 32; e += 512) racc[e] = 0.f;
-    __syncthreads();
-    load_rows<D, LD, 512>(QH, q, b, t0, nv, h, T, H, rq, tid);
-    load_rows<D, LD, 512>(KH, k, b, t0, nv, h, T, H, rk, tid);
-    load_rows<D, LD, 512>(B2, v, b, t0, nv, h, T, H, nullptr, tid);
-    load_rec<D, LD, 512>(B1, ws + w.dU + r * kCB * D, tid);
-    load_rec<kCB, kL64, 512>(Tm, ws + w.Tm + r * kCB * kCB, tid);
-    __syncthreads();
-    const float gC = expf(Lg[kCB - 1]);
-    // row of element e (0..3) of a tile
-    auto rowof = [&](int e) { return r0 + gid + (e >> 1) * 8; };
-    // add a per-lane value for each of the lane's two rows into a row accumulator (quad sum first)
+    if (warp == 0) sm100::tmem_alloc(tmem_slot, L::TCOLS);
+    // L2 prefetches: At and P (read late), the chunk's q and k rows (read in several epilogues)
+    if (warp == 1 && lane < 2) sm100::bulk_prefetch_l2(lane ? Pg : Atg, kCB * kCB * 4);
+    if (tid >= 64 && tid < 192 && ((tid - 64) & 63) < nv)
+        sm100::bulk_prefetch_l2((tid < 128 ? q : k) + tok_off(b, t0 + ((tid - 64) & 63), h, T, H) * D,
+                                (uint32_t)(D * sizeof(Tin)));
+    // dY and V rows into registers (stored once the barriers are set up)
+    constexpr int PER = D / 64;
+    const int rr = 32 * (warp & 1) + lane;  // the row this thread stages (see stage())
+    float xy[PER][8], xv[PER][8];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int m = 8 * ((warp >> 1) + 8 * u);
+        if (rr < nv) {
+            ld8(dy + tok_off(b, t0 + rr, h, T, H) * D + m, xy[u]);
+            ld8(v + tok_off(b, t0 + rr, h, T, H) * D + m, xv[u]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) xy[u][j] = xv[u][j] = 0.f;
+        }
+    }
+    for (int e = tid; e < L::NROW * kCB + 32; e += 512) racc[e] = 0.f;
+    sm100::tc_fence_before();
+    __syncthreads();  // barriers initialised, TMEM allocated
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    uint32_t copies = 0;  // (thread 0) the copy barriers armed so far
+    if (tid == 0) {  // dU, S rows 0..63 and T by TMA; the chunk scalars rq, rk, Lg, beta
+        copies |= 1u << LB_C0;
+        sm100::mbar_arrive_expect_tx(&bars[LB_C0], (uint32_t)(2 * L::BIG + L::SMALL + 4 * kCB * 4));
+        tma_rec(sm + L::B0, &map_d, D, y_dU, &bars[LB_C0]);
+        tma_rec(sm + L::B2, &map_d, D, y_S, &bars[LB_C0]);
+        tma_rec(sm + L::S1, &map_64, kCB, y_T, &bars[LB_C0]);
+        sm100::bulk_load(sm + L::SCAL, ws + w.SC + r * 256, 4 * kCB * 4, &bars[LB_C0]);
+    }
+
+    auto tok = [=](const Tin* p) {  // token rows of a [B, T, H, D] tensor (zero past the end)
+        return [=](int i, int m, float* x) {
+            if (i < nv) {
+                ld8(p + tok_off(b, t0 + i, h, T, H) * D + m, x);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) x[j] = 0.f;
+            }
+        };
+    };
+    // elements (i, n), (i, n + 1) of token row i of a [B, T, H, D] tensor (zero past the end)
+    auto gpair = [&](const Tin* p, int i, int n) {
+        return i < nv ? ld2(p + tok_off(b, t0 + i, h, T, H) * D + n) : make_float2(0.f, 0.f);
+    };
+    auto tpair = [&](int off, int i, int n) {  // elements (i, n), (i, n + 1) of a 64-row panel tile
+        return *reinterpret_cast<const float2*>(sm + off + pan(kCB, i, n));
+    };
+    // all threads: operand stores visible to the tensor core, TMEM reads ordered before the next
+    // products; then thread 0 issues
+    auto sync_issue = [&]() {
+        sm100::fence_proxy_async_smem();
+        sm100::tc_fence_before();
+        __syncthreads();
+        sm100::tc_fence_after();
+    };
+    // all threads: wait for barrier i (products or copies); the result is the same everywhere
+    auto wait_bar = [&](int i) {
+        bool okw = sm100::mbar_wait_warp(&bars[i], 0, abort_flag);
+        okw = __syncthreads_and(okw) != 0;
+        sm100::tc_fence_after();
+        return okw;
+    };
+    auto frag = [&](uint32_t col, auto& acc) {  // this warp's fragment of a 64-row result
+        sm100::tmem_ld_frag<sizeof(acc) / 16>(tmem + lq + col, &acc[0][0]);
+    };
     auto row_add = [&](float* acc, float lo, float hi) {
         lo = quad_sum(lo);
         hi = quad_sum(hi);
@@ -773,173 +930,275 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
             atomicAdd(&acc[r0 + gid + 8], hi);
         }
     };
-    auto aT = [&](const float* M) { return [M](int i, int kk) { return M[kk * kL64 + i]; }; };
-    auto aR = [&](const float* M, int ld) { return [M, ld](int i, int kk) { return M[i * ld + kk]; }; };
-    auto bR = [&](const float* M, int ld) { return [M, ld](int kk, int n) { return M[kk * ld + n]; }; };
-    auto bT = [&](const float* M, int ld) { return [M, ld](int kk, int n) { return M[n * ld + kk]; }; };
+    constexpr uint32_t ID_N = sm100::idesc_tf32(64, D), ID_64 = sm100::idesc_tf32(64, 64);
 
+    // ---- stage 1: dY -> B1, V -> B4; dU^T -> B3 and T^T -> S0 from the copies
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int cc = 8 * ((warp >> 1) + 8 * u);
+        float a[8], bb[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { a[j] = rtf(xy[u][j]); bb[j] = rtf(xv[u][j]); }
+        *reinterpret_cast<float4*>(sm + L::B1 + pan(kCB, rr, cc)) = make_float4(a[0], a[1], a[2], a[3]);
+        *reinterpret_cast<float4*>(sm + L::B1 + pan(kCB, rr, cc + 4)) = make_float4(a[4], a[5], a[6], a[7]);
+        *reinterpret_cast<float4*>(sm + L::B4 + pan(kCB, rr, cc)) = make_float4(bb[0], bb[1], bb[2], bb[3]);
+        *reinterpret_cast<float4*>(sm + L::B4 + pan(kCB, rr, cc + 4)) = make_float4(bb[4], bb[5], bb[6], bb[7]);
+    }
+    bool ok = wait_bar(LB_C0);
+    if (ok) {
+        if (tid < kCB) gam[tid] = expf(Lg[tid]);
+        const uint8_t* du = sm + L::B0;
+        const uint8_t* tt = sm + L::S1;
+        stage<D>(nullptr, sm + L::B3, [du](int i, int m, float* x) { pan_ld8(du, i, m, x); }, tid);
+        stage<kCB>(nullptr, sm + L::S0, [tt](int i, int m, float* x) { pan_ld8(tt, i, m, x); }, tid);
+        sync_issue();
+        if (tid == 0) {
+            tc_gemm(tmem + L::TZ, sa + L::S0, sa + L::B3, D, kCB, ID_N, false);  // Z1 = T^T dU
+            tc_gemm(tmem + L::TW, sa + L::B0, sa + L::B2, kCB, D, ID_64, false);  // dU S^T, columns 0..63
+            tc_gemm(tmem + L::TG, sa + L::B1, sa + L::B2, kCB, D, ID_64, false);  // dY S^T, columns 0..63
+            tc_gemm(tmem + L::TX, sa + L::B0, sa + L::B4, kCB, D, ID_64, false);  // X = dU V^T
+            sm100::mma_commit(&bars[LB_P0]);
+        }
+        ok = wait_bar(LB_P0);
+    }
+    if constexpr (D == 128) {
+        if (ok) {
+            if (tid == 0) {  // S rows 64..127
+                copies |= 1u << LB_C1;
+                sm100::mbar_arrive_expect_tx(&bars[LB_C1], (uint32_t)L::BIG);
+                tma_rec(sm + L::B2, &map_d, D, y_S + 64, &bars[LB_C1]);
+            }
+        }
+    }
     float dqa[CT][4], dka[CT][4];
-    zero_acc(dqa);
-    zero_acc(dka);
-    // 1. Z1 = T^T dU: dV = diag(beta) Z1, dbeta += v . Z1
-    {
+    if (ok) {
+        // Z1 = T^T dU: dV = diag(beta) Z1, dbeta += v . Z1
         float z[CT][4];
-        zero_acc(z);
-        wmma_acc(z, kCB, r0, cD, aT(Tm), bR(B1, LD), lane);
+        frag(L::TZ + cD, z);
         float lo = 0.f, hi = 0.f;
 #pragma unroll
         for (int t = 0; t < CT; ++t)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
-                const float pv = B2[i * LD + n] * z[t][e];
-                if (e < 2) lo += pv; else hi += pv;
-                if (i < nv) dv[tok_off(b, t0 + i, h, T, H) * D + n] = from_f32<Tin>(be[i] * z[t][e]);
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = r0 + gid + 8 * hh, n = cD + 8 * t + 2 * tig;
+                const float2 vv = tpair(L::B4, i, n);
+                const float pv = vv.x * z[t][2 * hh] + vv.y * z[t][2 * hh + 1];
+                if (hh == 0) lo += pv; else hi += pv;
+                if (i < nv) st2(dv + tok_off(b, t0 + i, h, T, H) * D + n, be[i] * z[t][2 * hh], be[i] * z[t][2 * hh + 1]);
             }
         row_add(r_dbe, lo, hi);
     }
-    // 2. dW = -dU S^T (S staged through M1..M2, free until step 4)
-    {
-        static_assert(2 * kCB * kL64 >= kCB * LD, "staging space");
-        float x[CT][4];
-        zero_acc(x);
-        gemm_staged<D, LD>(x, aR(B1, LD), Sg, M1, r0, cD, tid, lane);
-#pragma unroll
-        for (int t = 0; t < CT; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) B3[rowof(e) * LD + cD + 8 * t + 2 * tig + (e & 1)] = -x[t][e];
+    if constexpr (D == 128) {
+        if (ok) ok = wait_bar(LB_C1);
+        if (ok) {
+            sync_issue();
+            if (tid == 0) {
+                tc_gemm(tmem + L::TW + 64, sa + L::B0, sa + L::B2, kCB, D, ID_64, false);
+                tc_gemm(tmem + L::TG + 64, sa + L::B1, sa + L::B2, kCB, D, ID_64, false);
+                sm100::mma_commit(&bars[LB_P1]);
+            }
+            ok = wait_bar(LB_P1);
+        }
+    } else {
+        if (ok) sync_issue();  // every thread is past Z1's epilogue (V in B4 is read no more)
     }
-    __syncthreads();
-    // 3. Z2 = T^T dW: dk^ = diag(beta gam) Z2, d(beta gam) = k^ . Z2
-    {
+    if (ok) {
+        if (tid == 0) {  // U -> B4 (V is read no more)
+            copies |= 1u << LB_C2;
+            sm100::mbar_arrive_expect_tx(&bars[LB_C2], (uint32_t)L::BIG);
+            tma_rec(sm + L::B4, &map_d, D, y_U, &bars[LB_C2]);
+        }
+        // k -> B2 (loaded first: its latency overlaps the epilogues below)
+        {
+            float xk[PER][8];
+            auto lk = tok(k);
+#pragma unroll
+            for (int u = 0; u < PER; ++u) lk(rr, 8 * ((warp >> 1) + 8 * u), xk[u]);
+            // G1 = dY S^T: dq^ = scale gam G1, q^ . G1 for d gam
+            float x[CT][4];
+            frag(L::TG + cD, x);
+            float lo = 0.f, hi = 0.f;
+#pragma unroll
+            for (int t = 0; t < CT; ++t)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int i = r0 + gid + 8 * hh, n = cD + 8 * t + 2 * tig;
+                    const float2 qv = gpair(q, i, n);
+                    dqa[t][2 * hh] = scale * gam[i] * x[t][2 * hh];
+                    dqa[t][2 * hh + 1] = scale * gam[i] * x[t][2 * hh + 1];
+                    const float pv = rq[i] * (qv.x * x[t][2 * hh] + qv.y * x[t][2 * hh + 1]);
+                    if (hh == 0) lo += pv; else hi += pv;
+                }
+            row_add(r_g1, lo, hi);
+            // dW = -dU S^T -> B0 (row-major) and B3 (transposed)
+            frag(L::TW + cD, x);
+#pragma unroll
+            for (int t = 0; t < CT; ++t)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int i = r0 + gid + 8 * hh, n = cD + 8 * t + 2 * tig;
+                    const float w0 = rtf(-x[t][2 * hh]), w1 = rtf(-x[t][2 * hh + 1]);
+                    *reinterpret_cast<float2*>(sm + L::B0 + pan(kCB, i, n)) = make_float2(w0, w1);
+                    *reinterpret_cast<float*>(sm + L::B3 + pan(D, n, i)) = w0;
+                    *reinterpret_cast<float*>(sm + L::B3 + pan(D, n + 1, i)) = w1;
+                }
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int cc = 8 * ((warp >> 1) + 8 * u);
+                float a[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a[j] = rtf(xk[u][j]);
+                *reinterpret_cast<float4*>(sm + L::B2 + pan(kCB, rr, cc)) = make_float4(a[0], a[1], a[2], a[3]);
+                *reinterpret_cast<float4*>(sm + L::B2 + pan(kCB, rr, cc + 4)) = make_float4(a[4], a[5], a[6], a[7]);
+            }
+        }
+        sync_issue();
+        if (tid == 0) {
+            tc_gemm(tmem + L::TZ, sa + L::S0, sa + L::B3, D, kCB, ID_N, false);  // Z2 = T^T dW
+            tc_gemm(tmem + L::TY, sa + L::B0, sa + L::B2, kCB, D, ID_64, false);  // Y' = dW k^T
+            sm100::mma_commit(&bars[LB_P2]);
+        }
+        ok = wait_bar(LB_P2);
+    }
+    if (ok) {
+        if (tid == 0) {  // dS' rows 0..63 -> B0, 64..127 -> B3 (dW, dW^T are read no more)
+            copies |= 1u << LB_C3;
+            sm100::mbar_arrive_expect_tx(&bars[LB_C3], (uint32_t)(D / 64) * L::BIG);
+            tma_rec(sm + L::B0, &map_d, D, y_dS, &bars[LB_C3]);
+            if constexpr (D == 128) tma_rec(sm + L::B3, &map_d, D, y_dS + 64, &bars[LB_C3]);
+        }
+        // Z2 = T^T dW: dk^ = diag(beta gam) Z2, d(beta gam) = k^ . Z2
         float z[CT][4];
-        zero_acc(z);
-        wmma_acc(z, kCB, r0, cD, aT(Tm), bR(B3, LD), lane);
+        frag(L::TZ + cD, z);
         float lo = 0.f, hi = 0.f;
 #pragma unroll
         for (int t = 0; t < CT; ++t)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
-                dka[t][e] = be[i] * gam[i] * z[t][e];
-                const float pv = KH[i * LD + n] * z[t][e];
-                if (e < 2) lo += pv; else hi += pv;
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = r0 + gid + 8 * hh, n = cD + 8 * t + 2 * tig;
+                const float2 kv = tpair(L::B2, i, n);
+                dka[t][2 * hh] = be[i] * gam[i] * z[t][2 * hh];
+                dka[t][2 * hh + 1] = be[i] * gam[i] * z[t][2 * hh + 1];
+                const float pv = rk[i] * (kv.x * z[t][2 * hh] + kv.y * z[t][2 * hh + 1]);
+                if (hh == 0) lo += pv; else hi += pv;
             }
         row_add(r_dbg, lo, hi);
-    }
-    // 4. dT = (dU V^T + dW (gam K^)^T) diag(beta) -> M1
-    {
-        float x[2][4];
-        zero_acc(x);
-        wmma_acc(x, D, r0, c64, aR(B1, LD), bT(B2, LD), lane);
-        const float* gm = gam;
-        const float* kh = KH;
-        wmma_acc(x, D, r0, c64, aR(B3, LD), [kh, gm](int kk, int j) { return kh[j * LD + kk] * gm[j]; }, lane);
+        // dT = (dU V^T + dW (gam K^)^T) diag(beta), K^ = diag(rk) k -> S2 transposed
+        float xx[2][4], yy[2][4];
+        frag(L::TX + c64, xx);
+        frag(L::TY + c64, yy);
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int i = rowof(e), j = c64 + 8 * t + 2 * tig + (e & 1);
-                M1[i * kL64 + j] = be[j] * x[t][e];
+                const int i = r0 + gid + (e >> 1) * 8, j = c64 + 8 * t + 2 * tig + (e & 1);
+                *reinterpret_cast<float*>(sm + L::S2 + pan(kCB, j, i)) =
+                    rtf(be[j] * fmaf(gam[j] * rk[j], yy[t][e], xx[t][e]));
             }
+        ok = wait_bar(LB_C2) && wait_bar(LB_C3);
+        if (ok) {
+            sync_issue();
+            if (tid == 0) {
+                tc_gemm(tmem + L::TX, sa + L::S0, sa + L::S2, kCB, kCB, ID_64, false);  // M2 = T^T dT
+                tc_gemm(tmem + L::TW, sa + L::B4, sa + L::B0, kCB, D, ID_64, false);    // G2 = U dS'^T
+                if constexpr (D == 128) tc_gemm(tmem + L::TW + 64, sa + L::B4, sa + L::B3, kCB, D, ID_64, false);
+                tc_gemm(tmem + L::TG, sa + L::B1, sa + L::B4, kCB, D, ID_64, false);    // dP = dY U^T
+                sm100::mma_commit(&bars[LB_P3]);
+            }
+            ok = wait_bar(LB_P3);
+        }
     }
-    __syncthreads();
-    // B1 <- dY, B2 <- U for the second half
-    load_rows<D, LD, 512>(B1, dy, b, t0, nv, h, T, H, nullptr, tid);
-    load_rec<D, LD, 512>(B2, ws + w.U + r * kCB * D, tid);
-    // 5. dA = -(T^T dT) T^T, strictly lower -> M1
-    {
+    if (ok) {
+        // M2 -> S0 (T^T is read no more); dA' = M2 T^T
         float x[2][4];
-        zero_acc(x);
-        wmma_acc(x, kCB, r0, c64, aT(Tm), bR(M1, kL64), lane);
+        frag(L::TX + c64, x);
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) M2[rowof(e) * kL64 + c64 + 8 * t + 2 * tig + (e & 1)] = x[t][e];
-    }
-    __syncthreads();
-    {
-        float x[2][4];
-        zero_acc(x);
-        wmma_acc(x, kCB, r0, c64, aR(M2, kL64), bT(Tm, kL64), lane);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int i = rowof(e), j = c64 + 8 * t + 2 * tig + (e & 1);
-                M1[i * kL64 + j] = j < i ? -x[t][e] : 0.f;
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = r0 + gid + 8 * hh, j = c64 + 8 * t + 2 * tig;
+                *reinterpret_cast<float2*>(sm + L::S0 + pan(kCB, i, j)) =
+                    make_float2(rtf(x[t][2 * hh]), rtf(x[t][2 * hh + 1]));
             }
-    }
-    // 6. G1 = dY S^T: dq^ = scale gam G1, q^ . G1 for d gam
-    {
-        float x[CT][4];
-        zero_acc(x);
-        gemm_staged<D, LD>(x, aR(B1, LD), Sg, B3, r0, cD, tid, lane);  // S through B3 (free)
+        sync_issue();
+        if (tid == 0) {
+            tc_gemm(tmem + L::TY, sa + L::S0, sa + L::S1, kCB, kCB, ID_64, false);
+            sm100::mma_commit(&bars[LB_P4]);
+        }
+        // gC <S, dS'>: S from L2 (copied in by this CTA a moment ago), dS' from B0 / B3
+        const float gC = expf(Lg[kCB - 1]);
+        {
+            float s = 0.f;
+            constexpr int NE = D * D / 4 / 512;
+            float4 a4[NE];
+#pragma unroll
+            for (int u = 0; u < NE; ++u) a4[u] = __ldg(reinterpret_cast<const float4*>(Sg) + tid + u * 512);
+#pragma unroll
+            for (int u = 0; u < NE; ++u) {
+                const int e = (tid + u * 512) * 4, n = e / D, m = e % D;
+                const float4 dd = *reinterpret_cast<const float4*>(sm + (n < 64 ? L::B0 : L::B3) + pan(kCB, n & 63, m));
+                s = fmaf(a4[u].x, dd.x, fmaf(a4[u].y, dd.y, fmaf(a4[u].z, dd.z, fmaf(a4[u].w, dd.w, s))));
+            }
+            s = warp_sum(s);
+            if (lane == 0) atomicAdd(red, s * gC);
+        }
+        // G2 = U dS'^T: dk^ += (gC / gam) G2, k^ . G2 = d (gC / gam_i)
+        float y[CT][4];
+        frag(L::TW + cD, y);
         float lo = 0.f, hi = 0.f;
 #pragma unroll
         for (int t = 0; t < CT; ++t)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
-                dqa[t][e] = scale * gam[i] * x[t][e];
-                const float pv = QH[i * LD + n] * x[t][e];
-                if (e < 2) lo += pv; else hi += pv;
-            }
-        row_add(r_g1, lo, hi);
-    }
-    // 7. G2 = U dS'^T: dk^ += (gC / gam) G2, k^ . G2 = d (gC / gam_i); gC <S, dS'>
-    {
-        float x[CT][4];
-        zero_acc(x);
-        gemm_staged<D, LD>(x, aR(B2, LD), dSg, B3, r0, cD, tid, lane);  // dS' through B3
-        float lo = 0.f, hi = 0.f;
-#pragma unroll
-        for (int t = 0; t < CT; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
-                dka[t][e] = fmaf(expf(Lg[kCB - 1] - Lg[i]), x[t][e], dka[t][e]);
-                const float pv = KH[i * LD + n] * x[t][e];
-                if (e < 2) lo += pv; else hi += pv;
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = r0 + gid + 8 * hh, n = cD + 8 * t + 2 * tig;
+                const float dec = expf(Lg[kCB - 1] - Lg[i]);
+                const float2 kv = tpair(L::B2, i, n);
+                dka[t][2 * hh] = fmaf(dec, y[t][2 * hh], dka[t][2 * hh]);
+                dka[t][2 * hh + 1] = fmaf(dec, y[t][2 * hh + 1], dka[t][2 * hh + 1]);
+                const float pv = rk[i] * (kv.x * y[t][2 * hh] + kv.y * y[t][2 * hh + 1]);
+                if (hh == 0) lo += pv; else hi += pv;
             }
         row_add(r_dr, lo, hi);
-        float s = 0.f;
-        for (int e = tid; e < D * D / 4; e += 512) {
-            const float4 a4 = __ldg(reinterpret_cast<const float4*>(Sg) + e);
-            const float4 d4 = __ldg(reinterpret_cast<const float4*>(dSg) + e);
-            s = fmaf(a4.x, d4.x, fmaf(a4.y, d4.y, fmaf(a4.z, d4.z, fmaf(a4.w, d4.w, s))));
-        }
-        s = warp_sum(s);
-        if (lane == 0) atomicAdd(red, s * gC);
+        ok = wait_bar(LB_P4);
     }
-    __syncthreads();  // M1 = dA
-    // 8. dP = dY U^T (lower-incl); the scalar terms of dA and dP; E and F in place
-    {
+    if (ok) {
+        // dA = -(T^T dT) T^T, strictly lower
+        float da[2][4];
+        frag(L::TY + c64, da);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = r0 + gid + (e >> 1) * 8, j = c64 + 8 * t + 2 * tig + (e & 1);
+                da[t][e] = j < i ? -da[t][e] : 0.f;
+            }
+        // dP = dY U^T (lower-incl); the scalar terms of dA and dP; E = dA * beta_i Gam and
+        // F = scale dP * Gam, stored as the products below take them against the unnormalised
+        // k^T and q^T: E diag(rk), E^T diag(rk), F diag(rk) and F^T diag(rq)
         float x[2][4];
-        zero_acc(x);
-        wmma_acc(x, D, r0, c64, aR(B1, LD), bT(B2, LD), lane);
-        const float* Atg = ws + w.At + r * kCB * kCB;
-        const float* Pg = ws + w.P + r * kCB * kCB;
+        frag(L::TG + c64, x);
         float mlo = 0.f, mhi = 0.f, plo = 0.f, phi = 0.f;
         float cs[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int i = rowof(e), j = c64 + 8 * t + 2 * tig + (e & 1);
+                const int i = r0 + gid + (e >> 1) * 8, j = c64 + 8 * t + 2 * tig + (e & 1);
                 const float dp = j <= i ? x[t][e] : 0.f;
-                const float da = M1[i * kL64 + j];
                 const float at = Atg[i * kCB + j];
-                const float mij = da * be[i] * at + dp * Pg[i * kCB + j];
-                if (e < 2) { mlo += mij; plo += da * at; } else { mhi += mij; phi += da * at; }
+                const float mij = da[t][e] * be[i] * at + dp * Pg[i * kCB + j];
+                if (e < 2) { mlo += mij; plo += da[t][e] * at; } else { mhi += mij; phi += da[t][e] * at; }
                 cs[t][e & 1] += mij;
                 const float gm = j <= i ? expf(fminf(Lg[i] - Lg[j], 0.f)) : 0.f;
-                M1[i * kL64 + j] = da * be[i] * gm;     // E
-                M2[i * kL64 + j] = scale * dp * gm;     // F
+                const float ev = da[t][e] * be[i] * gm, fv = scale * dp * gm;
+                *reinterpret_cast<float*>(sm + L::S2 + pan(kCB, i, j)) = rtf(ev * rk[j]);  // E diag(rk)
+                *reinterpret_cast<float*>(sm + L::S1 + pan(kCB, j, i)) = rtf(ev * rk[i]);  // E^T diag(rk)
+                *reinterpret_cast<float*>(sm + L::B0 + pan(kCB, i, j)) = rtf(fv * rk[j]);  // F diag(rk)
+                *reinterpret_cast<float*>(sm + L::B3 + pan(kCB, j, i)) = rtf(fv * rq[i]);  // F^T diag(rq)
             }
         row_add(rowM, mlo, mhi);
         row_add(r_dbe, plo, phi);
-        // column sums: over the 8 rows-pairs of the quad column (lanes with equal tig)
+        // column sums: over the 8 row pairs of the quad column (lanes with equal tig)
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -950,86 +1209,165 @@ __global__ void __launch_bounds__(512, 1) bwdc_local(const Tin* __restrict__ q, 
                 v0 += __shfl_xor_sync(0xffffffffu, v0, 16);
                 if (gid == 0) atomicAdd(&colM[c64 + 8 * t + 2 * tig + u], v0);
             }
+        // ---- stage 4: k^T (from k in B2) -> B1, q^T -> B4 (dY and U are read no more)
+        const uint8_t* kk = sm + L::B2;
+        stage<D>(nullptr, sm + L::B1, [kk](int i, int m, float* x8) { pan_ld8(kk, i, m, x8); }, tid);
+        stage<D>(nullptr, sm + L::B4, tok(q), tid);
+        sync_issue();
+        if (tid == 0) {
+            // dk^ += E K^ + E^T K^ + F^T Q^;  dq^ += F K^
+            tc_gemm(tmem + L::TZ, sa + L::S2, sa + L::B1, D, kCB, ID_N, false);
+            tc_gemm(tmem + L::TZ, sa + L::S1, sa + L::B1, D, kCB, ID_N, true);
+            tc_gemm(tmem + L::TZ, sa + L::B3, sa + L::B4, D, kCB, ID_N, true);
+            tc_gemm(tmem + L::TW, sa + L::B0, sa + L::B1, D, kCB, ID_N, false);
+            sm100::mma_commit(&bars[LB_P5]);
+        }
+        ok = wait_bar(LB_P5);
     }
-    __syncthreads();
-    // 9. dk^ += E K^ + E^T K^ + F^T Q^;  dq^ += F K^
-    wmma_acc(dka, kCB, r0, cD, aR(M1, kL64), bR(KH, LD), lane);
-    wmma_acc(dka, kCB, r0, cD, aT(M1), bR(KH, LD), lane);
-    wmma_acc(dka, kCB, r0, cD, aT(M2), bR(QH, LD), lane);
-    wmma_acc(dqa, kCB, r0, cD, aR(M2, kL64), bR(KH, LD), lane);
-    // 11a. row dots for the norm backward
-    {
-        float ql = 0.f, qh2 = 0.f, kl = 0.f, kh2 = 0.f;
+    if (ok) {
+        float x[CT][4], qh[CT][4], kh2[CT][4];
+        frag(L::TZ + cD, x);
 #pragma unroll
         for (int t = 0; t < CT; ++t)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
-                const float pq = QH[i * LD + n] * dqa[t][e], pk = KH[i * LD + n] * dka[t][e];
-                if (e < 2) { ql += pq; kl += pk; } else { qh2 += pq; kh2 += pk; }
-            }
-        row_add(r_pq, ql, qh2);
-        row_add(r_pk, kl, kh2);
-    }
-    __syncthreads();
-    // 10. d Lg_i = gam_i d gam_i + rowM_i - colM_i (+ gC d gC for the last token); reverse cumsum
-    if (tid < kCB) {
-        const int i = tid;
-        const float dec = expf(Lg[kCB - 1] - Lg[i]);
-        const float dlg = r_dbg[i] * be[i] * gam[i] + scale * gam[i] * r_g1[i] - r_dr[i] * dec;
-        dLg[i] = dlg + rowM[i] - colM[i];
-        atomicAdd(red, r_dr[i] * dec);
-    }
-    __syncthreads();
-    if (tid == 0) {
-        float acc = red[0];
-        for (int ii = kCB - 1; ii >= 0; --ii) {
-            acc += dLg[ii];
-            dLg[ii] = acc;  // d ln(alpha_ii)
-        }
-    }
-    __syncthreads();
-    float pA = 0.f, pba = 0.f;  // this token's share of dA_log[h], db_alpha[h] (gated form)
-    if (tid < nv) {
-        const int i = tid;
-        const size_t o = tok_off(b, t0 + i, h, T, H);
-        const float dbe = r_dbe[i] + r_dbg[i] * gam[i];
-        if (A_log) {
-            // ln alpha = -e^A softplus(x), x = a + b_alpha: d a = -e^A sigmoid(x) d ln alpha,
-            // d A = ln alpha d ln alpha, d b_alpha = d a; beta = sigmoid(b): d b = beta (1-beta) d beta
-            const float xa = alpha[o] + b_alpha[h], ea = expf(A_log[h]);
-            const float da = -ea * gate_sigmoid(xa) * dLg[i];
-            dalpha[o] = da;
-            dbeta[o] = dbe * be[i] * (1.f - be[i]);
-            pA = -ea * gate_softplus(xa) * dLg[i];
-            pba = da;
-        } else {
-            dalpha[o] = dLg[i] / alpha[o];
-            dbeta[o] = dbe;
-        }
-    }
-    if (A_log && tid < kCB) {  // warps 0 and 1, whole warps
-        pA = warp_sum(pA);
-        pba = warp_sum(pba);
-        if (lane == 0) {
-            atomicAdd(&dA_log[h], pA);
-            atomicAdd(&db_alpha[h], pba);
-        }
-    }
-    // 11b. dx = r (dx^ - x^ (x^ . dx^))
+            for (int e = 0; e < 4; ++e) dka[t][e] += x[t][e];
+        frag(L::TW + cD, x);
 #pragma unroll
-    for (int t = 0; t < CT; ++t)
+        for (int t = 0; t < CT; ++t)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int i = rowof(e), n = cD + 8 * t + 2 * tig + (e & 1);
-            if (i < nv) {
-                const size_t o = tok_off(b, t0 + i, h, T, H) * D + n;
-                const float gq = l2norm ? rq[i] * (dqa[t][e] - QH[i * LD + n] * r_pq[i]) : dqa[t][e];
-                const float gk = l2norm ? rk[i] * (dka[t][e] - KH[i * LD + n] * r_pk[i]) : dka[t][e];
-                dq[o] = from_f32<Tin>(gq);
-                dk[o] = from_f32<Tin>(gk);
+            for (int e = 0; e < 4; ++e) dqa[t][e] += x[t][e];
+        // row dots for the norm backward (k from B2, q from q^T in B4)
+        float ql = 0.f, qh_ = 0.f, kl = 0.f, kh_ = 0.f;
+#pragma unroll
+        for (int t = 0; t < CT; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = r0 + gid + 8 * hh, n = cD + 8 * t + 2 * tig;
+                const float2 kv = tpair(L::B2, i, n);
+                qh[t][2 * hh] = rq[i] * *reinterpret_cast<const float*>(sm + L::B4 + pan(D, n, i));
+                qh[t][2 * hh + 1] = rq[i] * *reinterpret_cast<const float*>(sm + L::B4 + pan(D, n + 1, i));
+                kh2[t][2 * hh] = rk[i] * kv.x;
+                kh2[t][2 * hh + 1] = rk[i] * kv.y;
+                const float pq = qh[t][2 * hh] * dqa[t][2 * hh] + qh[t][2 * hh + 1] * dqa[t][2 * hh + 1];
+                const float pk = kh2[t][2 * hh] * dka[t][2 * hh] + kh2[t][2 * hh + 1] * dka[t][2 * hh + 1];
+                if (hh == 0) { ql += pq; kl += pk; } else { qh_ += pq; kh_ += pk; }
+            }
+        row_add(r_pq, ql, qh_);
+        row_add(r_pk, kl, kh_);
+        __syncthreads();
+        // d Lg_i = gam_i d gam_i + rowM_i - colM_i (+ gC d gC for the last token); reverse cumsum
+        if (warp < 2) {
+            const int i = tid;
+            const float dec = expf(Lg[kCB - 1] - Lg[i]);
+            const float dlg = r_dbg[i] * be[i] * gam[i] + scale * gam[i] * r_g1[i] - r_dr[i] * dec;
+            dLg[i] = dlg + rowM[i] - colM[i];
+            const float rs = warp_sum(r_dr[i] * dec);
+            if (lane == 0) atomicAdd(red, rs);
+        }
+        __syncthreads();
+        if (warp == 0) {  // d ln(alpha_i) = red + sum_{i' >= i} dLg_i': lane l holds 2 l, 2 l + 1
+            const float a0 = dLg[2 * lane], a1 = dLg[2 * lane + 1];
+            float suf = a0 + a1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_down_sync(0xffffffffu, suf, o);
+                if (lane + o < 32) suf += y;
+            }
+            const float base = red[0] + suf;
+            dLg[2 * lane] = base;
+            dLg[2 * lane + 1] = base - a0;
+        }
+        __syncthreads();
+        float pA = 0.f, pba = 0.f;  // this token's share of dA_log[h], db_alpha[h] (gated form)
+        if (tid < nv) {
+            const int i = tid;
+            const size_t o = tok_off(b, t0 + i, h, T, H);
+            const float dbe = r_dbe[i] + r_dbg[i] * gam[i];
+            if (A_log) {
+                // ln alpha = -e^A softplus(x), x = a + b_alpha: d a = -e^A sigmoid(x) d ln alpha,
+                // d A = ln alpha d ln alpha, d b_alpha = d a; beta = sigmoid(b): d b = beta (1-beta) d beta
+                const float xa = alpha[o] + b_alpha[h], ea = expf(A_log[h]);
+                const float dda = -ea * gate_sigmoid(xa) * dLg[i];
+                dalpha[o] = dda;
+                dbeta[o] = dbe * be[i] * (1.f - be[i]);
+                pA = -ea * gate_softplus(xa) * dLg[i];
+                pba = dda;
+            } else {
+                dalpha[o] = dLg[i] / alpha[o];
+                dbeta[o] = dbe;
             }
         }
+        if (A_log && tid < kCB) {  // warps 0 and 1, whole warps
+            pA = warp_sum(pA);
+            pba = warp_sum(pba);
+            if (lane == 0) {
+                atomicAdd(&dA_log[h], pA);
+                atomicAdd(&db_alpha[h], pba);
+            }
+        }
+        // dx = r (dx^ - x^ (x^ . dx^))
+#pragma unroll
+        for (int t = 0; t < CT; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = r0 + gid + 8 * hh, n = cD + 8 * t + 2 * tig;
+                if (i < nv) {
+                    const size_t o = tok_off(b, t0 + i, h, T, H) * D + n;
+                    float gq[2], gk[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int e = 2 * hh + u;
+                        gq[u] = l2norm ? rq[i] * (dqa[t][e] - qh[t][e] * r_pq[i]) : dqa[t][e];
+                        gk[u] = l2norm ? rk[i] * (dka[t][e] - kh2[t][e] * r_pk[i]) : dka[t][e];
+                    }
+                    st2(dq + o, gq[0], gq[1]);
+                    st2(dk + o, gk[0], gk[1]);
+                }
+            }
+    }
+    if (!ok && tid == 0) {
+        // a wait gave up: record it, let the issued products and copies drain, then release TMEM
+        record_status(status, GDN_ERR_TIMEOUT);
+        sm100::mma_commit(&bars[LB_DRAIN]);
+        sm100::mbar_wait(&bars[LB_DRAIN], 0, never, 100000000ull);
+        for (int i = LB_C0; i <= LB_C3; ++i)
+            if (copies & (1u << i)) sm100::mbar_wait(&bars[i], 0, never, 100000000ull);
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem, L::TCOLS);
+    }
+}
+
+// 2-D tensor map over the workspace viewed as rows of C fp32 values: box 32 x 64 (one 64-row panel
+// of 128-byte rows), 128-byte swizzle.
+typedef CUresult (*BwdEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                CUtensorMapFloatOOBfill);
+BwdEncodeFn bwd_encode_fn() {
+    static const BwdEncodeFn fn = [] {
+        cudaDriverEntryPointQueryResult qr;
+        void* f = nullptr;
+        return (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &qr) == cudaSuccess &&
+                qr == cudaDriverEntryPointSuccess)
+                   ? reinterpret_cast<BwdEncodeFn>(f)
+                   : nullptr;
+    }();
+    return fn;
+}
+bool make_ws_map(CUtensorMap* m, void* base, size_t rows, int C) {
+    const BwdEncodeFn enc = bwd_encode_fn();
+    if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u)) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)C * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)kCB};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int D, typename Tin>
@@ -1038,6 +1376,9 @@ cudaError_t launch_chunked(const BackwardArgs& a, cudaStream_t st) {
     const BwdChunkWs w = bwdc_ws(a.B, a.T, a.H, D);
     if (a.ws == nullptr || a.ws_bytes < w.total * sizeof(float)) return cudaErrorInvalidValue;
     float* ws = static_cast<float*>(a.ws);
+    CUtensorMap map_d, map_64;  // the workspace as rows of D and of 64 floats (bwdc_local's copies)
+    if (!make_ws_map(&map_d, ws, w.total / D, D) || !make_ws_map(&map_64, ws, w.total / kCB, kCB))
+        return cudaErrorInvalidValue;
     const Tin* q = static_cast<const Tin*>(a.q);
     const Tin* k = static_cast<const Tin*>(a.k);
     const Tin* v = static_cast<const Tin*>(a.v);
@@ -1070,7 +1411,7 @@ cudaError_t launch_chunked(const BackwardArgs& a, cudaStream_t st) {
     bwdc_local<D, Tin><<<R, 512, LocalB<D>::BYTES, st>>>(
         q, k, v, dy, a.alpha, static_cast<Tin*>(a.dq), static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv),
         a.dalpha, a.dbeta, ws, w, a.T, a.H, nch, a.scale, a.l2norm, a.A_log, a.b_alpha, a.dA_log,
-        a.db_alpha);
+        a.db_alpha, a.status, map_d, map_64);
     return cudaGetLastError();
 }
 

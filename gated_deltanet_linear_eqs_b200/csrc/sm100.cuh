@@ -11,6 +11,8 @@
 //   bits 15/16, N >> 3 in [17,23), M >> 4 in [24,29).
 // Operand tiles use the 128-byte swizzle: rows of 128 bytes, grouped by 8 into 1024-byte atoms,
 // the 16-byte chunk c of row r stored at chunk position c ^ (r % 8).
+// Accumulators: row i of an M = 128 product sits in TMEM lane i; row i of an M = 64 product
+// (cta_group::1) in lane 32 (i / 16) + i % 16, i.e. the first 16 lanes of each warp's quarter.
 #pragma once
 
 #include <cuda.h>
@@ -150,6 +152,13 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
         : "memory");
 }
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
 // Prefetch a tile into L2 (no shared-memory destination, no barrier).
 __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
     asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
@@ -230,6 +239,24 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// kind::tf32 instruction descriptor, both operands K-major, f32 accumulator.  (On this hardware
+// the MN-major flags give no result for 32-bit operands: transposed operands are stored
+// transposed instead.)  The MMA uses the upper 19 bits of each 32-bit operand (truncation).
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32_tc(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -391,6 +418,38 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
         "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
         GDN_W8(0), GDN_W8(8), GDN_W8(16), GDN_W8(24)
         : "memory");
+}
+
+// 16x256b shape over 16 lanes from the lane field of taddr, NG = 2 or 4 groups of 8 columns:
+// thread t of the warp receives, for group g, v[4 g + 0..1] = (lane + t / 4, columns
+// 8 g + 2 (t % 4) + 0..1) and v[4 g + 2..3] = (lane + t / 4 + 8, the same columns): the
+// accumulator fragment layout of the warp-level m16n8 MMA.  Completed before returning.
+template <int NG>
+__device__ __forceinline__ void tmem_ld_frag(uint32_t taddr, float* v) {
+    static_assert(NG == 2 || NG == 4, "8 or 16 registers");
+    __syncwarp();
+    if constexpr (NG == 2) {
+        uint32_t r[8];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+            "tcgen05.wait::ld.sync.aligned;"
+            : GDN_R8(0)
+            : "r"(taddr)
+            : "memory");
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+    } else {
+        uint32_t r[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+            "tcgen05.wait::ld.sync.aligned;"
+            : GDN_R8(0), GDN_R8(8)
+            : "r"(taddr)
+            : "memory");
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+    }
 }
 #undef GDN_R8
 #undef GDN_W8
