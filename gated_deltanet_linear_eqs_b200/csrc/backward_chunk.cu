@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -399,6 +400,332 @@ __global__ void __launch_bounds__(256, 2) bwdc_prep(const Tin* __restrict__ q, c
     if (tid < kCB) {
         float* sc = ws + w.SC + r * 256;
         sc[tid] = rq[tid]; sc[64 + tid] = rk[tid]; sc[128 + tid] = Lg[tid]; sc[192 + tid] = be[tid];
+    }
+}
+
+// ---------------------------------------------------------------------------- bwdc_prep_tc
+// The same chunk matrices for bf16 inputs, with the products on tcgen05 (kind::f16, M = 64
+// tiles, fp32 accumulators in TMEM).  q, k and v arrive by TMA as 128-byte-swizzled bf16 panels
+// (64 features x 64 tokens per box), unnormalised: K K^T and Q K^T are exact in fp32 from bf16
+// operands, and the row scales rq, rk enter in the epilogue.  The products with T, W and Ut,
+// take T diag(beta gam rk) and T diag(beta) as split images hi + lo (hi = bf16(x), lo =
+// bf16(x - hi): relative error below 2^-16, finer than tf32) against k and v as MN-major
+// operands, two MMAs each.  Eight warps: warp w reads the accumulator rows 16 (w % 4) .. +15 of
+// its TMEM lane quarter in the m16n8 fragment layout, columns by halves (w / 4).
+// byte offset of element (r, m) in a bf16 panel tile of R rows (64 elements per 128-byte row)
+__device__ __forceinline__ uint32_t bpan(int R, int r, int m) {
+    return (uint32_t)((((m >> 6) * R + r) << 7) + (((((m & 63) >> 3) ^ (r & 7))) << 4) + ((m & 7) << 1));
+}
+template <int D>
+struct PrepTC {
+    static constexpr int BF = kCB * D * 2;                 // a 64 x D bf16 tile
+    static constexpr int QV = 0, KP = QV + BF, TI = KP + BF;  // Q (then V), K, four 64 x 64 images
+    static constexpr int AM = TI + 4 * 8192, TM = AM + kCB * kL64 * 4, XS = TM + kCB * kL64 * 4;
+    static constexpr int SCAL = XS + 768 * 4;             // rq, rk, Lg, beta, gam
+    static constexpr int BAR = SCAL + 5 * kCB * 4;
+    static constexpr int MISC = BAR + 8 * 8;
+    static constexpr int BYTES = MISC + 16 + 1024;        // two CTAs per SM
+    static constexpr uint32_t TCOLS = 256;
+};
+enum PrepTcBar { PT_IN = 0, PT_V, PT_M1, PT_M2, PT_DRAIN };
+
+template <int D>
+__global__ void __launch_bounds__(256, 2) bwdc_prep_tc(const float* __restrict__ alpha,
+                                                    const float* __restrict__ beta, float* __restrict__ ws,
+                                                    const BwdChunkWs w, int T, int H, int nch, float scale,
+                                                    int l2norm, const float* __restrict__ A_log,
+                                                    const float* __restrict__ b_alpha, int* __restrict__ status,
+                                                    const __grid_constant__ CUtensorMap map_q,
+                                                    const __grid_constant__ CUtensorMap map_k,
+                                                    const __grid_constant__ CUtensorMap map_v) {
+    using L = PrepTC<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* Am = reinterpret_cast<float*>(sm + L::AM);
+    float* Tm = reinterpret_cast<float*>(sm + L::TM);
+    float* Xs = reinterpret_cast<float*>(sm + L::XS);
+    float* rq = reinterpret_cast<float*>(sm + L::SCAL);
+    float* rk = rq + kCB;
+    float* Lg = rk + kCB;
+    float* be = Lg + kCB;
+    float* gam = be + kCB;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
+    volatile int* never = reinterpret_cast<volatile int*>(sm + L::MISC + 8);
+    const size_t r = blockIdx.x;
+    const int h = (int)(r % H);
+    const int gr = (int)(r / H);
+    const int c = gr % nch, b = gr / nch;
+    const int t0 = c * kCB, nv = min(kCB, T - t0);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int r0 = (warp & 3) * 16;
+    const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t sa = sm100::smem_u32(sm);
+    const int z0 = b * T + t0;  // token row of the chunk's first token in the [B T, H, D] maps
+
+    if (tid == 0) {
+        for (int i = 0; i < 8; ++i) sm100::mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        *never = 0;
+        sm100::fence_mbar_init();
+        sm100::prefetch_tmap(&map_q);
+        sm100::prefetch_tmap(&map_k);
+        sm100::prefetch_tmap(&map_v);
+    }
+    if (warp == 0) sm100::tmem_alloc(tmem_slot, L::TCOLS);
+    if (tid < kCB) {
+        const size_t o = tok_off(b, t0 + tid, h, T, H);
+        float bt = 0.f, lg = 0.f;  // rows past the end: beta = 0, alpha = 1
+        if (tid < nv) {
+            // gated form: alpha, beta hold the logits of eqs. (9)-(10)
+            bt = A_log ? gate_sigmoid(beta[o]) : beta[o];
+            lg = A_log ? gate_log_decay(alpha[o], A_log[h], b_alpha[h]) : logf(alpha[o]);
+        }
+        be[tid] = bt;
+        Lg[tid] = lg;
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    uint32_t copies = 0;  // (thread 0) copy barriers armed
+    if (tid == 0) {
+        copies |= 1u << PT_IN;
+        sm100::mbar_arrive_expect_tx(&bars[PT_IN], 2u * L::BF);
+        for (int p = 0; p < D / 64; ++p) {
+            sm100::tma_load_3d(sm + L::QV + p * 8192, &map_q, 64 * p, h, z0, &bars[PT_IN]);
+            sm100::tma_load_3d(sm + L::KP + p * 8192, &map_k, 64 * p, h, z0, &bars[PT_IN]);
+        }
+    }
+    auto wait_bar = [&](int i) {
+        bool okw = sm100::mbar_wait_warp(&bars[i], 0, abort_flag);
+        okw = __syncthreads_and(okw) != 0;
+        sm100::tc_fence_after();
+        return okw;
+    };
+    bool ok = wait_bar(PT_IN);
+    if (ok) {
+        // rows past the end of the sequence are zero (the box may have read the next one's)
+        if (nv < kCB)
+            for (int e = tid; e < 2 * (D / 64) * (kCB - nv) * 8; e += 256) {
+                const int ch = e & 7, rowi = nv + ((e >> 3) % (kCB - nv)), pp = (e >> 3) / (kCB - nv);
+                *reinterpret_cast<uint4*>(sm + (pp & 1 ? L::KP : L::QV) + (pp >> 1) * 8192 + rowi * 128 + ch * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+        __syncthreads();
+        // sums of squares: thread t takes half (t % 2) of row t / 2 of [q; k]
+        {
+            const int row = tid >> 1, half = tid & 1;
+            const uint8_t* tile = sm + (row < kCB ? L::QV : L::KP);
+            const int i = row & (kCB - 1);
+            float s = 0.f;
+#pragma unroll
+            for (int u = 0; u < D / 16; ++u) {
+                const int m = half * (D / 2) + 8 * u;
+                const uint4 x = *reinterpret_cast<const uint4*>(tile + bpan(kCB, i, m));
+                const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float lo = __uint_as_float(wv[j] << 16), hi = __uint_as_float(wv[j] & 0xffff0000u);
+                    s = fmaf(lo, lo, fmaf(hi, hi, s));
+                }
+            }
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            if (half == 0) {
+                const float rn = l2norm ? 1.0f / sqrtf(s + kNormEps) : 1.0f;
+                if (row < kCB) rq[i] = rn; else rk[i] = rn;
+            }
+        }
+        if (warp == 0) {  // inclusive cumsum of ln alpha: lane l holds 2 l, 2 l + 1
+            const float a0 = Lg[2 * lane], a1 = Lg[2 * lane + 1];
+            float pre = a0 + a1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, pre, o);
+                if (lane >= o) pre += y;
+            }
+            Lg[2 * lane + 1] = pre;
+            Lg[2 * lane] = pre - a1;
+            gam[2 * lane + 1] = expf(pre);
+            gam[2 * lane] = expf(pre - a1);
+        }
+        sm100::fence_proxy_async_smem();
+        sm100::tc_fence_before();
+        __syncthreads();
+        sm100::tc_fence_after();
+        if (tid == 0) {
+            constexpr uint32_t ID = sm100::idesc_bf16(64, 64, false, false);
+            for (int kb = 0; kb < D / 64; ++kb)
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t off = kb * 8192 + kk * 32;
+                    const uint64_t dk_ = sm100::sdesc(sa + L::KP + off, 16, 1024);
+                    const uint64_t dq_ = sm100::sdesc(sa + L::QV + off, 16, 1024);
+                    sm100::mma_bf16(tmem + 0, dk_, dk_, ID, (kb | kk) != 0);    // K K^T
+                    sm100::mma_bf16(tmem + 64, dq_, dk_, ID, (kb | kk) != 0);   // Q K^T
+                }
+            sm100::mma_commit(&bars[PT_M1]);
+        }
+        ok = wait_bar(PT_M1);
+    }
+    if (ok) {
+        if (tid == 0) {  // V into Q's place (Q is read no more)
+            copies |= 1u << PT_V;
+            sm100::mbar_arrive_expect_tx(&bars[PT_V], (uint32_t)L::BF);
+            for (int p = 0; p < D / 64; ++p)
+                sm100::tma_load_3d(sm + L::QV + p * 8192, &map_v, 64 * p, h, z0, &bars[PT_V]);
+        }
+        // A / beta and P from the fragments of K K^T and Q K^T
+        float kk4[4][4], qk4[4][4];
+        const int c0 = (warp >> 2) * 32;
+        sm100::tmem_ld_frag<4>(tmem + lq + 0 + c0, &kk4[0][0]);
+        sm100::tmem_ld_frag<4>(tmem + lq + 64 + c0, &qk4[0][0]);
+        float* Atg = ws + w.At + r * kCB * kCB;
+        float* Pg = ws + w.P + r * kCB * kCB;
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = r0 + gid + 8 * hh, j = c0 + 8 * t + 2 * tig;
+                float at[2], pp[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const float gm = expf(fminf(Lg[i] - Lg[j + u], 0.f));
+                    at[u] = j + u < i ? rk[i] * rk[j + u] * kk4[t][2 * hh + u] * gm : 0.f;
+                    pp[u] = j + u <= i ? scale * rq[i] * rk[j + u] * qk4[t][2 * hh + u] * gm : 0.f;
+                    Am[i * kL64 + j + u] = be[i] * at[u];
+                }
+                *reinterpret_cast<float2*>(Atg + i * kCB + j) = make_float2(at[0], at[1]);
+                *reinterpret_cast<float2*>(Pg + i * kCB + j) = make_float2(pp[0], pp[1]);
+            }
+        __syncthreads();
+        // T = (I + A)^-1 by 16 x 16 blocks: the diagonal blocks by forward substitution (one
+        // column per thread), then T_ij = -T_ii sum_{j <= m < i} A_im T_mj for block distance 1, 2, 3
+        if (tid < kCB) {
+            const int bb = tid >> 4, m = tid & 15, o = 16 * bb;
+            for (int ii = 0; ii < 16; ++ii) {
+                float acc = 0.f;
+                for (int j = 0; j < ii; ++j) acc = fmaf(Am[(o + ii) * kL64 + o + j], Tm[(o + j) * kL64 + o + m], acc);
+                Tm[(o + ii) * kL64 + o + m] = ii < m ? 0.f : (ii == m ? 1.f : -acc);
+            }
+        }
+        for (int e = tid; e < kCB * kCB; e += 256) {  // zero the blocks above the diagonal
+            const int ii = e / kCB, j = e % kCB;
+            if ((j >> 4) > (ii >> 4)) Tm[ii * kL64 + j] = 0.f;
+        }
+        __syncthreads();
+        for (int dd = 1; dd < 4; ++dd) {
+            const int npair = 4 - dd;
+            for (int e = tid; e < npair * 256; e += 256) {  // X = sum_m A_im T_mj
+                const int pb = e >> 8, ii = (e >> 4) & 15, j = e & 15;
+                const int bi = pb + dd, bj = pb;
+                float acc = 0.f;
+                for (int m = 16 * bj; m < 16 * bi; ++m)
+                    acc = fmaf(Am[(16 * bi + ii) * kL64 + m], Tm[m * kL64 + 16 * bj + j], acc);
+                Xs[e] = acc;
+            }
+            __syncthreads();
+            for (int e = tid; e < npair * 256; e += 256) {  // T_ij = -T_ii X
+                const int pb = e >> 8, ii = (e >> 4) & 15, j = e & 15;
+                const int bi = pb + dd, bj = pb;
+                float acc = 0.f;
+                for (int m = 0; m < 16; ++m) acc = fmaf(Tm[(16 * bi + ii) * kL64 + 16 * bi + m], Xs[(pb << 8) + (m << 4) + j], acc);
+                Tm[(16 * bi + ii) * kL64 + 16 * bj + j] = -acc;
+            }
+            __syncthreads();
+        }
+        // T (tf32-rounded, for the local-gradient kernel) and the split images of
+        // T diag(beta gam rk) and T diag(beta): thread -> (row, 8-column group)
+        float* Tg = ws + w.Tm + r * kCB * kCB;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = tid + 256 * u, i = e >> 3, j0 = (e & 7) * 8;
+            float tv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) tv[j] = Tm[i * kL64 + j0 + j];
+            *reinterpret_cast<float4*>(Tg + i * kCB + j0) = make_float4(rtf(tv[0]), rtf(tv[1]), rtf(tv[2]), rtf(tv[3]));
+            *reinterpret_cast<float4*>(Tg + i * kCB + j0 + 4) = make_float4(rtf(tv[4]), rtf(tv[5]), rtf(tv[6]), rtf(tv[7]));
+            uint32_t wh[4], wl[4], uh[4], ul[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                float x2[2], y2[2];
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2) {
+                    const int j = j0 + 2 * jj + s2;
+                    x2[s2] = tv[2 * jj + s2] * be[j] * gam[j] * rk[j];
+                    y2[s2] = tv[2 * jj + s2] * be[j];
+                }
+                const __nv_bfloat162 xh = __floats2bfloat162_rn(x2[0], x2[1]);
+                const __nv_bfloat162 yh = __floats2bfloat162_rn(y2[0], y2[1]);
+                const float2 xf = __bfloat1622float2(xh), yf = __bfloat1622float2(yh);
+                const __nv_bfloat162 xl = __floats2bfloat162_rn(x2[0] - xf.x, x2[1] - xf.y);
+                const __nv_bfloat162 yl = __floats2bfloat162_rn(y2[0] - yf.x, y2[1] - yf.y);
+                wh[jj] = *reinterpret_cast<const uint32_t*>(&xh);
+                wl[jj] = *reinterpret_cast<const uint32_t*>(&xl);
+                uh[jj] = *reinterpret_cast<const uint32_t*>(&yh);
+                ul[jj] = *reinterpret_cast<const uint32_t*>(&yl);
+            }
+            const uint32_t off = bpan(kCB, i, j0);
+            *reinterpret_cast<uint4*>(sm + L::TI + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            *reinterpret_cast<uint4*>(sm + L::TI + 8192 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+            *reinterpret_cast<uint4*>(sm + L::TI + 16384 + off) = make_uint4(uh[0], uh[1], uh[2], uh[3]);
+            *reinterpret_cast<uint4*>(sm + L::TI + 24576 + off) = make_uint4(ul[0], ul[1], ul[2], ul[3]);
+        }
+        sm100::fence_proxy_async_smem();
+        sm100::tc_fence_before();
+        ok = wait_bar(PT_V);  // (a barrier for every thread, then the copy of V)
+        if (ok && tid == 0) {
+            // W = T diag(beta gam rk) k and Ut = T diag(beta) v, k and v as MN-major operands
+            constexpr uint32_t ID = sm100::idesc_bf16(64, D, false, true);
+            for (int half = 0; half < 2; ++half)
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ta = sm100::sdesc(sa + L::TI + half * 8192 + kk * 32, 16, 1024);
+                    const uint64_t tb = sm100::sdesc(sa + L::TI + 16384 + half * 8192 + kk * 32, 16, 1024);
+                    const uint64_t kb = sm100::sdesc(sa + L::KP + kk * 2048, 8192, 1024);
+                    const uint64_t vb = sm100::sdesc(sa + L::QV + kk * 2048, 8192, 1024);
+                    sm100::mma_bf16(tmem + 0, ta, kb, ID, (half | kk) != 0);
+                    sm100::mma_bf16(tmem + D, tb, vb, ID, (half | kk) != 0);
+                }
+            sm100::mma_commit(&bars[PT_M2]);
+        }
+        if (ok) ok = wait_bar(PT_M2);
+    }
+    if (ok) {
+        float* Wg = ws + w.W + r * kCB * D;
+        float* Ug = ws + w.Ut + r * kCB * D;
+        const int c0 = (warp >> 2) * (D / 2);
+#pragma unroll
+        for (int g = 0; g < D / 64; ++g) {  // 32 columns (4 tiles) at a time
+            float wa[4][4], ua[4][4];
+            sm100::tmem_ld_frag<4>(tmem + lq + 0 + c0 + 32 * g, &wa[0][0]);
+            sm100::tmem_ld_frag<4>(tmem + lq + D + c0 + 32 * g, &ua[0][0]);
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const size_t o = (size_t)(r0 + gid + 8 * hh) * D + c0 + 32 * g + 8 * t + 2 * tig;
+                    *reinterpret_cast<float2*>(Wg + o) = make_float2(wa[t][2 * hh], wa[t][2 * hh + 1]);
+                    *reinterpret_cast<float2*>(Ug + o) = make_float2(ua[t][2 * hh], ua[t][2 * hh + 1]);
+                }
+        }
+        if (tid < kCB) {
+            float* sc = ws + w.SC + r * 256;
+            sc[tid] = rq[tid]; sc[64 + tid] = rk[tid]; sc[128 + tid] = Lg[tid]; sc[192 + tid] = be[tid];
+        }
+    }
+    if (!ok && tid == 0) {
+        record_status(status, GDN_ERR_TIMEOUT);
+        sm100::mma_commit(&bars[PT_DRAIN]);
+        sm100::mbar_wait(&bars[PT_DRAIN], 0, never, 100000000ull);
+        for (int i = PT_IN; i <= PT_V; ++i)
+            if (copies & (1u << i)) sm100::mbar_wait(&bars[i], 0, never, 100000000ull);
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem, L::TCOLS);
     }
 }
 
@@ -1370,6 +1697,20 @@ bool make_ws_map(CUtensorMap* m, void* base, size_t rows, int C) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D tensor map over a [B T, H, D] bf16 token tensor: box 64 (features) x 1 (head) x 64 (tokens),
+// 128-byte swizzle.
+bool make_tok_map(CUtensorMap* m, const void* base, long tokens, int H, int D) {
+    const BwdEncodeFn enc = bwd_encode_fn();
+    if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u)) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)tokens};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kCB};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, typename Tin>
 cudaError_t launch_chunked(const BackwardArgs& a, cudaStream_t st) {
     const int nch = (a.T + kCB - 1) / kCB;
@@ -1395,8 +1736,21 @@ cudaError_t launch_chunked(const BackwardArgs& a, cudaStream_t st) {
         (e = cudaFuncSetAttribute(bwdc_local<D, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   LocalB<D>::BYTES)) != cudaSuccess)
         return e;
-    bwdc_prep<D, Tin><<<R, 256, PrepB<D>::BYTES, st>>>(q, k, v, a.alpha, a.beta, ws, w, a.T, a.H, nch,
-                                                        a.scale, a.l2norm, a.A_log, a.b_alpha);
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
+        CUtensorMap mq, mk, mv;
+        const long tokens = (long)a.B * a.T;
+        if (!make_tok_map(&mq, q, tokens, a.H, D) || !make_tok_map(&mk, k, tokens, a.H, D) ||
+            !make_tok_map(&mv, v, tokens, a.H, D))
+            return cudaErrorInvalidValue;
+        if ((e = cudaFuncSetAttribute(bwdc_prep_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      PrepTC<D>::BYTES)) != cudaSuccess)
+            return e;
+        bwdc_prep_tc<D><<<R, 256, PrepTC<D>::BYTES, st>>>(a.alpha, a.beta, ws, w, a.T, a.H, nch, a.scale,
+                                                          a.l2norm, a.A_log, a.b_alpha, a.status, mq, mk, mv);
+    } else {
+        bwdc_prep<D, Tin><<<R, 256, PrepB<D>::BYTES, st>>>(q, k, v, a.alpha, a.beta, ws, w, a.T, a.H, nch,
+                                                            a.scale, a.l2norm, a.A_log, a.b_alpha);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwdc_fwd<D, Tin><<<chains, 256, ChainB<D>::FWD_BYTES, st>>>(k, a.s0, ws, w, a.T, a.H, nch);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
