@@ -54,7 +54,7 @@ constexpr int kL64 = 68;  // row stride (floats) of 64 x 64 shared matrices
 
 // Workspace arrays (float offsets); one record per (sequence, chunk, head), r = (b nch + c) H + h.
 struct BwdChunkWs {
-    size_t W, Ut, P, Tm, At, SC, S, U, dSp, dU, total;
+    size_t W, Ut, P, Tm, At, SC, S, U, dSp, dU, Wi, Pi, total;
 };
 BwdChunkWs bwdc_ws(int B, int T, int H, int D) {
     const size_t nch = (size_t)(T + kCB - 1) / kCB, R = (size_t)B * nch * H;
@@ -70,6 +70,8 @@ BwdChunkWs bwdc_ws(int B, int T, int H, int D) {
     w.U = o;   o += R * kCB * D;
     w.dSp = o; o += R * D * D;
     w.dU = o;  o += R * kCB * D;
+    w.Wi = o;  o += R * kCB * D;    // -W as split bf16 images hi, lo (64 x D each)
+    w.Pi = o;  o += R * kCB * kCB;  // P as split bf16 images hi, lo (64 x 64 each)
     w.total = o;
     return w;
 }
@@ -405,6 +407,15 @@ __global__ void __launch_bounds__(256, 2) bwdc_prep(const Tin* __restrict__ q, c
     }
 }
 
+// hi = bf16(x), lo = bf16(x - hi) for a pair, as two packed bf16x2 words
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 // ---------------------------------------------------------------------------- bwdc_prep_tc
 // The same chunk matrices for bf16 inputs, with the products on tcgen05 (kind::f16, M = 64
 // tiles, fp32 accumulators in TMEM).  q, k and v arrive by TMA as 128-byte-swizzled bf16 panels
@@ -585,6 +596,7 @@ __global__ void __launch_bounds__(256, 2) bwdc_prep_tc(const float* __restrict__
         sm100::tmem_ld_frag<4>(tmem + lq + 64 + c0, &qk4[0][0]);
         float* Atg = ws + w.At + r * kCB * kCB;
         float* Pg = ws + w.P + r * kCB * kCB;
+        __nv_bfloat16* Pig = reinterpret_cast<__nv_bfloat16*>(ws + w.Pi) + r * 2 * kCB * kCB;
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
@@ -600,6 +612,10 @@ __global__ void __launch_bounds__(256, 2) bwdc_prep_tc(const float* __restrict__
                 }
                 *reinterpret_cast<float2*>(Atg + i * kCB + j) = make_float2(at[0], at[1]);
                 *reinterpret_cast<float2*>(Pg + i * kCB + j) = make_float2(pp[0], pp[1]);
+                uint32_t phi, plo;  // P's split images for the reverse chain
+                split2(pp[0], pp[1], phi, plo);
+                *reinterpret_cast<uint32_t*>(Pig + i * kCB + j) = phi;
+                *reinterpret_cast<uint32_t*>(Pig + (kCB + i) * kCB + j) = plo;
             }
         __syncthreads();
         // T = (I + A)^-1 by 16 x 16 blocks: the diagonal blocks by forward substitution (one
@@ -696,6 +712,7 @@ __global__ void __launch_bounds__(256, 2) bwdc_prep_tc(const float* __restrict__
     if (ok) {
         float* Wg = ws + w.W + r * kCB * D;
         float* Ug = ws + w.Ut + r * kCB * D;
+        __nv_bfloat16* Wig = reinterpret_cast<__nv_bfloat16*>(ws + w.Wi) + r * 2 * kCB * D;
         const int c0 = (warp >> 2) * (D / 2);
 #pragma unroll
         for (int g = 0; g < D / 64; ++g) {  // 32 columns (4 tiles) at a time
@@ -709,6 +726,10 @@ __global__ void __launch_bounds__(256, 2) bwdc_prep_tc(const float* __restrict__
                     const size_t o = (size_t)(r0 + gid + 8 * hh) * D + c0 + 32 * g + 8 * t + 2 * tig;
                     *reinterpret_cast<float2*>(Wg + o) = make_float2(wa[t][2 * hh], wa[t][2 * hh + 1]);
                     *reinterpret_cast<float2*>(Ug + o) = make_float2(ua[t][2 * hh], ua[t][2 * hh + 1]);
+                    uint32_t whi, wlo;  // -W's split images for the reverse chain
+                    split2(-wa[t][2 * hh], -wa[t][2 * hh + 1], whi, wlo);
+                    *reinterpret_cast<uint32_t*>(Wig + o) = whi;
+                    *reinterpret_cast<uint32_t*>(Wig + kCB * D + o) = wlo;
                 }
         }
         if (tid < kCB) {
@@ -722,6 +743,289 @@ __global__ void __launch_bounds__(256, 2) bwdc_prep_tc(const float* __restrict__
         sm100::mbar_wait(&bars[PT_DRAIN], 0, never, 100000000ull);
         for (int i = PT_IN; i <= PT_V; ++i)
             if (copies & (1u << i)) sm100::mbar_wait(&bars[i], 0, never, 100000000ull);
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem, L::TCOLS);
+    }
+}
+
+// ---------------------------------------------------------------------------- bwdc_rev_tc
+// The reverse chain for bf16 inputs on tcgen05 (kind::f16): one CTA per (sequence, head,
+// 64-column slice of the state gradient), 256 threads, chunks in reverse.  Per chunk, with dS the
+// slice of the state gradient at the chunk's end (fp32, in registers: thread = row, 32 columns):
+//   (i)   D1 = k dS (k exact in bf16; dS as split images hi + lo), D2 = P^T dY (P as split images)
+//   (ii)  dU = diag(dec rk) D1 + D2 -> workspace, and dU's split images
+//   (iii) D3 = q^T diag(s) dY - W^T dU (q exact; diag(s) dY and W as split images; the product of
+//         two split operands takes hi hi + hi lo + lo hi), s = scale gam rq
+//   (iv)  dS <- gC dS + D3
+// Split images keep a product's relative error below about 2^-16 (tf32: 2^-11).  k, q, dY arrive
+// by TMA as bf16 panels; the split images of -W and P were written by bwdc_prep_tc.  The copies
+// for chunk c-1 start as soon as chunk c's products are done with their buffers.
+template <int D>
+struct RevTC {
+    static constexpr int BF = kCB * D * 2, T8 = kCB * kCB * 2, SB = D * kCB * 2;  // 64 x D, 64 x 64, D x 64 bf16
+    static constexpr int KP = 0, QP = KP + BF, WH = QP + BF, WL = WH + BF, PH = WL + BF, PL = PH + T8,
+                         DY = PL + T8, SH = DY + T8, SL = SH + SB, UH = SL + SB, UL = UH + T8,
+                         YH = UL + T8, YL = YH + T8;
+    static constexpr int SC = YL + T8;              // the chunk's rq, rk, Lg, beta (copied)
+    static constexpr int SCL = SC + 4 * kCB * 4;    // dec rk, s
+    static constexpr int BAR = SCL + 2 * kCB * 4;
+    static constexpr int MISC = BAR + 8 * 8;
+    static constexpr int BYTES = MISC + 16 + 1024;
+    static constexpr uint32_t TD1 = 0, TD2 = 64, TD3 = 128, TCOLS = 256;
+};
+enum RevBar { RB_A = 0, RB_B, RB_M1, RB_M2, RB_DRAIN };
+
+
+template <int D>
+__global__ void __launch_bounds__(256, 1) bwdc_rev_tc(const float* __restrict__ ds_final, float* __restrict__ ds0,
+                                                   float* __restrict__ ws, const BwdChunkWs w, int T, int H, int nch,
+                                                   float scale, int* __restrict__ status,
+                                                   const __grid_constant__ CUtensorMap map_q,
+                                                   const __grid_constant__ CUtensorMap map_k,
+                                                   const __grid_constant__ CUtensorMap map_dy,
+                                                   const __grid_constant__ CUtensorMap map_wi,
+                                                   const __grid_constant__ CUtensorMap map_pi) {
+    using L = RevTC<D>;
+    constexpr int NSL = D / 64;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const float* sc = reinterpret_cast<const float*>(sm + L::SC);
+    float* decrk = reinterpret_cast<float*>(sm + L::SCL);
+    float* sy = decrk + kCB;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
+    volatile int* never = reinterpret_cast<volatile int*>(sm + L::MISC + 8);
+    const int jsl = blockIdx.x % NSL, h = (blockIdx.x / NSL) % H, b = blockIdx.x / (NSL * H);
+    const int n0 = 64 * jsl;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int r0 = (warp & 3) * 16;
+    const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t sa = sm100::smem_u32(sm);
+    // the thread's row of the state-gradient slice and its 32 columns (M = 128: row = TMEM lane;
+    // M = 64: rows 16 (w % 4) + lane for lanes 0..15)
+    const bool has_row = (D == 128) || lane < 16;
+    const int mrow = D == 128 ? 32 * (warp & 3) + lane : 16 * (warp & 3) + (lane & 15);
+    const int cb = 32 * (warp >> 2);
+
+    if (tid == 0) {
+        for (int i = 0; i < 8; ++i) sm100::mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        *never = 0;
+        sm100::fence_mbar_init();
+        sm100::prefetch_tmap(&map_q);
+        sm100::prefetch_tmap(&map_k);
+        sm100::prefetch_tmap(&map_dy);
+        sm100::prefetch_tmap(&map_wi);
+        sm100::prefetch_tmap(&map_pi);
+    }
+    if (warp == 0) sm100::tmem_alloc(tmem_slot, L::TCOLS);
+    // the state gradient at the end of the sequence
+    float dS[32];
+    {
+        const float* src = ds_final ? ds_final + (((size_t)b * H + h) * D + mrow) * D + n0 + cb : nullptr;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float4 x = (src && has_row) ? *reinterpret_cast<const float4*>(src + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+            dS[4 * u] = x.x; dS[4 * u + 1] = x.y; dS[4 * u + 2] = x.z; dS[4 * u + 3] = x.w;
+        }
+    }
+    // dS's split images (rows m, columns n of the slice: the MN-major operand of k dS)
+    auto write_dS_images = [&]() {
+        if (!has_row) return;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) split2(dS[8 * u + 2 * p], dS[8 * u + 2 * p + 1], hi[p], lo[p]);
+            const uint32_t off = bpan(D, mrow, cb + 8 * u);
+            *reinterpret_cast<uint4*>(sm + L::SH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(sm + L::SL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+    };
+    write_dS_images();
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    uint32_t pend = 0, ppar = 0;  // (thread 0) copy barriers armed and not yet waited for, their parities
+    auto arm = [&](int i, int par, uint32_t bytes) {
+        pend |= 1u << i;
+        ppar = (ppar & ~(1u << i)) | ((uint32_t)par << i);
+        sm100::mbar_arrive_expect_tx(&bars[i], bytes);
+    };
+    auto issue_A = [&](int cc, int par) {  // k, P's images, the dY slice and the scalars of chunk cc
+        const long rr = ((long)b * nch + cc) * H + h;
+        const int z = b * T + cc * kCB;
+        arm(RB_A, par, (uint32_t)(L::BF + 3 * L::T8 + 4 * kCB * 4));
+        for (int p = 0; p < D / 64; ++p) sm100::tma_load_3d(sm + L::KP + p * 8192, &map_k, 64 * p, h, z, &bars[RB_A]);
+        sm100::tma_load_2d(sm + L::PH, &map_pi, 0, (int)(rr * 128), &bars[RB_A]);
+        sm100::tma_load_2d(sm + L::PL, &map_pi, 0, (int)(rr * 128 + 64), &bars[RB_A]);
+        sm100::tma_load_3d(sm + L::DY, &map_dy, n0, h, z, &bars[RB_A]);
+        sm100::bulk_load(sm + L::SC, ws + w.SC + rr * 256, 4 * kCB * 4, &bars[RB_A]);
+    };
+    auto issue_B = [&](int cc, int par) {  // q and -W's images of chunk cc
+        const long rr = ((long)b * nch + cc) * H + h;
+        const int z = b * T + cc * kCB;
+        arm(RB_B, par, (uint32_t)(3 * L::BF));
+        for (int p = 0; p < D / 64; ++p) {
+            sm100::tma_load_3d(sm + L::QP + p * 8192, &map_q, 64 * p, h, z, &bars[RB_B]);
+            sm100::tma_load_2d(sm + L::WH + p * 8192, &map_wi, 64 * p, (int)(rr * 128), &bars[RB_B]);
+            sm100::tma_load_2d(sm + L::WL + p * 8192, &map_wi, 64 * p, (int)(rr * 128 + 64), &bars[RB_B]);
+        }
+    };
+    auto wait_bar = [&](int i, int par) {
+        bool okw = sm100::mbar_wait_warp(&bars[i], (uint32_t)par, abort_flag);
+        okw = __syncthreads_and(okw) != 0;
+        sm100::tc_fence_after();
+        if (tid == 0 && okw) pend &= ~(1u << i);
+        return okw;
+    };
+    auto sync_issue = [&]() {
+        sm100::fence_proxy_async_smem();
+        sm100::tc_fence_before();
+        __syncthreads();
+        sm100::tc_fence_after();
+    };
+    if (tid == 0) {
+        issue_A(nch - 1, 0);
+        issue_B(nch - 1, 0);
+    }
+    constexpr uint32_t ID64 = sm100::idesc_bf16(64, 64, false, true);     // k dS
+    constexpr uint32_t IDP = sm100::idesc_bf16(64, 64, true, true);       // P^T dY
+    constexpr uint32_t ID3 = sm100::idesc_bf16(D, 64, true, true);        // q^T sdY, (-W)^T dU
+    bool ok = true;
+    for (int it = 0, c = nch - 1; ok && c >= 0; ++it, --c) {
+        const int par = it & 1;
+        const long rr = ((long)b * nch + c) * H + h;
+        const int nvc = min(kCB, T - c * kCB);
+        // dS' of chunk c -> workspace (tf32-rounded, for the local-gradient kernel)
+        if (has_row) {
+            float* g = ws + w.dSp + rr * D * D + (size_t)mrow * D + n0 + cb;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<float4*>(g + 4 * u) =
+                    make_float4(rtf(dS[4 * u]), rtf(dS[4 * u + 1]), rtf(dS[4 * u + 2]), rtf(dS[4 * u + 3]));
+        }
+        ok = wait_bar(RB_A, par);
+        if (!ok) break;
+        if (nvc < kCB)  // token rows past the end of the sequence are zero (k, dY)
+            for (int e = tid; e < (D / 64 + 1) * (kCB - nvc) * 8; e += 256) {
+                const int ch = e & 7, rowi = nvc + ((e >> 3) % (kCB - nvc)), pp = (e >> 3) / (kCB - nvc);
+                *reinterpret_cast<uint4*>(sm + (pp < D / 64 ? L::KP + pp * 8192 : L::DY) + rowi * 128 + ch * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+        const float gC = expf(sc[128 + kCB - 1]);
+        if (tid < kCB) {
+            decrk[tid] = expf(sc[128 + kCB - 1] - sc[128 + tid]) * sc[64 + tid];
+            sy[tid] = scale * expf(sc[128 + tid]) * sc[tid];
+        }
+        __syncthreads();
+        {  // diag(s) dY as split images: thread -> row j = tid / 4, 16 columns
+            const int j = tid >> 2;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int c8 = (tid & 3) * 16 + 8 * u;
+                const uint32_t off = bpan(kCB, j, c8);
+                const uint4 x = *reinterpret_cast<const uint4*>(sm + L::DY + off);
+                const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    split2(sy[j] * __uint_as_float(wv[p] << 16), sy[j] * __uint_as_float(wv[p] & 0xffff0000u), hi[p], lo[p]);
+                *reinterpret_cast<uint4*>(sm + L::YH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(sm + L::YL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
+        sync_issue();
+        if (tid == 0) {
+            for (int hl = 0; hl < 2; ++hl)  // D1 = k dS_hi + k dS_lo
+                for (int kb = 0; kb < D / 64; ++kb)
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t a = sm100::sdesc(sa + L::KP + kb * 8192 + kk * 32, 16, 1024);
+                        const uint64_t bd = sm100::sdesc(sa + (hl ? L::SL : L::SH) + (kb * 4 + kk) * 2048, L::SB, 1024);
+                        sm100::mma_bf16(tmem + L::TD1, a, bd, ID64, (hl | kb | kk) != 0);
+                    }
+            for (int hl = 0; hl < 2; ++hl)  // D2 = P_hi^T dY + P_lo^T dY
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t a = sm100::sdesc(sa + (hl ? L::PL : L::PH) + kk * 2048, 8192, 1024);
+                    const uint64_t bd = sm100::sdesc(sa + L::DY + kk * 2048, 8192, 1024);
+                    sm100::mma_bf16(tmem + L::TD2, a, bd, IDP, (hl | kk) != 0);
+                }
+            sm100::mma_commit(&bars[RB_M1]);
+        }
+        ok = wait_bar(RB_M1, par);
+        if (!ok) break;
+        if (tid == 0 && c > 0) issue_A(c - 1, par ^ 1);  // k, P, dY and the scalars are read no more
+        {  // dU = diag(dec rk) D1 + D2 -> workspace (tf32-rounded) and its split images
+            const int c0 = 32 * (warp >> 2);
+            float d1[4][4], d2[4][4];
+            sm100::tmem_ld_frag<4>(tmem + lq + L::TD1 + c0, &d1[0][0]);
+            sm100::tmem_ld_frag<4>(tmem + lq + L::TD2 + c0, &d2[0][0]);
+            float* dUg = ws + w.dU + rr * kCB * D + n0;
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int i = r0 + gid + 8 * hh, n = c0 + 8 * t + 2 * tig;
+                    const float u0 = fmaf(decrk[i], d1[t][2 * hh], d2[t][2 * hh]);
+                    const float u1 = fmaf(decrk[i], d1[t][2 * hh + 1], d2[t][2 * hh + 1]);
+                    *reinterpret_cast<float2*>(dUg + (size_t)i * D + n) = make_float2(rtf(u0), rtf(u1));
+                    uint32_t hi, lo;
+                    split2(u0, u1, hi, lo);
+                    *reinterpret_cast<uint32_t*>(sm + L::UH + bpan(kCB, i, n)) = hi;
+                    *reinterpret_cast<uint32_t*>(sm + L::UL + bpan(kCB, i, n)) = lo;
+                }
+        }
+        ok = wait_bar(RB_B, par);
+        if (!ok) break;
+        sync_issue();
+        if (tid == 0) {
+            for (int kk = 0; kk < 4; ++kk) {  // q^T (sdY_hi + sdY_lo)
+                const uint64_t a = sm100::sdesc(sa + L::QP + kk * 2048, 8192, 1024);
+                sm100::mma_bf16(tmem + L::TD3, a, sm100::sdesc(sa + L::YH + kk * 2048, 8192, 1024), ID3, kk != 0);
+                sm100::mma_bf16(tmem + L::TD3, a, sm100::sdesc(sa + L::YL + kk * 2048, 8192, 1024), ID3, 1);
+            }
+            for (int kk = 0; kk < 4; ++kk) {  // (-W)^T dU: hi hi + hi lo + lo hi
+                const uint64_t ah = sm100::sdesc(sa + L::WH + kk * 2048, 8192, 1024);
+                const uint64_t al = sm100::sdesc(sa + L::WL + kk * 2048, 8192, 1024);
+                const uint64_t bh = sm100::sdesc(sa + L::UH + kk * 2048, 8192, 1024);
+                const uint64_t bl = sm100::sdesc(sa + L::UL + kk * 2048, 8192, 1024);
+                sm100::mma_bf16(tmem + L::TD3, ah, bh, ID3, 1);
+                sm100::mma_bf16(tmem + L::TD3, ah, bl, ID3, 1);
+                sm100::mma_bf16(tmem + L::TD3, al, bh, ID3, 1);
+            }
+            sm100::mma_commit(&bars[RB_M2]);
+        }
+        ok = wait_bar(RB_M2, par);
+        if (!ok) break;
+        if (tid == 0 && c > 0) issue_B(c - 1, par ^ 1);  // q and -W are read no more
+        {  // dS <- gC dS + D3, and its split images for the next chunk's k dS
+            float d3[32];
+            sm100::tmem_ld32(tmem + lq + L::TD3 + cb, d3);
+            if (has_row)
+#pragma unroll
+                for (int j = 0; j < 32; ++j) dS[j] = fmaf(gC, dS[j], d3[j]);
+            write_dS_images();
+        }
+    }
+    if (ok && ds0 && has_row) {
+        float* g = ds0 + (((size_t)b * H + h) * D + mrow) * D + n0 + cb;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<float4*>(g + 4 * u) = make_float4(dS[4 * u], dS[4 * u + 1], dS[4 * u + 2], dS[4 * u + 3]);
+    }
+    if (!ok && tid == 0) {
+        record_status(status, GDN_ERR_TIMEOUT);
+        sm100::mma_commit(&bars[RB_DRAIN]);
+        sm100::mbar_wait(&bars[RB_DRAIN], 0, never, 100000000ull);
+        for (int i = RB_A; i <= RB_B; ++i)
+            if (pend & (1u << i)) sm100::mbar_wait(&bars[i], (ppar >> i) & 1u, never, 100000000ull);
     }
     sm100::tc_fence_before();
     __syncthreads();
@@ -1713,6 +2017,20 @@ bool make_tok_map(CUtensorMap* m, const void* base, long tokens, int H, int D) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D tensor map over a row-major bf16 array of `rows` x C (C = 64 or 128): box 64 x 64, 128-byte
+// swizzle (the split images of -W and P).
+bool make_img_map(CUtensorMap* m, void* base, size_t rows, int C) {
+    const BwdEncodeFn enc = bwd_encode_fn();
+    if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u)) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)C * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kCB};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, typename Tin>
 cudaError_t launch_chunked(const BackwardArgs& a, cudaStream_t st) {
     const int nch = (a.T + kCB - 1) / kCB;
@@ -1739,26 +2057,37 @@ cudaError_t launch_chunked(const BackwardArgs& a, cudaStream_t st) {
                                   LocalB<D>::BYTES)) != cudaSuccess)
         return e;
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
-        CUtensorMap mq, mk, mv;
+        CUtensorMap mq, mk, mv, mdy, mwi, mpi;
         const long tokens = (long)a.B * a.T;
         if (!make_tok_map(&mq, q, tokens, a.H, D) || !make_tok_map(&mk, k, tokens, a.H, D) ||
-            !make_tok_map(&mv, v, tokens, a.H, D))
+            !make_tok_map(&mv, v, tokens, a.H, D) || !make_tok_map(&mdy, dy, tokens, a.H, D) ||
+            !make_img_map(&mwi, ws + w.Wi, (size_t)R * 2 * kCB, D) ||
+            !make_img_map(&mpi, ws + w.Pi, (size_t)R * 2 * kCB, kCB))
             return cudaErrorInvalidValue;
         if ((e = cudaFuncSetAttribute(bwdc_prep_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      PrepTC<D>::BYTES)) != cudaSuccess)
+                                      PrepTC<D>::BYTES)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(bwdc_rev_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      RevTC<D>::BYTES)) != cudaSuccess)
             return e;
         bwdc_prep_tc<D><<<R, 256, PrepTC<D>::BYTES, st>>>(a.alpha, a.beta, ws, w, a.T, a.H, nch, a.scale,
                                                           a.l2norm, a.A_log, a.b_alpha, a.status, mq, mk, mv);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        bwdc_fwd<D, Tin><<<chains, 256, ChainB<D>::FWD_BYTES, st>>>(k, a.s0, ws, w, a.T, a.H, nch);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const unsigned rev_ctas = (unsigned)(a.B * a.H * (D / 64));
+        bwdc_rev_tc<D><<<rev_ctas, 256, RevTC<D>::BYTES, st>>>(a.ds_final, a.ds0, ws, w, a.T, a.H, nch,
+                                                               a.scale, a.status, mq, mk, mdy, mwi, mpi);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     } else {
         bwdc_prep<D, Tin><<<R, 256, PrepB<D>::BYTES, st>>>(q, k, v, a.alpha, a.beta, ws, w, a.T, a.H, nch,
                                                             a.scale, a.l2norm, a.A_log, a.b_alpha);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        bwdc_fwd<D, Tin><<<chains, 256, ChainB<D>::FWD_BYTES, st>>>(k, a.s0, ws, w, a.T, a.H, nch);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        bwdc_rev<D, Tin><<<chains, 256, ChainB<D>::REV_BYTES, st>>>(q, k, dy, a.ds_final, a.ds0, ws, w, a.T,
+                                                                     a.H, nch, a.scale);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwdc_fwd<D, Tin><<<chains, 256, ChainB<D>::FWD_BYTES, st>>>(k, a.s0, ws, w, a.T, a.H, nch);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwdc_rev<D, Tin><<<chains, 256, ChainB<D>::REV_BYTES, st>>>(q, k, dy, a.ds_final, a.ds0, ws, w, a.T,
-                                                                 a.H, nch, a.scale);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (a.A_log) {
         if ((e = cudaMemsetAsync(a.dA_log, 0, sizeof(float) * a.H, st)) != cudaSuccess ||
             (e = cudaMemsetAsync(a.db_alpha, 0, sizeof(float) * a.H, st)) != cudaSuccess)

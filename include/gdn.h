@@ -159,8 +159,9 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* al
  * dbeta [B,T,H] fp32; ds0 [B,H,dk,dv] fp32.
  *   ws/ws_bytes: see gdn_workspace_bytes(GDN_OP_BACKWARD, ...): per (sequence, 64-token
  *   chunk, head) the chunk's fp32 matrices (W, Ut, P, T, A/beta; 4 * (2*64*dk + 3*64*64)
- *   bytes), 1 KB of scalars, its start state and end-state gradient (2 * 4*dk*dv bytes) and
- *   its pseudo-values and their gradient (2 * 4*64*dv bytes).
+ *   bytes), 1 KB of scalars, its start state and end-state gradient (2 * 4*dk*dv bytes), its
+ *   pseudo-values and their gradient (2 * 4*64*dv bytes), and split bf16 images (hi, lo) of
+ *   -W and P (4*64*dk + 4*64*64 bytes).
  * Runs the chunked form: a chunk-parallel pass (the chunk matrices), a forward and a reverse
  * pass over the chunks (states and state gradients), and a chunk-parallel pass for every
  * token's gradients, all in fp32.

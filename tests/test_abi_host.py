@@ -66,8 +66,9 @@ def test_workspace_bytes(lib):
                                    ctypes.byref(n)) == 0
     assert n.value == 0
     # chunked backward: per (sequence, chunk, head) record, fp32: W, Ut, U, dU (64 x d each),
-    # P, T, A/beta (64 x 64 each), 256 scalars, S^c and dS' (d x d each)
-    brec = lambda d: 4 * (4 * 64 * d + 3 * 64 * 64 + 256 + 2 * d * d)
+    # P, T, A/beta (64 x 64 each), 256 scalars, S^c and dS' (d x d each); bf16 split images
+    # (hi, lo) of -W (2 x 64 x d) and of P (2 x 64 x 64)
+    brec = lambda d: 4 * (4 * 64 * d + 3 * 64 * 64 + 256 + 2 * d * d) + 2 * (2 * 64 * d + 2 * 64 * 64)
     assert lib.gdn_workspace_bytes(_abi.GDN_OP_BACKWARD, 8, 4096, 32, 128, 128, 0,
                                    ctypes.byref(n)) == 0
     assert n.value == 8 * 64 * 32 * brec(128)
