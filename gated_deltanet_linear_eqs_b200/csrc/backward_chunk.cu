@@ -752,6 +752,237 @@ __global__ void __launch_bounds__(256, 2) bwdc_prep_tc(const float* __restrict__
     }
 }
 
+// ---------------------------------------------------------------------------- bwdc_fwd_tc
+// The forward chain for bf16 inputs on tcgen05 (kind::f16): one CTA per (sequence, head,
+// 64-column slice of the state), 256 threads, two per SM.  Per chunk, with S the state slice at
+// the chunk's start (fp32, in registers: thread = row, 32 columns):
+//   (i)   D1 = (-W) S  (-W's split images from bwdc_prep_tc; S as split images; hi hi + hi lo + lo hi)
+//   (ii)  U = Ut + D1 -> workspace, and U' = diag(dec rk) U as split images
+//   (iii) D2 = k^T U'  (k exact in bf16, as the MN-major operand)
+//   (iv)  S <- gC S + D2
+// The -W images and the chunk scalars for chunk c+1 are copied as soon as (i) and the U epilogue
+// are done with theirs; k for chunk c+1 once (iii) is.
+template <int D>
+struct FwdTC {
+    static constexpr int BF = kCB * D * 2, T8 = kCB * kCB * 2, SB = D * kCB * 2;
+    static constexpr int KP = 0, WH = KP + BF, WL = WH + BF, SH = WL + BF, SL = SH + SB, UH = SL + SB,
+                         UL = UH + T8;
+    static constexpr int SC = UL + T8;              // the chunk's rq, rk, Lg, beta (copied)
+    static constexpr int SCL = SC + 4 * kCB * 4;    // dec rk
+    static constexpr int BAR = SCL + kCB * 4;
+    static constexpr int MISC = BAR + 8 * 8;
+    static constexpr int BYTES = MISC + 16 + 1024;  // two CTAs per SM
+    static constexpr uint32_t TD1 = 0, TD2 = 64, TCOLS = 128;
+};
+enum FwdBar { FB_A = 0, FB_K, FB_M1, FB_M2, FB_DRAIN };
+
+template <int D>
+__global__ void __launch_bounds__(256, 2) bwdc_fwd_tc(const float* __restrict__ s0, float* __restrict__ ws,
+                                                   const BwdChunkWs w, int T, int H, int nch,
+                                                   int* __restrict__ status,
+                                                   const __grid_constant__ CUtensorMap map_k,
+                                                   const __grid_constant__ CUtensorMap map_wi) {
+    using L = FwdTC<D>;
+    constexpr int NSL = D / 64;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const float* sc = reinterpret_cast<const float*>(sm + L::SC);
+    float* decrk = reinterpret_cast<float*>(sm + L::SCL);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
+    volatile int* never = reinterpret_cast<volatile int*>(sm + L::MISC + 8);
+    const int jsl = blockIdx.x % NSL, h = (blockIdx.x / NSL) % H, b = blockIdx.x / (NSL * H);
+    const int n0 = 64 * jsl;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int r0 = (warp & 3) * 16;
+    const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t sa = sm100::smem_u32(sm);
+    const bool has_row = (D == 128) || lane < 16;
+    const int mrow = D == 128 ? 32 * (warp & 3) + lane : 16 * (warp & 3) + (lane & 15);
+    const int cb = 32 * (warp >> 2);
+    const int c0 = 32 * (warp >> 2);  // the warp's columns in 64 x 64 results
+
+    if (tid == 0) {
+        for (int i = 0; i < 8; ++i) sm100::mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        *never = 0;
+        sm100::fence_mbar_init();
+        sm100::prefetch_tmap(&map_k);
+        sm100::prefetch_tmap(&map_wi);
+    }
+    if (warp == 0) sm100::tmem_alloc(tmem_slot, L::TCOLS);
+    float S[32];  // the state slice (row mrow, columns n0 + cb ..)
+    {
+        const float* src = s0 ? s0 + (((size_t)b * H + h) * D + mrow) * D + n0 + cb : nullptr;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float4 x = (src && has_row) ? *reinterpret_cast<const float4*>(src + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+            S[4 * u] = x.x; S[4 * u + 1] = x.y; S[4 * u + 2] = x.z; S[4 * u + 3] = x.w;
+        }
+    }
+    auto write_S_images = [&]() {
+        if (!has_row) return;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) split2(S[8 * u + 2 * p], S[8 * u + 2 * p + 1], hi[p], lo[p]);
+            const uint32_t off = bpan(D, mrow, cb + 8 * u);
+            *reinterpret_cast<uint4*>(sm + L::SH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(sm + L::SL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+    };
+    write_S_images();
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    uint32_t pend = 0, ppar = 0;
+    auto arm = [&](int i, int par, uint32_t bytes) {
+        pend |= 1u << i;
+        ppar = (ppar & ~(1u << i)) | ((uint32_t)par << i);
+        sm100::mbar_arrive_expect_tx(&bars[i], bytes);
+    };
+    auto issue_A = [&](int cc, int par) {  // -W's images and the scalars of chunk cc
+        const long rr = ((long)b * nch + cc) * H + h;
+        arm(FB_A, par, (uint32_t)(2 * L::BF + 4 * kCB * 4));
+        for (int p = 0; p < D / 64; ++p) {
+            sm100::tma_load_2d(sm + L::WH + p * 8192, &map_wi, 64 * p, (int)(rr * 128), &bars[FB_A]);
+            sm100::tma_load_2d(sm + L::WL + p * 8192, &map_wi, 64 * p, (int)(rr * 128 + 64), &bars[FB_A]);
+        }
+        sm100::bulk_load(sm + L::SC, ws + w.SC + rr * 256, 4 * kCB * 4, &bars[FB_A]);
+    };
+    auto issue_K = [&](int cc, int par) {  // k of chunk cc
+        arm(FB_K, par, (uint32_t)L::BF);
+        for (int p = 0; p < D / 64; ++p)
+            sm100::tma_load_3d(sm + L::KP + p * 8192, &map_k, 64 * p, h, b * T + cc * kCB, &bars[FB_K]);
+    };
+    auto wait_bar = [&](int i, int par) {
+        bool okw = sm100::mbar_wait_warp(&bars[i], (uint32_t)par, abort_flag);
+        okw = __syncthreads_and(okw) != 0;
+        sm100::tc_fence_after();
+        if (tid == 0 && okw) pend &= ~(1u << i);
+        return okw;
+    };
+    auto sync_issue = [&]() {
+        sm100::fence_proxy_async_smem();
+        sm100::tc_fence_before();
+        __syncthreads();
+        sm100::tc_fence_after();
+    };
+    if (tid == 0) {
+        issue_A(0, 0);
+        issue_K(0, 0);
+    }
+    constexpr uint32_t ID1 = sm100::idesc_bf16(64, 64, false, true);   // (-W) S
+    constexpr uint32_t ID2 = sm100::idesc_bf16(D, 64, true, true);     // k^T U'
+    bool ok = true;
+    for (int c = 0; ok && c < nch; ++c) {
+        const int par = c & 1;
+        const long rr = ((long)b * nch + c) * H + h;
+        const int nvc = min(kCB, T - c * kCB);
+        // S^c -> workspace (tf32-rounded, for the local-gradient kernel)
+        if (has_row) {
+            float* g = ws + w.S + rr * D * D + (size_t)mrow * D + n0 + cb;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<float4*>(g + 4 * u) =
+                    make_float4(rtf(S[4 * u]), rtf(S[4 * u + 1]), rtf(S[4 * u + 2]), rtf(S[4 * u + 3]));
+        }
+        // this warp's fragment of Ut (read while the products run)
+        float2 ut[4][2];
+        {
+            const float* Utg = ws + w.Ut + rr * kCB * D + n0;
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    ut[t][hh] = *reinterpret_cast<const float2*>(Utg + (size_t)(r0 + gid + 8 * hh) * D + c0 + 8 * t + 2 * tig);
+        }
+        ok = wait_bar(FB_A, par);
+        if (!ok) break;
+        const float gC = expf(sc[128 + kCB - 1]);
+        if (tid < kCB) decrk[tid] = expf(sc[128 + kCB - 1] - sc[128 + tid]) * sc[64 + tid];
+        sync_issue();
+        if (tid == 0) {  // D1 = (-W) S: hi hi + hi lo + lo hi
+            for (int kb = 0; kb < D / 64; ++kb)
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t ao = kb * 8192 + kk * 32, bo = (kb * 4 + kk) * 2048;
+                    const uint64_t ah = sm100::sdesc(sa + L::WH + ao, 16, 1024);
+                    const uint64_t al = sm100::sdesc(sa + L::WL + ao, 16, 1024);
+                    const uint64_t bh = sm100::sdesc(sa + L::SH + bo, L::SB, 1024);
+                    const uint64_t bl = sm100::sdesc(sa + L::SL + bo, L::SB, 1024);
+                    sm100::mma_bf16(tmem + L::TD1, ah, bh, ID1, (kb | kk) != 0);
+                    sm100::mma_bf16(tmem + L::TD1, ah, bl, ID1, 1);
+                    sm100::mma_bf16(tmem + L::TD1, al, bh, ID1, 1);
+                }
+            sm100::mma_commit(&bars[FB_M1]);
+        }
+        ok = wait_bar(FB_M1, par);
+        if (!ok) break;
+        {  // U = Ut + D1 -> workspace (tf32-rounded); U' = diag(dec rk) U as split images
+            float d1[4][4];
+            sm100::tmem_ld_frag<4>(tmem + lq + L::TD1 + c0, &d1[0][0]);
+            float* Ug = ws + w.U + rr * kCB * D + n0;
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int i = r0 + gid + 8 * hh, n = c0 + 8 * t + 2 * tig;
+                    const float u0 = ut[t][hh].x + d1[t][2 * hh], u1 = ut[t][hh].y + d1[t][2 * hh + 1];
+                    *reinterpret_cast<float2*>(Ug + (size_t)i * D + n) = make_float2(rtf(u0), rtf(u1));
+                    uint32_t hi, lo;
+                    split2(decrk[i] * u0, decrk[i] * u1, hi, lo);
+                    *reinterpret_cast<uint32_t*>(sm + L::UH + bpan(kCB, i, n)) = hi;
+                    *reinterpret_cast<uint32_t*>(sm + L::UL + bpan(kCB, i, n)) = lo;
+                }
+        }
+        ok = wait_bar(FB_K, par);
+        if (!ok) break;
+        if (nvc < kCB)  // rows past the end of the sequence are zero
+            for (int e = tid; e < (D / 64) * (kCB - nvc) * 8; e += 256) {
+                const int ch = e & 7, rowi = nvc + ((e >> 3) % (kCB - nvc)), pp = (e >> 3) / (kCB - nvc);
+                *reinterpret_cast<uint4*>(sm + L::KP + pp * 8192 + rowi * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+            }
+        sync_issue();
+        if (tid == 0) {  // D2 = k^T (U'_hi + U'_lo)
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t a = sm100::sdesc(sa + L::KP + kk * 2048, 8192, 1024);
+                sm100::mma_bf16(tmem + L::TD2, a, sm100::sdesc(sa + L::UH + kk * 2048, 8192, 1024), ID2, kk != 0);
+                sm100::mma_bf16(tmem + L::TD2, a, sm100::sdesc(sa + L::UL + kk * 2048, 8192, 1024), ID2, 1);
+            }
+            sm100::mma_commit(&bars[FB_M2]);
+            if (c + 1 < nch) issue_A(c + 1, par ^ 1);  // -W and the scalars are read no more
+        }
+        ok = wait_bar(FB_M2, par);
+        if (!ok) break;
+        if (tid == 0 && c + 1 < nch) issue_K(c + 1, par ^ 1);  // k is read no more
+        {  // S <- gC S + D2, and its split images for the next chunk
+            float d2[32];
+            sm100::tmem_ld32(tmem + lq + L::TD2 + cb, d2);
+            if (has_row)
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[j] = fmaf(gC, S[j], d2[j]);
+            write_S_images();
+        }
+    }
+    if (!ok && tid == 0) {
+        record_status(status, GDN_ERR_TIMEOUT);
+        sm100::mma_commit(&bars[FB_DRAIN]);
+        sm100::mbar_wait(&bars[FB_DRAIN], 0, never, 100000000ull);
+        for (int i = FB_A; i <= FB_K; ++i)
+            if (pend & (1u << i)) sm100::mbar_wait(&bars[i], (ppar >> i) & 1u, never, 100000000ull);
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem, L::TCOLS);
+    }
+}
+
 // ---------------------------------------------------------------------------- bwdc_rev_tc
 // The reverse chain for bf16 inputs on tcgen05 (kind::f16): one CTA per (sequence, head,
 // 64-column slice of the state gradient), 256 threads, chunks in reverse.  Per chunk, with dS the
@@ -2066,17 +2297,19 @@ cudaError_t launch_chunked(const BackwardArgs& a, cudaStream_t st) {
             return cudaErrorInvalidValue;
         if ((e = cudaFuncSetAttribute(bwdc_prep_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       PrepTC<D>::BYTES)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(bwdc_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      FwdTC<D>::BYTES)) != cudaSuccess ||
             (e = cudaFuncSetAttribute(bwdc_rev_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       RevTC<D>::BYTES)) != cudaSuccess)
             return e;
         bwdc_prep_tc<D><<<R, 256, PrepTC<D>::BYTES, st>>>(a.alpha, a.beta, ws, w, a.T, a.H, nch, a.scale,
                                                           a.l2norm, a.A_log, a.b_alpha, a.status, mq, mk, mv);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        bwdc_fwd<D, Tin><<<chains, 256, ChainB<D>::FWD_BYTES, st>>>(k, a.s0, ws, w, a.T, a.H, nch);
+        const unsigned slice_ctas = (unsigned)(a.B * a.H * (D / 64));  // 64-column state slices
+        bwdc_fwd_tc<D><<<slice_ctas, 256, FwdTC<D>::BYTES, st>>>(a.s0, ws, w, a.T, a.H, nch, a.status, mk, mwi);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        const unsigned rev_ctas = (unsigned)(a.B * a.H * (D / 64));
-        bwdc_rev_tc<D><<<rev_ctas, 256, RevTC<D>::BYTES, st>>>(a.ds_final, a.ds0, ws, w, a.T, a.H, nch,
-                                                               a.scale, a.status, mq, mk, mdy, mwi, mpi);
+        bwdc_rev_tc<D><<<slice_ctas, 256, RevTC<D>::BYTES, st>>>(a.ds_final, a.ds0, ws, w, a.T, a.H, nch,
+                                                                 a.scale, a.status, mq, mk, mdy, mwi, mpi);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     } else {
         bwdc_prep<D, Tin><<<R, 256, PrepB<D>::BYTES, st>>>(q, k, v, a.alpha, a.beta, ws, w, a.T, a.H, nch,
