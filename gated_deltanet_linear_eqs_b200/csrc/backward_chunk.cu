@@ -1,9 +1,10 @@
 // backward_chunk.cu -- the backward pass of eqs. (1)-(4) (Qwen3.8-Flash-Next summary, picx.dev,
 // "Theoretical foundations"; the reverse recurrence of its Appendix B) in the chunked WY form of
-// the forward, on 64-token chunks, in fp32 with the products on tensor cores: tcgen05 tiles in
-// the chunk-parallel kernels (bwdc_prep_tc, bwdc_local), warp-level m16n8k8 tf32 tiles in the
-// sequential chains (the reverse chain's dS products with split 3 x tf32 operands, since their
-// rounding accumulates into dS0 along the whole chain).
+// the forward, on 64-token chunks, with fp32 states and accumulation and the products on tensor
+// cores.  For bf16 inputs every kernel runs tcgen05 tiles (bwdc_prep_tc, bwdc_fwd_tc,
+// bwdc_rev_tc with exact or split bf16 operands; bwdc_local with tf32 operands); for fp32 inputs
+// the chunk matrices and the chains run warp-level m16n8k8 tf32 tiles (the reverse chain's dS
+// products with split 3 x tf32 operands, since their rounding accumulates into dS0).
 //
 // Per chunk, with q^ = rq q, k^ = rk k the normalised rows, Lg the inclusive cumsum of ln(alpha),
 // gam = e^Lg, gC = gam of the chunk's last token, Gam_ij = e^(Lg_i - Lg_j), S = S^c the state at
@@ -31,9 +32,11 @@
 //
 // Kernels (one launch each, in stream order):
 //   bwdc_prep   one CTA per (chunk, head): norms, Lg, A / beta (kept for dbeta), P, T, W, Ut
-//               (bwdc_prep_tc for bf16 inputs, bwdc_prep for fp32)
-//   bwdc_fwd    one CTA per (sequence, head, 32 state columns): S^c and U of every chunk
-//   bwdc_rev    one CTA per (sequence, head, 32 state columns): dS' and dU of every chunk, dS0
+//               (bwdc_prep_tc for bf16 inputs, which also writes split images of -W and P)
+//   bwdc_fwd    one CTA per (sequence, head, state slice): S^c and U of every chunk
+//               (bwdc_fwd_tc for bf16 inputs: 64-column slices; bwdc_fwd: 32)
+//   bwdc_rev    one CTA per (sequence, head, state slice): dS' and dU of every chunk, dS0
+//               (bwdc_rev_tc for bf16 inputs: 64-column slices; bwdc_rev: 32)
 //   bwdc_local  one CTA per (chunk, head): all gradients of the chunk's tokens
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
