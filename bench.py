@@ -304,6 +304,9 @@ def run_ours(args, rank, world, local_rank):
 QSA_BUDGET = 512
 
 
+QSA_SRC = "gated_deltanet_linear_eqs_b200/csrc/qsa_indexer.cu"
+
+
 def run_qsa(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier):
     """The QSA block indexer over the prefill workload's stream (T = 32768, 4 documents) with
     4 indexer query heads and one key head of dim 128 and the budget of 512 blocks: the scores
@@ -345,12 +348,16 @@ def run_qsa(args, dev, uuid, peaks, peak_src, max_over_ranks, barrier):
             tf = flops / (ms / 1e3) / 1e12
             roof = {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
                     "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"], "flops_per_launch": flops,
-                    "traffic": None, "peak_source": peak_src}
+                    "traffic": profile_traffic("qsa_indexer_T32768.md", QSA_SRC,
+                                               key="score_dram_bytes_per_launch"),
+                    "peak_source": peak_src}
         else:
             gbs = sel_bytes / (ms / 1e3) / 1e9
             roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": sel_bytes,
-                    "traffic": None, "peak_source": peak_src}
+                    "traffic": profile_traffic("qsa_indexer_T32768.md", QSA_SRC,
+                                               key="select_dram_bytes_per_launch"),
+                    "peak_source": peak_src}
         res[name] = {"ms_per_launch": ms, "roofline": roof, "clocks": clk.summary()}
     res["config"] = {"workload": f"QSA indexer: {T_TOTAL} tokens in {NDOCS} seeded documents, "
                                  f"4 query heads + 1 key head of dim 128, blocks of 4 tokens, "
