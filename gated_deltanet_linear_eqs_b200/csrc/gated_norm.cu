@@ -10,22 +10,26 @@
 //     dy = r (dn - n mean(dn n)),  dw = sum over rows of do s n.
 //
 // Both are streaming passes (read y, z [, do], write o [, dy, dz]); nothing is reused, so the
-// bound is HBM.  Layout: a row of dv = 128 (64) values is read by 32 (16) lanes, four
-// consecutive values each (8-byte loads for bf16, 16-byte for fp32), so a warp instruction
-// covers whole 256-byte (bf16) rows.  Each warp takes four rows per step to keep more loads in
-// flight; the grid is at most 8 blocks per SM, with grid-stride loops over warp steps.
+// bound is HBM.  The reads are staged through shared memory by bulk copies so that many of them
+// are in flight independently of the registers: one persistent CTA per SM, one producer warp
+// that copies tiles of consecutive rows (8 KB of each input tensor per tile) into a ring of
+// stages, and eight consumer warps that normalise the rows of a stage (a row of 16 bytes per lane,
+// row sums by shuffles) and write the outputs straight to global memory with streaming stores.
+// Every wait is bounded: a wait that gives up records GDN_ERR_TIMEOUT and the CTA unwinds.
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace gdn {
 
 namespace {
 
-constexpr int kNormThreads = 256;
-constexpr int kRowsPerStep = 4;  // rows each lane group loads before computing
+constexpr int kConsumers = 8;                      // consumer warps
+constexpr int kNormThreads = 32 * (kConsumers + 1);  // + the producer warp
+constexpr int kTileBytes = 8192;                   // per input tensor per tile
 
-// sigmoid(x) = 1 / (1 + e^-x) and 1 / sqrt(x), with the fast exponential, divide and reciprocal
-// square root intrinsics (the outputs are rounded to the rows' dtype afterwards)
+// sigmoid(x) = 1 / (1 + e^-x) with the fast exponential and divide intrinsics (the outputs are
+// rounded to the rows' dtype afterwards)
 __device__ __forceinline__ float fast_sigmoid(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
 // sum over the LPR lanes that share a row (LPR a power of two, <= 32)
@@ -36,159 +40,205 @@ __device__ __forceinline__ float row_sum(float x) {
     return x;
 }
 
-__device__ __forceinline__ float dot4(float4 a, float4 b) {
-    return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
-}
-
-template <int DV, typename T>
-__global__ void __launch_bounds__(kNormThreads)
-gated_norm_kernel(const T* __restrict__ y, const T* __restrict__ z, const float* __restrict__ w,
-                  T* __restrict__ o, long long rows, float eps) {
-    constexpr int LPR = DV / 4;      // lanes per row
-    constexpr int RPW = 32 / LPR;    // rows per warp instruction
-    constexpr int RW = RPW * kRowsPerStep;  // rows of one warp step
-    const int lane = threadIdx.x & 31;
-    const int col = (lane % LPR) * 4;
-    // the loop runs per warp (its bound is warp-uniform), so every shuffle sees the whole warp
-    const long long gw = ((long long)blockIdx.x * kNormThreads + threadIdx.x) >> 5;
-    const long long nw = (long long)gridDim.x * (kNormThreads / 32);
-    const float4 wv = *reinterpret_cast<const float4*>(w + col);
-    const float4 g = make_float4(1.f + wv.x, 1.f + wv.y, 1.f + wv.z, 1.f + wv.w);
-    for (long long wb = gw * RW; wb < rows; wb += nw * RW) {
-        float4 yv[kRowsPerStep], zv[kRowsPerStep];
+// 16 bytes of a row in shared memory -> fp32 values; fp32 values -> 16 bytes of a row in global
+// memory (streaming store)
+__device__ __forceinline__ void ld16(const uint8_t* p, float* x, __nv_bfloat16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int u = 0; u < kRowsPerStep; ++u) {
-            const long long row = wb + u * RPW + lane / LPR;
-            if (row < rows) {
-                yv[u] = load4(y + row * DV + col);
-                zv[u] = load4(z + row * DV + col);
-            } else {
-                yv[u] = zv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kRowsPerStep; ++u) {
-            const long long row = wb + u * RPW + lane / LPR;
-            const float r = rsqrtf(row_sum<LPR>(dot4(yv[u], yv[u])) * (1.0f / DV) + eps);
-            float4 ov;
-            ov.x = g.x * yv[u].x * r * fast_sigmoid(zv[u].x);
-            ov.y = g.y * yv[u].y * r * fast_sigmoid(zv[u].y);
-            ov.z = g.z * yv[u].z * r * fast_sigmoid(zv[u].z);
-            ov.w = g.w * yv[u].w * r * fast_sigmoid(zv[u].w);
-            if (row < rows) store4(o + row * DV + col, ov);
-        }
+    for (int j = 0; j < 4; ++j) {
+        x[2 * j] = __uint_as_float(w[j] << 16);
+        x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
     }
 }
+__device__ __forceinline__ void ld16(const uint8_t* p, float* x, float) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+}
+__device__ __forceinline__ void st16(__nv_bfloat16* p, const float* x) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
+        w[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    __stcs(reinterpret_cast<uint4*>(p), make_uint4(w[0], w[1], w[2], w[3]));
+}
+__device__ __forceinline__ void st16(float* p, const float* x) {
+    __stcs(reinterpret_cast<float4*>(p), make_float4(x[0], x[1], x[2], x[3]));
+}
 
-template <int DV, typename T>
-__global__ void __launch_bounds__(kNormThreads)
-gated_norm_bwd_kernel(const T* __restrict__ y, const T* __restrict__ z,
-                      const float* __restrict__ w, const T* __restrict__ d_o, T* __restrict__ dy,
-                      T* __restrict__ dz, float* __restrict__ dw, long long rows, float eps) {
-    constexpr int LPR = DV / 4;
-    constexpr int RPW = 32 / LPR;
-    __shared__ float4 s_dw[kNormThreads / 32][LPR];
-    constexpr int RW = RPW * kRowsPerStep;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int col = (lane % LPR) * 4;
-    const long long gw = ((long long)blockIdx.x * kNormThreads + threadIdx.x) >> 5;
-    const long long nw = (long long)gridDim.x * (kNormThreads / 32);
-    const float4 wv = *reinterpret_cast<const float4*>(w + col);
-    const float4 g = make_float4(1.f + wv.x, 1.f + wv.y, 1.f + wv.z, 1.f + wv.w);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);  // this lane's columns of dw
-    for (long long wb = gw * RW; wb < rows; wb += nw * RW) {
-        float4 yv[kRowsPerStep], zv[kRowsPerStep], dv[kRowsPerStep];
-#pragma unroll
-        for (int u = 0; u < kRowsPerStep; ++u) {
-            const long long row = wb + u * RPW + lane / LPR;
-            if (row < rows) {
-                yv[u] = load4(y + row * DV + col);
-                zv[u] = load4(z + row * DV + col);
-                dv[u] = load4(d_o + row * DV + col);
-            } else {
-                yv[u] = zv[u] = dv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+template <int DV, typename T, bool BWD>
+struct NormCfg {
+    static constexpr int ROWB = DV * (int)sizeof(T);     // bytes per row
+    static constexpr int VPL = 16 / (int)sizeof(T);      // values per lane
+    static constexpr int LPR = DV / VPL;                 // lanes per row
+    static constexpr int RPW = 32 / LPR;                 // rows per warp instruction
+    static constexpr int R = kTileBytes / ROWB;          // rows per tile
+    static constexpr int NT = BWD ? 3 : 2;               // input tensors
+    static constexpr int STAGES = BWD ? 5 : 6;
+    static constexpr int STAGE = NT * kTileBytes;
+    static constexpr int BAR = STAGES * STAGE;           // full[STAGES], empty[STAGES]
+    static constexpr int MISC = BAR + 2 * STAGES * 8;    // abort flag
+    static constexpr int DWS = MISC + 16;                // dw partials: kConsumers x DV floats
+    static constexpr int BYTES = DWS + (BWD ? kConsumers * DV * 4 : 0) + 1024;
+    static_assert(R % (kConsumers * RPW) == 0, "rows of a tile split evenly over the warps");
+};
+
+template <int DV, typename T, bool BWD>
+__global__ void __launch_bounds__(kNormThreads, 1)
+gated_norm_kernel(const T* __restrict__ y, const T* __restrict__ z, const T* __restrict__ d_o,
+                  const float* __restrict__ w, T* __restrict__ o, T* __restrict__ dy,
+                  T* __restrict__ dz, float* __restrict__ dw, long long rows, float eps,
+                  int* __restrict__ status) {
+    using C = NormCfg<DV, T, BWD>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::BAR);
+    uint64_t* empty = full + C::STAGES;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::MISC);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long ntiles = (rows + C::R - 1) / C::R;
+    if (tid == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            sm100::mbar_init(&full[s], 1);
+            sm100::mbar_init(&empty[s], kConsumers);
         }
-#pragma unroll
-        for (int u = 0; u < kRowsPerStep; ++u) {
-            const long long row = wb + u * RPW + lane / LPR;
-            const float r = rsqrtf(row_sum<LPR>(dot4(yv[u], yv[u])) * (1.0f / DV) + eps);
-            const float4 n = make_float4(yv[u].x * r, yv[u].y * r, yv[u].z * r, yv[u].w * r);
-            const float4 s = make_float4(fast_sigmoid(zv[u].x), fast_sigmoid(zv[u].y),
-                                         fast_sigmoid(zv[u].z), fast_sigmoid(zv[u].w));
-            const float4 ds = make_float4(dv[u].x * s.x, dv[u].y * s.y, dv[u].z * s.z, dv[u].w * s.w);
-            const float4 dn = make_float4(ds.x * g.x, ds.y * g.y, ds.z * g.z, ds.w * g.w);
-            const float m = row_sum<LPR>(dot4(dn, n)) * (1.0f / DV);
-            float4 gy, gz;
-            gy.x = r * (dn.x - n.x * m); gy.y = r * (dn.y - n.y * m);
-            gy.z = r * (dn.z - n.z * m); gy.w = r * (dn.w - n.w * m);
-            gz.x = dn.x * n.x * (1.f - s.x); gz.y = dn.y * n.y * (1.f - s.y);
-            gz.z = dn.z * n.z * (1.f - s.z); gz.w = dn.w * n.w * (1.f - s.w);
-            if (row < rows) {  // rows past the end (zeros; r may be inf) add nothing
-                acc.x = fmaf(ds.x, n.x, acc.x); acc.y = fmaf(ds.y, n.y, acc.y);
-                acc.z = fmaf(ds.z, n.z, acc.z); acc.w = fmaf(ds.w, n.w, acc.w);
-                store4(dy + row * DV + col, gy);
-                store4(dz + row * DV + col, gz);
-            }
-        }
+        *abort_flag = 0;
+        sm100::fence_mbar_init();
     }
-    // lanes that share columns (the RPW rows of a warp instruction), then the block's warps
-#pragma unroll
-    for (int o = LPR; o < 32; o <<= 1) {
-        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
-        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
-        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
-        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
-    }
-    if (lane < LPR) s_dw[warp][lane] = acc;
     __syncthreads();
-    if (threadIdx.x < LPR) {
-        float4 t = s_dw[0][threadIdx.x];
-#pragma unroll
-        for (int k = 1; k < kNormThreads / 32; ++k) {
-            const float4 x = s_dw[k][threadIdx.x];
-            t.x += x.x; t.y += x.y; t.z += x.z; t.w += x.w;
+    if (warp == kConsumers) {
+        // ------------------------------------------------------------ producer (one lane)
+        if (lane == 0) {
+            int it = 0;
+            for (long long tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++it) {
+                const int s = it % C::STAGES;
+                if (it >= C::STAGES &&
+                    !sm100::mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1, abort_flag))
+                    break;
+                const long long r0 = tile * C::R;
+                const uint32_t bytes = (uint32_t)((rows - r0 < C::R ? rows - r0 : C::R) * C::ROWB);
+                sm100::mbar_arrive_expect_tx(&full[s], bytes * C::NT);
+                uint8_t* dst = sm + s * C::STAGE;
+                sm100::bulk_load(dst, reinterpret_cast<const uint8_t*>(y) + r0 * C::ROWB, bytes, &full[s]);
+                sm100::bulk_load(dst + kTileBytes, reinterpret_cast<const uint8_t*>(z) + r0 * C::ROWB, bytes,
+                                 &full[s]);
+                if (BWD)
+                    sm100::bulk_load(dst + 2 * kTileBytes, reinterpret_cast<const uint8_t*>(d_o) + r0 * C::ROWB,
+                                     bytes, &full[s]);
+            }
+            // copies still in flight land before the CTA may end (bounded)
+            for (int k = (it > C::STAGES ? it - C::STAGES : 0); k < it; ++k) {
+                int never = 0;
+                sm100::mbar_wait(&full[k % C::STAGES], (k / C::STAGES) & 1, &never, 100000000ull);
+            }
         }
-        float* p = dw + threadIdx.x * 4;
-        atomicAdd(p + 0, t.x);
-        atomicAdd(p + 1, t.y);
-        atomicAdd(p + 2, t.z);
-        atomicAdd(p + 3, t.w);
+        return;
+    }
+    // ---------------------------------------------------------------- consumers
+    const int col = (lane % C::LPR) * C::VPL;
+    float g[C::VPL], acc[C::VPL];  // the gain 1 + w of this lane's columns; its dw partial
+#pragma unroll
+    for (int j = 0; j < C::VPL; ++j) {
+        g[j] = 1.f + w[col + j];
+        acc[j] = 0.f;
+    }
+    int it = 0;
+    for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        const int s = it % C::STAGES;
+        if (!sm100::mbar_wait_warp(&full[s], (it / C::STAGES) & 1, abort_flag)) {
+            if (lane == 0 && atomicExch(const_cast<int*>(abort_flag), 1) == 0) record_status(status, GDN_ERR_TIMEOUT);
+            break;
+        }
+        const uint8_t* st = sm + s * C::STAGE;
+        const long long r0 = tile * C::R;
+#pragma unroll
+        for (int k = 0; k < C::R / (kConsumers * C::RPW); ++k) {
+            const int rr = (k * kConsumers + warp) * C::RPW + lane / C::LPR;  // row within the tile
+            const long long row = r0 + rr;
+            float yv[C::VPL], zv[C::VPL];
+            ld16(st + rr * C::ROWB + col * (int)sizeof(T), yv, T());
+            ld16(st + kTileBytes + rr * C::ROWB + col * (int)sizeof(T), zv, T());
+            float ss = 0.f;
+#pragma unroll
+            for (int j = 0; j < C::VPL; ++j) ss = fmaf(yv[j], yv[j], ss);
+            const float r = rsqrtf(row_sum<C::LPR>(ss) * (1.0f / DV) + eps);
+            if constexpr (!BWD) {
+                float ov[C::VPL];
+#pragma unroll
+                for (int j = 0; j < C::VPL; ++j) ov[j] = g[j] * yv[j] * r * fast_sigmoid(zv[j]);
+                if (row < rows) st16(o + row * DV + col, ov);
+            } else {
+                float dv[C::VPL];
+                ld16(st + 2 * kTileBytes + rr * C::ROWB + col * (int)sizeof(T), dv, T());
+                float n[C::VPL], sg[C::VPL], ds[C::VPL], dn[C::VPL];
+                float m = 0.f;
+#pragma unroll
+                for (int j = 0; j < C::VPL; ++j) {
+                    n[j] = yv[j] * r;
+                    sg[j] = fast_sigmoid(zv[j]);
+                    ds[j] = dv[j] * sg[j];
+                    dn[j] = ds[j] * g[j];
+                    m = fmaf(dn[j], n[j], m);
+                }
+                m = row_sum<C::LPR>(m) * (1.0f / DV);
+                float gy[C::VPL], gz[C::VPL];
+#pragma unroll
+                for (int j = 0; j < C::VPL; ++j) {
+                    gy[j] = r * (dn[j] - n[j] * m);
+                    gz[j] = dn[j] * n[j] * (1.f - sg[j]);
+                }
+                if (row < rows) {  // rows past the end of the tensor add nothing
+#pragma unroll
+                    for (int j = 0; j < C::VPL; ++j) acc[j] = fmaf(ds[j], n[j], acc[j]);
+                    st16(dy + row * DV + col, gy);
+                    st16(dz + row * DV + col, gz);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&empty[s]);
+    }
+    if constexpr (BWD) {
+        // dw: the lanes that share columns (the RPW rows of a warp instruction), then the warps
+        float* dws = reinterpret_cast<float*>(sm + C::DWS);
+#pragma unroll
+        for (int o2 = C::LPR; o2 < 32; o2 <<= 1)
+#pragma unroll
+            for (int j = 0; j < C::VPL; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o2);
+        if (lane < C::LPR)
+#pragma unroll
+            for (int j = 0; j < C::VPL; ++j) dws[warp * DV + col + j] = acc[j];
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * kConsumers) : "memory");  // the consumer warps
+        for (int c = tid; c < DV; c += 32 * kConsumers) {
+            float t = 0.f;
+#pragma unroll
+            for (int k2 = 0; k2 < kConsumers; ++k2) t += dws[k2 * DV + c];
+            atomicAdd(dw + c, t);
+        }
     }
 }
 
-// Blocks: enough for every row slot, at most 8 resident blocks (2048 threads) per SM.
-cudaError_t norm_grid(long long rows, int dv, unsigned* grid) {
+// One CTA per SM (its shared memory holds the ring), at most one per tile.
+template <int DV, typename T, bool BWD>
+cudaError_t launch(const GatedNormArgs& a, cudaStream_t st) {
+    using C = NormCfg<DV, T, BWD>;
     int dev = 0, nsm = 0;
     cudaError_t e;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
         (e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    const long long rows_per_block = (long long)(kNormThreads / 32) * (128 / dv) * kRowsPerStep;
-    const long long need = (rows + rows_per_block - 1) / rows_per_block;
-    const long long cap = 8LL * nsm;
-    *grid = (unsigned)(need < cap ? need : cap);
-    return cudaSuccess;
-}
-
-template <int DV, typename T>
-cudaError_t fwd(const GatedNormArgs& a, cudaStream_t st) {
-    unsigned grid = 0;
-    if (cudaError_t e = norm_grid(a.rows, DV, &grid)) return e;
-    gated_norm_kernel<DV, T><<<grid, kNormThreads, 0, st>>>(
-        static_cast<const T*>(a.y), static_cast<const T*>(a.z), a.w, static_cast<T*>(a.o), a.rows,
-        a.eps);
-    return cudaGetLastError();
-}
-
-template <int DV, typename T>
-cudaError_t bwd(const GatedNormArgs& a, cudaStream_t st) {
-    unsigned grid = 0;
-    if (cudaError_t e = norm_grid(a.rows, DV, &grid)) return e;
-    if (cudaError_t e = cudaMemsetAsync(a.dw, 0, sizeof(float) * DV, st)) return e;
-    gated_norm_bwd_kernel<DV, T><<<grid, kNormThreads, 0, st>>>(
-        static_cast<const T*>(a.y), static_cast<const T*>(a.z), a.w, static_cast<const T*>(a.d_o),
-        static_cast<T*>(a.dy), static_cast<T*>(a.dz), a.dw, a.rows, a.eps);
+    const long long ntiles = (a.rows + C::R - 1) / C::R;
+    const unsigned grid = (unsigned)(ntiles < nsm ? ntiles : nsm);
+    if ((e = cudaFuncSetAttribute(gated_norm_kernel<DV, T, BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  C::BYTES)) != cudaSuccess)
+        return e;
+    if (BWD && (e = cudaMemsetAsync(a.dw, 0, sizeof(float) * DV, st)) != cudaSuccess) return e;
+    gated_norm_kernel<DV, T, BWD><<<grid, kNormThreads, C::BYTES, st>>>(
+        static_cast<const T*>(a.y), static_cast<const T*>(a.z), static_cast<const T*>(a.d_o), a.w,
+        static_cast<T*>(a.o), static_cast<T*>(a.dy), static_cast<T*>(a.dz), a.dw, a.rows, a.eps,
+        a.status);
     return cudaGetLastError();
 }
 
@@ -197,15 +247,15 @@ cudaError_t bwd(const GatedNormArgs& a, cudaStream_t st) {
 cudaError_t launch_gated_norm(const GatedNormArgs& a, cudaStream_t st) {
     if (a.rows == 0) return cudaSuccess;
     if (a.dtype == GDN_BF16)
-        return a.dv == 128 ? fwd<128, __nv_bfloat16>(a, st) : fwd<64, __nv_bfloat16>(a, st);
-    return a.dv == 128 ? fwd<128, float>(a, st) : fwd<64, float>(a, st);
+        return a.dv == 128 ? launch<128, __nv_bfloat16, false>(a, st) : launch<64, __nv_bfloat16, false>(a, st);
+    return a.dv == 128 ? launch<128, float, false>(a, st) : launch<64, float, false>(a, st);
 }
 
 cudaError_t launch_gated_norm_backward(const GatedNormArgs& a, cudaStream_t st) {
     if (a.rows == 0) return cudaMemsetAsync(a.dw, 0, sizeof(float) * a.dv, st);
     if (a.dtype == GDN_BF16)
-        return a.dv == 128 ? bwd<128, __nv_bfloat16>(a, st) : bwd<64, __nv_bfloat16>(a, st);
-    return a.dv == 128 ? bwd<128, float>(a, st) : bwd<64, float>(a, st);
+        return a.dv == 128 ? launch<128, __nv_bfloat16, true>(a, st) : launch<64, __nv_bfloat16, true>(a, st);
+    return a.dv == 128 ? launch<128, float, true>(a, st) : launch<64, float, true>(a, st);
 }
 
 }  // namespace gdn

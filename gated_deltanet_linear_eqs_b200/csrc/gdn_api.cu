@@ -334,7 +334,7 @@ int gdn_gated_rmsnorm(const void* y, const void* z, const float* w, void* o, int
     DeviceInfo dev;
     if (int rc = current_device_info(&dev)) return rc;
     gdn::GatedNormArgs a{y, z, w, nullptr, o, nullptr, nullptr, nullptr, (long long)rows, dv,
-                         dtype, eps};
+                         dtype, eps, dev.status};
     return map_cuda(gdn::launch_gated_norm(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -350,7 +350,8 @@ int gdn_gated_rmsnorm_backward(const void* y, const void* z, const float* w, con
     if (dv != 64 && dv != 128) return GDN_ERR_UNSUPPORTED_SHAPE;
     DeviceInfo dev;
     if (int rc = current_device_info(&dev)) return rc;
-    gdn::GatedNormArgs a{y, z, w, d_o, nullptr, dy, dz, dw, (long long)rows, dv, dtype, eps};
+    gdn::GatedNormArgs a{y, z, w, d_o, nullptr, dy, dz, dw, (long long)rows, dv, dtype, eps,
+                         dev.status};
     return map_cuda(gdn::launch_gated_norm_backward(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -100,6 +100,7 @@ struct GatedNormArgs {
     long long rows;
     int dv, dtype;
     float eps;
+    int* status;           // device status word (bounded waits that give up)
 };
 cudaError_t launch_gated_norm(const GatedNormArgs& a, cudaStream_t st);
 cudaError_t launch_gated_norm_backward(const GatedNormArgs& a, cudaStream_t st);
