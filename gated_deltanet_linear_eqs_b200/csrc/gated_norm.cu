@@ -76,7 +76,7 @@ struct NormCfg {
     static constexpr int RPW = 32 / LPR;                 // rows per warp instruction
     static constexpr int R = kTileBytes / ROWB;          // rows per tile
     static constexpr int NT = BWD ? 3 : 2;               // input tensors
-    static constexpr int STAGES = BWD ? 5 : 6;
+    static constexpr int STAGES = BWD ? 5 : 8;
     static constexpr int STAGE = NT * kTileBytes;
     static constexpr int BAR = STAGES * STAGE;           // full[STAGES], empty[STAGES]
     static constexpr int MISC = BAR + 2 * STAGES * 8;    // abort flag
