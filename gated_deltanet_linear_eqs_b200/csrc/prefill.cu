@@ -107,13 +107,13 @@ __device__ __forceinline__ void load_half_row(const uint8_t* tile, int row, int 
 #pragma unroll
     for (int c = 0; c < 4; ++c) unpack8(*reinterpret_cast<const uint4*>(tile + swz(row, c0 + c)), x + 8 * c);
 }
-// Sum of squares of one swizzled bf16 row of 64 elements.
-__device__ __forceinline__ float row_sumsq(const uint8_t* tile, int row) {
+// Sum of squares of one half (columns 32 half .. +31) of a swizzled bf16 row of 64 elements.
+__device__ __forceinline__ float row_sumsq_half(const uint8_t* tile, int row, int half) {
     float s[8] = {};
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
         float x[8];
-        unpack8(*reinterpret_cast<const uint4*>(tile + swz(row, c)), x);
+        unpack8(*reinterpret_cast<const uint4*>(tile + swz(row, 4 * half + c)), x);
 #pragma unroll
         for (int e = 0; e < 8; ++e) s[e] = fmaf(x[e], x[e], s[e]);
     }
@@ -218,7 +218,7 @@ struct PrepLayout {
     static_assert(TWN % 1024 == 0 && TF + 64 * kLd * 2 >= TWN + 16384, "T_w / N_b tile");
     static_assert(2 * (BYTES + 1024 + 1024) <= 233472, "two prep CTAs per SM");
 };
-enum { PS_G = 0, PS_GAM, PS_BETA, PS_RK, PS_RQ, PS_FTW, PS_CARRY, PS_COLF };
+enum { PS_G = 0, PS_GAM, PS_BETA, PS_RK, PS_RQ, PS_FTW, PS_UNUSED, PS_COLF };
 enum { PB_FULL = 0, PB_TMEM, PB_M1, PB_RA1, PB_M3, PB_RW, PB_MX, PB_FIN, PB_COUNT };
 
 struct PrepParams {
@@ -459,72 +459,67 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         float* sRk = scal(PS_RK);
         float* sRq = scal(PS_RQ);
         float* sFtw = scal(PS_FTW);
-        float* sCarry = scal(PS_CARRY);
         float* sColf = scal(PS_COLF);
         float* rs = p.ws_s + rec * (kRecS / 4);
 
-        // (1) decay and norms
+        // (1) decay and norms.  Row t of [K; Q] is summed by both warps of its lane quadrant (hf:
+        // the first or the second half of each 64-column block); warp 8 scans log2(alpha) over
+        // the chunk, two tokens per lane.
+        float* sPart = reinterpret_cast<float*>(sm + L::XB);  // free until the T merges
         bool ok = wwait(PB_FULL, 0);
-        if (ok && hf == 0) {
-            if (t < 64) {
-                float gl = ab[t];  // log2(alpha)
+        float ss = 0.f;
+        if (ok) {
+            const uint8_t* rows = sm + L::KQ + (t < 64 ? 0 : 8192);
+#pragma unroll
+            for (int b = 0; b < KB; ++b) ss += row_sumsq_half(rows + b * 16384, t & 63, hf);
+            if (hf == 1) sPart[t] = ss;
+            if (warp == 8) {
+                const float a0 = ab[2 * lane], a1 = ab[2 * lane + 1];
+                float incl = a0 + a1;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
-                    const float x = __shfl_up_sync(0xffffffffu, gl, o);
-                    if (lane >= o) gl += x;
+                    const float x = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += x;
                 }
-                if (t == 31) sCarry[0] = gl;
-                float ss = 0.f;
-#pragma unroll
-                for (int b = 0; b < KB; ++b) ss += row_sumsq(sm + L::KQ + b * 16384, t);
-                sRk[t] = p.l2norm ? 1.0f / sqrtf(ss + kNormEps) : 1.0f;
-                sBeta[t] = ab[64 + t];
-                sG[t] = gl;
-            } else {
-                const int r = t - 64;
-                float ss = 0.f;
-#pragma unroll
-                for (int b = 0; b < KB; ++b) ss += row_sumsq(sm + L::KQ + b * 16384 + 8192, r);
-                sRq[r] = p.l2norm ? 1.0f / sqrtf(ss + kNormEps) : 1.0f;
+                sG[2 * lane] = incl - a1;
+                sG[2 * lane + 1] = incl;
+                sBeta[2 * lane] = ab[64 + 2 * lane];
+                sBeta[2 * lane + 1] = ab[65 + 2 * lane];
             }
         }
         named_sync(1, 256);
-        if (ok && hf == 0 && t >= 32 && t < 64) sG[t] += sCarry[0];
-        named_sync(1, 256);
         const float Glast = sG[nvalid - 1];
         if (ok && hf == 0) {
+            const float rn = p.l2norm ? 1.0f / sqrtf(ss + sPart[t] + kNormEps) : 1.0f;
             if (t < 64) {
                 const float G = sG[t], gam = ex2(G);
+                sRk[t] = rn;
                 sGam[t] = gam;
                 sColf[t] = ex2(sG[t | 15] - G);  // decay from token t to the end of its 16-block
-                sFtw[t] = sBeta[t] * gam * sRk[t];
-                rs[t] = (t < nvalid) ? ex2(Glast - G) * sRk[t] : 0.f;
+                sFtw[t] = sBeta[t] * gam * rn;
+                rs[t] = (t < nvalid) ? ex2(Glast - G) * rn : 0.f;
                 if (t == 0) rs[128] = ex2(Glast);
             } else {
                 const int r = t - 64;
-                rs[64 + r] = p.scale * ex2(sG[r]) * sRq[r];
+                sRq[r] = rn;
+                rs[64 + r] = p.scale * ex2(sG[r]) * rn;
             }
         }
         named_sync(1, 256);
 
         // (2) A (rows 0-63 of M1, to shared memory) and P (rows 64-127, to the workspace)
-        ok = wwait(PB_TMEM, 0) && ok;
-        tc_fence_after();
-        const uint32_t tmem = *tmem_slot;
-        ok = wwait(PB_M1, 0) && ok;
-        tc_fence_after();
         // Gam_ij = 2^(G_i - G_j) for j <= i.  Within the row's own 16-token block it is computed
         // directly; for an earlier block b it is the product 2^(G_i - G_e) 2^(G_e - G_j) through
         // the block's last token e = 16 b + 15.  Both exponents are <= 0 (G does not increase),
-        // so neither factor can overflow, and a row needs 20 exponentials instead of 64.
-        if (ok) {
-            const int i = t & 63, blk = i >> 4;
-            const bool arow = t < 64;  // rows of A (strictly lower) or of P (lower, diagonal incl.)
+        // so neither factor can overflow, and a row needs 20 exponentials instead of 64.  They
+        // are taken while the products run.
+        const int i = t & 63, blk = i >> 4;
+        const bool arow = t < 64;  // rows of A (strictly lower) or of P (lower, diagonal incl.)
+        // this warp's columns: blocks 2 hf and 2 hf + 1; the row's own block is among them when
+        // blk / 2 == hf (the same for the whole warp)
+        float rf[2], dg[16];
+        {
             const float Gi = sG[i];
-            const float sc = arow ? sBeta[i] * sRk[i] : p.scale * sRq[i];
-            // this warp's columns: blocks 2 hf and 2 hf + 1; the row's own block is among them
-            // when blk / 2 == hf (the same for the whole warp)
-            float rf[2], dg[16];
 #pragma unroll
             for (int k = 0; k < 2; ++k) rf[k] = ex2(Gi - sG[16 * (2 * hf + k) + 15]);
             if ((blk >> 1) == hf) {
@@ -534,6 +529,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                 for (int u = 0; u < 16; ++u) dg[u] = 0.f;
             }
+        }
+        ok = wwait(PB_TMEM, 0) && ok;
+        tc_fence_after();
+        const uint32_t tmem = *tmem_slot;
+        ok = wwait(PB_M1, 0) && ok;
+        tc_fence_after();
+        if (ok) {
+            const float sc = arow ? sBeta[i] * sRk[i] : p.scale * sRq[i];
             const int lim = arow ? i : i + 1;  // columns j < lim are kept
             uint8_t* P = p.ws_p + rec * kRecP;
             float d[32];
