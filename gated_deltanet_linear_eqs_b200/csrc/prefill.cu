@@ -1103,17 +1103,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                         for (int j = 0; j < 16; ++j) S[j] = fmaf(gprev, S[j], d[j] + e[j]);
                     }
-                    if (ywarp) {
-                        // P_{a-1} U_{a-1} (M4b(a), complete before M5(a-1) is): into registers,
-                        // so that the accumulator is released at once
-                        const int cy = a - 1;
-                        ok = wwait(CB_M4B + (cy & 1), (cy >> 1) & 1, cy) && ok;
-                        tc_fence_after();
-                        if (ok) tmem_ld16(tmem + L::T_D4B + (cy & 1) * 128 + 64 + lane_base + col0, pu);
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&bars[CB_YD + (cy & 1)]);
-                    }
                 }
                 if (a < nch) {
                     // S^a -> bf16 operand rows (columns col0 .. col0 + 15 of the 64-wide tile)
@@ -1133,8 +1122,17 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     }
                 }
                 if (ywarp && a >= 1) {
-                    // Y_{a-1} = ysc (Q_{a-1} S^{a-1}) + P_{a-1} U_{a-1}: rows 0-63 of M4a(a), M4b(a)
+                    // Y_{a-1} = ysc (Q_{a-1} S^{a-1}) + P_{a-1} U_{a-1}: rows 0-63 of M4a(a), M4b(a).
+                    // P_{a-1} U_{a-1} (M4b(a), complete before M5(a-1) is) goes into registers at
+                    // once, releasing the accumulator; both are read after the state image is out,
+                    // which the next product waits for.
                     const int cy = a - 1;
+                    ok = wwait(CB_M4B + (cy & 1), (cy >> 1) & 1, cy) && ok;
+                    tc_fence_after();
+                    if (ok) tmem_ld16(tmem + L::T_D4B + (cy & 1) * 128 + 64 + lane_base + col0, pu);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[CB_YD + (cy & 1)]);
                     ok = wwait(CB_M4A + (a & 1), (a >> 1) & 1, a) && ok;
                     tc_fence_after();
                     if (ok) {
