@@ -13,8 +13,9 @@
 // bound is HBM.  The reads are staged through shared memory by bulk copies so that many of them
 // are in flight independently of the registers: one persistent CTA per SM, one producer warp
 // that copies tiles of consecutive rows (8 KB of each input tensor per tile) into a ring of
-// stages, and eight consumer warps that normalise the rows of a stage (a row of 16 bytes per lane,
-// row sums by shuffles) and write the outputs straight to global memory with streaming stores.
+// stages, and consumer warps (16 in the forward, 8 in the backward) that normalise the rows of a
+// stage (a row of 16 bytes per lane, row sums by shuffles) and write the outputs straight to global
+// memory with streaming stores.
 // Every wait is bounded: a wait that gives up records GDN_ERR_TIMEOUT and the CTA unwinds.
 #include "common.cuh"
 #include "internal.h"
@@ -24,8 +25,12 @@ namespace gdn {
 
 namespace {
 
-constexpr int kConsumers = 8;                      // consumer warps
-constexpr int kNormThreads = 32 * (kConsumers + 1);  // + the producer warp
+// consumer warps: 16 in the forward (two inputs, one output: more warps keep more of the output
+// stores in flight), 8 in the backward (three inputs, two outputs and the dw partials)
+template <bool BWD>
+constexpr int consumers() { return BWD ? 8 : 16; }
+template <bool BWD>
+constexpr int norm_threads() { return 32 * (consumers<BWD>() + 1); }  // + the producer warp
 constexpr int kTileBytes = 8192;                   // per input tensor per tile
 
 // sigmoid(x) = 1 / (1 + e^-x) with the fast exponential and divide intrinsics (the outputs are
@@ -80,13 +85,14 @@ struct NormCfg {
     static constexpr int STAGE = NT * kTileBytes;
     static constexpr int BAR = STAGES * STAGE;           // full[STAGES], empty[STAGES]
     static constexpr int MISC = BAR + 2 * STAGES * 8;    // abort flag
-    static constexpr int DWS = MISC + 16;                // dw partials: kConsumers x DV floats
-    static constexpr int BYTES = DWS + (BWD ? kConsumers * DV * 4 : 0) + 1024;
-    static_assert(R % (kConsumers * RPW) == 0, "rows of a tile split evenly over the warps");
+    static constexpr int NC = consumers<BWD>();           // consumer warps
+    static constexpr int DWS = MISC + 16;                // dw partials: NC x DV floats
+    static constexpr int BYTES = DWS + (BWD ? NC * DV * 4 : 0) + 1024;
+    static_assert(R % (NC * RPW) == 0, "rows of a tile split evenly over the warps");
 };
 
 template <int DV, typename T, bool BWD>
-__global__ void __launch_bounds__(kNormThreads, 1)
+__global__ void __launch_bounds__(norm_threads<BWD>(), 1)
 gated_norm_kernel(const T* __restrict__ y, const T* __restrict__ z, const T* __restrict__ d_o,
                   const float* __restrict__ w, T* __restrict__ o, T* __restrict__ dy,
                   T* __restrict__ dz, float* __restrict__ dw, long long rows, float eps,
@@ -102,13 +108,13 @@ gated_norm_kernel(const T* __restrict__ y, const T* __restrict__ z, const T* __r
     if (tid == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             sm100::mbar_init(&full[s], 1);
-            sm100::mbar_init(&empty[s], kConsumers);
+            sm100::mbar_init(&empty[s], C::NC);
         }
         *abort_flag = 0;
         sm100::fence_mbar_init();
     }
     __syncthreads();
-    if (warp == kConsumers) {
+    if (warp == C::NC) {
         // ------------------------------------------------------------ producer (one lane)
         if (lane == 0) {
             int it = 0;
@@ -154,8 +160,8 @@ gated_norm_kernel(const T* __restrict__ y, const T* __restrict__ z, const T* __r
         const uint8_t* st = sm + s * C::STAGE;
         const long long r0 = tile * C::R;
 #pragma unroll
-        for (int k = 0; k < C::R / (kConsumers * C::RPW); ++k) {
-            const int rr = (k * kConsumers + warp) * C::RPW + lane / C::LPR;  // row within the tile
+        for (int k = 0; k < C::R / (C::NC * C::RPW); ++k) {
+            const int rr = (k * C::NC + warp) * C::RPW + lane / C::LPR;  // row within the tile
             const long long row = r0 + rr;
             float yv[C::VPL], zv[C::VPL];
             ld16(st + rr * C::ROWB + col * (int)sizeof(T), yv, T());
@@ -210,11 +216,11 @@ gated_norm_kernel(const T* __restrict__ y, const T* __restrict__ z, const T* __r
         if (lane < C::LPR)
 #pragma unroll
             for (int j = 0; j < C::VPL; ++j) dws[warp * DV + col + j] = acc[j];
-        asm volatile("bar.sync 1, %0;" ::"r"(32 * kConsumers) : "memory");  // the consumer warps
-        for (int c = tid; c < DV; c += 32 * kConsumers) {
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * C::NC) : "memory");  // the consumer warps
+        for (int c = tid; c < DV; c += 32 * C::NC) {
             float t = 0.f;
 #pragma unroll
-            for (int k2 = 0; k2 < kConsumers; ++k2) t += dws[k2 * DV + c];
+            for (int k2 = 0; k2 < C::NC; ++k2) t += dws[k2 * DV + c];
             atomicAdd(dw + c, t);
         }
     }
@@ -235,7 +241,7 @@ cudaError_t launch(const GatedNormArgs& a, cudaStream_t st) {
                                   C::BYTES)) != cudaSuccess)
         return e;
     if (BWD && (e = cudaMemsetAsync(a.dw, 0, sizeof(float) * DV, st)) != cudaSuccess) return e;
-    gated_norm_kernel<DV, T, BWD><<<grid, kNormThreads, C::BYTES, st>>>(
+    gated_norm_kernel<DV, T, BWD><<<grid, norm_threads<BWD>(), C::BYTES, st>>>(
         static_cast<const T*>(a.y), static_cast<const T*>(a.z), static_cast<const T*>(a.d_o), a.w,
         static_cast<T*>(a.o), static_cast<T*>(a.dy), static_cast<T*>(a.dz), a.dw, a.rows, a.eps,
         a.status);
