@@ -13,9 +13,9 @@
 // bound is HBM.  The reads are staged through shared memory by bulk copies so that many of them
 // are in flight independently of the registers: one persistent CTA per SM, one producer warp
 // that copies tiles of consecutive rows (8 KB of each input tensor per tile) into a ring of
-// stages, and consumer warps (16 in the forward, 8 in the backward) that normalise the rows of a
-// stage (a row of 16 bytes per lane, row sums by shuffles) and write the outputs straight to global
-// memory with streaming stores.
+// stages (six in the forward, five in the backward), and consumer warps (16 in the forward, 8 in
+// the backward) that normalise the rows of a stage (a row of 16 bytes per lane, row sums by
+// shuffles) and write the outputs straight to global memory with streaming stores.
 // Every wait is bounded: a wait that gives up records GDN_ERR_TIMEOUT and the CTA unwinds.
 #include "common.cuh"
 #include "internal.h"
@@ -81,7 +81,7 @@ struct NormCfg {
     static constexpr int RPW = 32 / LPR;                 // rows per warp instruction
     static constexpr int R = kTileBytes / ROWB;          // rows per tile
     static constexpr int NT = BWD ? 3 : 2;               // input tensors
-    static constexpr int STAGES = BWD ? 5 : 8;
+    static constexpr int STAGES = BWD ? 5 : 6;          // the fastest in a sweep of 3 .. 12
     static constexpr int STAGE = NT * kTileBytes;
     static constexpr int BAR = STAGES * STAGE;           // full[STAGES], empty[STAGES]
     static constexpr int MISC = BAR + 2 * STAGES * 8;    // abort flag
